@@ -1,0 +1,330 @@
+/*
+ * oracle.c -- plain, slow, obviously correct CPU oracle for the
+ * SmoothQuant-style W8A8 linear path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * CPU-baseline leg of the benchmark may load this library.  The CUDA product
+ * path never links, calls or includes anything from here, and this file
+ * includes nothing from the product path.
+ *
+ * Sources (web pages on LLM post-training quantization):
+ *   [SQ]  "SmoothQuant大模型量化技术深度解析" (developer.baidu.com),
+ *         section 1 "SmoothQuant技术原理": smoothing factor
+ *         s_j = max|X_j|^a / max|W_j|^(1-a), activations divided by s and
+ *         weights multiplied by s so the product is unchanged.
+ *   [SSZ] "SSZ：权重量化算法说明" (msModelSlim docs), sections
+ *         "算法流程" (MinMax init, least-squares update, greedy keep,
+ *         repeat until converged or out of iterations), "迭代优化阶段"
+ *         (symmetric: offset fixed at 0, only the scale is optimised),
+ *         "收敛判断" (relative and absolute change tests; stop when every
+ *         channel has converged), "算法参数" (20 iterations, threshold
+ *         1e-10, minimum scale 1e-5), "使用限制" (int8 / int4 per-channel
+ *         symmetric, 2-D weights only).
+ *   [CQ]  CUDA INT8 quantization notes (aicoding.csdn.net), section 2.1
+ *         "量化基础理论": Q = round(R/S) + Z with range calibration,
+ *         parameter computation and saturation; section 3.2 (INT8 matrix
+ *         multiply with 32-bit accumulation); section 4.2 (dequantization
+ *         fused after the integer product).
+ *   [PTQ] "训练后量化（PTQ）" tutorial, "PTQ 的基本流程" (calibrate on a
+ *         small set, then compute scales) and "逐层量化 vs 逐通道量化"
+ *         (one scale per output channel).
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *   - channel j of W in the smoothing factor is input channel j (column j of
+ *     the [N,K] weight); it is the only reading under which diag(s) cancels.
+ *   - s_j = 1 when max|X_j| == 0 or max|W_j| == 0.
+ *   - pow is evaluated in fp64 and rounded once to fp32.
+ *   - "round" is round-half-to-even; activations clamp to [-127, 127];
+ *     int4 codes clamp to [-7, 7] (qmax = 2^(bits-1) - 1).
+ *   - the minimum scale floors every weight scale (init and candidates).
+ *   - the quantization error is the mean over K of the squared residual,
+ *     summed in fp64; a candidate's error is measured after re-quantising
+ *     with the candidate scale.
+ *   - the relative and absolute convergence tests are OR-ed, evaluated
+ *     before the greedy update, and convergence is per channel and sticky.
+ *   - the activation scale of an all-zero row is 0 and its codes are 0.
+ *
+ * Arithmetic: IEEE binary32 for every quantity that decides a code, fp64
+ * for error and least-squares sums, exact integers for the matrix product.
+ * Build with -ffp-contract=off and without fast-math.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define SSZ_CONVERGE_THRESHOLD 1e-10 /* [SSZ] 算法参数 */
+#define SSZ_MIN_SCALE 1e-5f          /* [SSZ] 算法参数 */
+#define ACT_QMAX 127                 /* symmetric int8, narrow range */
+
+/* ---------------------------------------------------------------- step 1 */
+/* Per-input-channel activation absmax, [SQ] max(|X_j|), gathered over the
+ * calibration tokens ([PTQ] calibration step).  x is [M,K] row-major.
+ * accumulate != 0 folds the new batch into the running max in ax. */
+void oracle_calib_absmax(const float *x, int64_t M, int64_t K, float *ax,
+                         int accumulate)
+{
+    for (int64_t j = 0; j < K; ++j)
+        if (!accumulate)
+            ax[j] = 0.0f;
+    for (int64_t t = 0; t < M; ++t) {
+        const float *row = x + t * K;
+        for (int64_t j = 0; j < K; ++j) {
+            float a = fabsf(row[j]);
+            if (a > ax[j])
+                ax[j] = a;
+        }
+    }
+}
+
+/* ---------------------------------------------------------------- step 2a */
+/* Per-input-channel weight absmax, [SQ] max(|W_j|): w is [N,K] row-major,
+ * aw[j] = max_n |w[n,j]|. */
+void oracle_weight_col_absmax(const float *w, int64_t N, int64_t K, float *aw)
+{
+    oracle_calib_absmax(w, N, K, aw, 0);
+}
+
+/* ---------------------------------------------------------------- step 2b */
+/* Smoothing factor [SQ]: s_j = ax_j^alpha / aw_j^(1-alpha), evaluated in
+ * fp64 and rounded once; inv_s_j = 1/s_j in fp32. */
+void oracle_smooth_factor(const float *ax, const float *aw, int64_t K,
+                          float alpha, float *s, float *inv_s)
+{
+    double a = (double)alpha;
+    for (int64_t j = 0; j < K; ++j) {
+        float sj;
+        if (ax[j] == 0.0f || aw[j] == 0.0f)
+            sj = 1.0f;
+        else
+            sj = (float)(pow((double)ax[j], a) / pow((double)aw[j], 1.0 - a));
+        s[j] = sj;
+        inv_s[j] = 1.0f / sj;
+    }
+}
+
+/* ---------------------------------------------------------------- step 2c */
+/* Fold [SQ]: every column j of a [R,K] matrix times f[j] (one fp32 multiply).
+ * With f = s this is W' = W diag(s); with f = 1/s it is X' = X diag(s)^-1. */
+void oracle_scale_columns(const float *a, int64_t R, int64_t K, const float *f,
+                          float *out)
+{
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t j = 0; j < K; ++j)
+            out[r * K + j] = a[r * K + j] * f[j];
+}
+
+/* ---------------------------------------------------------------- step 3 */
+/* Symmetric code [CQ] 2.1 with Z = 0: clamp(round(w / s), -qmax, qmax),
+ * fp32 division, ties to even. */
+static float sym_code(float w, float s, int qmax)
+{
+    float r = rintf(w / s);
+    if (r > (float)qmax)
+        r = (float)qmax;
+    if (r < -(float)qmax)
+        r = -(float)qmax;
+    return r;
+}
+
+/* Quantization error of one channel at scale s: mean over K of
+ * (w_k - s*Q(w_k,s))^2, accumulated in fp64 in index order. */
+static double channel_mse(const float *w, int64_t K, float s, int qmax)
+{
+    double acc = 0.0;
+    for (int64_t k = 0; k < K; ++k) {
+        double e = (double)w[k] - (double)s * (double)sym_code(w[k], s, qmax);
+        acc += e * e;
+    }
+    return acc / (double)K;
+}
+
+/* SSZ scale search for one output channel ([SSZ] 算法流程, 迭代优化阶段,
+ * 收敛判断), symmetric per-channel.  Returns the number of least-squares
+ * rounds taken.  trace (nullable) gets the best error after the MinMax init
+ * (trace[0]) and after each round (trace[1..max_iters]); unused rounds
+ * repeat the final value. */
+static int ssz_channel(const float *w, int64_t K, int qmax, int max_iters,
+                       float *scale, double *mse, double *trace)
+{
+    /* MinMax observer, symmetric: scale = max|w| / qmax, offset 0. */
+    float amax = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+        float a = fabsf(w[k]);
+        if (a > amax)
+            amax = a;
+    }
+    float s_best = amax / (float)qmax;
+    if (s_best < SSZ_MIN_SCALE)
+        s_best = SSZ_MIN_SCALE;
+    double m_best = channel_mse(w, K, s_best, qmax);
+    if (trace)
+        trace[0] = m_best;
+
+    int it = 0;
+    int done = 0;
+    while (it < max_iters && !done) {
+        ++it;
+        /* Least squares for the codes of the current best scale:
+         * argmin_s sum (w - s q)^2 = sum(w q) / sum(q q). */
+        double num = 0.0;
+        int64_t den = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            float q = sym_code(w[k], s_best, qmax);
+            num += (double)w[k] * (double)q;
+            den += (int64_t)q * (int64_t)q;
+        }
+        float s_cand = s_best;
+        if (den != 0) {
+            s_cand = (float)(num / (double)den);
+            if (s_cand < SSZ_MIN_SCALE)
+                s_cand = SSZ_MIN_SCALE;
+        }
+        double m_cand = channel_mse(w, K, s_cand, qmax);
+        /* Convergence: relative OR absolute change below the threshold,
+         * measured before the greedy update. */
+        double delta = m_best - m_cand;
+        done = (m_best == 0.0) || (delta / m_best < SSZ_CONVERGE_THRESHOLD) ||
+               (fabs(delta) < SSZ_CONVERGE_THRESHOLD);
+        /* Greedy: keep the candidate only if it lowers the error. */
+        if (m_cand < m_best) {
+            s_best = s_cand;
+            m_best = m_cand;
+        }
+        if (trace)
+            trace[it] = m_best;
+    }
+    if (trace)
+        for (int r = it + 1; r <= max_iters; ++r)
+            trace[r] = m_best;
+    *scale = s_best;
+    *mse = m_best;
+    return it;
+}
+
+/* Per-output-channel symmetric weight quantization with the SSZ search.
+ * w is the already-smoothed [N,K] fp32 weight.  bits is 8 or 4.
+ * Outputs: codes q [N,K] (int4 codes stored one per byte), scale [N],
+ * mse [N] (nullable), iters [N] (nullable), trace [N, max_iters+1]
+ * (nullable).  Returns 0, or -1 on an argument the pages do not support. */
+int oracle_ssz_quant_weight(const float *w, int64_t N, int64_t K, int bits,
+                            int max_iters, int8_t *q, float *scale,
+                            double *mse, int32_t *iters, double *trace)
+{
+    if (bits != 8 && bits != 4)
+        return -1; /* [SSZ] 使用限制: int8 and int4 only */
+    if (N < 0 || K <= 0 || max_iters < 0)
+        return -1;
+    int qmax = (1 << (bits - 1)) - 1;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t n = 0; n < N; ++n) {
+        const float *row = w + n * K;
+        float s;
+        double m;
+        int it = ssz_channel(row, K, qmax, max_iters, &s, &m,
+                             trace ? trace + n * (int64_t)(max_iters + 1) : 0);
+        scale[n] = s;
+        if (mse)
+            mse[n] = m;
+        if (iters)
+            iters[n] = it;
+        for (int64_t k = 0; k < K; ++k)
+            q[n * K + k] = (int8_t)sym_code(row[k], s, qmax);
+    }
+    return 0;
+}
+
+/* Codes of a [N,K] weight at given per-row scales (stage-wise parity: the
+ * codes a scale implies). */
+void oracle_weight_codes(const float *w, int64_t N, int64_t K, int bits,
+                         const float *scale, int8_t *q)
+{
+    int qmax = (1 << (bits - 1)) - 1;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            q[n * K + k] = (int8_t)sym_code(w[n * K + k], scale[n], qmax);
+}
+
+/* The error of one channel at a given scale (exposed for the pins). */
+double oracle_channel_mse(const float *w, int64_t K, float s, int bits)
+{
+    return channel_mse(w, K, s, (1 << (bits - 1)) - 1);
+}
+
+/* ---------------------------------------------------------------- step 4 */
+/* Per-token symmetric activation quantization ([CQ] 2.1, Z = 0): with
+ * x' = x * inv_s (inv_s nullable: no smoothing), sx_t = max_j|x'_tj| / 127
+ * and q_tj = clamp(rint(x'_tj / sx_t), -127, 127); an all-zero row gives
+ * sx_t = 0 and zero codes. */
+void oracle_quant_act_per_token(const float *x, int64_t M, int64_t K,
+                                const float *inv_s, int8_t *q, float *sx)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < M; ++t) {
+        const float *row = x + t * K;
+        float amax = 0.0f;
+        for (int64_t j = 0; j < K; ++j) {
+            float v = inv_s ? row[j] * inv_s[j] : row[j];
+            float a = fabsf(v);
+            if (a > amax)
+                amax = a;
+        }
+        float s = amax / (float)ACT_QMAX;
+        sx[t] = s;
+        for (int64_t j = 0; j < K; ++j) {
+            float v = inv_s ? row[j] * inv_s[j] : row[j];
+            q[t * K + j] = (s == 0.0f) ? (int8_t)0 : (int8_t)sym_code(v, s, ACT_QMAX);
+        }
+    }
+}
+
+/* ---------------------------------------------------------------- step 5 */
+/* Exact integer product [CQ] 3.2: acc[t,n] = sum_k qx[t,k] * qw[n,k], both
+ * operands K-contiguous (the weight in [N,K] linear-layer layout).  The sum
+ * is taken in int64; |acc| <= K * 127^2 < 2^31 for K < 133144. */
+void oracle_gemm_i8(const int8_t *qx, const int8_t *qw, int64_t M, int64_t N,
+                    int64_t K, int32_t *acc)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < M; ++t)
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t sum = 0;
+            for (int64_t k = 0; k < K; ++k)
+                sum += (int64_t)qx[t * K + k] * (int64_t)qw[n * K + k];
+            acc[t * N + n] = (int32_t)sum;
+        }
+}
+
+/* fp32 -> bf16 with round-to-nearest-even; NaN maps to a quiet NaN. */
+static uint16_t f32_to_bf16_rne(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7fffffffu) > 0x7f800000u)
+        return (uint16_t)((u >> 16) | 0x0040u);
+    u += 0x7fffu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+/* Dequantization [CQ] 4.2: y[t,n] = ((float)acc[t,n] * sx[t]) * sw[n], two
+ * fp32 multiplies in that order.  y_f32 and y_bf16 are each nullable. */
+void oracle_dequant(const int32_t *acc, const float *sx, const float *sw,
+                    int64_t M, int64_t N, float *y_f32, uint16_t *y_bf16)
+{
+    for (int64_t t = 0; t < M; ++t)
+        for (int64_t n = 0; n < N; ++n) {
+            float y = ((float)acc[t * N + n] * sx[t]) * sw[n];
+            if (y_f32)
+                y_f32[t * N + n] = y;
+            if (y_bf16)
+                y_bf16[t * N + n] = f32_to_bf16_rne(y);
+        }
+}
+
+/* Elementwise fp32 -> bf16 (RNE) for arrays, so callers round exactly as
+ * the dequant does. */
+void oracle_to_bf16(const float *a, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = f32_to_bf16_rne(a[i]);
+}

@@ -1,0 +1,106 @@
+"""Mutation check of the oracle's pins.
+
+Each case plants one plausible slip in a copy of oracle/oracle.c (a dropped
+term, a wrong sign or exponent, a transposed operand, a wrong rounding mode,
+an off-by-one range), builds it on the CPU, and runs the pins of
+tests/test_oracle_pins.py against it.  At least one pin must fail for every
+planted slip; the unmodified source must pass them all.
+
+Not planted: dropping the greedy keep-if-better test of the SSZ search.  In
+exact arithmetic it never rejects: the least-squares candidate minimises the
+residual for the current codes, and re-rounding at the candidate scale gives
+each element its nearest code, so the candidate's error is never larger.  The
+keep only matters at fp rounding ties, so that mutant is equivalent.
+"""
+import inspect
+import os
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = open(os.path.join(os.path.dirname(oracle.__file__), "oracle.c")).read()
+
+# (name, original text, replacement)
+MUTANTS = [
+    ("calib_drops_abs", "float a = fabsf(row[j]);", "float a = row[j];"),
+    ("smooth_weight_exponent_is_alpha", "pow((double)aw[j], 1.0 - a)", "pow((double)aw[j], a)"),
+    ("smooth_swaps_x_and_w", "pow((double)ax[j], a) / pow((double)aw[j], 1.0 - a)",
+     "pow((double)aw[j], a) / pow((double)ax[j], 1.0 - a)"),
+    ("fold_wrong_column", "out[r * K + j] = a[r * K + j] * f[j];",
+     "out[r * K + j] = a[r * K + j] * f[(j + 1) % K];"),
+    ("round_half_away", "float r = rintf(w / s);", "float r = roundf(w / s);"),
+    ("asymmetric_clamp", "if (r < -(float)qmax)\n        r = -(float)qmax;",
+     "if (r < -(float)(qmax + 1))\n        r = -(float)(qmax + 1);"),
+    ("mse_is_sum_not_mean", "return acc / (double)K;", "return acc;"),
+    ("ls_inverted", "s_cand = (float)(num / (double)den);", "s_cand = (float)((double)den / num);"),
+    ("ls_drops_square", "den += (int64_t)q * (int64_t)q;", "den += (int64_t)(q < 0 ? -q : q);"),
+    ("convergence_sign_flipped", "(delta / m_best < SSZ_CONVERGE_THRESHOLD)",
+     "(delta / m_best > SSZ_CONVERGE_THRESHOLD)"),
+    ("minmax_uses_qmax_plus_one", "float s_best = amax / (float)qmax;",
+     "float s_best = amax / (float)(qmax + 1);"),
+    ("candidate_not_floored", "if (s_cand < SSZ_MIN_SCALE)\n                s_cand = SSZ_MIN_SCALE;", ""),
+    ("act_scale_128", "float s = amax / (float)ACT_QMAX;", "float s = amax / 128.0f;"),
+    ("act_divides_by_inv_s", "float v = inv_s ? row[j] * inv_s[j] : row[j];\n            q[",
+     "float v = inv_s ? row[j] / inv_s[j] : row[j];\n            q["),
+    ("gemm_transposed_weight", "(int64_t)qw[n * K + k]", "(int64_t)qw[k * N + n]"),
+    ("dequant_drops_token_scale", "((float)acc[t * N + n] * sx[t]) * sw[n]",
+     "((float)acc[t * N + n]) * sw[n]"),
+    ("bf16_rounds_half_up", "u += 0x7fffu + ((u >> 16) & 1u);", "u += 0x8000u;"),
+]
+
+PIN_TESTS = []
+for _name, _fn in inspect.getmembers(pins, inspect.isfunction):
+    if not _name.startswith("test_"):
+        continue
+    marks = getattr(_fn, "pytestmark", [])
+    params = [m for m in marks if m.name == "parametrize"]
+    if params:
+        argname, values = params[0].args
+        for v in values:
+            PIN_TESTS.append((f"{_name}[{v}]", _fn, {argname: v}))
+    else:
+        PIN_TESTS.append((_name, _fn, {}))
+
+
+# the brute-force grid is the slowest pin: run it last
+PIN_TESTS.sort(key=lambda t: "brute_force" in t[0])
+
+
+def _failing_pins(stop_at_first: bool = False):
+    failed = []
+    for name, fn, kw in PIN_TESTS:
+        try:
+            fn(oracle, **kw)
+        except Exception:  # an assertion, or a crash-free numeric error
+            failed.append(name)
+            if stop_at_first:
+                break
+    return failed
+
+
+@pytest.fixture(scope="module")
+def workdir(tmp_path_factory):
+    return tmp_path_factory.mktemp("oracle_mutants")
+
+
+def test_unmodified_oracle_passes_every_pin(workdir):
+    path = oracle.build_variant(SRC, str(workdir / "lib_orig.so"))
+    oracle.load_library(path)
+    try:
+        assert _failing_pins() == []
+    finally:
+        oracle.load_library(None)
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_slip_is_caught(workdir, name, old, new):
+    assert SRC.count(old) == 1, "mutation site not unique: %s" % name
+    path = oracle.build_variant(SRC.replace(old, new), str(workdir / ("lib_%s.so" % name)))
+    oracle.load_library(path)
+    try:
+        failed = _failing_pins(stop_at_first=True)
+    finally:
+        oracle.load_library(None)
+    assert failed, "no pin caught the planted slip %s" % name

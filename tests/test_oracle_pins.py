@@ -1,0 +1,398 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test checks the oracle against what the pages and mathematics fix:
+library routines (numpy/torch), closed forms, invariants, hand-derived golden
+values under tests/golden/, and brute force on tiny inputs.  They are chosen so
+that a plausible slip (a dropped term, a wrong sign or index, a transposed
+operand, a swapped exponent) fails at least one; tests/test_oracle_mutants.py
+plants such slips in a copy of the oracle and checks that they are caught.
+
+Sources: SmoothQuant deep-dive (developer.baidu.com) section 1 for the
+smoothing factor and the equivalence; "SSZ：权重量化算法说明" (msModelSlim)
+sections 算法流程 / 迭代优化阶段 / 收敛判断 / 算法参数 for the weight search;
+CUDA INT8 notes (aicoding.csdn.net) section 2.1 for Q = round(R/S) + Z.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+rng = np.random.default_rng(1234)
+
+
+def _llm_like(M, K, n_out=2, scale=40.0, seed=0):
+    r = np.random.default_rng(seed)
+    x = r.standard_normal((M, K)).astype(np.float32)
+    cols = r.permutation(K)[:n_out]
+    x[:, cols] *= scale
+    return x
+
+
+# ----------------------------------------------------------------- step 1 / 2a
+def test_calib_absmax_matches_numpy(orc):
+    x = _llm_like(37, 80)
+    np.testing.assert_array_equal(orc.calib_absmax(x), np.abs(x).max(axis=0))
+
+
+def test_calib_absmax_running_max_equals_concatenation(orc):
+    x1, x2 = _llm_like(9, 48, seed=1), _llm_like(13, 48, seed=2)
+    run = orc.calib_absmax(x2, ax=orc.calib_absmax(x1))
+    np.testing.assert_array_equal(run, orc.calib_absmax(np.concatenate([x1, x2])))
+    # a larger prior max survives
+    big = np.full(48, 1e6, np.float32)
+    np.testing.assert_array_equal(orc.calib_absmax(x1, ax=big), big)
+
+
+def test_weight_col_absmax_is_per_input_channel(orc):
+    w = rng.standard_normal((11, 24)).astype(np.float32)
+    np.testing.assert_array_equal(orc.weight_col_absmax(w), np.abs(w).max(axis=0))
+    # column (input channel) reduction, not row: a planted column max shows up at j
+    w[3, 5] = 100.0
+    assert orc.weight_col_absmax(w)[5] == 100.0
+
+
+# ----------------------------------------------------------------- step 2
+def _ax_aw(K=64, seed=3):
+    r = np.random.default_rng(seed)
+    ax = (np.abs(r.standard_normal(K)) * 5 + 0.1).astype(np.float32)
+    aw = (np.abs(r.standard_normal(K)) * 0.05 + 0.01).astype(np.float32)
+    return ax, aw
+
+
+def test_smooth_factor_special_alphas(orc):
+    ax, aw = _ax_aw()
+    s1, inv1 = orc.smooth_factor(ax, aw, 1.0)           # alpha = 1: s = max|X_j|
+    np.testing.assert_array_equal(s1, ax)
+    s0, _ = orc.smooth_factor(ax, aw, 0.0)              # alpha = 0: s = 1 / max|W_j|
+    np.testing.assert_array_equal(s0, (1.0 / aw.astype(np.float64)).astype(np.float32))
+    sh, _ = orc.smooth_factor(ax, aw, 0.5)              # alpha = 1/2: sqrt(ax / aw)
+    np.testing.assert_allclose(sh, np.sqrt(ax.astype(np.float64) / aw), rtol=2e-7)
+    np.testing.assert_array_equal(inv1, np.float32(1.0) / s1)
+
+
+def test_smooth_factor_matches_torch_pow(orc):
+    ax, aw = _ax_aw(K=128, seed=4)
+    for alpha in (0.2, 0.5, 0.8):
+        s, _ = orc.smooth_factor(ax, aw, alpha)
+        a = torch.tensor(ax, dtype=torch.float64)
+        b = torch.tensor(aw, dtype=torch.float64)
+        ref = (a.pow(float(np.float32(alpha))) / b.pow(1.0 - float(np.float32(alpha)))).float().numpy()
+        np.testing.assert_allclose(s, ref, rtol=1.2e-7)
+
+
+def test_smooth_factor_zero_channel_is_identity(orc):
+    ax, aw = _ax_aw(K=8)
+    ax[2] = 0.0
+    aw[5] = 0.0
+    s, inv = orc.smooth_factor(ax, aw, 0.5)
+    assert s[2] == 1.0 and inv[2] == 1.0 and s[5] == 1.0
+
+
+def test_smoothing_balances_ranges(orc):
+    # alpha = 1/2: after the fold, max|X'_j| and max|W'_j| both equal
+    # sqrt(max|X_j| * max|W_j|)  (the "balance" the page describes)
+    x = _llm_like(64, 96, n_out=4, scale=50.0, seed=5)
+    w = (np.random.default_rng(6).standard_normal((40, 96)) * 0.02).astype(np.float32)
+    ax, aw = orc.calib_absmax(x), orc.weight_col_absmax(w)
+    s, inv_s = orc.smooth_factor(ax, aw, 0.5)
+    xs, ws = orc.scale_columns(x, inv_s), orc.scale_columns(w, s)
+    target = np.sqrt(ax.astype(np.float64) * aw)
+    np.testing.assert_allclose(np.abs(xs).max(0), target, rtol=4e-7)
+    np.testing.assert_allclose(np.abs(ws).max(0), target, rtol=4e-7)
+    # alpha = 1 makes every activation channel range 1; alpha = 0 every weight column range 1
+    s1, inv1 = orc.smooth_factor(ax, aw, 1.0)
+    np.testing.assert_allclose(np.abs(orc.scale_columns(x, inv1)).max(0), 1.0, rtol=1.2e-7)
+    s0, _ = orc.smooth_factor(ax, aw, 0.0)
+    np.testing.assert_allclose(np.abs(orc.scale_columns(w, s0)).max(0), 1.0, rtol=1.2e-7)
+
+
+def test_smoothing_is_equivalent_transform(orc):
+    # (X diag(s)^-1)(W diag(s))^T = X W^T, up to the fp32 rounding of the fold
+    x = _llm_like(32, 128, n_out=3, scale=60.0, seed=7)
+    w = (np.random.default_rng(8).standard_normal((48, 128)) * 0.02).astype(np.float32)
+    for alpha in (0.0, 0.5, 0.8, 1.0):
+        s, inv_s = orc.smooth_factor(orc.calib_absmax(x), orc.weight_col_absmax(w), alpha)
+        lhs = orc.scale_columns(x, inv_s).astype(np.float64) @ orc.scale_columns(w, s).astype(np.float64).T
+        rhs = x.astype(np.float64) @ w.astype(np.float64).T
+        # each product term carries at most ~3 fp32 roundings
+        bound = 4e-7 * (np.abs(x).astype(np.float64) @ np.abs(w).astype(np.float64).T)
+        assert np.all(np.abs(lhs - rhs) <= bound + 1e-30)
+
+
+def test_scale_columns_matches_numpy(orc):
+    a = rng.standard_normal((7, 33)).astype(np.float32)
+    f = rng.standard_normal(33).astype(np.float32)
+    np.testing.assert_array_equal(orc.scale_columns(a, f), a * f[None, :])
+
+
+# ----------------------------------------------------------------- step 3: SSZ
+def _q(w, s, qmax):
+    return np.clip(np.rint(np.float32(w) / np.float32(s)), -qmax, qmax)
+
+
+def _mse_np(w, s, qmax):
+    q = _q(w, s, qmax).astype(np.float64)
+    return float(np.mean((w.astype(np.float64) - np.float64(np.float32(s)) * q) ** 2))
+
+
+def test_ssz_golden_hand_cases(orc):
+    # see tests/golden/ssz_hand.txt for the derivations
+    w = np.array([[1.0, 0.3]], np.float32)
+    r = orc.ssz_quant_weight(w, bits=4)
+    w2 = np.float64(np.float32(0.3))
+    assert r["scale"][0] == np.float32((7.0 + 2.0 * w2) / 53.0)
+    assert r["q"].tolist() == [[7, 2]] and r["iters"][0] == 2
+
+    c = np.float32(2.0 ** -6)
+    k = np.random.default_rng(9).integers(-127, 128, size=64).astype(np.float32)
+    k[10] = 127
+    r = orc.ssz_quant_weight((c * k)[None, :], bits=8)
+    assert r["scale"][0] == c and r["mse"][0] == 0.0 and r["iters"][0] == 1
+    np.testing.assert_array_equal(r["q"][0], k.astype(np.int8))
+
+    row = np.zeros((1, 32), np.float32)
+    row[0, 17] = 0.7
+    r = orc.ssz_quant_weight(row, bits=8)
+    s0 = np.float32(np.float32(0.7) / np.float32(127))
+    assert r["scale"][0] == s0
+    assert r["q"][0, 17] == 127 and r["iters"][0] == 1
+    assert r["mse"][0] == pytest.approx((float(np.float32(0.7)) - 127.0 * float(s0)) ** 2 / 32, rel=1e-12)
+    assert np.count_nonzero(r["q"]) == 1
+
+    r = orc.ssz_quant_weight(np.zeros((1, 16), np.float32), bits=8)
+    assert r["scale"][0] == np.float32(1e-5) and not r["q"].any() and r["iters"][0] == 1
+
+    tiny = np.full((1, 16), 1e-7, np.float32)
+    r = orc.ssz_quant_weight(tiny, bits=8)
+    assert r["scale"][0] == np.float32(1e-5) and not r["q"].any() and r["iters"][0] == 1
+    assert r["mse"][0] == pytest.approx(float(np.float32(1e-7)) ** 2, rel=1e-12)
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_ssz_never_worse_than_minmax_and_monotone(orc, bits):
+    w = (np.random.default_rng(10).standard_normal((64, 256)) * 0.02).astype(np.float32)
+    w[np.random.default_rng(11).random(w.shape) < 0.003] *= 10.0
+    qmax = (1 << (bits - 1)) - 1
+    r = orc.ssz_quant_weight(w, bits=bits, trace=True)
+    tr = r["trace"]
+    assert np.all(np.diff(tr, axis=1) <= 0.0)                 # greedy: never increases
+    mm = orc.ssz_quant_weight(w, bits=bits, max_iters=0)
+    assert np.all(mm["iters"] == 0)
+    np.testing.assert_array_equal(mm["scale"], np.maximum(np.abs(w).max(1) / np.float32(qmax), np.float32(1e-5)))
+    assert np.all(r["mse"] <= mm["mse"])
+    # the search does real work: strictly better on most channels
+    assert np.mean(r["mse"] < mm["mse"]) > 0.8
+    np.testing.assert_array_equal(tr[:, 0], mm["mse"])
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_ssz_reported_error_and_codes_are_consistent(orc, bits):
+    w = (np.random.default_rng(12).standard_normal((16, 64)) * 0.02).astype(np.float32)
+    qmax = (1 << (bits - 1)) - 1
+    r = orc.ssz_quant_weight(w, bits=bits)
+    for n in range(w.shape[0]):
+        np.testing.assert_array_equal(r["q"][n], _q(w[n], r["scale"][n], qmax).astype(np.int8))
+        assert r["mse"][n] == pytest.approx(_mse_np(w[n], r["scale"][n], qmax), rel=1e-12)
+    assert np.abs(r["q"]).max() <= qmax
+    np.testing.assert_array_equal(orc.weight_codes(w, r["scale"], bits), r["q"])
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_ssz_scale_is_least_squares_for_its_codes(orc, bits):
+    # closed form: for fixed codes q the residual sum (w - s q)^2 is minimised
+    # at s* = sum(w q) / sum(q q); a converged channel sits at (or within a
+    # rounding of) s* of its own codes, so s +/- 1% is never better.
+    w = (np.random.default_rng(13).standard_normal((48, 128)) * 0.02).astype(np.float32)
+    r = orc.ssz_quant_weight(w, bits=bits)
+    conv = r["iters"] < 20
+    assert conv.mean() > 0.9
+    for n in np.nonzero(conv)[0]:
+        q = r["q"][n].astype(np.float64)
+        wd = w[n].astype(np.float64)
+        s = float(r["scale"][n])
+        s_star = (wd @ q) / (q @ q)
+        assert abs(s - s_star) <= 2e-3 * s_star
+        res = lambda t: float(np.sum((wd - t * q) ** 2))
+        assert res(s) <= res(s * 1.01) and res(s) <= res(s * 0.99)
+
+
+def test_ssz_close_to_brute_force_optimum(orc):
+    # brute force on tiny rows: a dense grid of scales in [0.25, 1.5] x MinMax.
+    # The search is local, so it may stop above the global optimum, but it can
+    # never go below it, never ends above MinMax, and closes much of the gap.
+    r8 = np.random.default_rng(14)
+    for bits in (8, 4):
+        qmax = (1 << (bits - 1)) - 1
+        gs, gm = [], []
+        for K in (24, 64):
+            w = (r8.standard_normal((20, K)) * 0.02).astype(np.float32)
+            r = orc.ssz_quant_weight(w, bits=bits)
+            for n in range(w.shape[0]):
+                s0 = np.abs(w[n]).max() / qmax
+                grid = (np.linspace(0.25, 1.5, 100001) * s0).astype(np.float32)
+                wd = w[n].astype(np.float64)[None, :]
+                q = np.clip(np.rint(w[n][None, :] / grid[:, None]), -qmax, qmax)
+                best = np.mean((wd - grid[:, None].astype(np.float64) * q) ** 2, axis=1).min()
+                m_mm = _mse_np(w[n], s0, qmax)
+                assert r["mse"][n] >= best * (1 - 1e-6)   # grid spacing 1.25e-5 relative
+                assert r["mse"][n] <= m_mm
+                gs.append(r["mse"][n] / best)
+                gm.append(m_mm / best)
+        assert np.median(gs) < np.median(gm) - 0.05
+        assert max(gs) < 2.0
+
+
+def test_ssz_rows_are_independent(orc):
+    w = (np.random.default_rng(15).standard_normal((20, 64)) * 0.02).astype(np.float32)
+    perm = np.random.default_rng(16).permutation(20)
+    a = orc.ssz_quant_weight(w)
+    b = orc.ssz_quant_weight(w[perm])
+    np.testing.assert_array_equal(a["scale"][perm], b["scale"])
+    np.testing.assert_array_equal(a["q"][perm], b["q"])
+
+
+def test_ssz_fused_fold_equals_prefolded(orc):
+    w = (np.random.default_rng(17).standard_normal((8, 32)) * 0.02).astype(np.float32)
+    s = (np.random.default_rng(18).random(32) * 3 + 0.2).astype(np.float32)
+    a = orc.ssz_quant_weight(w, s=s)
+    b = orc.ssz_quant_weight(w * s[None, :])
+    np.testing.assert_array_equal(a["scale"], b["scale"])
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_ssz_minimum_scale_floors_every_scale(orc, bits):
+    # minimum scale 1e-5 (the page's algorithm parameters): weights of
+    # magnitude ~1e-5 have least-squares optima below the floor, and every
+    # returned scale must still be >= 1e-5, with the codes that scale implies.
+    r = np.random.default_rng(27)
+    w = (r.standard_normal((32, 64)) * 2e-5).astype(np.float32)
+    out = orc.ssz_quant_weight(w, bits=bits)
+    assert np.all(out["scale"] >= np.float32(1e-5))
+    assert np.any(out["scale"] == np.float32(1e-5))
+    qmax = (1 << (bits - 1)) - 1
+    for n in range(32):
+        np.testing.assert_array_equal(out["q"][n], _q(w[n], out["scale"][n], qmax).astype(np.int8))
+
+
+def test_ssz_rejects_unsupported(orc):
+    with pytest.raises(ValueError):
+        orc.ssz_quant_weight(np.ones((2, 16), np.float32), bits=6)
+
+
+# ----------------------------------------------------------------- step 4
+def test_act_quant_golden_ties(orc):
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "act_round_half_even.txt"))
+            if l.strip() and not l.startswith("#")]
+    x = np.array([[float(a) for a, _ in rows]], np.float32)
+    want = np.array([[int(b) for _, b in rows]], np.int8)
+    q, sx = orc.quant_act_per_token(x)
+    assert sx[0] == 1.0
+    np.testing.assert_array_equal(q, want)
+
+
+def test_act_quant_matches_numpy_rint(orc):
+    x = _llm_like(40, 96, seed=19)
+    inv = (np.random.default_rng(20).random(96) + 0.5).astype(np.float32)
+    q, sx = orc.quant_act_per_token(x, inv)
+    xs = x * inv[None, :]
+    np.testing.assert_array_equal(sx, np.abs(xs).max(1) / np.float32(127))
+    want = np.clip(np.rint(xs / sx[:, None]), -127, 127).astype(np.int8)
+    np.testing.assert_array_equal(q, want)
+
+
+def test_act_quant_error_bound_and_extremes(orc):
+    x = _llm_like(64, 128, seed=21)
+    q, sx = orc.quant_act_per_token(x)
+    err = np.abs(x.astype(np.float64) - q.astype(np.float64) * sx[:, None].astype(np.float64))
+    assert np.all(err <= sx[:, None] * (0.5 + 1e-6))
+    # the row's absmax element lands on +/-127
+    j = np.abs(x).argmax(1)
+    assert np.all(np.abs(q[np.arange(64), j]) == 127)
+    # sign is preserved
+    assert np.all(np.sign(q) * np.sign(x) >= 0)
+
+
+def test_act_quant_zero_row_and_identity_smoothing(orc):
+    x = _llm_like(4, 32, seed=22)
+    x[2] = 0.0
+    q, sx = orc.quant_act_per_token(x)
+    assert sx[2] == 0.0 and not q[2].any()
+    q1, sx1 = orc.quant_act_per_token(x, np.ones(32, np.float32))
+    np.testing.assert_array_equal(q, q1)
+    np.testing.assert_array_equal(sx, sx1)
+
+
+# ----------------------------------------------------------------- step 5
+@pytest.mark.parametrize("shape", [(1, 1, 16), (7, 5, 32), (33, 17, 48), (64, 64, 64)])
+def test_gemm_matches_numpy_int64(orc, shape):
+    M, N, K = shape
+    r = np.random.default_rng(M * 1000 + N)
+    qx = r.integers(-127, 128, size=(M, K), dtype=np.int8)
+    qw = r.integers(-127, 128, size=(N, K), dtype=np.int8)
+    want = qx.astype(np.int64) @ qw.astype(np.int64).T
+    np.testing.assert_array_equal(orc.gemm_i8(qx, qw), want.astype(np.int32))
+
+
+def test_gemm_operand_orientation(orc):
+    # acc[t, n] uses row t of qx and row n of qw (both K-contiguous)
+    qx = np.zeros((3, 16), np.int8)
+    qw = np.zeros((5, 16), np.int8)
+    qx[1, 4] = 3
+    qw[2, 4] = -7
+    acc = orc.gemm_i8(qx, qw)
+    assert acc[1, 2] == -21 and np.count_nonzero(acc) == 1
+
+
+def test_gemm_extremes_do_not_overflow(orc):
+    K = 8192
+    qx = np.full((2, K), 127, np.int8)
+    qw = np.full((3, K), -127, np.int8)
+    qw[1] = 127
+    acc = orc.gemm_i8(qx, qw)
+    assert acc[0, 0] == -K * 127 * 127 and acc[1, 1] == K * 127 * 127
+
+
+def test_dequant_matches_library_casts(orc):
+    r = np.random.default_rng(23)
+    acc = r.integers(-2 ** 27, 2 ** 27, size=(9, 13), dtype=np.int32)
+    sx = (r.random(9) * 0.1).astype(np.float32)
+    sw = (r.random(13) * 1e-3).astype(np.float32)
+    yf = orc.dequant(acc, sx, sw, out="f32")
+    want = (acc.astype(np.float32) * sx[:, None]) * sw[None, :]
+    np.testing.assert_array_equal(yf, want)
+    yb = orc.dequant(acc, sx, sw, out="bf16")
+    tb = torch.from_numpy(want).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(yb, tb)
+
+
+def test_bf16_rounding_matches_torch(orc):
+    r = np.random.default_rng(24)
+    a = (r.standard_normal(4096) * 10.0 ** r.integers(-30, 30, 4096)).astype(np.float32)
+    a[:4] = [0.0, -0.0, np.inf, -np.inf]
+    # exact ties (low 16 bits 0x8000) with even and odd kept parts: RNE goes
+    # to the even neighbour, which a round-half-up slip gets wrong
+    ties = np.array([0x3F808000, 0x3F818000, 0xBF808000, 0xC0418000, 0x00018000, 0x7F7F8000],
+                    dtype=np.uint32).view(np.float32)
+    a[4:4 + ties.size] = ties
+    want = torch.from_numpy(a).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(orc.to_bf16_bits(a), want)
+
+
+# ----------------------------------------------------------------- whole path
+def test_smoothing_lowers_w8a8_error_with_outliers(orc):
+    # the point of the method: with activation outlier channels, smoothing
+    # (alpha = 0.5) gives a more accurate W8A8 product than no smoothing.
+    x = _llm_like(64, 256, n_out=4, scale=50.0, seed=25)
+    w = (np.random.default_rng(26).standard_normal((128, 256)) * 0.02).astype(np.float32)
+    ref = x.astype(np.float64) @ w.astype(np.float64).T
+    y_s = orc.linear(x, w, alpha=0.5, out="f32")["y"]
+    y_0 = orc.linear(x, w, alpha=0.0, out="f32")["y"]      # alpha=0 still rescales; use s=1 below
+    qw = orc.ssz_quant_weight(w)
+    qx, sx = orc.quant_act_per_token(x)
+    y_none = orc.dequant(orc.gemm_i8(qx, qw["q"]), sx, qw["scale"], out="f32")
+    e = lambda y: np.linalg.norm(y - ref) / np.linalg.norm(ref)
+    assert e(y_s) < 0.5 * e(y_none)
+    assert e(y_s) < 0.05
+    assert np.isfinite(y_0).all()
