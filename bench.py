@@ -1,0 +1,452 @@
+"""Throughput of the SmoothQuant W8A8 linear path on B200.
+
+A step is one pass of the whole path over one batch: per-input-channel
+activation absmax (calibration) -> smoothing factor and weight column absmax
+-> SSZ int8 weight quantization of the smoothed weight -> per-token int8
+activation quantization -> INT8 GEMM with fused dequant.  Inputs are seeded
+synthetic LLM-shaped data resident in HBM; L2 is flushed (a 512 MB write)
+before every timed step, outside the timed events.
+
+value  = 2*M*N*K int8 ops of the linear per step, over all ranks, divided by
+         the step time (max over ranks), in TOPS.
+e2e    = the same, through the C ABI with the inputs copied from pinned host
+         memory every step and the output copied back (copies timed).
+
+Multi-GPU (torchrun): data parallel, each rank a replica of the layer with its
+own batch of tokens (weak scaling).  The one exchange is the calibration
+statistic: the [K] activation absmax is all-reduced with MAX over NCCL so all
+replicas derive the same smoothing factor and the same quantized weight.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "prefill_2048x4096x4096"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--e2e-steps", type=int, default=20)
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def algorithmic_work(cfg):
+    """Bytes (or int8 ops) each kernel must move (or do) per launch."""
+    M, K, N = cfg.M, cfg.K, cfg.N
+    xb = 2 if cfg.in_dtype == "bf16" else 4
+    yb = 2 if cfg.out_dtype == "bf16" else 4
+    return {
+        "calib_absmax": {"bytes": xb * M * K + 4 * K},
+        "smooth_fold": {"bytes": xb * N * K + 3 * 4 * K},
+        "ssz_quant_weight": {"bytes": xb * N * K + N * K + 4 * K + 4 * N + 8 * N + 4 * N},
+        "quant_act_per_token": {"bytes": xb * M * K + M * K + 4 * K + 4 * M},
+        "w8a8_gemm_dequant": {"ops": 2 * M * N * K, "bytes": M * K + N * K + 4 * M + 4 * N + yb * M * N},
+    }
+
+
+KERNEL_SOURCES = {
+    "calib_absmax": "smooth.cu", "smooth_fold": "smooth.cu", "ssz_quant_weight": "ssz.cu",
+    "quant_act_per_token": "quant_act.cu", "w8a8_gemm_dequant": "gemm.cu",
+}
+
+
+def source_sha(fname):
+    h = hashlib.sha256()
+    for f in (fname, "common.cuh"):
+        with open(os.path.join(ROOT, "w8a8_linear_layers_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def dram_traffic(step_name, workload):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's
+    source is unchanged since it was captured."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(workload, {}).get(step_name)
+    if not e or e.get("src_sha") != source_sha(KERNEL_SOURCES[step_name]):
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.result = None
+        if self.proc is None:
+            return
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if sm:
+            self.result = {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                           "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import synthetic
+    import w8a8_linear_layers_b200 as w
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = synthetic.CONFIGS[args.workload]
+    M, K, N = cfg.M, cfg.K, cfg.N
+    # each replica draws its own token batch (seed = rank) and the same weight
+    x_cpu, w_cpu = synthetic.make_linear(cfg, seed=0)
+    if rank > 0:
+        x_cpu, _ = synthetic.make_linear(cfg, seed=rank)
+    x = x_cpu.to(dev)
+    wt = w_cpu.to(dev)
+    f32 = dict(device=dev, dtype=torch.float32)
+    ax, aw, s, inv = (torch.empty(K, **f32) for _ in range(4))
+    qw = torch.empty(N, K, device=dev, dtype=torch.int8)
+    sw = torch.empty(N, **f32)
+    qx = torch.empty(M, K, device=dev, dtype=torch.int8)
+    sx = torch.empty(M, **f32)
+    ydt = torch.bfloat16 if cfg.out_dtype == "bf16" else torch.float32
+    y = torch.empty(M, N, device=dev, dtype=ydt)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    names = ["calib_absmax", "smooth_fold", "ssz_quant_weight", "quant_act_per_token", "w8a8_gemm_dequant"]
+
+    def step(xin, evs=None):
+        def mark(i):
+            if evs is not None:
+                evs[i].record(stream)
+        mark(0)
+        w.sq_calib_absmax(xin, ax)
+        mark(1)
+        if world > 1:
+            dist.all_reduce(ax, op=dist.ReduceOp.MAX)
+        w.sq_smooth_fold(ax, wt, cfg.alpha, aw, s, inv)
+        mark(2)
+        w.ssz_quant_weight(wt, s, cfg.bits, cfg.max_iters, qw, sw)
+        mark(3)
+        w.quant_act_per_token(xin, inv, qx, sx)
+        mark(4)
+        w.w8a8_gemm_dequant(qx, sx, qw, sw, y)
+        mark(5)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(x)
+    torch.cuda.synchronize()
+    if w.device_fault() != 0:
+        raise RuntimeError("a kernel gave up on a bounded wait during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        wall0 = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()          # L2 flush, outside the timed events
+            step(x, evs[i])
+        torch.cuda.synchronize()
+        wall1 = time.perf_counter()
+    if world > 1:
+        dist.barrier()
+    step_ms = [e[0].elapsed_time(e[5]) for e in evs]
+    kern_ms = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, n in enumerate(names)}
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    if w.device_fault() != 0:
+        raise RuntimeError("a kernel gave up on a bounded wait during timing")
+
+    ops_per_step = 2.0 * M * N * K
+    value = ops_per_step * world * args.steps / (total_ms * 1e-3) / 1e12
+
+    # ---- end to end through the C ABI with host buffers
+    xh = x_cpu.pin_memory()
+    wh = w_cpu.pin_memory()
+    yh = torch.empty(M, N, dtype=ydt).pin_memory()
+    xd = torch.empty_like(x)
+    wd = torch.empty_like(wt)
+    e2e_ms = []
+    for i in range(args.warmup + args.e2e_steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        xd.copy_(xh, non_blocking=True)
+        wd.copy_(wh, non_blocking=True)
+        w.sq_calib_absmax(xd, ax)
+        if world > 1:
+            dist.all_reduce(ax, op=dist.ReduceOp.MAX)
+        w.sq_smooth_fold(ax, wd, cfg.alpha, aw, s, inv)
+        w.ssz_quant_weight(wd, s, cfg.bits, cfg.max_iters, qw, sw)
+        w.quant_act_per_token(xd, inv, qx, sx)
+        w.w8a8_gemm_dequant(qx, sx, qw, sw, y)
+        yh.copy_(y, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e_total = sum(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    e2e_value = ops_per_step * world * len(e2e_ms) / (e2e_total * 1e-3) / 1e12
+    h2d = x.numel() * x.element_size() + wt.numel() * wt.element_size()
+    d2h = y.numel() * y.element_size()
+
+    # ---- rooflines per kernel
+    peaks, src = load_peaks()
+    work = algorithmic_work(cfg)
+    kernels = {}
+    for n in names:
+        t_s = kern_ms[n] * 1e-3
+        entry = {"us": round(kern_ms[n] * 1e3, 2)}
+        if "ops" in work[n]:
+            ach = work[n]["ops"] / t_s / 1e12
+            peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+            entry.update(bound="tensor", achieved=round(ach, 1), peak=round(peak, 1), unit="TFLOP/s",
+                         frac=round(ach / peak, 4))
+        else:
+            ach = work[n]["bytes"] / t_s / 1e9
+            peak = peaks["hbm_gbs"]
+            entry.update(bound="hbm", achieved=round(ach, 1), peak=round(peak, 1), unit="GB/s",
+                         frac=round(ach / peak, 4))
+        entry["algorithmic"] = work[n]
+        entry["traffic"] = dram_traffic(n, args.workload)
+        kernels[n] = entry
+    dom = max(names, key=lambda n: kern_ms[n])
+    roof = {k: kernels[dom][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
+    roof["kernel"] = dom
+    roof["peak_source"] = "%s (%s)" % (src, "bf16 burst x2 for int8" if roof["bound"] == "tensor" else "hbm copy")
+
+    launches_per_step = {"calib_absmax": 1, "smooth_fold": 2, "ssz_quant_weight": 1, "quant_act_per_token": 1,
+                         "w8a8_gemm_dequant": 1}
+    result = {
+        "metric": "W8A8 linear INT8 TOPS (% of peak); quant/SSZ GB/s (% of HBM) on 1 B200",
+        "value": round(value, 2),
+        "unit": "TOPS",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8 codes, int32 acc, %s in/out, fp32 scales" % cfg.in_dtype,
+        "data": "synthetic (seeded LLM-shaped activations with outlier channels, N(0,std) weights)",
+        "config": {"workload": args.workload, "M_tokens_per_gpu": M, "K": K, "N": N, "alpha": cfg.alpha,
+                   "weight_bits": cfg.bits, "ssz_max_iters": cfg.max_iters,
+                   "parallelism": "dp%d (replicas; MAX all-reduce of the calibration absmax)" % world,
+                   "l2": "flushed (512 MB write) before every timed step, outside the timed events"},
+        "roofline": roof,
+        "kernels": kernels,
+        "e2e": {"value": round(e2e_value, 3), "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_total / len(e2e_ms), 4)},
+        "gpu_launches": sum(launches_per_step.values()) * args.steps,
+        "clocks": clk.result,
+        "wall_s_timed_region": round(wall1 - wall0, 3),
+    }
+    return result
+
+
+# ------------------------------------------------------------------ oracle arm
+def oracle_sample(cfg, frac=1.0):
+    """Time the CPU oracle on one step of the workload.  frac < 1 runs the
+    SSZ search, the activation quantization and the GEMM+dequant on that
+    fraction of their rows (rows are independent in all three) and scales
+    their times back up; the calibration and weight-absmax passes always run
+    in full.  Returns (seconds per full step, per-stage seconds, description)."""
+    import oracle
+    import synthetic
+    x, wt = _oracle_inputs(cfg)
+    M, K, N = cfg.M, cfg.K, cfg.N
+    t = {}
+    t0 = time.perf_counter()
+    ax = oracle.calib_absmax(x)
+    t["calib_absmax"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    aw = oracle.weight_col_absmax(wt)
+    s, inv_s = oracle.smooth_factor(ax, aw, cfg.alpha)
+    t["smooth_fold"] = time.perf_counter() - t0
+    n_s = max(1, min(N, int(round(N * frac))))
+    m_s = max(1, min(M, int(round(M * frac))))
+    t0 = time.perf_counter()
+    wq = oracle.ssz_quant_weight(wt[:n_s], bits=cfg.bits, max_iters=cfg.max_iters, s=s)
+    t["ssz_quant_weight"] = (time.perf_counter() - t0) * N / n_s
+    t0 = time.perf_counter()
+    qx, sx = oracle.quant_act_per_token(x[:m_s], inv_s)
+    t["quant_act_per_token"] = (time.perf_counter() - t0) * M / m_s
+    t0 = time.perf_counter()
+    acc = oracle.gemm_i8(qx, wq["q"])
+    oracle.dequant(acc, sx, wq["scale"])
+    t["w8a8_gemm_dequant"] = (time.perf_counter() - t0) * (M * N) / (m_s * n_s)
+    if frac >= 1.0:
+        sample = "the whole workload, one step (%d tokens x %d -> %d)" % (M, K, N)
+    else:
+        sample = ("calibration and weight absmax in full; SSZ on %d of %d channels, activation quantization on "
+                  "%d of %d tokens, GEMM+dequant on their %dx%d block; each scaled to the full step"
+                  % (n_s, N, m_s, M, m_s, n_s))
+    return sum(t.values()), t, sample
+
+
+_INPUTS = {}
+
+
+def _oracle_inputs(cfg):
+    import synthetic
+    if cfg.name not in _INPUTS:
+        x, wt = synthetic.make_linear(cfg, seed=0)
+        _INPUTS[cfg.name] = (x.float().numpy(), wt.float().numpy())
+    return _INPUTS[cfg.name]
+
+
+def cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def run_reference(args, rank):
+    """The oracle as it stands, timed on the host cores.  Each step is a
+    sample of the workload sized so that warm-up + steps take about two
+    minutes; its time is scaled to one full step."""
+    import synthetic
+    if rank != 0:
+        return None
+    cfg = synthetic.CONFIGS[args.workload]
+    probe, _, _ = oracle_sample(cfg, frac=1.0 / 16)
+    budget = 120.0 / max(1, args.warmup + args.steps)
+    frac = min(1.0, max(1.0 / 256, budget / max(probe, 1e-9)))
+    steps = []
+    for _ in range(args.warmup + args.steps):
+        total, parts, sample = oracle_sample(cfg, frac)
+        steps.append(total)
+    timed = steps[args.warmup:]
+    ops = 2.0 * cfg.M * cfg.N * cfg.K
+    value = ops * len(timed) / sum(timed) / 1e12
+    return {
+        "impl": "reference",
+        "metric": "W8A8 linear INT8 TOPS (% of peak); quant/SSZ GB/s (% of HBM) on 1 B200",
+        "value": value, "unit": "TOPS", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * sum(timed) / len(timed), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8 codes, int32 acc, fp32 decisions, fp64 sums (CPU)",
+        "data": "synthetic", "config": {"workload": args.workload, "M_tokens_per_gpu": cfg.M, "K": cfg.K, "N": cfg.N},
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cores(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores()))
+    if args.impl == "reference":
+        res = run_reference(args, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            import synthetic
+            total, parts, sample = oracle_sample(synthetic.CONFIGS[args.workload], frac=1.0)
+            cfg = synthetic.CONFIGS[args.workload]
+            res["cpu_baseline"] = {"value": round(2.0 * cfg.M * cfg.N * cfg.K / total / 1e12, 6), "unit": "TOPS",
+                                   "cores": cores(), "kind": "oracle", "sample": sample,
+                                   "seconds_per_step": round(total, 3),
+                                   "stage_seconds": {k: round(v, 3) for k, v in parts.items()}}
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

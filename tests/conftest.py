@@ -13,6 +13,16 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "slow: full-size parity case (minutes of oracle time)")
 
 
+def build_cuda_library() -> str:
+    """Build libw8a8.so (by file path: importing the package needs the .so)."""
+    import importlib.util
+    path = os.path.join(ROOT, "w8a8_linear_layers_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("w8a8_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()
+
+
 @pytest.fixture(scope="session")
 def orc():
     import oracle

@@ -1,0 +1,223 @@
+"""Python binding of libw8a8.so, the B200 (sm_100a) SmoothQuant-style W8A8
+linear layer.
+
+Argument marshalling only: every function here has the name and the meaning
+of the C entry point declared in include/w8a8.h, takes torch CUDA tensors
+(the caller owns them; outputs are written in place), passes their device
+pointers and the current CUDA stream, and raises W8A8Error on a non-OK status.
+All computation happens in the library's CUDA kernels; there is no CPU or
+PyTorch fallback, and importing fails loudly if the library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libw8a8.so")
+
+SQ_F32, SQ_BF16 = 0, 1
+STATUS = ["SQ_OK", "SQ_ERR_NULL", "SQ_ERR_SHAPE", "SQ_ERR_DTYPE", "SQ_ERR_ALIGN", "SQ_ERR_ARG",
+          "SQ_ERR_UNSUPPORTED", "SQ_ERR_CUDA", "SQ_ERR_DEVICE"]
+
+# every symbol include/w8a8.h declares
+EXPORTS = ["sq_status_string", "sq_last_error_detail", "sq_abi_version", "sq_device_fault",
+           "sq_selftest_bounded_wait",
+           "sq_calib_absmax", "sq_smooth_fold", "ssz_quant_weight", "quant_act_per_token",
+           "w8a8_gemm_dequant"]
+
+
+class W8A8Error(RuntimeError):
+    def __init__(self, fn: str, status: int, detail: str):
+        self.status = status
+        self.status_name = STATUS[status] if 0 <= status < len(STATUS) else "SQ_ERR_UNKNOWN"
+        self.detail = detail
+        super().__init__("%s failed: %s (%s)" % (fn, self.status_name, detail))
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            "libw8a8.so is not built (%s); run `python -m w8a8_linear_layers_b200.build`" % LIB_PATH)
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I64, I, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+    sig = {
+        "sq_status_string": ([I], ctypes.c_char_p),
+        "sq_last_error_detail": ([], ctypes.c_char_p),
+        "sq_abi_version": ([], I),
+        "sq_device_fault": ([P, P], I),
+        "sq_selftest_bounded_wait": ([ctypes.c_uint32, P], I),
+        "sq_calib_absmax": ([P, I, I64, I64, P, I, P], I),
+        "sq_smooth_fold": ([P, P, I, I64, I64, F, P, P, P, P, P], I),
+        "ssz_quant_weight": ([P, I, I64, I64, P, I, I, P, P, P, P, P], I),
+        "quant_act_per_token": ([P, I, I64, I64, P, P, P, P], I),
+        "w8a8_gemm_dequant": ([P, P, P, P, I64, I64, I64, P, I, P, P], I),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+lib = _load()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise W8A8Error(fn, status, lib.sq_last_error_detail().decode())
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor, got one on %s" % t.device)
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return SQ_F32
+    if t.dtype == torch.bfloat16:
+        return SQ_BF16
+    raise ValueError("unsupported dtype %s (float32 or bfloat16)" % t.dtype)
+
+
+def _need(t: torch.Tensor | None, dtype: torch.dtype, name: str) -> None:
+    if t is not None and t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def abi_version() -> int:
+    return lib.sq_abi_version()
+
+
+def device_fault(stream=None) -> int:
+    """Read and clear the device fault word (0: no kernel gave up on a wait)."""
+    out = ctypes.c_uint32(0)
+    _check("sq_device_fault", lib.sq_device_fault(_stream(stream), ctypes.byref(out)))
+    return out.value
+
+
+def selftest_bounded_wait(limit_ms: int = 50, stream=None) -> None:
+    """Launch the bounded-wait self test (see include/w8a8.h)."""
+    _check("sq_selftest_bounded_wait", lib.sq_selftest_bounded_wait(int(limit_ms), _stream(stream)))
+
+
+def sq_calib_absmax(x: torch.Tensor, absmax: torch.Tensor, accumulate: bool = False, stream=None) -> None:
+    """absmax[j] = max(accumulate ? absmax[j] : 0, max_t |x[t,j]|)."""
+    _need(absmax, torch.float32, "absmax")
+    M, K = x.shape
+    _check("sq_calib_absmax", lib.sq_calib_absmax(_ptr(x), _dtype(x), M, K, _ptr(absmax),
+                                                   1 if accumulate else 0, _stream(stream)))
+
+
+def sq_smooth_fold(x_absmax: torch.Tensor, w: torch.Tensor, alpha: float, w_absmax_out: torch.Tensor,
+                   s_out: torch.Tensor, inv_s_out: torch.Tensor, w_folded_out: torch.Tensor | None = None,
+                   stream=None) -> None:
+    """Weight column absmax, s = ax^alpha / aw^(1-alpha), 1/s, optional W diag(s)."""
+    for t, n in ((x_absmax, "x_absmax"), (w_absmax_out, "w_absmax_out"), (s_out, "s_out"),
+                 (inv_s_out, "inv_s_out"), (w_folded_out, "w_folded_out")):
+        _need(t, torch.float32, n)
+    N, K = w.shape
+    _check("sq_smooth_fold", lib.sq_smooth_fold(_ptr(x_absmax), _ptr(w), _dtype(w), N, K, float(alpha),
+                                                 _ptr(w_absmax_out), _ptr(s_out), _ptr(inv_s_out),
+                                                 _ptr(w_folded_out), _stream(stream)))
+
+
+def ssz_quant_weight(w: torch.Tensor, s: torch.Tensor | None, bits: int, max_iters: int, q_out: torch.Tensor,
+                     scale_out: torch.Tensor, mse_out: torch.Tensor | None = None,
+                     iters_out: torch.Tensor | None = None, stream=None) -> None:
+    """SSZ per-output-channel symmetric quantization of w [N,K] (folded by s)."""
+    _need(s, torch.float32, "s")
+    _need(q_out, torch.int8, "q_out")
+    _need(scale_out, torch.float32, "scale_out")
+    _need(mse_out, torch.float64, "mse_out")
+    _need(iters_out, torch.int32, "iters_out")
+    N, K = w.shape
+    _check("ssz_quant_weight", lib.ssz_quant_weight(_ptr(w), _dtype(w), N, K, _ptr(s), int(bits), int(max_iters),
+                                                     _ptr(q_out), _ptr(scale_out), _ptr(mse_out),
+                                                     _ptr(iters_out), _stream(stream)))
+
+
+def quant_act_per_token(x: torch.Tensor, inv_s: torch.Tensor | None, q_out: torch.Tensor,
+                        scale_out: torch.Tensor, stream=None) -> None:
+    """Per-token int8 codes and scales of x * inv_s."""
+    _need(inv_s, torch.float32, "inv_s")
+    _need(q_out, torch.int8, "q_out")
+    _need(scale_out, torch.float32, "scale_out")
+    M, K = x.shape
+    _check("quant_act_per_token", lib.quant_act_per_token(_ptr(x), _dtype(x), M, K, _ptr(inv_s), _ptr(q_out),
+                                                           _ptr(scale_out), _stream(stream)))
+
+
+def w8a8_gemm_dequant(qx: torch.Tensor, sx: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor, y: torch.Tensor,
+                      acc_out: torch.Tensor | None = None, stream=None) -> None:
+    """y = ((float)(qx @ qw^T) * sx[:,None]) * sw[None,:], int32 accumulation."""
+    _need(qx, torch.int8, "qx")
+    _need(qw, torch.int8, "qw")
+    _need(sx, torch.float32, "sx")
+    _need(sw, torch.float32, "sw")
+    _need(acc_out, torch.int32, "acc_out")
+    M, K = qx.shape
+    N, K2 = qw.shape
+    if K != K2 or tuple(y.shape) != (M, N):
+        raise ValueError("shape mismatch: qx %s, qw %s, y %s" % (tuple(qx.shape), tuple(qw.shape), tuple(y.shape)))
+    _check("w8a8_gemm_dequant", lib.w8a8_gemm_dequant(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), M, N, K, _ptr(y),
+                                                       _dtype(y), _ptr(acc_out), _stream(stream)))
+
+
+class W8A8Linear:
+    """A calibrated SmoothQuant W8A8 linear layer built from the five calls.
+
+    calibrate(x) accumulates the activation absmax; quantize() smooths and
+    SSZ-quantizes the weight; forward(x) quantizes x per token and runs the
+    integer GEMM with the fused dequant.  Buffers are torch tensors on the
+    weight's device (memory plumbing only)."""
+
+    def __init__(self, w: torch.Tensor, alpha: float = 0.5, bits: int = 8, max_iters: int = 20,
+                 out_dtype: torch.dtype | None = None):
+        self.w = w.contiguous()
+        self.N, self.K = w.shape
+        self.alpha, self.bits, self.max_iters = alpha, bits, max_iters
+        self.out_dtype = out_dtype or w.dtype
+        dev = w.device
+        f32 = dict(device=dev, dtype=torch.float32)
+        self.ax = torch.zeros(self.K, **f32)
+        self.aw = torch.empty(self.K, **f32)
+        self.s = torch.empty(self.K, **f32)
+        self.inv_s = torch.empty(self.K, **f32)
+        self.qw = torch.empty(self.N, self.K, device=dev, dtype=torch.int8)
+        self.sw = torch.empty(self.N, **f32)
+        self.mse = torch.empty(self.N, device=dev, dtype=torch.float64)
+        self.iters = torch.empty(self.N, device=dev, dtype=torch.int32)
+        self._calibrated = False
+
+    def calibrate(self, x: torch.Tensor) -> None:
+        sq_calib_absmax(x, self.ax, accumulate=self._calibrated)
+        self._calibrated = True
+
+    def quantize(self) -> None:
+        sq_smooth_fold(self.ax, self.w, self.alpha, self.aw, self.s, self.inv_s)
+        ssz_quant_weight(self.w, self.s, self.bits, self.max_iters, self.qw, self.sw, self.mse, self.iters)
+
+    def forward(self, x: torch.Tensor, y: torch.Tensor | None = None) -> torch.Tensor:
+        M = x.shape[0]
+        qx = torch.empty(M, self.K, device=x.device, dtype=torch.int8)
+        sx = torch.empty(M, device=x.device, dtype=torch.float32)
+        quant_act_per_token(x, self.inv_s, qx, sx)
+        if y is None:
+            y = torch.empty(M, self.N, device=x.device, dtype=self.out_dtype)
+        w8a8_gemm_dequant(qx, sx, self.qw, self.sw, y)
+        return y

@@ -1,0 +1,120 @@
+// common.cuh -- helpers shared by the libw8a8 kernels and entry points.
+//
+// Device side: 16-byte vector loads of bf16/fp32 rows, warp/block
+// reductions, and the exact symmetric quantizer.  Host side: argument
+// checking, the thread-local error detail, device queries.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <stdarg.h>
+
+#include <algorithm>
+
+#include "w8a8.h"
+
+namespace w8a8 {
+
+// ----------------------------------------------------------------- host side
+void set_detail(const char *fmt, ...);
+
+inline sq_status fail(sq_status s, const char *fmt, ...) {
+    char buf[256];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    set_detail("%s", buf);
+    return s;
+}
+
+// Compute capability 10.0 check for the current device; fills the SM count.
+sq_status check_device(int *sm_count);
+
+inline bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+inline sq_status launch_status(const char *what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return fail(SQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return SQ_OK;
+}
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ----------------------------------------------------------------- device side
+// Load 8 consecutive elements (16 bytes of bf16, or 32 bytes of fp32) as fp32.
+// bf16 widens exactly (its bits are the high half of an fp32).
+template <typename T> struct Vec8;
+
+template <> struct Vec8<__nv_bfloat16> {
+    static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float (&v)[8]) {
+        uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
+        uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[2 * i] = __uint_as_float(w[i] << 16);
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+};
+
+template <> struct Vec8<float> {
+    static __device__ __forceinline__ void load(const float *p, float (&v)[8]) {
+        float4 a = __ldg(reinterpret_cast<const float4 *>(p));
+        float4 b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+};
+
+__device__ __forceinline__ void load8_f32(const float *p, float (&v)[8]) {
+    Vec8<float>::load(p, v);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// Symmetric code clamp(rint(v / s), -qmax, qmax) with round-half-to-even,
+// bit-identical to an IEEE fp32 division followed by rint.
+//
+// Fast path: y = v * r with r = RN(1/s).  Error analysis (two roundings of
+// relative size <= 2^-24 each, plus the rounding of the true quotient) gives
+// |y - RN(v/s)| < 0.75 * 2^-22 * |y|.  rint has its only discontinuities at
+// half-integers, so unless a half-integer lies within 2^-22 * |y| of y, the
+// two round to the same integer.  Inside that window (about one element in
+// 10^6) the exact IEEE quotient is used.  `exact_only` forces the division
+// (r is not finite when s is below ~2^-126).
+__device__ __forceinline__ float sym_code(float v, float s, float r, float qmax, bool exact_only) {
+    float q;
+    if (exact_only) {
+        q = rintf(__fdiv_rn(v, s));
+    } else {
+        float y = v * r;
+        float h = floorf(y) + 0.5f;
+        if (fabsf(y - h) <= fabsf(y) * 2.384185791015625e-07f)  // 2^-22
+            q = rintf(__fdiv_rn(v, s));
+        else
+            q = rintf(y);
+    }
+    return fminf(fmaxf(q, -qmax), qmax);
+}
+
+// Pack 8 codes (already integral floats in [-127,127]) into 8 bytes.
+__device__ __forceinline__ uint2 pack8_codes(const float (&q)[8]) {
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        lo |= ((uint32_t)(int32_t)q[i] & 0xffu) << (8 * i);
+        hi |= ((uint32_t)(int32_t)q[4 + i] & 0xffu) << (8 * i);
+    }
+    return make_uint2(lo, hi);
+}
+
+}  // namespace w8a8

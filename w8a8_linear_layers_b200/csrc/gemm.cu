@@ -1,0 +1,567 @@
+// gemm.cu -- step 5: INT8 x INT8 -> INT32 GEMM with a fused per-token x
+// per-output-channel dequantization epilogue, for sm_100a (B200).
+//
+// Source: CUDA INT8 quantization notes (aicoding.csdn.net), section 3.2
+// ("低精度矩阵乘实现": an INT8 tensor-core matrix multiply, tiled, with
+// double-buffered operand staging) and section 4.2 ("内核融合优化":
+// quantize -> integer product -> dequantize fused in one kernel, persistent
+// thread blocks).  The WMMA/Ampere kernel described there is prior art only;
+// this kernel is built for the 5th-generation tensor cores:
+//
+//   * tcgen05.mma.cta_group::1.kind::i8, 128 x BN x 32 per instruction, int32
+//     accumulators in tensor memory (TMEM), issued by one thread;
+//   * operands staged by TMA (cp.async.bulk.tensor.2d, 128-byte swizzle,
+//     zero fill past the matrix edges) into a STAGES-deep shared-memory ring
+//     guarded by mbarriers (full: TMA bytes landed; empty: the MMAs that read
+//     the stage completed, signalled by tcgen05.commit);
+//   * persistent CTAs (one per SM) walking the output tiles; two TMEM
+//     accumulator buffers so the epilogue of one tile overlaps the main loop
+//     of the next;
+//   * warp roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
+//     warps 2..5 epilogue (TMEM lanes 32*(warp%4) .. +31 each).
+//
+// Epilogue: tcgen05.ld of 32 accumulator columns per thread (thread = output
+// row), y = ((float)acc * sx[row]) * sw[col] (two fp32 multiplies, int->fp32
+// round-to-nearest-even), converted to bf16 (RNE) or kept fp32, stored with
+// 16-byte stores.  Optionally the raw int32 accumulators are stored too.
+//
+// No TMA multicast is used anywhere (each CTA loads its own tiles).
+//
+// Every mbarrier wait is bounded: after kWaitNs without progress the waiting
+// thread records a fault code in a device word (read by sq_device_fault),
+// raises a CTA-wide abort flag, and every role leaves its loop; in-flight TMA
+// copies and MMAs are drained (again with a bound) before TMEM is freed and
+// the kernel returns.  Nothing traps.
+#include "common.cuh"
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+namespace w8a8 {
+
+__device__ unsigned int g_gemm_fault;
+
+namespace gemm {
+
+constexpr int BM = 128;          // rows of X per tile (= MMA M, = TMEM lanes)
+constexpr int BK = 128;          // K bytes per stage (one 128-byte swizzle row)
+constexpr int UMMA_K = 32;       // K per tcgen05.mma of kind::i8
+constexpr int kThreads = 192;    // 6 warps
+constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s
+
+enum : unsigned {
+    kFaultProducer = 1,
+    kFaultMmaFull = 2,
+    kFaultMmaTmemEmpty = 3,
+    kFaultEpilogue = 4,
+    kFaultDrain = 5,
+    kFaultSelftest = 6,
+};
+
+// ------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long globaltimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait for the phase of `bar` with the given parity.  Returns false
+// if the CTA aborted (this thread timed out, or another role did).
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                             unsigned code, unsigned long long limit_ns = kWaitNs) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer() - t0 > limit_ns) {
+            atomicCAS(&g_gemm_fault, 0u, code);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(dst), "l"((uint64_t)map), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t slot_smem, uint32_t cols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_smem), "r"(cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, int8 x int8 -> int32.
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on `bar` once every tcgen05 op this thread issued so far completes.
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+// 32 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor for a K-major operand tile written by TMA
+// with 128-byte swizzle: rows of 128 bytes, 8-row core groups 1024 bytes
+// apart (stride byte offset), leading byte offset unused for swizzled
+// K-major (encoded 1), descriptor version 1 (sm_100), layout 2 = 128B swizzle.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3fffu);        // start address
+    d |= (uint64_t)1u << 16;                       // leading byte offset (16 B units)
+    d |= (uint64_t)(1024u >> 4) << 32;             // stride byte offset (16 B units)
+    d |= (uint64_t)1u << 46;                       // version
+    d |= (uint64_t)2u << 61;                       // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor, kind::i8: D int32, A and B signed int8, both
+// K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t idesc_i8(int m, int n) {
+    return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+template <int BN>
+struct Cfg {
+    static constexpr int STAGES = 4;
+    static constexpr int A_BYTES = BM * BK;
+    static constexpr int B_BYTES = BN * BK;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int TMEM_COLS = 2 * BN;  // two accumulator buffers
+    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024;  // + alignment slack
+    static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
+};
+
+template <typename OutT>
+__device__ __forceinline__ void store_row_chunk(OutT *yrow, const uint32_t (&acc)[32], float sxr,
+                                                const float *__restrict__ swc, int valid, bool vec_ok);
+
+template <>
+__device__ __forceinline__ void store_row_chunk<__nv_bfloat16>(__nv_bfloat16 *yrow, const uint32_t (&acc)[32],
+                                                               float sxr, const float *__restrict__ swc,
+                                                               int valid, bool vec_ok) {
+    if (vec_ok && valid >= 32) {
+        uint32_t packed[16];
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+            float4 f = __ldg(reinterpret_cast<const float4 *>(swc + j));
+            float sv[4] = {f.x, f.y, f.z, f.w};
+            float y[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) y[i] = (__int2float_rn((int)acc[j + i]) * sxr) * sv[i];
+            __nv_bfloat162 lo = __floats2bfloat162_rn(y[0], y[1]);
+            __nv_bfloat162 hi = __floats2bfloat162_rn(y[2], y[3]);
+            packed[j / 2] = *reinterpret_cast<uint32_t *>(&lo);
+            packed[j / 2 + 1] = *reinterpret_cast<uint32_t *>(&hi);
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(yrow);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (j < valid) yrow[j] = __float2bfloat16_rn((__int2float_rn((int)acc[j]) * sxr) * swc[j]);
+    }
+}
+
+template <>
+__device__ __forceinline__ void store_row_chunk<float>(float *yrow, const uint32_t (&acc)[32], float sxr,
+                                                       const float *__restrict__ swc, int valid, bool vec_ok) {
+    if (vec_ok && valid >= 32) {
+        float4 *dst = reinterpret_cast<float4 *>(yrow);
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+            float4 f = __ldg(reinterpret_cast<const float4 *>(swc + j));
+            dst[j / 4] = make_float4((__int2float_rn((int)acc[j]) * sxr) * f.x,
+                                     (__int2float_rn((int)acc[j + 1]) * sxr) * f.y,
+                                     (__int2float_rn((int)acc[j + 2]) * sxr) * f.z,
+                                     (__int2float_rn((int)acc[j + 3]) * sxr) * f.w);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (j < valid) yrow[j] = (__int2float_rn((int)acc[j]) * sxr) * swc[j];
+    }
+}
+
+template <int BN, typename OutT>
+__global__ void __launch_bounds__(kThreads, 1)
+w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                 const float *__restrict__ sx, const float *__restrict__ sw, OutT *__restrict__ y,
+                 int32_t *__restrict__ acc_out, int M, int N, int K) {
+    using C = Cfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full_bar[C::STAGES];
+    __shared__ __align__(8) uint64_t empty_bar[C::STAGES];
+    __shared__ __align__(8) uint64_t tfull_bar[2];
+    __shared__ __align__(8) uint64_t tempty_bar[2];
+    __shared__ __align__(8) uint64_t drain_bar;
+    __shared__ uint32_t tmem_slot;
+    __shared__ volatile int abort_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;  // 1024-aligned for 128B swizzle
+
+    const int tiles_m = (M + BM - 1) / BM;
+    const int tiles_n = (N + BN - 1) / BN;
+    const int num_tiles = tiles_m * tiles_n;
+    const int num_kb = (K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(smem_u32(&full_bar[s]), 1);
+            mbar_init(smem_u32(&empty_bar[s]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&tfull_bar[b]), 1);
+            mbar_init(smem_u32(&tempty_bar[b]), 4 * 32);
+        }
+        mbar_init(smem_u32(&drain_bar), 1);
+        abort_flag = 0;
+        fence_barrier_init();
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tmap_a) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tmap_b) : "memory");
+    }
+    if (warp == 1) tmem_alloc(smem_u32(&tmem_slot), C::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;  // stages whose loads were issued (for the abort drain)
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int m0 = (tile % tiles_m) * BM, n0 = (tile / tiles_m) * BN;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, &abort_flag, kFaultProducer)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t a_dst = smem_base + stage * C::STAGE_BYTES;
+                    const uint32_t b_dst = a_dst + C::A_BYTES;
+                    const uint32_t fb = smem_u32(&full_bar[stage]);
+                    mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+                    tma_load_2d(a_dst, &tmap_a, fb, kb * BK, m0);
+                    tma_load_2d(b_dst, &tmap_b, fb, kb * BK, n0);
+                    ++issued;
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // drain: wait (bounded) for the copies of the last issued stages
+                int outstanding = issued < C::STAGES ? issued : C::STAGES;
+                int s = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < outstanding; ++i) {
+                    if (--s < 0) {
+                        s = C::STAGES - 1;
+                        ph ^= 1u;
+                    }
+                    const unsigned long long t0 = globaltimer();
+                    while (!mbar_try_wait(smem_u32(&full_bar[s]), ph) && globaltimer() - t0 < kWaitNs) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_i8(BM, BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int buf = 0;
+            uint32_t buf_phase = 0;
+            bool ok = true;
+            bool issued_any = false;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                if (!wait_bounded(smem_u32(&tempty_bar[buf]), buf_phase ^ 1u, &abort_flag, kFaultMmaTmemEmpty)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!wait_bounded(smem_u32(&full_bar[stage]), phase, &abort_flag, kFaultMmaFull)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_base + stage * C::STAGE_BYTES;
+                    const uint32_t b_addr = a_addr + C::A_BYTES;
+#pragma unroll
+                    for (int k = 0; k < BK / UMMA_K; ++k) {
+                        mma_i8(d_tmem, smem_desc_sw128(a_addr + k * UMMA_K), smem_desc_sw128(b_addr + k * UMMA_K),
+                               idesc, (kb | k) != 0 ? 1u : 0u);
+                    }
+                    issued_any = true;
+                    mma_commit(smem_u32(&empty_bar[stage]));
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(smem_u32(&tfull_bar[buf]));
+                buf ^= 1;
+                if (buf == 0) buf_phase ^= 1u;
+            }
+            if (!ok && issued_any) {
+                // drain: every MMA issued so far completes before TMEM is freed
+                mma_commit(smem_u32(&drain_bar));
+                const unsigned long long t0 = globaltimer();
+                while (!mbar_try_wait(smem_u32(&drain_bar), 0) && globaltimer() - t0 < kWaitNs) {
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue (warps 2..5)
+        const int quarter = warp & 3;  // TMEM lanes this warp may access
+        const int row_in_tile = quarter * 32 + lane;
+        const bool vec_ok = (N % (16 / (int)sizeof(OutT))) == 0;
+        const bool acc_vec_ok = (N % 4) == 0;
+        int buf = 0;
+        uint32_t buf_phase = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+            const int m0 = (tile % tiles_m) * BM, n0 = (tile / tiles_m) * BN;
+            const int row = m0 + row_in_tile;
+            const float sxr = row < M ? sx[row] : 0.0f;
+            // the TMEM loads below are warp-collective: leave together or not at all
+            const bool ok = wait_bounded(smem_u32(&tfull_bar[buf]), buf_phase, &abort_flag, kFaultEpilogue);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                uint32_t acc[32];
+                tmem_ld32(tbase + (uint32_t)c0, acc);  // warp-collective: every lane takes part
+                const int col = n0 + c0;
+                if (row < M && col < N) {
+                    const int valid = N - col;
+                    OutT *yrow = y + (int64_t)row * N + col;
+                    store_row_chunk<OutT>(yrow, acc, sxr, sw + col, valid, vec_ok);
+                    if (acc_out) {
+                        int32_t *arow = acc_out + (int64_t)row * N + col;
+                        if (acc_vec_ok && valid >= 32) {
+#pragma unroll
+                            for (int j = 0; j < 32; j += 4)
+                                *reinterpret_cast<int4 *>(arow + j) =
+                                    make_int4((int)acc[j], (int)acc[j + 1], (int)acc[j + 2], (int)acc[j + 3]);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (j < valid) arow[j] = (int)acc[j];
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(smem_u32(&tempty_bar[buf]));
+            buf ^= 1;
+            if (buf == 0) buf_phase ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// One CTA waits, with the same bounded wait the GEMM uses, on an mbarrier
+// that nothing ever arrives at: the wait must run out, record
+// kFaultSelftest and return, leaving the context usable.
+__global__ void bounded_wait_selftest_kernel(unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ volatile int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    wait_bounded(smem_u32(&bar), 0, &abort_flag, kFaultSelftest, limit_ns);
+}
+
+// ------------------------------------------------------------ host side
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
+    }
+    return fn;
+}
+
+// 2-D int8 tensor [rows, K] (K contiguous), box [box_rows, 128 bytes], 128B swizzle.
+static bool make_map(CUtensorMap *map, const void *base, int64_t rows, int64_t K, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K};
+    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int BN, typename OutT>
+static sq_status launch(const int8_t *qx, const float *sx, const int8_t *qw, const float *sw, int M, int N,
+                        int K, void *y, int32_t *acc_out, int sms, cudaStream_t st) {
+    using C = Cfg<BN>;
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, qx, M, K, BM) || !make_map(&mb, qw, N, K, BN))
+        return fail(SQ_ERR_CUDA, "w8a8_gemm_dequant: cuTensorMapEncodeTiled failed");
+    auto kern = w8a8_gemm_kernel<BN, OutT>;
+    static int configured_dev[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !configured_dev[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e != cudaSuccess) return fail(SQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        configured_dev[dev] = 1;
+    }
+    const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int grid = std::min(tiles, sms);
+    kern<<<grid, kThreads, C::SMEM, st>>>(ma, mb, sx, sw, (OutT *)y, acc_out, M, N, K);
+    return launch_status("w8a8_gemm_kernel");
+}
+
+}  // namespace gemm
+}  // namespace w8a8
+
+using namespace w8a8;
+
+extern "C" sq_status w8a8_gemm_dequant(const int8_t *qx, const float *sx, const int8_t *qw, const float *sw,
+                                       int64_t M, int64_t N, int64_t K, void *y, sq_dtype yt, int32_t *acc_out,
+                                       void *stream) {
+    if (M > 0 && N > 0 && (!qx || !sx || !qw || !sw || !y))
+        return fail(SQ_ERR_NULL, "w8a8_gemm_dequant: NULL pointer");
+    if (yt != SQ_F32 && yt != SQ_BF16) return fail(SQ_ERR_DTYPE, "w8a8_gemm_dequant: output dtype %d", (int)yt);
+    if (M < 0 || N < 0 || K <= 0 || K % 16 != 0 || K > 133144 || M > INT32_MAX || N > INT32_MAX)
+        return fail(SQ_ERR_SHAPE, "w8a8_gemm_dequant: M=%lld N=%lld K=%lld (K a multiple of 16 in [16, 133144])",
+                    (long long)M, (long long)N, (long long)K);
+    if (M == 0 || N == 0) return SQ_OK;
+    const int out_vec = (yt == SQ_BF16) ? 8 : 4;
+    if (N % out_vec != 0)
+        return fail(SQ_ERR_SHAPE, "w8a8_gemm_dequant: N=%lld must be a multiple of %d for this output dtype",
+                    (long long)N, out_vec);
+    if (acc_out && N % 4 != 0) return fail(SQ_ERR_SHAPE, "w8a8_gemm_dequant: acc_out needs N %% 4 == 0");
+    if (!aligned(qx, 16) || !aligned(qw, 16) || !aligned(y, 16) || !aligned(sw, 16) || !aligned(sx, 4) ||
+        (acc_out && !aligned(acc_out, 16)))
+        return fail(SQ_ERR_ALIGN, "w8a8_gemm_dequant: misaligned pointer (qx, qw, y, sw, acc_out need 16 bytes)");
+    int sms;
+    sq_status st = check_device(&sms);
+    if (st != SQ_OK) return st;
+    cudaStream_t cs = (cudaStream_t)stream;
+    if (yt == SQ_BF16)
+        return gemm::launch<256, __nv_bfloat16>(qx, sx, qw, sw, (int)M, (int)N, (int)K, y, acc_out, sms, cs);
+    return gemm::launch<256, float>(qx, sx, qw, sw, (int)M, (int)N, (int)K, y, acc_out, sms, cs);
+}
+
+extern "C" sq_status sq_selftest_bounded_wait(uint32_t limit_ms, void *stream) {
+    if (limit_ms == 0 || limit_ms > 10000)
+        return fail(SQ_ERR_ARG, "sq_selftest_bounded_wait: limit_ms=%u outside [1, 10000]", limit_ms);
+    int sms;
+    sq_status st = check_device(&sms);
+    if (st != SQ_OK) return st;
+    gemm::bounded_wait_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((unsigned long long)limit_ms * 1000000ull);
+    return launch_status("bounded_wait_selftest_kernel");
+}
+
+extern "C" sq_status sq_device_fault(void *stream, uint32_t *fault_out) {
+    if (!fault_out) return fail(SQ_ERR_NULL, "sq_device_fault: NULL pointer");
+    cudaStream_t cs = (cudaStream_t)stream;
+    unsigned int v = 0, zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_gemm_fault, sizeof v, 0, cudaMemcpyDeviceToHost, cs);
+    if (e == cudaSuccess) e = cudaMemcpyToSymbolAsync(g_gemm_fault, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, cs);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+    if (e != cudaSuccess) return fail(SQ_ERR_CUDA, "sq_device_fault: %s", cudaGetErrorString(e));
+    *fault_out = v;
+    return SQ_OK;
+}
