@@ -81,38 +81,57 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
-// Symmetric code clamp(rint(v / s), -qmax, qmax) with round-half-to-even,
-// bit-identical to an IEEE fp32 division followed by rint.
+// Symmetric code clamp(rint(v / s), -qmax, qmax) (round half to even),
+// bit-identical to an IEEE fp32 division followed by rint, for qmax <= 127.
 //
-// Fast path: y = v * r with r = RN(1/s).  Error analysis (two roundings of
-// relative size <= 2^-24 each, plus the rounding of the true quotient) gives
-// |y - RN(v/s)| < 0.75 * 2^-22 * |y|.  rint has its only discontinuities at
-// half-integers, so unless a half-integer lies within 2^-22 * |y| of y, the
-// two round to the same integer.  Inside that window (about one element in
-// 10^6) the exact IEEE quotient is used.  `exact_only` forces the division
-// (r is not finite when s is below ~2^-126).
-__device__ __forceinline__ float sym_code(float v, float s, float r, float qmax, bool exact_only) {
-    float q;
-    if (exact_only) {
-        q = rintf(__fdiv_rn(v, s));
-    } else {
-        float y = v * r;
-        float h = floorf(y) + 0.5f;
-        if (fabsf(y - h) <= fabsf(y) * 2.384185791015625e-07f)  // 2^-22
-            q = rintf(__fdiv_rn(v, s));
-        else
-            q = rintf(y);
-    }
-    return fminf(fmaxf(q, -qmax), qmax);
+// Fast path: y = v * r with r = RN(1/s).  Two roundings of relative size
+// <= 2^-24 plus the rounding of the true quotient give
+// |y - RN(v/s)| < 0.75 * 2^-22 * |y|.  rint only jumps at half-integers, so
+// y and RN(v/s) round to the same integer unless a half-integer lies within
+// 2^-22 |y| of y.  Whenever |y| <= 128 that window is below 2^-15; whenever
+// |y| > 128 both sides clamp to +/-qmax anyway.  So the exact IEEE quotient
+// is needed only when y's distance to its nearest integer is at least
+// 0.5 - 2^-15 (about one element in 16000).
+//
+// Rounding uses the magic constant 1.5 * 2^23: for |y| < 2^22 the sum
+// t = y + 1.5*2^23 is y rounded to an integer (ties to even, as the constant
+// is even) plus the constant, computed on the FP32 pipe; the clamped code is
+// then read from t's bit pattern.  Larger |y| only ever clamps.
+// Returns the code as an int; the caller converts as it needs.
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr int kRoundMagicBits = 0x4B400000;
+
+__device__ __forceinline__ int sym_code_i(float v, float s, float r, float qmax) {
+    const float y = v * r;
+    float t = y + kRoundMagic;
+    const float d = y - (t - kRoundMagic);
+    if (fabsf(d) >= 0.5f - 3.0517578125e-05f)  // within 2^-15 of a tie: exact quotient
+        t = rintf(__fdiv_rn(v, s)) + kRoundMagic;
+    t = fminf(fmaxf(t, kRoundMagic - qmax), kRoundMagic + qmax);
+    return __float_as_int(t) - kRoundMagicBits;
 }
 
-// Pack 8 codes (already integral floats in [-127,127]) into 8 bytes.
-__device__ __forceinline__ uint2 pack8_codes(const float (&q)[8]) {
+// Same code as a float; `exact_only` forces the IEEE division (used when
+// r = 1/s is not finite, i.e. s below ~2^-126).
+__device__ __forceinline__ float sym_code(float v, float s, float r, float qmax, bool exact_only) {
+    if (exact_only) return fminf(fmaxf(rintf(__fdiv_rn(v, s)), -qmax), qmax);
+    return (float)sym_code_i(v, s, r, qmax);
+}
+
+// Exact fp64 value of a small integer code without a conversion instruction:
+// the double with high word 0x43300000 and low word (q + 2^31) is
+// 2^52 + 2^31 + q.
+__device__ __forceinline__ double code_to_f64(int q) {
+    return __hiloint2double(0x43300000, q ^ (int)0x80000000) - 4503601774854144.0;
+}
+
+// Pack 8 integer codes in [-127,127] into 8 bytes.
+__device__ __forceinline__ uint2 pack8_codes(const int (&q)[8]) {
     uint32_t lo = 0, hi = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        lo |= ((uint32_t)(int32_t)q[i] & 0xffu) << (8 * i);
-        hi |= ((uint32_t)(int32_t)q[4 + i] & 0xffu) << (8 * i);
+        lo |= ((uint32_t)q[i] & 0xffu) << (8 * i);
+        hi |= ((uint32_t)q[4 + i] & 0xffu) << (8 * i);
     }
     return make_uint2(lo, hi);
 }

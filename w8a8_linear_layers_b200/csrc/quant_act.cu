@@ -78,10 +78,17 @@ quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__r
 #pragma unroll
         for (int c = 0; c < C; ++c) {
             if (!live[c]) continue;
-            float code[8];
+            int code[8];
+            if (s == 0.0f) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                code[i] = (s == 0.0f) ? 0.0f : sym_code(v[c][i], s, r, 127.0f, exact_only);
+                for (int i = 0; i < 8; ++i) code[i] = 0;
+            } else if (exact_only) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) code[i] = (int)sym_code(v[c][i], s, r, 127.0f, true);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) code[i] = sym_code_i(v[c][i], s, r, 127.0f);
+            }
             *reinterpret_cast<uint2 *>(qr + ((int64_t)c * T_ + threadIdx.x) * 8) = pack8_codes(code);
         }
     }

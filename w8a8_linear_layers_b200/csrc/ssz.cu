@@ -34,6 +34,15 @@
 
 namespace w8a8 {
 
+// Elements per thread for 2048 < K <= W8A8_SSZ_MID_MAX_K (a build-time
+// tuning choice; 32 elements per thread otherwise above 2048).
+#ifndef W8A8_SSZ_MID_E
+#define W8A8_SSZ_MID_E 32
+#endif
+#ifndef W8A8_SSZ_MID_MAX_K
+#define W8A8_SSZ_MID_MAX_K 8192
+#endif
+
 constexpr double kSszThreshold = 1e-10;
 constexpr float kSszMinScale = 1e-5f;
 
@@ -43,28 +52,65 @@ struct Sums {
     int den;      // sum q q  (<= 32768 * 127^2 < 2^31)
 };
 
+// One pass over this thread's elements at scale c.  Per element: the code
+// on the FP32 pipe (magic-constant rounding, as sym_code_i), the code widened
+// to fp64 from its bits, w widened by one F2F, the residual w - c q rounded
+// once (c*q is exact in fp64), and three accumulations, split four ways so
+// the fp64 adds do not form one long dependency chain.  The distance of each
+// scaled value to its nearest integer is folded into a running max instead
+// of branching per element; if any element of this thread came within 2^-15
+// of a tie, the thread redoes its sums from the shared-memory copy of its
+// elements with the exact IEEE quotient where needed (rare: about one thread
+// in 500 per pass).
 template <int C>
-__device__ __forceinline__ Sums row_pass(const float (&w)[C][8], const bool (&live)[C], float c,
-                                         float qmax) {
+__device__ __forceinline__ Sums row_pass(const float (&w)[C][8], const bool (&live)[C],
+                                         const float *__restrict__ wsh, float c, float qmax) {
     const float r = __fdiv_rn(1.0f, c);  // c >= 1e-5, so r is finite
     const double cd = (double)c;
-    double err = 0.0, wq = 0.0;
+    const float lo = kRoundMagic - qmax, hi = kRoundMagic + qmax;
+    double err[4] = {0.0, 0.0, 0.0, 0.0}, wq[4] = {0.0, 0.0, 0.0, 0.0};
     int den = 0;
+    float dmax = 0.0f;
 #pragma unroll
     for (int k = 0; k < C; ++k) {
         if (!live[k]) continue;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            float q = sym_code(w[k][i], c, r, qmax, false);
-            double wd = (double)w[k][i], qd = (double)q;
-            double e = fma(-cd, qd, wd);  // c*q is exact in fp64, so this is w - c q rounded once
-            err = fma(e, e, err);
-            wq = fma(wd, qd, wq);          // w*q is exact in fp64
-            int qi = (int)q;
-            den += qi * qi;
+            const float y = w[k][i] * r;
+            const float t = y + kRoundMagic;
+            dmax = fmaxf(dmax, fabsf(y - (t - kRoundMagic)));
+            const int q = __float_as_int(fminf(fmaxf(t, lo), hi)) - kRoundMagicBits;
+            const double qd = code_to_f64(q);
+            const double wd = (double)w[k][i];
+            const double e = fma(-cd, qd, wd);
+            err[i & 3] = fma(e, e, err[i & 3]);
+            wq[i & 3] = fma(wd, qd, wq[i & 3]);  // w*q is exact in fp64
+            den += q * q;
         }
     }
-    return {err, wq, den};
+    if (dmax >= 0.5f - 3.0517578125e-05f) {
+        // rare exact path, rolled over the shared-memory copy (same order)
+        const int T_ = blockDim.x;
+        double err_x = 0.0, wq_x = 0.0;
+        den = 0;
+#pragma unroll 1
+        for (int k = 0; k < C; ++k) {
+            if (!live[k]) continue;
+            const float *p = wsh + (k * T_ + threadIdx.x) * 8;
+#pragma unroll 1
+            for (int i = 0; i < 8; ++i) {
+                const int q = sym_code_i(p[i], c, r, qmax);
+                const double qd = code_to_f64(q);
+                const double wd = (double)p[i];
+                const double e = fma(-cd, qd, wd);
+                err_x = fma(e, e, err_x);
+                wq_x = fma(wd, qd, wq_x);
+                den += q * q;
+            }
+        }
+        return {err_x, wq_x, den};
+    }
+    return {(err[0] + err[1]) + (err[2] + err[3]), (wq[0] + wq[1]) + (wq[2] + wq[3]), den};
 }
 
 // Block-wide sum of Sums; every thread gets the same result (warps are
@@ -97,6 +143,7 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int64_t K, const float *__restri
     constexpr int C = E / 8;
     __shared__ Sums red[2][32];
     __shared__ float redmax[32];
+    extern __shared__ float wsh[];  // this channel's folded row (exact-path copy)
     const int T_ = blockDim.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = T_ >> 5;
 
@@ -117,6 +164,9 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int64_t K, const float *__restri
 #pragma unroll
                     for (int i = 0; i < 8; ++i) w[k][i] = w[k][i] * f[i];
                 }
+                float4 *dst = reinterpret_cast<float4 *>(wsh + j);
+                dst[0] = make_float4(w[k][0], w[k][1], w[k][2], w[k][3]);
+                dst[1] = make_float4(w[k][4], w[k][5], w[k][6], w[k][7]);
             } else {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) w[k][i] = 0.0f;
@@ -131,29 +181,37 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int64_t K, const float *__restri
         amax = redmax[0];
         for (int i = 1; i < nwarps; ++i) amax = fmaxf(amax, redmax[i]);
 
-        float s_best = fmaxf(__fdiv_rn(amax, qmax), kSszMinScale);
+        // Round 0 evaluates the MinMax scale; round it >= 1 evaluates the
+        // least-squares candidate built from the sums of the kept scale.  One
+        // inlined pass serves both, which keeps the kernel small.
         const double kd = (double)K;
-        int slot = 0;
-        Sums cur = block_sum(row_pass<C>(w, live, s_best, qmax), red, slot);
-        double m_best = cur.err / kd;
-
-        // ---- least-squares rounds
+        float s_best = fmaxf(__fdiv_rn(amax, qmax), kSszMinScale);
+        float c = s_best;
+        double m_best = 0.0;
+        Sums cur = {0.0, 0.0, 0};
         int it = 0;
-        bool done = false;
-        while (it < max_iters && !done) {
-            ++it;
-            float s_cand = s_best;
-            if (cur.den != 0) s_cand = fmaxf((float)(cur.wq / (double)cur.den), kSszMinScale);
+        int slot = 0;
+        for (;;) {
+            const Sums nxt = block_sum(row_pass<C>(w, live, wsh, c, qmax), red, slot);
             slot ^= 1;
-            Sums nxt = block_sum(row_pass<C>(w, live, s_cand, qmax), red, slot);
-            double m_cand = nxt.err / kd;
-            double delta = m_best - m_cand;
-            done = (m_best == 0.0) || (delta / m_best < kSszThreshold) || (fabs(delta) < kSszThreshold);
-            if (m_cand < m_best) {
-                s_best = s_cand;
-                m_best = m_cand;
+            const double m_c = nxt.err / kd;
+            if (it == 0) {
+                m_best = m_c;
                 cur = nxt;
+            } else {
+                const double delta = m_best - m_c;
+                const bool done = (m_best == 0.0) || (delta / m_best < kSszThreshold) ||
+                                  (fabs(delta) < kSszThreshold);
+                if (m_c < m_best) {
+                    s_best = c;
+                    m_best = m_c;
+                    cur = nxt;
+                }
+                if (done) break;
             }
+            if (it == max_iters) break;
+            ++it;
+            c = (cur.den != 0) ? fmaxf((float)(cur.wq / (double)cur.den), kSszMinScale) : s_best;
         }
 
         // ---- codes at the kept scale
@@ -161,9 +219,9 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int64_t K, const float *__restri
 #pragma unroll
         for (int k = 0; k < C; ++k) {
             if (!live[k]) continue;
-            float code[8];
+            int code[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) code[i] = sym_code(w[k][i], s_best, r, qmax, false);
+            for (int i = 0; i < 8; ++i) code[i] = sym_code_i(w[k][i], s_best, r, qmax);
             *reinterpret_cast<uint2 *>(q_out + n * K + ((int64_t)k * T_ + threadIdx.x) * 8) =
                 pack8_codes(code);
         }
@@ -185,12 +243,10 @@ static void launch_ssz(const void *w, int64_t N, int64_t K, const float *s, int 
     const float qmax = (float)((1 << (bits - 1)) - 1);
     const int per_sm = std::max(1, 2048 / threads);
     const int64_t grid = std::min<int64_t>(N, (int64_t)sms * per_sm * 4);
-    if (s)
-        ssz_kernel<T, E, true><<<(unsigned)grid, threads, 0, st>>>((const T *)w, N, K, s, qmax, max_iters,
-                                                                   q, scale, mse, iters);
-    else
-        ssz_kernel<T, E, false><<<(unsigned)grid, threads, 0, st>>>((const T *)w, N, K, s, qmax, max_iters,
-                                                                    q, scale, mse, iters);
+    const size_t smem = (size_t)threads * E * sizeof(float);  // <= 512 * 64 * 4 = 128 KB
+    auto kern = s ? ssz_kernel<T, E, true> : ssz_kernel<T, E, false>;
+    if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    kern<<<(unsigned)grid, threads, smem, st>>>((const T *)w, N, K, s, qmax, max_iters, q, scale, mse, iters);
 }
 
 }  // namespace w8a8
@@ -226,6 +282,7 @@ extern "C" sq_status ssz_quant_weight(const void *w, sq_dtype wt, int64_t N, int
     // elements per thread: at most 512 threads per channel row
     if (K <= 512) SSZ_LAUNCH(8);
     else if (K <= 2048) SSZ_LAUNCH(16);
+    else if (K <= W8A8_SSZ_MID_MAX_K) SSZ_LAUNCH(W8A8_SSZ_MID_E);
     else if (K <= 16384) SSZ_LAUNCH(32);
     else SSZ_LAUNCH(64);
 #undef SSZ_LAUNCH
