@@ -14,239 +14,379 @@
 // The SmoothQuant fold W' = W diag(s) ("SmoothQuant大模型量化技术深度解析",
 // section 1) is applied as the row is loaded.
 //
-// Readings (shared with the CPU oracle): the error is the mean over K of
-// (w - c Q(w,c))^2 summed in fp64 after re-quantising at the candidate c;
-// the relative and absolute tests are OR-ed, taken before the greedy update,
-// and a channel stops for good once it meets them; the minimum scale floors
-// the MinMax scale and every candidate; int4 codes are [-7, 7].
+// Readings (shared with the CPU oracle): the error of a scale c is the mean
+// over K of (w - c Q(w,c))^2 after re-quantising at c; the relative and
+// absolute tests are OR-ed, taken before the greedy update, and a channel
+// stops for good once it meets them; the minimum scale floors the MinMax
+// scale and every candidate; int4 codes are [-7, 7].
 //
-// Design: one CTA per output channel.  The folded row stays in registers for
-// the whole search (E fp32 values per thread), so W is read from HBM once and
-// the codes written once.  Each round is ONE pass over the row that computes,
-// for the candidate scale c, the codes Q(w,c), the error sum (w - c q)^2, and
-// the least-squares sums sum(w q), sum(q q) for the next candidate: when the
-// candidate is kept, the next round's least squares needs exactly these sums;
-// when it is not kept the channel has converged (d <= 0 passes the relative
-// test), so no round ever needs the sums of an older scale.  The three sums
-// are reduced across the CTA (warp shuffles, then the warps in a fixed order
-// so every thread takes the same decisions).
+// Design.  One CTA of R warps per output channel; the folded fp32 row stays
+// resident in shared memory for the whole search (W is read from HBM once,
+// the codes written once), next to two code buffers (kept / candidate).
+//
+// The error is evaluated exactly instead of by a per-element fp64 sum:
+//     K e(c) = W2 - 2 c NUM + c^2 DEN,  W2 = sum w^2, NUM = sum w q, DEN = sum q^2,
+// with W2 and NUM held in double-double (error-free transformations: Knuth's
+// TwoSum and the FMA TwoProduct), DEN exact, and the cancelling sum taken
+// with TwoSum, so e(c) is the exact error rounded once -- never further from
+// the true value than a direct fp64 sum.  NUM and DEN change only where a
+// code changes, so a round is one pass that computes the codes at the
+// candidate scale on the FP32 pipe (magic-constant rounding), compares them
+// 8 at a time with the kept codes and updates NUM/DEN for the few that moved.
+// Codes are exact: an element whose scaled value lies within |y| 2^-21 of a
+// half-integer takes the IEEE quotient (see sym_code_i for the bound).
+//
+// The search is a chain of rounds per channel, so the kernel is latency
+// bound; it keeps many channels in flight (small CTAs, shared-memory rows)
+// and keeps each round's serial tail short: warp trees skip warps whose
+// codes did not move, every warp takes the (identical) decision itself after
+// one barrier, and the next candidate is computed alongside the error.
 #include "common.cuh"
 
 namespace w8a8 {
 
-// Elements per thread for 2048 < K <= W8A8_SSZ_MID_MAX_K (a build-time
-// tuning choice; 32 elements per thread otherwise above 2048).
-#ifndef W8A8_SSZ_MID_E
-#define W8A8_SSZ_MID_E 32
-#endif
-#ifndef W8A8_SSZ_MID_MAX_K
-#define W8A8_SSZ_MID_MAX_K 8192
-#endif
-
 constexpr double kSszThreshold = 1e-10;
 constexpr float kSszMinScale = 1e-5f;
 
-struct Sums {
-    double err;   // sum (w - c q)^2
-    double wq;    // sum w q
-    int den;      // sum q q  (<= 32768 * 127^2 < 2^31)
+// ------------------------------------------------------------ double-double
+struct dd {
+    double hi, lo;
 };
 
-// One pass over this thread's elements at scale c.  Per element: the code
-// on the FP32 pipe (magic-constant rounding, as sym_code_i), the code widened
-// to fp64 from its bits, w widened by one F2F, the residual w - c q rounded
-// once (c*q is exact in fp64), and three accumulations, split four ways so
-// the fp64 adds do not form one long dependency chain.  The distance of each
-// scaled value to its nearest integer is folded into a running max instead
-// of branching per element; if any element of this thread came within 2^-15
-// of a tie, the thread redoes its sums from the shared-memory copy of its
-// elements with the exact IEEE quotient where needed (rare: about one thread
-// in 500 per pass).
-template <int C>
-__device__ __forceinline__ Sums row_pass(const float (&w)[C][8], const bool (&live)[C],
-                                         const float *__restrict__ wsh, float c, float qmax) {
-    const float r = __fdiv_rn(1.0f, c);  // c >= 1e-5, so r is finite
-    const double cd = (double)c;
-    const float lo = kRoundMagic - qmax, hi = kRoundMagic + qmax;
-    double err[4] = {0.0, 0.0, 0.0, 0.0}, wq[4] = {0.0, 0.0, 0.0, 0.0};
-    int den = 0;
-    float dmax = 0.0f;
+__device__ __forceinline__ dd two_sum(double a, double b) {
+    const double s = a + b;
+    const double bb = s - a;
+    return {s, (a - (s - bb)) + (b - bb)};
+}
+
+// a += b (b a double-double), cascaded: exact in hi/lo pairs up to the
+// rounding of the small lo sum.  TwoSum's error term is exact and symmetric
+// in its arguments, so butterfly reductions give identical results on all
+// lanes.
+__device__ __forceinline__ dd dd_add_cascade(dd a, dd b) {
+    const dd s = two_sum(a.hi, b.hi);
+    return {s.hi, (a.lo + b.lo) + s.lo};
+}
+
+__device__ __forceinline__ void dd_acc(dd &a, double t) {
+    const dd s = two_sum(a.hi, t);
+    a.hi = s.hi;
+    a.lo += s.lo;
+}
+
+__device__ __forceinline__ dd warp_sum_dd(dd a) {
 #pragma unroll
-    for (int k = 0; k < C; ++k) {
-        if (!live[k]) continue;
+    for (int o = 16; o > 0; o >>= 1)
+        a = dd_add_cascade(a, {__shfl_xor_sync(0xffffffffu, a.hi, o), __shfl_xor_sync(0xffffffffu, a.lo, o)});
+    return a;
+}
+
+__device__ __forceinline__ int warp_sum_i(int v) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float y = w[k][i] * r;
-            const float t = y + kRoundMagic;
-            dmax = fmaxf(dmax, fabsf(y - (t - kRoundMagic)));
-            const int q = __float_as_int(fminf(fmaxf(t, lo), hi)) - kRoundMagicBits;
-            const double qd = code_to_f64(q);
-            const double wd = (double)w[k][i];
-            const double e = fma(-cd, qd, wd);
-            err[i & 3] = fma(e, e, err[i & 3]);
-            wq[i & 3] = fma(wd, qd, wq[i & 3]);  // w*q is exact in fp64
-            den += q * q;
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// K e(c) = W2 - 2 c NUM + c^2 DEN, exact up to one final rounding.  The
+// search compares these K-scaled errors directly (K > 0 cancels), and
+// divides by K only for the reported error.
+__device__ __forceinline__ double exact_error_k(dd W2, dd NUM, int den, float c) {
+    const double c2x = 2.0 * (double)c;               // exact
+    const double p1 = c2x * NUM.hi;                   // 2 c NUM.hi = p1 + e1 exactly
+    const double e1 = fma(c2x, NUM.hi, -p1);
+    const double cc = (double)c * (double)c;           // exact (24-bit x 24-bit)
+    const double dend = (double)den;
+    const double p2 = dend * cc;                       // c^2 DEN = p2 + e2 exactly
+    const double e2 = fma(dend, cc, -p2);
+    const dd s1 = two_sum(W2.hi, -p1);
+    const dd s2 = two_sum(s1.hi, p2);
+    const double tail = ((s1.lo + s2.lo) + (W2.lo - e1)) + (e2 - c2x * NUM.lo);
+    const double v = s2.hi + tail;
+    // below the evaluation error (a few 2^-100 W2) the error is zero
+    return fabs(v) <= W2.hi * 0x1p-96 ? 0.0 : v;
+}
+
+// Next least-squares candidate from the kept sums (oracle: fp32 of the fp64
+// quotient, floored at the minimum scale; no codes: keep the scale).
+__device__ __forceinline__ float ls_candidate(dd NUM, int den, float keep) {
+    return den != 0 ? fmaxf((float)((NUM.hi + NUM.lo) / (double)den), kSszMinScale) : keep;
+}
+
+// The exact code of one element (IEEE quotient), out of line: only taken for
+// the rare elements near a rounding tie.
+__device__ __noinline__ int exact_code(float v, float c, float qmax) {
+    return (int)fminf(fmaxf(rintf(__fdiv_rn(v, c)), -qmax), qmax);
+}
+
+__device__ __forceinline__ int code_byte(uint2 p, int b) {
+    const uint32_t w = b < 4 ? p.x : p.y;
+    return (int)(int8_t)((w >> (8 * (b & 3))) & 0xffu);
+}
+
+struct PassOut {
+    dd num;     // init: NUM; update: change of NUM
+    dd w2;      // init only
+    int den;    // init: DEN; update: change of DEN
+    bool moved;
+};
+
+// Codes of 8 consecutive elements at scale c (fast path) packed in 8 bytes;
+// dmax collects max |y - rint(y)| for the tie test.
+__device__ __forceinline__ uint2 fast_codes8(const float4 a, const float4 b, float r, float lo, float hi,
+                                             float &dmax) {
+    const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t t[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float y = v[i] * r;
+        const float tt = y + kRoundMagic;
+        dmax = fmaxf(dmax, fabsf(y - (tt - kRoundMagic)));
+        t[i] = __float_as_uint(fminf(fmaxf(tt, lo), hi));  // code = low byte
+    }
+    const uint32_t p0 = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
+    const uint32_t p1 = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
+    return make_uint2(p0, p1);
+}
+
+// Change of NUM and DEN for one chunk whose packed codes moved from od to nw.
+__device__ __forceinline__ void chunk_delta(const float *__restrict__ wc, uint2 nw, uint2 od, PassOut &out) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int qn = code_byte(nw, i), qo = code_byte(od, i);
+        if (qn != qo) {
+            out.den += qn * qn - qo * qo;
+            dd_acc(out.num, (double)wc[i] * code_to_f64(qn - qo));  // exact product
         }
     }
-    if (dmax >= 0.5f - 3.0517578125e-05f) {
-        // rare exact path, rolled over the shared-memory copy (same order)
-        const int T_ = blockDim.x;
-        double err_x = 0.0, wq_x = 0.0;
-        den = 0;
+}
+
+// One pass at scale c over this thread's chunks of the row in shared memory.
+// Writes the codes at c into qc.  init: accumulates W2, NUM, DEN.  update:
+// accumulates the change of NUM and DEN against the kept codes qk; the main
+// loop only marks moved chunks (a warp would otherwise run the update path
+// whenever any lane had a moved chunk), which are then visited once.
+// wmax is the thread's max |w|, for the tie bound.
+template <bool INIT>
+__device__ __forceinline__ PassOut row_pass(const float *__restrict__ wrow, int K, float c, float qmax, float wmax,
+                                            const int8_t *__restrict__ qk, int8_t *__restrict__ qc) {
+    const int T_ = blockDim.x;
+    const int stride = T_ * 8;
+    const float r = __fdiv_rn(1.0f, c);  // c >= 1e-5, so r is finite
+    const float lo = kRoundMagic - qmax, hi = kRoundMagic + qmax;
+    PassOut out = {{0.0, 0.0}, {0.0, 0.0}, 0, false};
+    float dmax = 0.0f;
+    uint32_t moved = 0u;  // bit m: chunk m of this thread moved (at most 32 chunks per thread)
+    int m = 0;
+#pragma unroll 2
+    for (int j = threadIdx.x * 8; j < K; j += stride, ++m) {
+        const float4 a = *reinterpret_cast<const float4 *>(wrow + j);
+        const float4 b = *reinterpret_cast<const float4 *>(wrow + j + 4);
+        const uint2 nw = fast_codes8(a, b, r, lo, hi, dmax);
+        *reinterpret_cast<uint2 *>(qc + j) = nw;
+        if (INIT) {
+            const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int q = code_byte(nw, i);
+                const double wd = (double)v[i];
+                dd_acc(out.w2, wd * wd);               // exact product
+                dd_acc(out.num, wd * code_to_f64(q));  // exact product
+                out.den += q * q;
+            }
+        } else {
+            const uint2 od = *reinterpret_cast<const uint2 *>(qk + j);
+            if ((nw.x ^ od.x) | (nw.y ^ od.y)) moved |= 1u << m;
+        }
+    }
+    if (!INIT) {
+        out.moved = moved != 0u;
+        while (moved) {
+            const int mm = __ffs(moved) - 1;
+            moved &= moved - 1u;
+            const int j = threadIdx.x * 8 + mm * stride;
+            chunk_delta(wrow + j, *reinterpret_cast<const uint2 *>(qc + j), *reinterpret_cast<const uint2 *>(qk + j),
+                        out);
+        }
+    }
+    // Tie test: the fast code equals the exact one unless |y - rint(y)| is
+    // within |y| 2^-21 of 0.5 (|y| <= wmax r); rare, and then the thread
+    // takes the exact quotient for its near-tie elements.
+    if (dmax >= 0.5f - wmax * r * 4.76837158203125e-07f) {
 #pragma unroll 1
-        for (int k = 0; k < C; ++k) {
-            if (!live[k]) continue;
-            const float *p = wsh + (k * T_ + threadIdx.x) * 8;
+        for (int j = threadIdx.x * 8; j < K; j += stride) {
 #pragma unroll 1
             for (int i = 0; i < 8; ++i) {
-                const int q = sym_code_i(p[i], c, r, qmax);
-                const double qd = code_to_f64(q);
-                const double wd = (double)p[i];
-                const double e = fma(-cd, qd, wd);
-                err_x = fma(e, e, err_x);
-                wq_x = fma(wd, qd, wq_x);
-                den += q * q;
+                const float v = wrow[j + i];
+                const float y = v * r;
+                const float t = y + kRoundMagic;
+                const float d = y - (t - kRoundMagic);
+                if (fmaf(fabsf(y), 4.76837158203125e-07f, fabsf(d)) >= 0.5f) {
+                    const int qf = __float_as_int(fminf(fmaxf(t, lo), hi)) - kRoundMagicBits;
+                    const int qe = exact_code(v, c, qmax);
+                    if (qe != qf) {
+                        qc[j + i] = (int8_t)qe;
+                        out.den += qe * qe - qf * qf;
+                        dd_acc(out.num, (double)v * code_to_f64(qe - qf));
+                        out.moved = true;
+                    }
+                }
             }
         }
-        return {err_x, wq_x, den};
     }
-    return {(err[0] + err[1]) + (err[2] + err[3]), (wq[0] + wq[1]) + (wq[2] + wq[3]), den};
+    return out;
 }
 
-// Block-wide sum of Sums; every thread gets the same result (warps are
-// combined in index order).  `slot` alternates so one barrier per call is
-// enough.
-__device__ __forceinline__ Sums block_sum(Sums s, Sums (*red)[32], int slot) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        s.err += __shfl_xor_sync(0xffffffffu, s.err, o);
-        s.wq += __shfl_xor_sync(0xffffffffu, s.wq, o);
-        s.den += __shfl_xor_sync(0xffffffffu, s.den, o);
-    }
-    if (lane == 0) red[slot][warp] = s;
-    __syncthreads();
-    Sums t = red[slot][0];
-    for (int w = 1; w < nwarps; ++w) {
-        t.err += red[slot][w].err;
-        t.wq += red[slot][w].wq;
-        t.den += red[slot][w].den;
-    }
-    return t;
-}
+struct WarpPart {
+    dd num, w2;
+    int den;
+};
 
-template <typename T, int E, bool FOLD>
+template <typename T, bool FOLD>
 __global__ void __launch_bounds__(512)
-ssz_kernel(const T *__restrict__ wg, int64_t N, int64_t K, const float *__restrict__ s, float qmax,
-           int max_iters, int8_t *__restrict__ q_out, float *__restrict__ scale_out,
-           double *__restrict__ mse_out, int32_t *__restrict__ iters_out) {
-    constexpr int C = E / 8;
-    __shared__ Sums red[2][32];
-    __shared__ float redmax[32];
-    extern __shared__ float wsh[];  // this channel's folded row (exact-path copy)
+ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__ s, float qmax, int max_iters,
+           int8_t *__restrict__ q_out, float *__restrict__ scale_out, double *__restrict__ mse_out,
+           int32_t *__restrict__ iters_out) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    float *wrow = reinterpret_cast<float *>(smem);            // K floats: the folded row
+    int8_t *qbuf = reinterpret_cast<int8_t *>(wrow + K);      // 2 x K codes: kept / candidate
+    __shared__ WarpPart part[2][16];                          // per-warp partials, by round parity
+    __shared__ float redmax[16];
     const int T_ = blockDim.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = T_ >> 5;
+    const double kd = (double)K;
+    const double thr_k = kSszThreshold * kd;  // absolute threshold on K-scaled errors
 
     for (int64_t n = blockIdx.x; n < N; n += gridDim.x) {
-        // ---- load the folded row into registers
-        float w[C][8];
-        bool live[C];
+        // ---- stage the folded row in shared memory
         float amax = 0.0f;
+#pragma unroll 4
+        for (int j = threadIdx.x * 8; j < K; j += T_ * 8) {
+            float v[8];
+            Vec8<T>::load(wg + n * K + j, v);
+            if (FOLD) {
+                float f[8];
+                load8_f32(s + j, f);
 #pragma unroll
-        for (int k = 0; k < C; ++k) {
-            int64_t j = ((int64_t)k * T_ + threadIdx.x) * 8;
-            live[k] = j < K;
-            if (live[k]) {
-                Vec8<T>::load(wg + n * K + j, w[k]);
-                if (FOLD) {
-                    float f[8];
-                    load8_f32(s + j, f);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) w[k][i] = w[k][i] * f[i];
-                }
-                float4 *dst = reinterpret_cast<float4 *>(wsh + j);
-                dst[0] = make_float4(w[k][0], w[k][1], w[k][2], w[k][3]);
-                dst[1] = make_float4(w[k][4], w[k][5], w[k][6], w[k][7]);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) w[k][i] = 0.0f;
+                for (int i = 0; i < 8; ++i) v[i] = v[i] * f[i];
             }
 #pragma unroll
-            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(w[k][i]));
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+            float4 *dst = reinterpret_cast<float4 *>(wrow + j);
+            dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+            dst[1] = make_float4(v[4], v[5], v[6], v[7]);
         }
-        // ---- MinMax init
+        const float wmax = amax;  // this thread's max |w| (tie bound)
         amax = warp_max(amax);
         if (lane == 0) redmax[warp] = amax;
         __syncthreads();
         amax = redmax[0];
         for (int i = 1; i < nwarps; ++i) amax = fmaxf(amax, redmax[i]);
 
-        // Round 0 evaluates the MinMax scale; round it >= 1 evaluates the
-        // least-squares candidate built from the sums of the kept scale.  One
-        // inlined pass serves both, which keeps the kernel small.
-        const double kd = (double)K;
+        // ---- MinMax init: codes into buffer 0, exact W2 / NUM / DEN
+        int8_t *qk = qbuf, *qc = qbuf + K;
         float s_best = fmaxf(__fdiv_rn(amax, qmax), kSszMinScale);
-        float c = s_best;
-        double m_best = 0.0;
-        Sums cur = {0.0, 0.0, 0};
+        int par = 0;
+        {
+            PassOut p = row_pass<true>(wrow, K, s_best, qmax, wmax, nullptr, qk);
+            p.num = warp_sum_dd(p.num);
+            p.w2 = warp_sum_dd(p.w2);
+            p.den = warp_sum_i(p.den);
+            if (lane == 0) part[par][warp] = {p.num, p.w2, p.den};
+        }
+        __syncthreads();
+        // every thread holds the (identical) channel state
+        dd W2 = part[par][0].w2, NUM = part[par][0].num;
+        int DEN = part[par][0].den;
+        for (int i = 1; i < nwarps; ++i) {
+            W2 = dd_add_cascade(W2, part[par][i].w2);
+            NUM = dd_add_cascade(NUM, part[par][i].num);
+            DEN += part[par][i].den;
+        }
+        double m_best = exact_error_k(W2, NUM, DEN, s_best);  // K x error
+        float c = ls_candidate(NUM, DEN, s_best);
         int it = 0;
-        int slot = 0;
-        for (;;) {
-            const Sums nxt = block_sum(row_pass<C>(w, live, wsh, c, qmax), red, slot);
-            slot ^= 1;
-            const double m_c = nxt.err / kd;
-            if (it == 0) {
-                m_best = m_c;
-                cur = nxt;
+        bool done = max_iters == 0;
+
+        // ---- least-squares rounds
+        while (!done) {
+            par ^= 1;
+            PassOut p = row_pass<false>(wrow, K, c, qmax, wmax, qk, qc);
+            if (__any_sync(0xffffffffu, p.moved)) {
+                p.num = warp_sum_dd(p.num);
+                p.den = warp_sum_i(p.den);
             } else {
-                const double delta = m_best - m_c;
-                const bool done = (m_best == 0.0) || (delta / m_best < kSszThreshold) ||
-                                  (fabs(delta) < kSszThreshold);
-                if (m_c < m_best) {
-                    s_best = c;
-                    m_best = m_c;
-                    cur = nxt;
-                }
-                if (done) break;
+                p.num = {0.0, 0.0};
+                p.den = 0;
             }
-            if (it == max_iters) break;
+            if (lane == 0) part[par][warp] = {p.num, {0.0, 0.0}, p.den};
+            __syncthreads();  // the candidate codes and all partials are in place
             ++it;
-            c = (cur.den != 0) ? fmaxf((float)(cur.wq / (double)cur.den), kSszMinScale) : s_best;
+            dd num_c = NUM;
+            int den_c = DEN;
+            for (int i = 0; i < nwarps; ++i) {
+                num_c = dd_add_cascade(num_c, part[par][i].num);
+                den_c += part[par][i].den;
+            }
+            const double m_c = exact_error_k(W2, num_c, den_c, c);
+            const float c_next = ls_candidate(num_c, den_c, c);  // used only if c is kept
+            // on K-scaled errors: d/e < thr  <=>  dK < thr eK (eK > 0), |d| < thr  <=>  |dK| < thr K
+            const double delta = m_best - m_c;
+            done = (m_best == 0.0) || (delta < kSszThreshold * m_best) || (fabs(delta) < thr_k) ||
+                   it == max_iters;
+            if (m_c < m_best) {  // keep c: its codes become the kept codes
+                s_best = c;
+                m_best = m_c;
+                NUM = num_c;
+                DEN = den_c;
+                int8_t *t = qk;
+                qk = qc;
+                qc = t;
+                c = c_next;
+            }
+            // part[par] is rewritten two rounds from now, after another barrier
         }
 
-        // ---- codes at the kept scale
-        const float r = __fdiv_rn(1.0f, s_best);
-#pragma unroll
-        for (int k = 0; k < C; ++k) {
-            if (!live[k]) continue;
-            int code[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) code[i] = sym_code_i(w[k][i], s_best, r, qmax);
-            *reinterpret_cast<uint2 *>(q_out + n * K + ((int64_t)k * T_ + threadIdx.x) * 8) =
-                pack8_codes(code);
-        }
+        // ---- kept codes out (each thread wrote and now reads its own chunks)
+        for (int j = threadIdx.x * 8; j < K; j += T_ * 8)
+            *reinterpret_cast<uint2 *>(q_out + n * K + j) = *reinterpret_cast<const uint2 *>(qk + j);
         if (threadIdx.x == 0) {
             scale_out[n] = s_best;
-            if (mse_out) mse_out[n] = m_best;
+            if (mse_out) mse_out[n] = m_best / kd;
             if (iters_out) iters_out[n] = it;
         }
-        // redmax / red slots are reused by the next row: make sure every
-        // thread has read them
-        __syncthreads();
+        __syncthreads();  // shared row and buffers are reused by the next channel
     }
 }
 
-template <typename T, int E>
-static void launch_ssz(const void *w, int64_t N, int64_t K, const float *s, int bits, int max_iters,
-                       int8_t *q, float *scale, double *mse, int32_t *iters, int sms, cudaStream_t st) {
-    const int threads = (int)ceil_div(ceil_div(K, E), 32) * 32;
+// Warps per channel: enough channels in flight per SM to cover each round's
+// serial tail, enough warps per channel to spread a pass.
+static int ssz_warps(int64_t K) {
+#ifdef W8A8_SSZ_WARPS
+    int64_t w = W8A8_SSZ_WARPS;
+#else
+    int64_t w = ceil_div(K, 2048);
+#endif
+    // at most 32 chunks of 8 per thread (the moved-chunk mask is 32 bits)
+    w = std::max<int64_t>(w, ceil_div(K, 32 * 32 * 8));
+    return (int)std::min<int64_t>(16, std::max<int64_t>(1, w));
+}
+
+template <typename T>
+static sq_status launch_ssz(const void *w, int64_t N, int64_t K, const float *s, int bits, int max_iters,
+                            int8_t *q, float *scale, double *mse, int32_t *iters, int sms, cudaStream_t st) {
+    const int threads = 32 * ssz_warps(K);
     const float qmax = (float)((1 << (bits - 1)) - 1);
-    const int per_sm = std::max(1, 2048 / threads);
-    const int64_t grid = std::min<int64_t>(N, (int64_t)sms * per_sm * 4);
-    const size_t smem = (size_t)threads * E * sizeof(float);  // <= 512 * 64 * 4 = 128 KB
-    auto kern = s ? ssz_kernel<T, E, true> : ssz_kernel<T, E, false>;
-    if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    kern<<<(unsigned)grid, threads, smem, st>>>((const T *)w, N, K, s, qmax, max_iters, q, scale, mse, iters);
+    const size_t smem = 6 * (size_t)K;  // fp32 row + kept + candidate codes
+    auto kern = s ? ssz_kernel<T, true> : ssz_kernel<T, false>;
+    if (smem > 32 * 1024) {  // dynamic + static shared memory may pass the 48 KB default
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return fail(SQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    }
+    int per_sm = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
+    const int64_t grid = std::min<int64_t>(N, (int64_t)sms * std::max(per_sm, 1) * 8);
+    kern<<<(unsigned)grid, threads, smem, st>>>((const T *)w, N, (int)K, s, qmax, max_iters, q, scale, mse, iters);
+    return launch_status("ssz_kernel");
 }
 
 }  // namespace w8a8
@@ -273,18 +413,7 @@ extern "C" sq_status ssz_quant_weight(const void *w, sq_dtype wt, int64_t N, int
     sq_status st = check_device(&sms);
     if (st != SQ_OK) return st;
     cudaStream_t cs = (cudaStream_t)stream;
-    const bool bf = wt == SQ_BF16;
-#define SSZ_LAUNCH(E)                                                                              \
-    (bf ? launch_ssz<__nv_bfloat16, E>(w, N, K, s, bits, max_iters, q_out, scale_out, mse_out,     \
-                                       iters_out, sms, cs)                                         \
-        : launch_ssz<float, E>(w, N, K, s, bits, max_iters, q_out, scale_out, mse_out, iters_out, \
-                               sms, cs))
-    // elements per thread: at most 512 threads per channel row
-    if (K <= 512) SSZ_LAUNCH(8);
-    else if (K <= 2048) SSZ_LAUNCH(16);
-    else if (K <= W8A8_SSZ_MID_MAX_K) SSZ_LAUNCH(W8A8_SSZ_MID_E);
-    else if (K <= 16384) SSZ_LAUNCH(32);
-    else SSZ_LAUNCH(64);
-#undef SSZ_LAUNCH
-    return launch_status("ssz_kernel");
+    if (wt == SQ_BF16)
+        return launch_ssz<__nv_bfloat16>(w, N, K, s, bits, max_iters, q_out, scale_out, mse_out, iters_out, sms, cs);
+    return launch_ssz<float>(w, N, K, s, bits, max_iters, q_out, scale_out, mse_out, iters_out, sms, cs);
 }
