@@ -47,6 +47,9 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=20)
+    p.add_argument("--record-traffic", metavar="NCU_CSV",
+                   help="read an ncu --csv capture (gpu__time_duration.sum, dram__bytes_read.sum, "
+                        "dram__bytes_write.sum) of this workload and write profiles/dram_traffic.json")
     return p.parse_args()
 
 
@@ -159,6 +162,7 @@ def run_ours(args, rank, world, local_rank):
 
     import synthetic
     import w8a8_linear_layers_b200 as w
+    from w8a8_linear_layers_b200 import distributed as wdist
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -190,8 +194,7 @@ def run_ours(args, rank, world, local_rank):
         mark(0)
         w.sq_calib_absmax(xin, ax)
         mark(1)
-        if world > 1:
-            dist.all_reduce(ax, op=dist.ReduceOp.MAX)
+        wdist.allreduce_calibration(ax)
         w.sq_smooth_fold(ax, wt, cfg.alpha, aw, s, inv)
         mark(2)
         w.ssz_quant_weight(wt, s, cfg.bits, cfg.max_iters, qw, sw)
@@ -223,11 +226,7 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     step_ms = [e[0].elapsed_time(e[5]) for e in evs]
     kern_ms = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, n in enumerate(names)}
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = wdist.max_over_ranks(sum(step_ms), device=dev)
     if w.device_fault() != 0:
         raise RuntimeError("a kernel gave up on a bounded wait during timing")
 
@@ -237,12 +236,12 @@ def run_ours(args, rank, world, local_rank):
     # ---- end to end through the C ABI with host buffers
     e2e = None
     if args.e2e_steps > 0:
-        e2e = run_e2e(args, w, dist, world, x_cpu, w_cpu, x, wt, cfg, ax, aw, s, inv, qw, sw, qx, sx, y, flush,
+        e2e = run_e2e(args, w, wdist, world, x_cpu, w_cpu, x, wt, cfg, ax, aw, s, inv, qw, sw, qx, sx, y, flush,
                       stream)
     return finish(args, world, cfg, names, kern_ms, total_ms, value, e2e, clk, wall1 - wall0)
 
 
-def run_e2e(args, w, dist, world, x_cpu, w_cpu, x, wt, cfg, ax, aw, s, inv, qw, sw, qx, sx, y, flush, stream):
+def run_e2e(args, w, wdist, world, x_cpu, w_cpu, x, wt, cfg, ax, aw, s, inv, qw, sw, qx, sx, y, flush, stream):
     import torch
     M, K, N = cfg.M, cfg.K, cfg.N
     ydt = y.dtype
@@ -260,8 +259,7 @@ def run_e2e(args, w, dist, world, x_cpu, w_cpu, x, wt, cfg, ax, aw, s, inv, qw, 
         xd.copy_(xh, non_blocking=True)
         wd.copy_(wh, non_blocking=True)
         w.sq_calib_absmax(xd, ax)
-        if world > 1:
-            dist.all_reduce(ax, op=dist.ReduceOp.MAX)
+        wdist.allreduce_calibration(ax)
         w.sq_smooth_fold(ax, wd, cfg.alpha, aw, s, inv)
         w.ssz_quant_weight(wd, s, cfg.bits, cfg.max_iters, qw, sw)
         w.quant_act_per_token(xd, inv, qx, sx)
@@ -271,11 +269,7 @@ def run_e2e(args, w, dist, world, x_cpu, w_cpu, x, wt, cfg, ax, aw, s, inv, qw, 
         e1.synchronize()
         if i >= args.warmup:
             e2e_ms.append(e0.elapsed_time(e1))
-    e2e_total = sum(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
+    e2e_total = wdist.max_over_ranks(sum(e2e_ms), device=x.device)
     e2e_value = ops_per_step * world * len(e2e_ms) / (e2e_total * 1e-3) / 1e12
     h2d = x.numel() * x.element_size() + wt.numel() * wt.element_size()
     d2h = y.numel() * y.element_size()
@@ -427,8 +421,68 @@ def run_reference(args, rank):
     }
 
 
+# kernel name prefix in an ncu capture -> step of the path
+NCU_KERNELS = [("col_absmax_kernel", None), ("smooth_factor_kernel", "smooth_fold"), ("ssz_kernel", "ssz_quant_weight"),
+               ("quant_act_kernel", "quant_act_per_token"), ("w8a8_gemm_kernel", "w8a8_gemm_dequant")]
+
+
+def record_traffic(csv_path, workload):
+    """DRAM bytes per launch of each kernel from an ncu capture of this
+    bench's workload; written with the hash of each kernel's source so the
+    numbers are dropped once the kernel changes."""
+    import csv
+    import collections
+    rows = [r for r in csv.reader(open(csv_path)) if r]
+    hdr = next(r for r in rows if r[0] == "ID")
+    per = collections.defaultdict(lambda: collections.defaultdict(dict))
+    for r in rows[rows.index(hdr) + 1:]:
+        if len(r) != len(hdr):
+            continue
+        d = dict(zip(hdr, r))
+        scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "nsecond": 1e-9, "usecond": 1e-6,
+                 "msecond": 1e-3}.get(d["Metric Unit"], 1.0)
+        per[d["Kernel Name"]][d["ID"]][d["Metric Name"]] = float(d["Metric Value"].replace(",", "")) * scale
+    # launches in ID order; a step launches col_absmax twice (X, then W),
+    # smooth_factor, ssz, quant_act, gemm
+    launches = []
+    for kname, ls in per.items():
+        for lid, v in ls.items():
+            launches.append((int(lid), kname, v))
+    launches.sort()
+    acc = collections.defaultdict(list)
+    n_col = 0
+    for _, kname, v in launches:
+        if "dram__bytes_read.sum" not in v:
+            continue
+        t = v["dram__bytes_read.sum"] + v.get("dram__bytes_write.sum", 0.0)
+        if "col_absmax_kernel" in kname:
+            acc["calib_absmax" if n_col % 2 == 0 else "smooth_fold"].append(t)
+            n_col += 1
+            continue
+        for prefix, step in NCU_KERNELS:
+            if step and prefix in kname:
+                if step == "smooth_fold" and acc["smooth_fold"]:
+                    acc["smooth_fold"][-1] += t  # same step as the preceding W absmax
+                else:
+                    acc[step].append(t)
+    out = {}
+    for step, ts in acc.items():
+        if ts:
+            out[step] = {"bytes_per_launch": int(sum(ts) / len(ts)), "launches": len(ts),
+                         "src_sha": source_sha(KERNEL_SOURCES[step])}
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    allw = json.load(open(path)) if os.path.exists(path) else {}
+    allw[workload] = out
+    with open(path, "w") as f:
+        json.dump(allw, f, indent=1, sort_keys=True)
+    print(json.dumps(out, indent=1))
+
+
 def main():
     args = parse()
+    if args.record_traffic:
+        record_traffic(args.record_traffic, args.workload)
+        return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
