@@ -84,29 +84,25 @@ __device__ __forceinline__ float warp_max(float v) {
 // Symmetric code clamp(rint(v / s), -qmax, qmax) (round half to even),
 // bit-identical to an IEEE fp32 division followed by rint, for qmax <= 127.
 //
-// Fast path: y = v * r with r = RN(1/s).  Two roundings of relative size
-// <= 2^-24 plus the rounding of the true quotient give
-// |y - RN(v/s)| < 0.75 * 2^-22 * |y|.  rint only jumps at half-integers, so
-// y and RN(v/s) round to the same integer unless a half-integer lies within
-// 2^-22 |y| of y.  Whenever |y| <= 128 that window is below 2^-15; whenever
-// |y| > 128 both sides clamp to +/-qmax anyway.  So the exact IEEE quotient
-// is needed only when y's distance to its nearest integer is at least
-// 0.5 - 2^-15 (about one element in 16000).
-//
-// Rounding uses the magic constant 1.5 * 2^23: for |y| < 2^22 the sum
-// t = y + 1.5*2^23 is y rounded to an integer (ties to even, as the constant
-// is even) plus the constant, computed on the FP32 pipe; the clamped code is
-// then read from t's bit pattern.  Larger |y| only ever clamps.
-// Returns the code as an int; the caller converts as it needs.
+// Fast path, all on the FMA pipe: with r = RN(1/s) and the magic constant
+// M = 1.5 * 2^23, t = fma(v, r, M) = RN(v r + M), which for |v r| < 2^22 is M
+// plus v r rounded to an integer (ties to even; M is even) -- the EXACT
+// product v r, rounded once.  Since r carries one rounding (2^-24 relative)
+// and the IEEE quotient another, |v r - RN(v/s)| <= 2^-23 |y|, so the two
+// round to the same integer unless a half-integer lies within 2^-23 |y|.
+// d = fma(v, r, M - t) = RN(v r - rint(v r)) measures the distance to the
+// nearest integer (M - t is exact); when |d| comes within
+// |rint| 2^-21 + 2^-22 (>= 2^-21 |y|, a 4x margin) of 0.5 the exact quotient
+// is taken.  Larger |v r| only ever clamps.  Returns the code as an int.
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
 constexpr int kRoundMagicBits = 0x4B400000;
 
 __device__ __forceinline__ int sym_code_i(float v, float s, float r, float qmax) {
-    const float y = v * r;
-    float t = y + kRoundMagic;
-    const float d = y - (t - kRoundMagic);
-    if (fabsf(d) >= 0.5f - 3.0517578125e-05f)  // within 2^-15 of a tie: exact quotient
-        t = rintf(__fdiv_rn(v, s)) + kRoundMagic;
+    float t = fmaf(v, r, kRoundMagic);
+    const float rq = t - kRoundMagic;
+    const float d = fmaf(v, r, -rq);
+    if (fabsf(d) + fmaf(fabsf(rq), 4.76837158203125e-07f, 2.384185791015625e-07f) >= 0.5f)
+        t = rintf(__fdiv_rn(v, s)) + kRoundMagic;  // near a tie: exact quotient
     t = fminf(fmaxf(t, kRoundMagic - qmax), kRoundMagic + qmax);
     return __float_as_int(t) - kRoundMagicBits;
 }
@@ -123,6 +119,27 @@ __device__ __forceinline__ float sym_code(float v, float s, float r, float qmax,
 // 2^52 + 2^31 + q.
 __device__ __forceinline__ double code_to_f64(int q) {
     return __hiloint2double(0x43300000, q ^ (int)0x80000000) - 4503601774854144.0;
+}
+
+// Packed two-lane fp32 arithmetic of sm_100 (fma/sub .rn.f32x2): each lane
+// rounds exactly like the scalar IEEE operation.  Only fused multiply-adds
+// and subtractions are used, so there is no separate product for the
+// compiler to fuse with a later add.
+union F2U {
+    float2 f;
+    unsigned long long u;
+};
+
+__device__ __forceinline__ float2 f2_fma(float2 a, float2 b, float2 c) {
+    F2U x{a}, y{b}, z{c}, r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r.u) : "l"(x.u), "l"(y.u), "l"(z.u));
+    return r.f;
+}
+
+__device__ __forceinline__ float2 f2_sub(float2 a, float2 b) {
+    F2U x{a}, y{b}, r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r.u) : "l"(x.u), "l"(y.u));
+    return r.f;
 }
 
 // Pack 8 integer codes in [-127,127] into 8 bytes.

@@ -448,6 +448,315 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     }
 }
 
+// ============================================================ 2-CTA pair kernel
+// A cluster of two CTAs (a "pair") computes a 256 x 256 output tile with
+// tcgen05.mma.cta_group::2: each CTA stages 128 rows of A (its half of the
+// tile's M) and 128 rows of B (its half of N) per stage, and the pair's
+// tensor cores compute 128 x 256 each into their own TMEM, reading both B
+// halves.  Per SM this halves the B operand traffic of a 1-CTA 128 x 256 tile
+// (64 instead of 96 shared-memory bytes per MMA cycle) and doubles the work
+// each staged byte feeds.
+//
+// Synchronisation (leader = CTA rank 0 of the pair):
+//   full[s]   (leader) : leader's producer posts arrive.expect_tx for both
+//                        CTAs' bytes; both CTAs' TMA loads complete_tx on it;
+//   empty[s]  (each)   : the leader's MMA commit multicasts to both CTAs;
+//   tfull[b]  (each)   : the leader's commit after a tile's last k-block,
+//                        multicast to both CTAs;
+//   tempty[b] (leader) : all 2 x 128 epilogue threads of the pair arrive.
+// TMEM (512 columns) is allocated and freed by warp 1 of both CTAs
+// (cta_group::2); cluster barriers order barrier init before any remote
+// arrival and keep both CTAs alive until the pair is done.
+
+constexpr uint32_t kPeerMask = 0xFEFFFFFFu;  // shared::cluster address -> same offset in rank 0
+
+// Tile t -> (m tile, n tile).  Consecutive pairs walk down M within a band of
+// N tiles, so concurrently running pairs share B tiles in L2.
+__device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, int &tm, int &tn) {
+#ifdef W8A8_TILE_N_FASTEST
+    tm = tile / tiles_n;
+    tn = tile % tiles_n;
+#else
+    tm = tile % tiles_m;
+    tn = tile / tiles_m;
+    (void)tiles_n;
+#endif
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, uint32_t leader_bar, int x,
+                                                 int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+        "[%2];" ::"r"(dst),
+        "l"((uint64_t)map), "r"(leader_bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t slot_smem, uint32_t cols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_smem), "r"(cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t cols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
+}
+
+__device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on `bar` (same offset) in both CTAs of the pair once this thread's
+// issued tcgen05 ops complete.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}"
+        ::"r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_leader(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar & kPeerMask) : "memory");
+}
+
+template <typename OutT>
+__device__ __forceinline__ void epilogue_tile(uint32_t tbase, int row, int M, int n0, int N, const float sxr,
+                                              const float *__restrict__ sw, OutT *__restrict__ y,
+                                              int32_t *__restrict__ acc_out, int BNc) {
+    const bool vec_ok = (N % (16 / (int)sizeof(OutT))) == 0;
+    const bool acc_vec_ok = (N % 4) == 0;
+#pragma unroll 1
+    for (int c0 = 0; c0 < BNc; c0 += 32) {
+        uint32_t acc[32];
+        tmem_ld32(tbase + (uint32_t)c0, acc);  // warp-collective
+        const int col = n0 + c0;
+        if (row < M && col < N) {
+            const int valid = N - col;
+            store_row_chunk<OutT>(y + (int64_t)row * N + col, acc, sxr, sw + col, valid, vec_ok);
+            if (acc_out) {
+                int32_t *arow = acc_out + (int64_t)row * N + col;
+                if (acc_vec_ok && valid >= 32) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<int4 *>(arow + j) =
+                            make_int4((int)acc[j], (int)acc[j + 1], (int)acc[j + 2], (int)acc[j + 3]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (j < valid) arow[j] = (int)acc[j];
+                }
+            }
+        }
+    }
+}
+
+#ifndef W8A8_PAIR_STAGES
+#define W8A8_PAIR_STAGES 6
+#endif
+
+struct Cfg2 {
+    static constexpr int BN = 256;              // pair tile N (each CTA stages BN/2 rows of B)
+    static constexpr int PM = 2 * BM;           // pair tile M
+    static constexpr int STAGES = W8A8_PAIR_STAGES;
+    static constexpr int A_BYTES = BM * BK;     // 16 KB: this CTA's 128 rows of A
+    static constexpr int B_BYTES = (BN / 2) * BK;  // 16 KB: this CTA's half of B
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int TMEM_COLS = 2 * BN;    // two 128 x 256 accumulator buffers
+    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024;
+};
+
+template <typename OutT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+w8a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                      const float *__restrict__ sx, const float *__restrict__ sw, OutT *__restrict__ y,
+                      int32_t *__restrict__ acc_out, int M, int N, int K) {
+    using C = Cfg2;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full_bar[C::STAGES];
+    __shared__ __align__(8) uint64_t empty_bar[C::STAGES];
+    __shared__ __align__(8) uint64_t tfull_bar[2];
+    __shared__ __align__(8) uint64_t tempty_bar[2];
+    __shared__ __align__(8) uint64_t drain_bar;
+    __shared__ uint32_t tmem_slot;
+    __shared__ volatile int abort_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;  // same offset in both CTAs
+
+    const int tiles_m = (M + C::PM - 1) / C::PM;
+    const int tiles_n = (N + C::BN - 1) / C::BN;
+    const int num_tiles = tiles_m * tiles_n;
+    const int num_kb = (K + BK - 1) / BK;
+    const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(smem_u32(&full_bar[s]), 1);
+            mbar_init(smem_u32(&empty_bar[s]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&tfull_bar[b]), 1);
+            mbar_init(smem_u32(&tempty_bar[b]), 2 * 4 * 32);
+        }
+        mbar_init(smem_u32(&drain_bar), 1);
+        abort_flag = 0;
+        fence_barrier_init();
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tmap_a) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tmap_b) : "memory");
+    }
+    if (warp == 1) tmem_alloc_pair(smem_u32(&tmem_slot), C::TMEM_COLS);
+    tc_fence_before();
+    cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            bool ok = true;
+            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+                int tm, tn;
+                tile_coords(tile, tiles_m, tiles_n, tm, tn);
+                const int m0 = tm * C::PM + (int)rank * BM;
+                const int n0 = tn * C::BN + (int)rank * (C::BN / 2);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, &abort_flag, kFaultProducer)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t a_dst = smem_base + stage * C::STAGE_BYTES;
+                    const uint32_t b_dst = a_dst + C::A_BYTES;
+                    const uint32_t fb = smem_u32(&full_bar[stage]);
+                    if (leader) mbar_arrive_expect_tx(fb, 2 * C::STAGE_BYTES);  // both CTAs' bytes
+                    tma_load_2d_pair(a_dst, &tmap_a, fb & kPeerMask, kb * BK, m0);
+                    tma_load_2d_pair(b_dst, &tmap_b, fb & kPeerMask, kb * BK, n0);
+                    ++issued;
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok && leader) {
+                // drain: wait (bounded) for the last issued stages to land
+                int outstanding = issued < C::STAGES ? issued : C::STAGES;
+                int s = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < outstanding; ++i) {
+                    if (--s < 0) {
+                        s = C::STAGES - 1;
+                        ph ^= 1u;
+                    }
+                    const unsigned long long t0 = globaltimer();
+                    while (!mbar_try_wait(smem_u32(&full_bar[s]), ph) && globaltimer() - t0 < kWaitNs) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (leader CTA only)
+        if (leader && lane == 0) {
+            constexpr uint32_t idesc = idesc_i8(C::PM, C::BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int buf = 0;
+            uint32_t buf_phase = 0;
+            bool ok = true;
+            bool issued_any = false;
+            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+                if (!wait_bounded(smem_u32(&tempty_bar[buf]), buf_phase ^ 1u, &abort_flag, kFaultMmaTmemEmpty)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(buf * C::BN);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!wait_bounded(smem_u32(&full_bar[stage]), phase, &abort_flag, kFaultMmaFull)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_base + stage * C::STAGE_BYTES;
+                    const uint32_t b_addr = a_addr + C::A_BYTES;
+#pragma unroll
+                    for (int k = 0; k < BK / UMMA_K; ++k) {
+                        mma_i8_pair(d_tmem, smem_desc_sw128(a_addr + k * UMMA_K),
+                                    smem_desc_sw128(b_addr + k * UMMA_K), idesc, (kb | k) != 0 ? 1u : 0u);
+                    }
+                    issued_any = true;
+                    mma_commit_pair(smem_u32(&empty_bar[stage]));
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit_pair(smem_u32(&tfull_bar[buf]));
+                buf ^= 1;
+                if (buf == 0) buf_phase ^= 1u;
+            }
+            if (!ok && issued_any) {
+                mma_commit_pair(smem_u32(&drain_bar));
+                const unsigned long long t0 = globaltimer();
+                while (!mbar_try_wait(smem_u32(&drain_bar), 0) && globaltimer() - t0 < kWaitNs) {
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue (warps 2..5, both CTAs)
+        const int quarter = warp & 3;
+        const int row_in_tile = (int)rank * BM + quarter * 32 + lane;
+        int buf = 0;
+        uint32_t buf_phase = 0;
+        for (int tile = pair; tile < num_tiles; tile += num_pairs) {
+            int tm, tn;
+            tile_coords(tile, tiles_m, tiles_n, tm, tn);
+            const int m0 = tm * C::PM, n0 = tn * C::BN;
+            const int row = m0 + row_in_tile;
+            const float sxr = row < M ? sx[row] : 0.0f;
+            const bool ok = wait_bounded(smem_u32(&tfull_bar[buf]), buf_phase, &abort_flag, kFaultEpilogue);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * C::BN);
+            epilogue_tile<OutT>(tbase, row, M, n0, N, sxr, sw, y, acc_out, C::BN);
+            tc_fence_before();
+            mbar_arrive_leader(smem_u32(&tempty_bar[buf]));
+            buf ^= 1;
+            if (buf == 0) buf_phase ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();  // the pair is done with TMEM and with each other's barriers
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    }
+}
+
 // One CTA waits, with the same bounded wait the GEMM uses, on an mbarrier
 // that nothing ever arrives at: the wait must run out, record
 // kFaultSelftest and return, leaving the context usable.
@@ -512,6 +821,28 @@ static sq_status launch(const int8_t *qx, const float *sx, const int8_t *qw, con
     return launch_status("w8a8_gemm_kernel");
 }
 
+template <typename OutT>
+static sq_status launch_pair(const int8_t *qx, const float *sx, const int8_t *qw, const float *sw, int M, int N,
+                             int K, void *y, int32_t *acc_out, int sms, cudaStream_t st) {
+    using C = Cfg2;
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, qx, M, K, BM) || !make_map(&mb, qw, N, K, C::BN / 2))
+        return fail(SQ_ERR_CUDA, "w8a8_gemm_dequant: cuTensorMapEncodeTiled failed");
+    auto kern = w8a8_gemm_pair_kernel<OutT>;
+    static int configured_dev[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !configured_dev[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e != cudaSuccess) return fail(SQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        configured_dev[dev] = 1;
+    }
+    const int tiles = ((M + C::PM - 1) / C::PM) * ((N + C::BN - 1) / C::BN);
+    const int pairs = std::min(tiles, sms / 2);
+    kern<<<2 * pairs, kThreads, C::SMEM, st>>>(ma, mb, sx, sw, (OutT *)y, acc_out, M, N, K);
+    return launch_status("w8a8_gemm_pair_kernel");
+}
+
 }  // namespace gemm
 }  // namespace w8a8
 
@@ -539,6 +870,12 @@ extern "C" sq_status w8a8_gemm_dequant(const int8_t *qx, const float *sx, const 
     sq_status st = check_device(&sms);
     if (st != SQ_OK) return st;
     cudaStream_t cs = (cudaStream_t)stream;
+    // M > 128: 256-row tiles on CTA pairs; otherwise one CTA per 128 x 256 tile
+    if (M > gemm::BM) {
+        if (yt == SQ_BF16)
+            return gemm::launch_pair<__nv_bfloat16>(qx, sx, qw, sw, (int)M, (int)N, (int)K, y, acc_out, sms, cs);
+        return gemm::launch_pair<float>(qx, sx, qw, sw, (int)M, (int)N, (int)K, y, acc_out, sms, cs);
+    }
     if (yt == SQ_BF16)
         return gemm::launch<256, __nv_bfloat16>(qx, sx, qw, sw, (int)M, (int)N, (int)K, y, acc_out, sms, cs);
     return gemm::launch<256, float>(qx, sx, qw, sw, (int)M, (int)N, (int)K, y, acc_out, sms, cs);

@@ -130,18 +130,21 @@ struct PassOut {
     bool moved;
 };
 
-// Codes of 8 consecutive elements at scale c (fast path) packed in 8 bytes;
-// dmax collects max |y - rint(y)| for the tie test.
+// Codes of 8 consecutive elements at scale c (fast path, see sym_code_i)
+// packed in 8 bytes, two elements per instruction: t = fma(v, r, M) and
+// d = fma(v, r, M - t).  dmax collects max |d| for the tie test.
 __device__ __forceinline__ uint2 fast_codes8(const float4 a, const float4 b, float r, float lo, float hi,
                                              float &dmax) {
-    const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    const float2 v[4] = {make_float2(a.x, a.y), make_float2(a.z, a.w), make_float2(b.x, b.y), make_float2(b.z, b.w)};
+    const float2 r2 = make_float2(r, r), m2 = make_float2(kRoundMagic, kRoundMagic);
     uint32_t t[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float y = v[i] * r;
-        const float tt = y + kRoundMagic;
-        dmax = fmaxf(dmax, fabsf(y - (tt - kRoundMagic)));
-        t[i] = __float_as_uint(fminf(fmaxf(tt, lo), hi));  // code = low byte
+    for (int i = 0; i < 4; ++i) {
+        const float2 tt = f2_fma(v[i], r2, m2);
+        const float2 d = f2_fma(v[i], r2, f2_sub(m2, tt));
+        dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
+        t[2 * i] = __float_as_uint(fminf(fmaxf(tt.x, lo), hi));  // code = low byte
+        t[2 * i + 1] = __float_as_uint(fminf(fmaxf(tt.y, lo), hi));
     }
     const uint32_t p0 = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
     const uint32_t p1 = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
@@ -211,16 +214,16 @@ __device__ __forceinline__ PassOut row_pass(const float *__restrict__ wrow, int 
     // Tie test: the fast code equals the exact one unless |y - rint(y)| is
     // within |y| 2^-21 of 0.5 (|y| <= wmax r); rare, and then the thread
     // takes the exact quotient for its near-tie elements.
-    if (dmax >= 0.5f - wmax * r * 4.76837158203125e-07f) {
+    if (dmax >= 0.5f - fmaf(wmax * r, 4.76837158203125e-07f, 2.384185791015625e-07f)) {
 #pragma unroll 1
         for (int j = threadIdx.x * 8; j < K; j += stride) {
 #pragma unroll 1
             for (int i = 0; i < 8; ++i) {
                 const float v = wrow[j + i];
-                const float y = v * r;
-                const float t = y + kRoundMagic;
-                const float d = y - (t - kRoundMagic);
-                if (fmaf(fabsf(y), 4.76837158203125e-07f, fabsf(d)) >= 0.5f) {
+                const float t = fmaf(v, r, kRoundMagic);
+                const float rq = t - kRoundMagic;
+                const float d = fmaf(v, r, -rq);
+                if (fabsf(d) + fmaf(fabsf(rq), 4.76837158203125e-07f, 2.384185791015625e-07f) >= 0.5f) {
                     const int qf = __float_as_int(fminf(fmaxf(t, lo), hi)) - kRoundMagicBits;
                     const int qe = exact_code(v, c, qmax);
                     if (qe != qf) {
