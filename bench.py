@@ -62,18 +62,22 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
-def algorithmic_work(cfg):
+def algorithmic_work_mnk(M, K, N, xb, yb, bits=8):
     """Bytes (or int8 ops) each kernel must move (or do) per launch."""
-    M, K, N = cfg.M, cfg.K, cfg.N
-    xb = 2 if cfg.in_dtype == "bf16" else 4
-    yb = 2 if cfg.out_dtype == "bf16" else 4
     return {
         "calib_absmax": {"bytes": xb * M * K + 4 * K},
         "smooth_fold": {"bytes": xb * N * K + 3 * 4 * K},
         "ssz_quant_weight": {"bytes": xb * N * K + N * K + 4 * K + 4 * N + 8 * N + 4 * N},
         "quant_act_per_token": {"bytes": xb * M * K + M * K + 4 * K + 4 * M},
-        "w8a8_gemm_dequant": {"ops": 2 * M * N * K, "bytes": M * K + N * K + 4 * M + 4 * N + yb * M * N},
+        "w8a8_gemm_dequant": ({"ops": 2 * M * N * K, "bytes": M * K + N * K + 4 * M + 4 * N + yb * M * N}
+                              if bits == 8 else {"ops": 0, "bytes": 0}),
     }
+
+
+def algorithmic_work(cfg):
+    xb = 2 if cfg.in_dtype == "bf16" else 4
+    yb = 2 if cfg.out_dtype == "bf16" else 4
+    return algorithmic_work_mnk(cfg.M, cfg.K, cfg.N, xb, yb, cfg.bits)
 
 
 KERNEL_SOURCES = {
@@ -156,62 +160,89 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ our arm
+NAMES = ["calib_absmax", "smooth_fold", "ssz_quant_weight", "quant_act_per_token", "w8a8_gemm_dequant"]
+GPT_WORKLOAD = "gpt345m_8x1024"
+
+
+class Problem:
+    """One linear layer of the workload with its device buffers."""
+
+    def __init__(self, torch, x, wt, alpha, bits, max_iters, ydt):
+        dev = x.device
+        M, K = x.shape
+        N = wt.shape[0]
+        self.x, self.wt, self.alpha, self.bits, self.max_iters = x, wt, alpha, bits, max_iters
+        self.M, self.K, self.N = M, K, N
+        f32 = dict(device=dev, dtype=torch.float32)
+        self.ax, self.aw, self.s, self.inv = (torch.empty(K, **f32) for _ in range(4))
+        self.qw = torch.empty(N, K, device=dev, dtype=torch.int8)
+        self.sw = torch.empty(N, **f32)
+        self.qx = torch.empty(M, K, device=dev, dtype=torch.int8)
+        self.sx = torch.empty(M, **f32)
+        self.y = torch.empty(M, N, device=dev, dtype=ydt)
+
+
+def make_problems(args, torch, rank, dev):
+    """The workload's linears on this rank: each replica draws its own tokens
+    (seed = rank) and the same weights."""
+    import synthetic
+    if args.workload == GPT_WORKLOAD:
+        from synthetic import gpt
+        weights = gpt.make_weights(0, dev)
+        cap = {}
+        gpt.forward(weights, gpt.make_tokens(rank), capture=cap)
+        return [Problem(torch, cap[k], weights[k], 0.5, 8, 20, torch.bfloat16) for k in sorted(cap)]
+    cfg = synthetic.CONFIGS[args.workload]
+    x_cpu, w_cpu = synthetic.make_linear(cfg, seed=0)
+    if rank > 0:
+        x_cpu, _ = synthetic.make_linear(cfg, seed=rank)
+    ydt = torch.bfloat16 if cfg.out_dtype == "bf16" else torch.float32
+    return [Problem(torch, x_cpu.to(dev), w_cpu.to(dev), cfg.alpha, cfg.bits, cfg.max_iters, ydt)]
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
 
-    import synthetic
     import w8a8_linear_layers_b200 as w
     from w8a8_linear_layers_b200 import distributed as wdist
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    cfg = synthetic.CONFIGS[args.workload]
-    M, K, N = cfg.M, cfg.K, cfg.N
-    # each replica draws its own token batch (seed = rank) and the same weight
-    x_cpu, w_cpu = synthetic.make_linear(cfg, seed=0)
-    if rank > 0:
-        x_cpu, _ = synthetic.make_linear(cfg, seed=rank)
-    x = x_cpu.to(dev)
-    wt = w_cpu.to(dev)
-    f32 = dict(device=dev, dtype=torch.float32)
-    ax, aw, s, inv = (torch.empty(K, **f32) for _ in range(4))
-    qw = torch.empty(N, K, device=dev, dtype=torch.int8)
-    sw = torch.empty(N, **f32)
-    qx = torch.empty(M, K, device=dev, dtype=torch.int8)
-    sx = torch.empty(M, **f32)
-    ydt = torch.bfloat16 if cfg.out_dtype == "bf16" else torch.float32
-    y = torch.empty(M, N, device=dev, dtype=ydt)
+    probs = make_problems(args, torch, rank, dev)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    names = ["calib_absmax", "smooth_fold", "ssz_quant_weight", "quant_act_per_token", "w8a8_gemm_dequant"]
-
-    def step(xin, evs=None):
+    def run(p, xin, wt, evs=None, base=0):
         def mark(i):
             if evs is not None:
-                evs[i].record(stream)
+                evs[base + i].record(stream)
         mark(0)
-        w.sq_calib_absmax(xin, ax)
+        w.sq_calib_absmax(xin, p.ax)
         mark(1)
-        wdist.allreduce_calibration(ax)
-        w.sq_smooth_fold(ax, wt, cfg.alpha, aw, s, inv)
+        wdist.allreduce_calibration(p.ax)
+        w.sq_smooth_fold(p.ax, wt, p.alpha, p.aw, p.s, p.inv)
         mark(2)
-        w.ssz_quant_weight(wt, s, cfg.bits, cfg.max_iters, qw, sw)
+        w.ssz_quant_weight(wt, p.s, p.bits, p.max_iters, p.qw, p.sw)
         mark(3)
-        w.quant_act_per_token(xin, inv, qx, sx)
+        w.quant_act_per_token(xin, p.inv, p.qx, p.sx)
         mark(4)
-        w.w8a8_gemm_dequant(qx, sx, qw, sw, y)
+        if p.bits == 8:
+            w.w8a8_gemm_dequant(p.qx, p.sx, p.qw, p.sw, p.y)
         mark(5)
+
+    def step(evs=None):
+        for i, p in enumerate(probs):
+            run(p, p.x, p.wt, evs, 6 * i)
 
     for _ in range(args.warmup):
         flush.zero_()
-        step(x)
+        step()
     torch.cuda.synchronize()
     if w.device_fault() != 0:
         raise RuntimeError("a kernel gave up on a bounded wait during warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6 * len(probs))] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -219,69 +250,64 @@ def run_ours(args, rank, world, local_rank):
         wall0 = time.perf_counter()
         for i in range(args.steps):
             flush.zero_()          # L2 flush, outside the timed events
-            step(x, evs[i])
+            step(evs[i])
         torch.cuda.synchronize()
         wall1 = time.perf_counter()
     if world > 1:
         dist.barrier()
-    step_ms = [e[0].elapsed_time(e[5]) for e in evs]
-    kern_ms = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, n in enumerate(names)}
+    step_ms = [sum(e[6 * j].elapsed_time(e[6 * j + 5]) for j in range(len(probs))) for e in evs]
+    kern_ms = {n: statistics.mean(sum(e[6 * j + i].elapsed_time(e[6 * j + i + 1]) for j in range(len(probs)))
+                                  for e in evs) for i, n in enumerate(NAMES)}
     total_ms = wdist.max_over_ranks(sum(step_ms), device=dev)
     if w.device_fault() != 0:
         raise RuntimeError("a kernel gave up on a bounded wait during timing")
 
-    ops_per_step = 2.0 * M * N * K
+    ops_per_step = sum(2.0 * p.M * p.N * p.K for p in probs)
     value = ops_per_step * world * args.steps / (total_ms * 1e-3) / 1e12
 
     # ---- end to end through the C ABI with host buffers
     e2e = None
     if args.e2e_steps > 0:
-        e2e = run_e2e(args, w, wdist, world, x_cpu, w_cpu, x, wt, cfg, ax, aw, s, inv, qw, sw, qx, sx, y, flush,
-                      stream)
-    return finish(args, world, cfg, names, kern_ms, total_ms, value, e2e, clk, wall1 - wall0)
+        e2e = run_e2e(args, w, wdist, torch, probs, run, flush, stream, ops_per_step, world)
+    return finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall1 - wall0)
 
 
-def run_e2e(args, w, wdist, world, x_cpu, w_cpu, x, wt, cfg, ax, aw, s, inv, qw, sw, qx, sx, y, flush, stream):
-    import torch
-    M, K, N = cfg.M, cfg.K, cfg.N
-    ydt = y.dtype
-    ops_per_step = 2.0 * M * N * K
-    xh = x_cpu.pin_memory()
-    wh = w_cpu.pin_memory()
-    yh = torch.empty(M, N, dtype=ydt).pin_memory()
-    xd = torch.empty_like(x)
-    wd = torch.empty_like(wt)
+def run_e2e(args, w, wdist, torch, probs, run, flush, stream, ops_per_step, world):
+    """Inputs copied from pinned host memory and outputs copied back every
+    step, inside the timed region."""
+    hosts = [(p.x.cpu().pin_memory(), p.wt.cpu().pin_memory(), torch.empty_like(p.y, device="cpu").pin_memory(),
+              torch.empty_like(p.x), torch.empty_like(p.wt)) for p in probs]
     e2e_ms = []
     for i in range(args.warmup + args.e2e_steps):
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        xd.copy_(xh, non_blocking=True)
-        wd.copy_(wh, non_blocking=True)
-        w.sq_calib_absmax(xd, ax)
-        wdist.allreduce_calibration(ax)
-        w.sq_smooth_fold(ax, wd, cfg.alpha, aw, s, inv)
-        w.ssz_quant_weight(wd, s, cfg.bits, cfg.max_iters, qw, sw)
-        w.quant_act_per_token(xd, inv, qx, sx)
-        w.w8a8_gemm_dequant(qx, sx, qw, sw, y)
-        yh.copy_(y, non_blocking=True)
+        for p, (xh, wh, yh, xd, wd) in zip(probs, hosts):
+            xd.copy_(xh, non_blocking=True)
+            wd.copy_(wh, non_blocking=True)
+            run(p, xd, wd)
+            yh.copy_(p.y, non_blocking=True)
         e1.record(stream)
         e1.synchronize()
         if i >= args.warmup:
             e2e_ms.append(e0.elapsed_time(e1))
-    e2e_total = wdist.max_over_ranks(sum(e2e_ms), device=x.device)
+    e2e_total = wdist.max_over_ranks(sum(e2e_ms), device=probs[0].x.device)
     e2e_value = ops_per_step * world * len(e2e_ms) / (e2e_total * 1e-3) / 1e12
-    h2d = x.numel() * x.element_size() + wt.numel() * wt.element_size()
-    d2h = y.numel() * y.element_size()
+    h2d = sum(p.x.numel() * p.x.element_size() + p.wt.numel() * p.wt.element_size() for p in probs)
+    d2h = sum(p.y.numel() * p.y.element_size() for p in probs)
     return {"value": round(e2e_value, 3), "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(e2e_total / len(e2e_ms), 4)}
 
 
-def finish(args, world, cfg, names, kern_ms, total_ms, value, e2e, clk, wall_s):
-    M, K, N = cfg.M, cfg.K, cfg.N
-    # ---- rooflines per kernel
+def finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall_s):
+    names = NAMES
+    # ---- rooflines per kernel (algorithmic work summed over the workload's linears)
     peaks, src = load_peaks()
-    work = algorithmic_work(cfg)
+    work = {n: {} for n in names}
+    for p in probs:
+        for n, v in algorithmic_work_mnk(p.M, p.K, p.N, p.x.element_size(), p.y.element_size(), p.bits).items():
+            for key, val in v.items():
+                work[n][key] = work[n].get(key, 0) + val
     kernels = {}
     for n in names:
         t_s = kern_ms[n] * 1e-3
@@ -306,6 +332,8 @@ def finish(args, world, cfg, names, kern_ms, total_ms, value, e2e, clk, wall_s):
 
     launches_per_step = {"calib_absmax": 1, "smooth_fold": 2, "ssz_quant_weight": 1, "quant_act_per_token": 1,
                          "w8a8_gemm_dequant": 1}
+    p0 = probs[0]
+    M, K, N = p0.M, p0.K, p0.N
     result = {
         "metric": "W8A8 linear INT8 TOPS (% of peak); quant/SSZ GB/s (% of HBM) on 1 B200",
         "value": round(value, 2),
@@ -317,16 +345,16 @@ def finish(args, world, cfg, names, kern_ms, total_ms, value, e2e, clk, wall_s):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "int8 codes, int32 acc, %s in/out, fp32 scales" % cfg.in_dtype,
+        "dtype": "int8 codes, int32 acc, %s in/out, fp32 scales" % ("bf16" if p0.x.element_size() == 2 else "f32"),
         "data": "synthetic (seeded LLM-shaped activations with outlier channels, N(0,std) weights)",
-        "config": {"workload": args.workload, "M_tokens_per_gpu": M, "K": K, "N": N, "alpha": cfg.alpha,
-                   "weight_bits": cfg.bits, "ssz_max_iters": cfg.max_iters,
+        "config": {"workload": args.workload, "linears": len(probs), "M_tokens_per_gpu": M, "K": K, "N": N,
+                   "alpha": p0.alpha, "weight_bits": p0.bits, "ssz_max_iters": p0.max_iters,
                    "parallelism": "dp%d (replicas; MAX all-reduce of the calibration absmax)" % world,
                    "l2": "flushed (512 MB write) before every timed step, outside the timed events"},
         "roofline": roof,
         "kernels": kernels,
         "e2e": e2e,
-        "gpu_launches": sum(launches_per_step.values()) * args.steps,
+        "gpu_launches": sum(launches_per_step.values()) * len(probs) * args.steps,
         "clocks": clk.result,
         "wall_s_timed_region": round(wall_s, 3),
     }
@@ -398,6 +426,8 @@ def run_reference(args, rank):
     import synthetic
     if rank != 0:
         return None
+    if args.workload not in synthetic.CONFIGS:
+        return {"impl": "reference", "unavailable": "the oracle arm times the single-linear workloads only"}
     cfg = synthetic.CONFIGS[args.workload]
     probe, _, _ = oracle_sample(cfg, frac=1.0 / 16)
     budget = 120.0 / max(1, args.warmup + args.steps)
@@ -503,7 +533,7 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
     try:
         res = run_ours(args, rank, world, local_rank)
-        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload != GPT_WORKLOAD:
             import synthetic
             total, parts, sample = oracle_sample(synthetic.CONFIGS[args.workload], frac=1.0)
             cfg = synthetic.CONFIGS[args.workload]
