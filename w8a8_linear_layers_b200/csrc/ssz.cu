@@ -176,15 +176,20 @@ __device__ __forceinline__ PassOut row_pass(const float *__restrict__ wrow, int 
     const int stride = T_ * 8;
     const float r = __fdiv_rn(1.0f, c);  // c >= 1e-5, so r is finite
     const float lo = kRoundMagic - qmax, hi = kRoundMagic + qmax;
+    // Tie bound: a fast code can differ from the exact one only where |d|
+    // comes within |y| 2^-21 + 2^-22 of 0.5, and |y| <= wmax r.
+    const float tie_bound = 0.5f - fmaf(wmax * r, 4.76837158203125e-07f, 2.384185791015625e-07f);
     PassOut out = {{0.0, 0.0}, {0.0, 0.0}, 0, false};
-    float dmax = 0.0f;
     uint32_t moved = 0u;  // bit m: chunk m of this thread moved (at most 32 chunks per thread)
+    uint32_t tie = 0u;    // bit m: chunk m holds an element near a rounding tie
     int m = 0;
 #pragma unroll 2
     for (int j = threadIdx.x * 8; j < K; j += stride, ++m) {
         const float4 a = *reinterpret_cast<const float4 *>(wrow + j);
         const float4 b = *reinterpret_cast<const float4 *>(wrow + j + 4);
+        float dmax = 0.0f;
         const uint2 nw = fast_codes8(a, b, r, lo, hi, dmax);
+        if (dmax >= tie_bound) tie |= 1u << m;
         *reinterpret_cast<uint2 *>(qc + j) = nw;
         if (INIT) {
             const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
@@ -211,27 +216,27 @@ __device__ __forceinline__ PassOut row_pass(const float *__restrict__ wrow, int 
                         out);
         }
     }
-    // Tie test: the fast code equals the exact one unless |y - rint(y)| is
-    // within |y| 2^-21 of 0.5 (|y| <= wmax r); rare, and then the thread
-    // takes the exact quotient for its near-tie elements.
-    if (dmax >= 0.5f - fmaf(wmax * r, 4.76837158203125e-07f, 2.384185791015625e-07f)) {
+    // Near-tie chunks (rare): the exact quotient decides their flagged
+    // elements.  Visiting only the flagged chunks keeps the warp's detour
+    // short when one lane has a near tie.
+    while (tie) {
+        const int mm = __ffs(tie) - 1;
+        tie &= tie - 1u;
+        const int j = threadIdx.x * 8 + mm * stride;
 #pragma unroll 1
-        for (int j = threadIdx.x * 8; j < K; j += stride) {
-#pragma unroll 1
-            for (int i = 0; i < 8; ++i) {
-                const float v = wrow[j + i];
-                const float t = fmaf(v, r, kRoundMagic);
-                const float rq = t - kRoundMagic;
-                const float d = fmaf(v, r, -rq);
-                if (fabsf(d) + fmaf(fabsf(rq), 4.76837158203125e-07f, 2.384185791015625e-07f) >= 0.5f) {
-                    const int qf = __float_as_int(fminf(fmaxf(t, lo), hi)) - kRoundMagicBits;
-                    const int qe = exact_code(v, c, qmax);
-                    if (qe != qf) {
-                        qc[j + i] = (int8_t)qe;
-                        out.den += qe * qe - qf * qf;
-                        dd_acc(out.num, (double)v * code_to_f64(qe - qf));
-                        out.moved = true;
-                    }
+        for (int i = 0; i < 8; ++i) {
+            const float v = wrow[j + i];
+            const float t = fmaf(v, r, kRoundMagic);
+            const float rq = t - kRoundMagic;
+            const float d = fmaf(v, r, -rq);
+            if (fabsf(d) + fmaf(fabsf(rq), 4.76837158203125e-07f, 2.384185791015625e-07f) >= 0.5f) {
+                const int qf = __float_as_int(fminf(fmaxf(t, lo), hi)) - kRoundMagicBits;
+                const int qe = exact_code(v, c, qmax);
+                if (qe != qf) {
+                    qc[j + i] = (int8_t)qe;
+                    out.den += qe * qe - qf * qf;
+                    dd_acc(out.num, (double)v * code_to_f64(qe - qf));
+                    out.moved = true;
                 }
             }
         }
