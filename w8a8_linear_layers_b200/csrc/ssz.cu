@@ -130,11 +130,27 @@ struct PassOut {
     bool moved;
 };
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t clamp_s16x2(uint32_t w, uint32_t lo2, uint32_t hi2) {
+    asm("max.s16x2 %0, %0, %1;" : "+r"(w) : "r"(lo2));
+    asm("min.s16x2 %0, %0, %1;" : "+r"(w) : "r"(hi2));
+    return w;
+}
+
 // Codes of 8 consecutive elements at scale c (fast path, see sym_code_i)
 // packed in 8 bytes, two elements per instruction: t = fma(v, r, M) and
 // d = fma(v, r, M - t).  dmax collects max |d| for the tie test.
+// NARROW (every |v r| < 2^14): bits(t) - bits(M) is the code, so the low
+// halves of bits(t) are the codes as int16 and are clamped two at a time;
+// otherwise t is clamped as a float (|v r| may leave the integer range of M).
+template <bool NARROW>
 __device__ __forceinline__ uint2 fast_codes8(const float4 a, const float4 b, float r, float lo, float hi,
-                                             float &dmax) {
+                                             uint32_t lo2, uint32_t hi2, float &dmax) {
     const float2 v[4] = {make_float2(a.x, a.y), make_float2(a.z, a.w), make_float2(b.x, b.y), make_float2(b.z, b.w)};
     const float2 r2 = make_float2(r, r), m2 = make_float2(kRoundMagic, kRoundMagic);
     uint32_t t[8];
@@ -142,9 +158,15 @@ __device__ __forceinline__ uint2 fast_codes8(const float4 a, const float4 b, flo
     for (int i = 0; i < 4; ++i) {
         const float2 tt = f2_fma(v[i], r2, m2);
         const float2 d = f2_fma(v[i], r2, f2_sub(m2, tt));
-        dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
-        t[2 * i] = __float_as_uint(fminf(fmaxf(tt.x, lo), hi));  // code = low byte
-        t[2 * i + 1] = __float_as_uint(fminf(fmaxf(tt.y, lo), hi));
+        dmax = fmax3(dmax, fabsf(d.x), fabsf(d.y));
+        t[2 * i] = __float_as_uint(NARROW ? tt.x : fminf(fmaxf(tt.x, lo), hi));  // code = low byte
+        t[2 * i + 1] = __float_as_uint(NARROW ? tt.y : fminf(fmaxf(tt.y, lo), hi));
+    }
+    if (NARROW) {
+        uint32_t h[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) h[i] = clamp_s16x2(__byte_perm(t[2 * i], t[2 * i + 1], 0x5410), lo2, hi2);
+        return make_uint2(__byte_perm(h[0], h[1], 0x6420), __byte_perm(h[2], h[3], 0x6420));
     }
     const uint32_t p0 = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
     const uint32_t p1 = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
@@ -169,26 +191,19 @@ __device__ __forceinline__ void chunk_delta(const float *__restrict__ wc, uint2 
 // loop only marks moved chunks (a warp would otherwise run the update path
 // whenever any lane had a moved chunk), which are then visited once.
 // wmax is the thread's max |w|, for the tie bound.
-template <bool INIT>
-__device__ __forceinline__ PassOut row_pass(const float *__restrict__ wrow, int K, float c, float qmax, float wmax,
-                                            const int8_t *__restrict__ qk, int8_t *__restrict__ qc) {
-    const int T_ = blockDim.x;
-    const int stride = T_ * 8;
-    const float r = __fdiv_rn(1.0f, c);  // c >= 1e-5, so r is finite
-    const float lo = kRoundMagic - qmax, hi = kRoundMagic + qmax;
-    // Tie bound: a fast code can differ from the exact one only where |d|
-    // comes within |y| 2^-21 + 2^-22 of 0.5, and |y| <= wmax r.
-    const float tie_bound = 0.5f - fmaf(wmax * r, 4.76837158203125e-07f, 2.384185791015625e-07f);
-    PassOut out = {{0.0, 0.0}, {0.0, 0.0}, 0, false};
-    uint32_t moved = 0u;  // bit m: chunk m of this thread moved (at most 32 chunks per thread)
-    uint32_t tie = 0u;    // bit m: chunk m holds an element near a rounding tie
+template <bool INIT, bool NARROW>
+__device__ __forceinline__ void pass_chunks(const float *__restrict__ wrow, int K, float r, float lo, float hi,
+                                            uint32_t lo2, uint32_t hi2, float tie_bound,
+                                            const int8_t *__restrict__ qk, int8_t *__restrict__ qc, PassOut &out,
+                                            uint32_t &moved, uint32_t &tie) {
+    const int stride = blockDim.x * 8;
     int m = 0;
 #pragma unroll 2
     for (int j = threadIdx.x * 8; j < K; j += stride, ++m) {
         const float4 a = *reinterpret_cast<const float4 *>(wrow + j);
         const float4 b = *reinterpret_cast<const float4 *>(wrow + j + 4);
         float dmax = 0.0f;
-        const uint2 nw = fast_codes8(a, b, r, lo, hi, dmax);
+        const uint2 nw = fast_codes8<NARROW>(a, b, r, lo, hi, lo2, hi2, dmax);
         if (dmax >= tie_bound) tie |= 1u << m;
         *reinterpret_cast<uint2 *>(qc + j) = nw;
         if (INIT) {
@@ -206,6 +221,32 @@ __device__ __forceinline__ PassOut row_pass(const float *__restrict__ wrow, int 
             if ((nw.x ^ od.x) | (nw.y ^ od.y)) moved |= 1u << m;
         }
     }
+}
+
+// One pass at scale c over this thread's chunks of the row in shared memory.
+// Writes the codes at c into qc.  init: accumulates W2, NUM, DEN.  update:
+// accumulates the change of NUM and DEN against the kept codes qk; the main
+// loop only marks moved chunks (a warp would otherwise run the update path
+// whenever any lane had a moved chunk), which are then visited once.
+// wmax is the thread's max |w|, for the tie bound.  Called by whole warps.
+template <bool INIT>
+__device__ __forceinline__ PassOut row_pass(const float *__restrict__ wrow, int K, float c, float qmax, float wmax,
+                                            const int8_t *__restrict__ qk, int8_t *__restrict__ qc) {
+    const int stride = blockDim.x * 8;
+    const float r = __fdiv_rn(1.0f, c);  // c >= 1e-5, so r is finite
+    const float lo = kRoundMagic - qmax, hi = kRoundMagic + qmax;
+    const uint32_t qm = (uint32_t)(int)qmax;
+    const uint32_t hi2 = qm | (qm << 16), lo2 = ((0x10000u - qm) & 0xffffu) * 0x10001u;
+    // Tie bound: a fast code can differ from the exact one only where |d|
+    // comes within |y| 2^-21 + 2^-22 of 0.5, and |y| <= wmax r.
+    const float tie_bound = 0.5f - fmaf(wmax * r, 4.76837158203125e-07f, 2.384185791015625e-07f);
+    PassOut out = {{0.0, 0.0}, {0.0, 0.0}, 0, false};
+    uint32_t moved = 0u;  // bit m: chunk m of this thread moved (at most 32 chunks per thread)
+    uint32_t tie = 0u;    // bit m: chunk m holds an element near a rounding tie
+    if (__all_sync(0xffffffffu, wmax * r < 16384.0f))
+        pass_chunks<INIT, true>(wrow, K, r, lo, hi, lo2, hi2, tie_bound, qk, qc, out, moved, tie);
+    else
+        pass_chunks<INIT, false>(wrow, K, r, lo, hi, lo2, hi2, tie_bound, qk, qc, out, moved, tie);
     if (!INIT) {
         out.moved = moved != 0u;
         while (moved) {
@@ -250,7 +291,7 @@ struct WarpPart {
 };
 
 template <typename T, bool FOLD>
-__global__ void __launch_bounds__(512)
+__global__ void __launch_bounds__(512, 2)
 ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__ s, float qmax, int max_iters,
            int8_t *__restrict__ q_out, float *__restrict__ scale_out, double *__restrict__ mse_out,
            int32_t *__restrict__ iters_out) {
