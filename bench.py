@@ -62,6 +62,12 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
+B200_SMS = 148
+FP32_LANES_PER_SM = 128
+NOMINAL_SM_MHZ = 1965.0
+SSZ_OPS_PER_ELEMENT_ROUND = 10  # codes, residual, clamp, compare and sums per element and round
+
+
 def algorithmic_work_mnk(M, K, N, xb, yb, bits=8):
     """Bytes (or int8 ops) each kernel must move (or do) per launch."""
     return {
@@ -177,6 +183,7 @@ class Problem:
         self.ax, self.aw, self.s, self.inv = (torch.empty(K, **f32) for _ in range(4))
         self.qw = torch.empty(N, K, device=dev, dtype=torch.int8)
         self.sw = torch.empty(N, **f32)
+        self.iters = torch.empty(N, device=dev, dtype=torch.int32)  # SSZ rounds per channel (ALU work)
         self.qx = torch.empty(M, K, device=dev, dtype=torch.int8)
         self.sx = torch.empty(M, **f32)
         self.y = torch.empty(M, N, device=dev, dtype=ydt)
@@ -223,7 +230,7 @@ def run_ours(args, rank, world, local_rank):
         wdist.allreduce_calibration(p.ax)
         w.sq_smooth_fold(p.ax, wt, p.alpha, p.aw, p.s, p.inv)
         mark(2)
-        w.ssz_quant_weight(wt, p.s, p.bits, p.max_iters, p.qw, p.sw)
+        w.ssz_quant_weight(wt, p.s, p.bits, p.max_iters, p.qw, p.sw, iters_out=p.iters)
         mark(3)
         w.quant_act_per_token(xin, p.inv, p.qx, p.sx)
         mark(4)
@@ -308,11 +315,27 @@ def finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall_s):
         for n, v in algorithmic_work_mnk(p.M, p.K, p.N, p.x.element_size(), p.y.element_size(), p.bits).items():
             for key, val in v.items():
                 work[n][key] = work[n].get(key, 0) + val
+    # SSZ is bound by its search rounds, not by HBM: ALU work = c N K (1 + iters)
+    # operations (c = 10 per element and round), against every FP32 lane of
+    # every SM at the SM clock sampled during the timed region
+    iters = sum(float(p.iters.double().sum().item()) for p in probs) / sum(p.N for p in probs)
+    ssz_ops = sum(SSZ_OPS_PER_ELEMENT_ROUND * p.N * p.K * (1.0 + float(p.iters.double().mean().item()))
+                  for p in probs)
+    sm_mhz = (clk.result or {}).get("sm_mhz") or NOMINAL_SM_MHZ
+    alu_peak = B200_SMS * FP32_LANES_PER_SM * sm_mhz * 1e6 / 1e12  # T ops/s
     kernels = {}
     for n in names:
         t_s = kern_ms[n] * 1e-3
         entry = {"us": round(kern_ms[n] * 1e3, 2)}
-        if "ops" in work[n]:
+        if n == "ssz_quant_weight":
+            ach = ssz_ops / t_s / 1e12
+            hbm = work[n]["bytes"] / t_s / 1e9
+            entry.update(bound="alu", achieved=round(ach, 2), peak=round(alu_peak, 2), unit="Tops/s",
+                         frac=round(ach / alu_peak, 4), mean_iters=round(iters, 3),
+                         hbm={"achieved": round(hbm, 1), "peak": round(peaks["hbm_gbs"], 1), "unit": "GB/s",
+                              "frac": round(hbm / peaks["hbm_gbs"], 4)})
+            work[n] = dict(work[n], ops=ssz_ops)
+        elif "ops" in work[n]:
             ach = work[n]["ops"] / t_s / 1e12
             peak = peaks["bf16_tflops"] * INT8_OVER_BF16
             entry.update(bound="tensor", achieved=round(ach, 1), peak=round(peak, 1), unit="TFLOP/s",
@@ -328,7 +351,9 @@ def finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall_s):
     dom = max(names, key=lambda n: kern_ms[n])
     roof = {k: kernels[dom][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
     roof["kernel"] = dom
-    roof["peak_source"] = "%s (%s)" % (src, "bf16 burst x2 for int8" if roof["bound"] == "tensor" else "hbm copy")
+    roof["peak_source"] = {"tensor": "%s (bf16 burst x2 for int8)" % src, "hbm": "%s (hbm copy)" % src,
+                           "alu": "derived: %d SMs x %d FP32 lanes x sampled SM clock" % (B200_SMS, FP32_LANES_PER_SM)
+                           }[roof["bound"]]
 
     launches_per_step = {"calib_absmax": 1, "smooth_fold": 2, "ssz_quant_weight": 1, "quant_act_per_token": 1,
                          "w8a8_gemm_dequant": 1}

@@ -153,4 +153,54 @@ __device__ __forceinline__ uint2 pack8_codes(const int (&q)[8]) {
     return make_uint2(lo, hi);
 }
 
+// The exact code of one element (IEEE quotient), out of line: only taken for
+// the rare elements near a rounding tie, so the division stays off the fast
+// path (inlined, the compiler may predicate it onto every element).
+static __device__ __noinline__ int exact_code(float v, float c, float qmax) {
+    return (int)fminf(fmaxf(rintf(__fdiv_rn(v, c)), -qmax), qmax);
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t clamp_s16x2(uint32_t w, uint32_t lo2, uint32_t hi2) {
+    asm("max.s16x2 %0, %0, %1;" : "+r"(w) : "r"(lo2));
+    asm("min.s16x2 %0, %0, %1;" : "+r"(w) : "r"(hi2));
+    return w;
+}
+
+// Codes of 8 consecutive elements at scale c (fast path, see sym_code_i)
+// packed in 8 bytes, two elements per instruction: t = fma(v, r, M) and
+// d = fma(v, r, M - t).  dmax collects max |d| for the tie test.
+// NARROW (every |v r| < 2^14): bits(t) - bits(M) is the code, so the low
+// halves of bits(t) are the codes as int16 and are clamped two at a time;
+// otherwise t is clamped as a float (|v r| may leave the integer range of M).
+template <bool NARROW>
+__device__ __forceinline__ uint2 fast_codes8(const float4 a, const float4 b, float r, float lo, float hi,
+                                             uint32_t lo2, uint32_t hi2, float &dmax) {
+    const float2 v[4] = {make_float2(a.x, a.y), make_float2(a.z, a.w), make_float2(b.x, b.y), make_float2(b.z, b.w)};
+    const float2 r2 = make_float2(r, r), m2 = make_float2(kRoundMagic, kRoundMagic);
+    uint32_t t[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 tt = f2_fma(v[i], r2, m2);
+        const float2 d = f2_fma(v[i], r2, f2_sub(m2, tt));
+        dmax = fmax3(dmax, fabsf(d.x), fabsf(d.y));
+        t[2 * i] = __float_as_uint(NARROW ? tt.x : fminf(fmaxf(tt.x, lo), hi));  // code = low byte
+        t[2 * i + 1] = __float_as_uint(NARROW ? tt.y : fminf(fmaxf(tt.y, lo), hi));
+    }
+    if (NARROW) {
+        uint32_t h[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) h[i] = clamp_s16x2(__byte_perm(t[2 * i], t[2 * i + 1], 0x5410), lo2, hi2);
+        return make_uint2(__byte_perm(h[0], h[1], 0x6420), __byte_perm(h[2], h[3], 0x6420));
+    }
+    const uint32_t p0 = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
+    const uint32_t p1 = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
+    return make_uint2(p0, p1);
+}
+
 }  // namespace w8a8

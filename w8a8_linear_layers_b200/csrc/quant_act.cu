@@ -7,23 +7,88 @@
 // ("SmoothQuant大模型量化技术深度解析", section 1: activations divided by s)
 // is applied on the fly as x * inv_s.
 //
-// Design: one CTA per token row (grid-stride), the row held in registers
-// between its two uses (absmax, then codes), so X is read from HBM once and
-// the codes written once: 2 (bf16) + 1 bytes per element.  Each thread owns
-// E/8 chunks of 8 consecutive columns; chunk c of thread t starts at column
-// (c * T + t) * 8, so a warp's loads are 512 contiguous bytes (bf16).
+// Design: one small CTA per token row (grid-stride), the row held in
+// registers between its two uses (absmax, then codes), so X is read from HBM
+// once and the codes written once: 2 (bf16) + 1 bytes per element.  Each
+// thread owns E/8 chunks of 8 consecutive columns; chunk c of thread t starts
+// at column (c * T + t) * 8, so a warp's loads are 512 contiguous bytes
+// (bf16).  Codes come 8 at a time from the packed fast path (fast_codes8);
+// only chunks with an element near a rounding tie take the exact quotient.
 #include "common.cuh"
 
 namespace w8a8 {
 
-template <typename T, int E>
+// 8 consecutive elements as loaded (16 bytes of bf16 or 32 bytes of fp32),
+// widened to fp32 only where used, so a CTA can keep several rows in flight.
+template <typename T> struct Raw8;
+template <> struct Raw8<__nv_bfloat16> {
+    uint4 u;
+    __device__ __forceinline__ void load(const __nv_bfloat16 *p) { u = __ldg(reinterpret_cast<const uint4 *>(p)); }
+    __device__ __forceinline__ void zero() { u = make_uint4(0u, 0u, 0u, 0u); }
+    __device__ __forceinline__ void widen(float (&v)[8]) const {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[2 * i] = __uint_as_float(w[i] << 16);
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+};
+template <> struct Raw8<float> {
+    float4 a, b;
+    __device__ __forceinline__ void load(const float *p) {
+        a = __ldg(reinterpret_cast<const float4 *>(p));
+        b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+    }
+    __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+    __device__ __forceinline__ void widen(float (&v)[8]) const {
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+};
+
+// Clamp bounds of the int8 codes: t in [M - 127, M + 127]; int16 pairs in
+// [-127, 127].
+constexpr float kLo = kRoundMagic - 127.0f, kHi = kRoundMagic + 127.0f;
+constexpr uint32_t kLo2 = 0xFF81FF81u, kHi2 = 0x007F007Fu;
+
+// Codes of 8 scaled elements at scale s (r = 1/s): packed fast path, then
+// the exact quotient for any element near a rounding tie (rare).
+__device__ __forceinline__ uint2 fast_codes_tied(const float (&v)[8], float s, float r, bool narrow,
+                                                 float tie_bound) {
+    const float4 a = make_float4(v[0], v[1], v[2], v[3]), b = make_float4(v[4], v[5], v[6], v[7]);
+    float dmax = 0.0f;
+    uint2 code = narrow ? fast_codes8<true>(a, b, r, kLo, kHi, kLo2, kHi2, dmax)
+                        : fast_codes8<false>(a, b, r, kLo, kHi, kLo2, kHi2, dmax);
+    if (dmax >= tie_bound) {
+#pragma unroll  // unrolled: v stays in registers
+        for (int i = 0; i < 8; ++i) {
+            const float t = fmaf(v[i], r, kRoundMagic);
+            const float rq = t - kRoundMagic;
+            const float d = fmaf(v[i], r, -rq);
+            if (fabsf(d) + fmaf(fabsf(rq), 4.76837158203125e-07f, 2.384185791015625e-07f) >= 0.5f) {
+                const uint32_t qe = (uint32_t)exact_code(v[i], s, 127.0f) & 0xffu;
+                const int sh = 8 * (i & 3);
+                uint32_t &w = i < 4 ? code.x : code.y;
+                w = (w & ~(0xffu << sh)) | (qe << sh);
+            }
+        }
+    }
+    return code;
+}
+
+// ROWS token rows per CTA iteration, all loaded before the first reduction.
+// Measured on B200: one row per CTA of one or two warps (E = 32 or 64) with
+// many CTAs per SM beats several rows per larger CTA and beats staging rows
+// in shared memory with bulk copies.
+template <typename T, int E, int ROWS>
 __global__ void __launch_bounds__(512)
 quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__restrict__ inv_s,
                  int8_t *__restrict__ q, float *__restrict__ scale) {
     constexpr int C = E / 8;  // chunks per thread
-    // inv_s is kept in registers across rows unless that would spill (E = 64)
-    constexpr bool kCacheInvS = C <= 4;
-    __shared__ float red[2][32];
+    // inv_s is kept in registers across rows unless that would spill
+    constexpr bool kCacheInvS = C * ROWS <= 4;
+    __shared__ float red[2][ROWS][32];
     const int T_ = blockDim.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = T_ >> 5;
 
@@ -42,66 +107,90 @@ quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__r
             }
         }
     }
+    // x * inv_s of chunk c (inv_s from registers or from L1)
+    auto scaled = [&](const Raw8<T> &raw, int c, float (&v)[8]) {
+        raw.widen(v);
+        if (inv_s) {
+            if (!kCacheInvS) load8_f32(inv_s + ((int64_t)c * T_ + threadIdx.x) * 8, f[0]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = v[i] * f[kCacheInvS ? c : 0][i];
+        }
+    };
 
     int parity = 0;
-    for (int64_t row = blockIdx.x; row < M; row += gridDim.x, parity ^= 1) {
-        const T *xr = x + row * K;
-        float v[C][8];
-        float amax = 0.0f;
+    for (int64_t row0 = (int64_t)blockIdx.x * ROWS; row0 < M; row0 += (int64_t)gridDim.x * ROWS, parity ^= 1) {
+        Raw8<T> raw[ROWS][C];
 #pragma unroll
-        for (int c = 0; c < C; ++c) {
-            if (live[c]) {
-                Vec8<T>::load(xr + ((int64_t)c * T_ + threadIdx.x) * 8, v[c]);
-                if (inv_s) {
-                    if (!kCacheInvS) load8_f32(inv_s + ((int64_t)c * T_ + threadIdx.x) * 8, f[0]);
+        for (int rr = 0; rr < ROWS; ++rr) {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) v[c][i] = v[c][i] * f[kCacheInvS ? c : 0][i];
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) v[c][i] = 0.0f;
+            for (int c = 0; c < C; ++c) {
+                if (live[c] && row0 + rr < M)
+                    raw[rr][c].load(x + (row0 + rr) * K + ((int64_t)c * T_ + threadIdx.x) * 8);
+                else
+                    raw[rr][c].zero();
             }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[c][i]));
         }
-        amax = warp_max(amax);
-        if (lane == 0) red[parity][warp] = amax;
-        __syncthreads();  // red[parity] complete; red[parity^1] free for the next row
-        amax = red[parity][0];
-        for (int w = 1; w < nwarps; ++w) amax = fmaxf(amax, red[parity][w]);
-
-        const float s = __fdiv_rn(amax, 127.0f);
-        if (threadIdx.x == 0) scale[row] = s;
-        const float r = __fdiv_rn(1.0f, s);
-        const bool exact_only = !(fabsf(r) <= 3.402823466e38f);  // 1/s overflowed (or s == 0)
-        int8_t *qr = q + row * K;
+        float amax[ROWS];
 #pragma unroll
-        for (int c = 0; c < C; ++c) {
-            if (!live[c]) continue;
-            int code[8];
-            if (s == 0.0f) {
+        for (int rr = 0; rr < ROWS; ++rr) {
+            amax[rr] = 0.0f;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) code[i] = 0;
-            } else if (exact_only) {
+            for (int c = 0; c < C; ++c) {
+                float v[8];
+                scaled(raw[rr][c], c, v);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) code[i] = (int)sym_code(v[c][i], s, r, 127.0f, true);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) code[i] = sym_code_i(v[c][i], s, r, 127.0f);
+                for (int i = 0; i < 8; ++i) amax[rr] = fmaxf(amax[rr], fabsf(v[i]));
             }
-            *reinterpret_cast<uint2 *>(qr + ((int64_t)c * T_ + threadIdx.x) * 8) = pack8_codes(code);
+            amax[rr] = warp_max(amax[rr]);
+            if (lane == 0) red[parity][rr][warp] = amax[rr];
+        }
+        __syncthreads();  // red[parity] complete; red[parity^1] free for the next rows
+#pragma unroll
+        for (int rr = 0; rr < ROWS; ++rr) {
+            const int64_t row = row0 + rr;
+            if (row >= M) break;
+            float am = red[parity][rr][0];
+            for (int w = 1; w < nwarps; ++w) am = fmaxf(am, red[parity][rr][w]);
+            const float s = __fdiv_rn(am, 127.0f);
+            if (threadIdx.x == 0) scale[row] = s;
+            const float r = __fdiv_rn(1.0f, s);
+            const bool exact_only = !(fabsf(r) <= 3.402823466e38f);  // 1/s overflowed (or s == 0)
+            // |v r| <= am r (about 127): the int16 clamp of fast_codes8 applies;
+            // a fast code can differ from the exact one only where |d| comes
+            // within |y| 2^-21 + 2^-22 of 0.5
+            const bool narrow = am * r < 16384.0f;
+            const float tie_bound = 0.5f - fmaf(am * r, 4.76837158203125e-07f, 2.384185791015625e-07f);
+            int8_t *qr = q + row * K;
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                if (!live[c]) continue;
+                float v[8];
+                scaled(raw[rr][c], c, v);
+                uint2 code = make_uint2(0u, 0u);
+                if (s == 0.0f) {
+                    // all-zero row: every code is 0
+                } else if (exact_only) {
+                    int e[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) e[i] = (int)sym_code(v[i], s, r, 127.0f, true);
+                    code = pack8_codes(e);
+                } else {
+                    code = fast_codes_tied(v, s, r, narrow, tie_bound);
+                }
+                *reinterpret_cast<uint2 *>(qr + ((int64_t)c * T_ + threadIdx.x) * 8) = code;
+            }
         }
     }
 }
 
-template <typename T, int E>
+template <typename T, int E, int ROWS>
 static void launch_quant_act(const void *x, int64_t M, int64_t K, const float *inv_s, int8_t *q,
                              float *scale, int sms, cudaStream_t st) {
     int threads = (int)ceil_div(ceil_div(K, E), 32) * 32;
-    // enough CTAs to fill the machine; each strides over rows
-    int per_sm = std::max(1, 2048 / threads);
-    int64_t grid = std::min<int64_t>(M, (int64_t)sms * per_sm);
-    quant_act_kernel<T, E><<<(unsigned)grid, threads, 0, st>>>((const T *)x, M, K, inv_s, q, scale);
+    // enough CTAs to fill the machine; each strides over groups of ROWS rows
+    int per_sm = std::max(1, std::min(32, 2048 / threads));
+    int64_t grid = std::min<int64_t>(ceil_div(M, ROWS), (int64_t)sms * per_sm);
+    quant_act_kernel<T, E, ROWS><<<(unsigned)grid, threads, 0, st>>>((const T *)x, M, K, inv_s, q, scale);
 }
 
 }  // namespace w8a8
@@ -123,20 +212,22 @@ extern "C" sq_status quant_act_per_token(const void *x, sq_dtype xt, int64_t M, 
     sq_status st = check_device(&sms);
     if (st != SQ_OK) return st;
     cudaStream_t cs = (cudaStream_t)stream;
-    // elements per thread: at most 512 threads per row
     const bool bf = xt == SQ_BF16;
-    if (K <= 2048) {
-        if (bf) launch_quant_act<__nv_bfloat16, 8>(x, M, K, inv_s, q_out, scale_out, sms, cs);
-        else launch_quant_act<float, 8>(x, M, K, inv_s, q_out, scale_out, sms, cs);
-    } else if (K <= 8192) {
-        if (bf) launch_quant_act<__nv_bfloat16, 16>(x, M, K, inv_s, q_out, scale_out, sms, cs);
-        else launch_quant_act<float, 16>(x, M, K, inv_s, q_out, scale_out, sms, cs);
-    } else if (K <= 16384) {
-        if (bf) launch_quant_act<__nv_bfloat16, 32>(x, M, K, inv_s, q_out, scale_out, sms, cs);
-        else launch_quant_act<float, 32>(x, M, K, inv_s, q_out, scale_out, sms, cs);
+    // E elements per thread: one warp per row up to K = 32 E, at most 64
+    // elements per thread
+    if (K <= 256) {
+        if (bf) launch_quant_act<__nv_bfloat16, 8, 1>(x, M, K, inv_s, q_out, scale_out, sms, cs);
+        else launch_quant_act<float, 8, 1>(x, M, K, inv_s, q_out, scale_out, sms, cs);
+    } else if (K <= 512) {
+        if (bf) launch_quant_act<__nv_bfloat16, 16, 1>(x, M, K, inv_s, q_out, scale_out, sms, cs);
+        else launch_quant_act<float, 16, 1>(x, M, K, inv_s, q_out, scale_out, sms, cs);
+    } else if (K <= 1024) {
+        if (bf) launch_quant_act<__nv_bfloat16, 32, 1>(x, M, K, inv_s, q_out, scale_out, sms, cs);
+        else launch_quant_act<float, 32, 1>(x, M, K, inv_s, q_out, scale_out, sms, cs);
+    } else if (bf) {
+        launch_quant_act<__nv_bfloat16, 64, 1>(x, M, K, inv_s, q_out, scale_out, sms, cs);
     } else {
-        if (bf) launch_quant_act<__nv_bfloat16, 64>(x, M, K, inv_s, q_out, scale_out, sms, cs);
-        else launch_quant_act<float, 64>(x, M, K, inv_s, q_out, scale_out, sms, cs);
+        launch_quant_act<float, 64, 1>(x, M, K, inv_s, q_out, scale_out, sms, cs);
     }
     return launch_status("quant_act_kernel");
 }

@@ -22,7 +22,9 @@
 //
 // Design.  One CTA of R warps per output channel; the folded fp32 row stays
 // resident in shared memory for the whole search (W is read from HBM once,
-// the codes written once), next to two code buffers (kept / candidate).
+// the codes written once), next to one buffer of kept codes: a candidate
+// that is not kept ends the search, so a round writes its codes over the
+// kept ones and the chunks it touched are restored in that one case.
 //
 // The error is evaluated exactly instead of by a per-element fp64 sum:
 //     K e(c) = W2 - 2 c NUM + c^2 DEN,  W2 = sum w^2, NUM = sum w q, DEN = sum q^2,
@@ -112,154 +114,98 @@ __device__ __forceinline__ float ls_candidate(dd NUM, int den, float keep) {
     return den != 0 ? fmaxf((float)((NUM.hi + NUM.lo) / (double)den), kSszMinScale) : keep;
 }
 
-// The exact code of one element (IEEE quotient), out of line: only taken for
-// the rare elements near a rounding tie.
-__device__ __noinline__ int exact_code(float v, float c, float qmax) {
-    return (int)fminf(fmaxf(rintf(__fdiv_rn(v, c)), -qmax), qmax);
-}
-
 __device__ __forceinline__ int code_byte(uint2 p, int b) {
     const uint32_t w = b < 4 ? p.x : p.y;
     return (int)(int8_t)((w >> (8 * (b & 3))) & 0xffu);
 }
 
 struct PassOut {
-    dd num;     // init: NUM; update: change of NUM
-    dd w2;      // init only
-    int den;    // init: DEN; update: change of DEN
-    bool moved;
+    dd num;          // init: NUM; update: change of NUM
+    dd w2;           // init only
+    int den;         // init: DEN; update: change of DEN
+    bool moved;      // update: some code of this thread changed
+    uint32_t touched;  // update: chunks whose codes were rewritten (moved or near a tie)
 };
 
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-    float r;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
-}
-
-__device__ __forceinline__ uint32_t clamp_s16x2(uint32_t w, uint32_t lo2, uint32_t hi2) {
-    asm("max.s16x2 %0, %0, %1;" : "+r"(w) : "r"(lo2));
-    asm("min.s16x2 %0, %0, %1;" : "+r"(w) : "r"(hi2));
-    return w;
-}
-
-// Codes of 8 consecutive elements at scale c (fast path, see sym_code_i)
-// packed in 8 bytes, two elements per instruction: t = fma(v, r, M) and
-// d = fma(v, r, M - t).  dmax collects max |d| for the tie test.
-// NARROW (every |v r| < 2^14): bits(t) - bits(M) is the code, so the low
-// halves of bits(t) are the codes as int16 and are clamped two at a time;
-// otherwise t is clamped as a float (|v r| may leave the integer range of M).
+// Fast codes of the chunk at j for scale 1/r (see fast_codes8); dmax as there.
 template <bool NARROW>
-__device__ __forceinline__ uint2 fast_codes8(const float4 a, const float4 b, float r, float lo, float hi,
+__device__ __forceinline__ uint2 chunk_codes(const float *__restrict__ wrow, int j, float r, float lo, float hi,
                                              uint32_t lo2, uint32_t hi2, float &dmax) {
-    const float2 v[4] = {make_float2(a.x, a.y), make_float2(a.z, a.w), make_float2(b.x, b.y), make_float2(b.z, b.w)};
-    const float2 r2 = make_float2(r, r), m2 = make_float2(kRoundMagic, kRoundMagic);
-    uint32_t t[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 tt = f2_fma(v[i], r2, m2);
-        const float2 d = f2_fma(v[i], r2, f2_sub(m2, tt));
-        dmax = fmax3(dmax, fabsf(d.x), fabsf(d.y));
-        t[2 * i] = __float_as_uint(NARROW ? tt.x : fminf(fmaxf(tt.x, lo), hi));  // code = low byte
-        t[2 * i + 1] = __float_as_uint(NARROW ? tt.y : fminf(fmaxf(tt.y, lo), hi));
-    }
-    if (NARROW) {
-        uint32_t h[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) h[i] = clamp_s16x2(__byte_perm(t[2 * i], t[2 * i + 1], 0x5410), lo2, hi2);
-        return make_uint2(__byte_perm(h[0], h[1], 0x6420), __byte_perm(h[2], h[3], 0x6420));
-    }
-    const uint32_t p0 = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
-    const uint32_t p1 = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
-    return make_uint2(p0, p1);
+    const float4 a = *reinterpret_cast<const float4 *>(wrow + j);
+    const float4 b = *reinterpret_cast<const float4 *>(wrow + j + 4);
+    return fast_codes8<NARROW>(a, b, r, lo, hi, lo2, hi2, dmax);
 }
 
-// Change of NUM and DEN for one chunk whose packed codes moved from od to nw.
-__device__ __forceinline__ void chunk_delta(const float *__restrict__ wc, uint2 nw, uint2 od, PassOut &out) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int qn = code_byte(nw, i), qo = code_byte(od, i);
-        if (qn != qo) {
-            out.den += qn * qn - qo * qo;
-            dd_acc(out.num, (double)wc[i] * code_to_f64(qn - qo));  // exact product
-        }
-    }
-}
-
-// One pass at scale c over this thread's chunks of the row in shared memory.
-// Writes the codes at c into qc.  init: accumulates W2, NUM, DEN.  update:
-// accumulates the change of NUM and DEN against the kept codes qk; the main
-// loop only marks moved chunks (a warp would otherwise run the update path
-// whenever any lane had a moved chunk), which are then visited once.
-// wmax is the thread's max |w|, for the tie bound.
+// Main loop of a pass over this thread's chunks.  init: writes the codes
+// into q and accumulates W2, NUM, DEN.  update: only compares the codes at
+// the candidate with the kept codes in q and marks the chunks that moved;
+// they are rewritten afterwards, once (a warp would otherwise run the update
+// path whenever any lane had a moved chunk).  Both mark near-tie chunks.
 template <bool INIT, bool NARROW>
 __device__ __forceinline__ void pass_chunks(const float *__restrict__ wrow, int K, float r, float lo, float hi,
-                                            uint32_t lo2, uint32_t hi2, float tie_bound,
-                                            const int8_t *__restrict__ qk, int8_t *__restrict__ qc, PassOut &out,
-                                            uint32_t &moved, uint32_t &tie) {
+                                            uint32_t lo2, uint32_t hi2, float tie_bound, int8_t *__restrict__ q,
+                                            PassOut &out, uint32_t &moved, uint32_t &tie) {
     const int stride = blockDim.x * 8;
     int m = 0;
 #pragma unroll 2
     for (int j = threadIdx.x * 8; j < K; j += stride, ++m) {
-        const float4 a = *reinterpret_cast<const float4 *>(wrow + j);
-        const float4 b = *reinterpret_cast<const float4 *>(wrow + j + 4);
         float dmax = 0.0f;
-        const uint2 nw = fast_codes8<NARROW>(a, b, r, lo, hi, lo2, hi2, dmax);
+        const uint2 nw = chunk_codes<NARROW>(wrow, j, r, lo, hi, lo2, hi2, dmax);
         if (dmax >= tie_bound) tie |= 1u << m;
-        *reinterpret_cast<uint2 *>(qc + j) = nw;
         if (INIT) {
+            *reinterpret_cast<uint2 *>(q + j) = nw;
+            const float4 a = *reinterpret_cast<const float4 *>(wrow + j);
+            const float4 b = *reinterpret_cast<const float4 *>(wrow + j + 4);
             const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const int q = code_byte(nw, i);
+                const int qq = code_byte(nw, i);
                 const double wd = (double)v[i];
-                dd_acc(out.w2, wd * wd);               // exact product
-                dd_acc(out.num, wd * code_to_f64(q));  // exact product
-                out.den += q * q;
+                dd_acc(out.w2, wd * wd);                // exact product
+                dd_acc(out.num, wd * code_to_f64(qq));  // exact product
+                out.den += qq * qq;
             }
         } else {
-            const uint2 od = *reinterpret_cast<const uint2 *>(qk + j);
+            const uint2 od = *reinterpret_cast<const uint2 *>(q + j);
             if ((nw.x ^ od.x) | (nw.y ^ od.y)) moved |= 1u << m;
         }
     }
 }
 
-// One pass at scale c over this thread's chunks of the row in shared memory.
-// Writes the codes at c into qc.  init: accumulates W2, NUM, DEN.  update:
-// accumulates the change of NUM and DEN against the kept codes qk; the main
-// loop only marks moved chunks (a warp would otherwise run the update path
-// whenever any lane had a moved chunk), which are then visited once.
-// wmax is the thread's max |w|, for the tie bound.  Called by whole warps.
-template <bool INIT>
-__device__ __forceinline__ PassOut row_pass(const float *__restrict__ wrow, int K, float c, float qmax, float wmax,
-                                            const int8_t *__restrict__ qk, int8_t *__restrict__ qc) {
+// Moved chunks: the change of NUM and DEN, and the new codes written over
+// the kept ones.
+template <bool NARROW>
+__device__ __forceinline__ void rewrite_moved(const float *__restrict__ wrow, uint32_t moved, float r, float lo,
+                                              float hi, uint32_t lo2, uint32_t hi2, int8_t *__restrict__ q,
+                                              PassOut &out) {
     const int stride = blockDim.x * 8;
-    const float r = __fdiv_rn(1.0f, c);  // c >= 1e-5, so r is finite
-    const float lo = kRoundMagic - qmax, hi = kRoundMagic + qmax;
-    const uint32_t qm = (uint32_t)(int)qmax;
-    const uint32_t hi2 = qm | (qm << 16), lo2 = ((0x10000u - qm) & 0xffffu) * 0x10001u;
-    // Tie bound: a fast code can differ from the exact one only where |d|
-    // comes within |y| 2^-21 + 2^-22 of 0.5, and |y| <= wmax r.
-    const float tie_bound = 0.5f - fmaf(wmax * r, 4.76837158203125e-07f, 2.384185791015625e-07f);
-    PassOut out = {{0.0, 0.0}, {0.0, 0.0}, 0, false};
-    uint32_t moved = 0u;  // bit m: chunk m of this thread moved (at most 32 chunks per thread)
-    uint32_t tie = 0u;    // bit m: chunk m holds an element near a rounding tie
-    if (__all_sync(0xffffffffu, wmax * r < 16384.0f))
-        pass_chunks<INIT, true>(wrow, K, r, lo, hi, lo2, hi2, tie_bound, qk, qc, out, moved, tie);
-    else
-        pass_chunks<INIT, false>(wrow, K, r, lo, hi, lo2, hi2, tie_bound, qk, qc, out, moved, tie);
-    if (!INIT) {
-        out.moved = moved != 0u;
-        while (moved) {
-            const int mm = __ffs(moved) - 1;
-            moved &= moved - 1u;
-            const int j = threadIdx.x * 8 + mm * stride;
-            chunk_delta(wrow + j, *reinterpret_cast<const uint2 *>(qc + j), *reinterpret_cast<const uint2 *>(qk + j),
-                        out);
+    while (moved) {
+        const int mm = __ffs(moved) - 1;
+        moved &= moved - 1u;
+        const int j = threadIdx.x * 8 + mm * stride;
+        float dmax = 0.0f;
+        const uint2 nw = chunk_codes<NARROW>(wrow, j, r, lo, hi, lo2, hi2, dmax);
+        const uint2 od = *reinterpret_cast<const uint2 *>(q + j);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int qn = code_byte(nw, i), qo = code_byte(od, i);
+            if (qn != qo) {
+                out.den += qn * qn - qo * qo;
+                dd_acc(out.num, (double)wrow[j + i] * code_to_f64(qn - qo));  // exact product
+            }
         }
+        *reinterpret_cast<uint2 *>(q + j) = nw;
     }
-    // Near-tie chunks (rare): the exact quotient decides their flagged
-    // elements.  Visiting only the flagged chunks keeps the warp's detour
-    // short when one lane has a near tie.
+}
+
+// Near-tie chunks (rare): the exact quotient decides their flagged elements,
+// whose fast codes are already in q.  With SUMS, the change of NUM and DEN
+// is accumulated.  Visiting only the flagged chunks keeps the warp's detour
+// short when one lane has a near tie.
+template <bool SUMS>
+__device__ __forceinline__ void fix_ties(const float *__restrict__ wrow, uint32_t tie, float c, float r, float qmax,
+                                         int8_t *__restrict__ q, PassOut &out) {
+    const int stride = blockDim.x * 8;
     while (tie) {
         const int mm = __ffs(tie) - 1;
         tie &= tie - 1u;
@@ -271,18 +217,88 @@ __device__ __forceinline__ PassOut row_pass(const float *__restrict__ wrow, int 
             const float rq = t - kRoundMagic;
             const float d = fmaf(v, r, -rq);
             if (fabsf(d) + fmaf(fabsf(rq), 4.76837158203125e-07f, 2.384185791015625e-07f) >= 0.5f) {
-                const int qf = __float_as_int(fminf(fmaxf(t, lo), hi)) - kRoundMagicBits;
+                const int qf = (int)q[j + i];
                 const int qe = exact_code(v, c, qmax);
                 if (qe != qf) {
-                    qc[j + i] = (int8_t)qe;
-                    out.den += qe * qe - qf * qf;
-                    dd_acc(out.num, (double)v * code_to_f64(qe - qf));
-                    out.moved = true;
+                    q[j + i] = (int8_t)qe;
+                    if (SUMS) {
+                        out.den += qe * qe - qf * qf;
+                        dd_acc(out.num, (double)v * code_to_f64(qe - qf));
+                        out.moved = true;
+                    }
                 }
             }
         }
     }
+}
+
+struct ScaleConsts {
+    float r, lo, hi, tie_bound;
+    uint32_t lo2, hi2;
+    bool narrow;
+};
+
+// Per-scale constants of a pass; narrow is warp-uniform.  Called by whole warps.
+__device__ __forceinline__ ScaleConsts scale_consts(float c, float qmax, float wmax) {
+    ScaleConsts k;
+    k.r = __fdiv_rn(1.0f, c);  // c >= 1e-5, so r is finite
+    k.lo = kRoundMagic - qmax;
+    k.hi = kRoundMagic + qmax;
+    const uint32_t qm = (uint32_t)(int)qmax;
+    k.hi2 = qm | (qm << 16);
+    k.lo2 = ((0x10000u - qm) & 0xffffu) * 0x10001u;
+    // a fast code can differ from the exact one only where |d| comes within
+    // |y| 2^-21 + 2^-22 of 0.5, and |y| <= wmax r
+    k.tie_bound = 0.5f - fmaf(wmax * k.r, 4.76837158203125e-07f, 2.384185791015625e-07f);
+    k.narrow = __all_sync(0xffffffffu, wmax * k.r < 16384.0f);
+    return k;
+}
+
+// One pass at scale c over this thread's chunks of the row in shared memory,
+// against the codes in q (one buffer).  init: q receives the codes at c and
+// W2, NUM, DEN are accumulated.  update: the codes at c are written over q
+// where they differ and the change of NUM and DEN is returned; `touched`
+// names the chunks rewritten, so that the kept codes can be restored if c
+// is rejected.  wmax is the thread's max |w|.  Called by whole warps.
+template <bool INIT>
+__device__ __forceinline__ PassOut row_pass(const float *__restrict__ wrow, int K, float c, float qmax, float wmax,
+                                            int8_t *__restrict__ q) {
+    const ScaleConsts k = scale_consts(c, qmax, wmax);
+    PassOut out = {{0.0, 0.0}, {0.0, 0.0}, 0, false, 0u};
+    uint32_t moved = 0u;  // bit m: chunk m of this thread moved (at most 32 chunks per thread)
+    uint32_t tie = 0u;    // bit m: chunk m holds an element near a rounding tie
+    if (k.narrow)
+        pass_chunks<INIT, true>(wrow, K, k.r, k.lo, k.hi, k.lo2, k.hi2, k.tie_bound, q, out, moved, tie);
+    else
+        pass_chunks<INIT, false>(wrow, K, k.r, k.lo, k.hi, k.lo2, k.hi2, k.tie_bound, q, out, moved, tie);
+    if (!INIT) {
+        out.moved = moved != 0u;
+        out.touched = moved | tie;
+        if (k.narrow) rewrite_moved<true>(wrow, moved, k.r, k.lo, k.hi, k.lo2, k.hi2, q, out);
+        else rewrite_moved<false>(wrow, moved, k.r, k.lo, k.hi, k.lo2, k.hi2, q, out);
+    }
+    fix_ties<true>(wrow, tie, c, k.r, qmax, q, out);
     return out;
+}
+
+// Writes the exact codes at scale c over the chunks named in `touched`.
+__device__ __forceinline__ void restore_chunks(const float *__restrict__ wrow, uint32_t touched, float c,
+                                               float qmax, float wmax, int8_t *__restrict__ q) {
+    const ScaleConsts k = scale_consts(c, qmax, wmax);
+    const int stride = blockDim.x * 8;
+    uint32_t tie = 0u;
+    for (uint32_t t = touched; t;) {
+        const int mm = __ffs(t) - 1;
+        t &= t - 1u;
+        const int j = threadIdx.x * 8 + mm * stride;
+        float dmax = 0.0f;
+        const uint2 nw = k.narrow ? chunk_codes<true>(wrow, j, k.r, k.lo, k.hi, k.lo2, k.hi2, dmax)
+                                  : chunk_codes<false>(wrow, j, k.r, k.lo, k.hi, k.lo2, k.hi2, dmax);
+        if (dmax >= k.tie_bound) tie |= 1u << mm;
+        *reinterpret_cast<uint2 *>(q + j) = nw;
+    }
+    PassOut unused;
+    fix_ties<false>(wrow, tie, c, k.r, qmax, q, unused);
 }
 
 struct WarpPart {
@@ -297,7 +313,7 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
            int32_t *__restrict__ iters_out) {
     extern __shared__ __align__(16) uint8_t smem[];
     float *wrow = reinterpret_cast<float *>(smem);            // K floats: the folded row
-    int8_t *qbuf = reinterpret_cast<int8_t *>(wrow + K);      // 2 x K codes: kept / candidate
+    int8_t *q = reinterpret_cast<int8_t *>(wrow + K);         // K codes: the kept codes
     __shared__ WarpPart part[2][16];                          // per-warp partials, by round parity
     __shared__ float redmax[16];
     const int T_ = blockDim.x;
@@ -331,12 +347,11 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
         amax = redmax[0];
         for (int i = 1; i < nwarps; ++i) amax = fmaxf(amax, redmax[i]);
 
-        // ---- MinMax init: codes into buffer 0, exact W2 / NUM / DEN
-        int8_t *qk = qbuf, *qc = qbuf + K;
+        // ---- MinMax init: codes into q, exact W2 / NUM / DEN
         float s_best = fmaxf(__fdiv_rn(amax, qmax), kSszMinScale);
         int par = 0;
         {
-            PassOut p = row_pass<true>(wrow, K, s_best, qmax, wmax, nullptr, qk);
+            PassOut p = row_pass<true>(wrow, K, s_best, qmax, wmax, q);
             p.num = warp_sum_dd(p.num);
             p.w2 = warp_sum_dd(p.w2);
             p.den = warp_sum_i(p.den);
@@ -355,11 +370,17 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
         float c = ls_candidate(NUM, DEN, s_best);
         int it = 0;
         bool done = max_iters == 0;
+        uint32_t touched = 0u;  // this thread's chunks rewritten by the last round
+        bool rejected = false;  // the last round's candidate was not kept
 
-        // ---- least-squares rounds
+        // ---- least-squares rounds.  A round whose candidate is not kept
+        // ends the search (its improvement is <= 0, below both thresholds),
+        // so the candidate's codes can be written over the kept ones and the
+        // touched chunks restored in that one case.
         while (!done) {
             par ^= 1;
-            PassOut p = row_pass<false>(wrow, K, c, qmax, wmax, qk, qc);
+            PassOut p = row_pass<false>(wrow, K, c, qmax, wmax, q);
+            touched = p.touched;
             if (__any_sync(0xffffffffu, p.moved)) {
                 p.num = warp_sum_dd(p.num);
                 p.den = warp_sum_i(p.den);
@@ -382,22 +403,23 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
             const double delta = m_best - m_c;
             done = (m_best == 0.0) || (delta < kSszThreshold * m_best) || (fabs(delta) < thr_k) ||
                    it == max_iters;
-            if (m_c < m_best) {  // keep c: its codes become the kept codes
+            if (m_c < m_best) {  // keep c: its codes are now the kept codes
                 s_best = c;
                 m_best = m_c;
                 NUM = num_c;
                 DEN = den_c;
-                int8_t *t = qk;
-                qk = qc;
-                qc = t;
                 c = c_next;
+            } else {
+                rejected = true;
+                done = true;  // implied by the tests above (m_best >= 0); stated for the restore below
             }
             // part[par] is rewritten two rounds from now, after another barrier
         }
+        if (rejected) restore_chunks(wrow, touched, s_best, qmax, wmax, q);
 
         // ---- kept codes out (each thread wrote and now reads its own chunks)
         for (int j = threadIdx.x * 8; j < K; j += T_ * 8)
-            *reinterpret_cast<uint2 *>(q_out + n * K + j) = *reinterpret_cast<const uint2 *>(qk + j);
+            *reinterpret_cast<uint2 *>(q_out + n * K + j) = *reinterpret_cast<const uint2 *>(q + j);
         if (threadIdx.x == 0) {
             scale_out[n] = s_best;
             if (mse_out) mse_out[n] = m_best / kd;
@@ -425,7 +447,7 @@ static sq_status launch_ssz(const void *w, int64_t N, int64_t K, const float *s,
                             int8_t *q, float *scale, double *mse, int32_t *iters, int sms, cudaStream_t st) {
     const int threads = 32 * ssz_warps(K);
     const float qmax = (float)((1 << (bits - 1)) - 1);
-    const size_t smem = 6 * (size_t)K;  // fp32 row + kept + candidate codes
+    const size_t smem = 5 * (size_t)K;  // fp32 row + codes
     auto kern = s ? ssz_kernel<T, true> : ssz_kernel<T, false>;
     if (smem > 32 * 1024) {  // dynamic + static shared memory may pass the 48 KB default
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
