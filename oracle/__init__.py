@@ -78,6 +78,9 @@ def _L():
             "oracle_quant_act_per_token": [P, I64, I64, P, P, P],
             "oracle_gemm_i8": [P, P, I64, I64, I64, P],
             "oracle_dequant": [P, P, P, I64, I64, P, P],
+            "oracle_static_batch_absmax": [P, I64, I64, P],
+            "oracle_static_ema": [ctypes.c_float, ctypes.c_float, ctypes.c_float, I],
+            "oracle_quant_act_static": [P, I64, I64, P, ctypes.c_float, P],
             "oracle_to_bf16": [P, I64, P],
         }
         for name, args in sig.items():
@@ -86,6 +89,8 @@ def _L():
             fn.restype = None
         _lib.oracle_ssz_quant_weight.restype = ctypes.c_int
         _lib.oracle_channel_mse.restype = ctypes.c_double
+        _lib.oracle_static_batch_absmax.restype = ctypes.c_float
+        _lib.oracle_static_ema.restype = ctypes.c_float
     return _lib
 
 
@@ -187,6 +192,46 @@ def quant_act_per_token(x, inv_s=None):
     sx = np.empty(M, np.float32)
     _L().oracle_quant_act_per_token(_ptr(x), M, K, _ptr(inv), _ptr(q), _ptr(sx))
     return q, sx
+
+
+# ------------------------------------------------------ static activation scale
+STATIC_EMA_RATE = np.float32(0.9)
+
+
+def static_batch_absmax(x, inv_s=None) -> np.float32:
+    """max |x * inv_s| over one calibration batch x [M,K]."""
+    x = _f32(x)
+    M, K = x.shape
+    inv = None if inv_s is None else _f32(inv_s)
+    return np.float32(_L().oracle_static_batch_absmax(_ptr(x), M, K, _ptr(inv)))
+
+
+def static_ema(state, a, rate=STATIC_EMA_RATE, first=False) -> np.float32:
+    """One moving-average step of the per-tensor activation range (fp32)."""
+    return np.float32(_L().oracle_static_ema(float(state), float(a), float(rate), 1 if first else 0))
+
+
+def static_range(batches, inv_s=None, rate=STATIC_EMA_RATE) -> np.float32:
+    """Moving-average abs-max over a sequence of calibration batches."""
+    m = np.float32(0.0)
+    for i, xb in enumerate(batches):
+        m = static_ema(m, static_batch_absmax(xb, inv_s), rate, first=(i == 0))
+    return m
+
+
+def quant_act_static(x, inv_s, m):
+    """Codes of x [M,K] (times inv_s) at the static scale S = m / 127."""
+    x = _f32(x)
+    M, K = x.shape
+    inv = None if inv_s is None else _f32(inv_s)
+    q = np.empty((M, K), np.int8)
+    _L().oracle_quant_act_static(_ptr(x), M, K, _ptr(inv), float(np.float32(m)), _ptr(q))
+    return q
+
+
+def static_scale(m) -> np.float32:
+    """S = m / 127 in fp32."""
+    return np.float32(np.float32(m) / np.float32(127.0))
 
 
 # --------------------------------------------------------------------- step 5

@@ -28,6 +28,10 @@
  *   [PTQ] "训练后量化（PTQ）" tutorial, "PTQ 的基本流程" (calibrate on a
  *         small set, then compute scales) and "逐层量化 vs 逐通道量化"
  *         (one scale per output channel).
+ *   [QAT] "PaddleNLP GPT 量化感知训练（QAT）实战指南", section 六 (the
+ *         Compress configuration): activation_quantize_type
+ *         'moving_average_abs_max' tracks the activation range with a
+ *         moving average of the abs-max.
  *
  * Readings where the pages are silent (each also listed in the design notes):
  *   - channel j of W in the smoothing factor is input channel j (column j of
@@ -43,6 +47,11 @@
  *   - the relative and absolute convergence tests are OR-ed, evaluated
  *     before the greedy update, and convergence is per channel and sticky.
  *   - the activation scale of an all-zero row is 0 and its codes are 0.
+ *   - static activation scale: one per tensor, S = m / 127 with m the
+ *     moving average over calibration batches of each batch's abs-max of the
+ *     smoothed activations, m_1 = a_1, m_t = rate m_{t-1} + (1 - rate) a_t
+ *     in fp32 (products and sum each rounded once); values beyond the range
+ *     saturate to +-127.
  *
  * Arithmetic: IEEE binary32 for every quantity that decides a code, fp64
  * for error and least-squares sums, exact integers for the matrix product.
@@ -276,6 +285,50 @@ void oracle_quant_act_per_token(const float *x, int64_t M, int64_t K,
             q[t * K + j] = (s == 0.0f) ? (int8_t)0 : (int8_t)sym_code(v, s, ACT_QMAX);
         }
     }
+}
+
+/* ------------------------------------------------- static activation scale */
+/* Abs-max of the smoothed activations x' = x * inv_s over one calibration
+ * batch x [M,K] (inv_s nullable): the per-tensor range [CQ] 2.1 "范围校准". */
+float oracle_static_batch_absmax(const float *x, int64_t M, int64_t K, const float *inv_s)
+{
+    float amax = 0.0f;
+    for (int64_t t = 0; t < M; ++t)
+        for (int64_t j = 0; j < K; ++j) {
+            float v = inv_s ? x[t * K + j] * inv_s[j] : x[t * K + j];
+            float a = fabsf(v);
+            if (a > amax)
+                amax = a;
+        }
+    return amax;
+}
+
+/* Moving average of the per-batch abs-max ([QAT] moving_average_abs_max;
+ * [CQ] 2.1: a moving average of the range is more robust than raw min/max):
+ * the first batch sets the state, later ones blend in with weight 1 - rate. */
+float oracle_static_ema(float state, float a, float rate, int first)
+{
+    if (first)
+        return a;
+    float keep = rate * state;
+    float w = 1.0f - rate;
+    float add = w * a;
+    return keep + add;
+}
+
+/* Static per-tensor activation quantization ([CQ] 2.1 with Z = 0, one scale
+ * for the whole tensor): S = m / 127, q = clamp(rint(x' / S), -127, 127);
+ * S == 0 gives zero codes. */
+void oracle_quant_act_static(const float *x, int64_t M, int64_t K, const float *inv_s, float m,
+                             int8_t *q)
+{
+    float S = m / (float)ACT_QMAX;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < M; ++t)
+        for (int64_t j = 0; j < K; ++j) {
+            float v = inv_s ? x[t * K + j] * inv_s[j] : x[t * K + j];
+            q[t * K + j] = (S == 0.0f) ? (int8_t)0 : (int8_t)sym_code(v, S, ACT_QMAX);
+        }
 }
 
 /* ---------------------------------------------------------------- step 5 */

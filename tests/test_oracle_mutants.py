@@ -48,6 +48,12 @@ MUTANTS = [
     ("dequant_drops_token_scale", "((float)acc[t * N + n] * sx[t]) * sw[n]",
      "((float)acc[t * N + n]) * sw[n]"),
     ("bf16_rounds_half_up", "u += 0x7fffu + ((u >> 16) & 1u);", "u += 0x8000u;"),
+    ("static_ema_swaps_weights", "float keep = rate * state;\n    float w = 1.0f - rate;",
+     "float keep = (1.0f - rate) * state;\n    float w = rate;"),
+    ("static_ema_ignores_first", "    if (first)\n        return a;\n", ""),
+    ("static_range_drops_smoothing", "float v = inv_s ? x[t * K + j] * inv_s[j] : x[t * K + j];\n            float a",
+     "float v = x[t * K + j];\n            float a"),
+    ("static_scale_128", "float S = m / (float)ACT_QMAX;", "float S = m / 128.0f;"),
 ]
 
 PIN_TESTS = []

@@ -10,7 +10,9 @@ plants such slips in a copy of the oracle and checks that they are caught.
 Sources: SmoothQuant deep-dive (developer.baidu.com) section 1 for the
 smoothing factor and the equivalence; "SSZ：权重量化算法说明" (msModelSlim)
 sections 算法流程 / 迭代优化阶段 / 收敛判断 / 算法参数 for the weight search;
-CUDA INT8 notes (aicoding.csdn.net) section 2.1 for Q = round(R/S) + Z.
+CUDA INT8 notes (aicoding.csdn.net) section 2.1 for Q = round(R/S) + Z;
+"PaddleNLP GPT 量化感知训练（QAT）实战指南" section 六 for the moving-average
+activation range.
 """
 import os
 
@@ -322,6 +324,73 @@ def test_act_quant_zero_row_and_identity_smoothing(orc):
     q1, sx1 = orc.quant_act_per_token(x, np.ones(32, np.float32))
     np.testing.assert_array_equal(q, q1)
     np.testing.assert_array_equal(sx, sx1)
+
+
+# ------------------------------------------------- static activation scale
+# "PaddleNLP GPT 量化感知训练（QAT）实战指南" section 六 (moving_average_abs_max)
+# and the CUDA INT8 notes section 2.1 (range calibration, saturation).
+def test_static_batch_absmax_matches_numpy_and_column_route(orc):
+    x = _llm_like(50, 96, seed=31)
+    inv = (np.random.default_rng(32).random(96) + 0.25).astype(np.float32)
+    a = orc.static_batch_absmax(x, inv)
+    assert a == np.abs(x * inv[None, :]).max()
+    # the same value from the per-channel absmax: |x| * c is monotonic in |x|
+    assert a == (orc.calib_absmax(x) * inv).max()
+    assert orc.static_batch_absmax(x) == np.abs(x).max()
+
+
+def test_static_ema_closed_forms(orc):
+    a = np.float32([3.0, 5.0, 2.0, 7.0])
+    # rate 0: the last batch; rate 1: the first batch; first call sets the state
+    assert orc.static_ema(123.0, 4.0, 0.9, first=True) == np.float32(4.0)
+    m = a[0]
+    for v in a[1:]:
+        m = orc.static_ema(m, v, 0.0)
+    assert m == a[-1]
+    m = a[0]
+    for v in a[1:]:
+        m = orc.static_ema(m, v, 1.0)
+    assert m == a[0]
+    # rate 1/2 on small integers is exact: m = (((3+5)/2 + 2)/2 + 7)/2
+    m = a[0]
+    for v in a[1:]:
+        m = orc.static_ema(m, v, 0.5)
+    assert m == np.float32(((3.0 + 5.0) / 2 + 2.0) / 2 / 2 + 7.0 / 2)
+    # general rate against the fp64 closed form rate^(T-1) a_1 + sum (1-rate) rate^(T-t) a_t
+    r = np.random.default_rng(33)
+    seq = (r.random(12) * 10).astype(np.float32)
+    m = orc.static_range([np.full((1, 16), v, np.float32) for v in seq], rate=0.9)
+    T = len(seq)
+    want = 0.9 ** (T - 1) * float(seq[0]) + sum(0.1 * 0.9 ** (T - 1 - t) * float(seq[t]) for t in range(1, T))
+    assert abs(float(m) - want) <= 1e-5 * want
+
+
+def test_static_quant_matches_numpy_and_saturates(orc):
+    x = _llm_like(24, 64, seed=34)
+    inv = (np.random.default_rng(35).random(64) + 0.5).astype(np.float32)
+    m = np.float32(np.abs(x * inv[None, :]).max() * np.float32(0.25))  # a range well below the max
+    q = orc.quant_act_static(x, inv, m)
+    S = orc.static_scale(m)
+    assert S == m / np.float32(127)
+    want = np.clip(np.rint((x * inv[None, :]) / S), -127, 127).astype(np.int8)
+    np.testing.assert_array_equal(q, want)
+    big = np.abs(x * inv[None, :]) > 128 * S
+    assert big.any() and np.all(np.abs(q[big]) == 127)
+    assert not orc.quant_act_static(x, inv, np.float32(0.0)).any()
+
+
+def test_static_quant_equals_dynamic_at_the_row_range(orc):
+    # with the static range equal to one row's abs-max, that row's codes are
+    # the per-token codes (an independently pinned function)
+    x = _llm_like(16, 80, seed=36)
+    inv = (np.random.default_rng(37).random(80) + 0.5).astype(np.float32)
+    qd, sx = orc.quant_act_per_token(x, inv)
+    for t in (0, 7, 15):
+        m = np.float32(sx[t] * np.float32(127))
+        if orc.static_scale(m) != sx[t]:
+            continue  # m / 127 does not round back to sx (rare); nothing to compare
+        qs = orc.quant_act_static(x[t:t + 1], inv, m)
+        np.testing.assert_array_equal(qs[0], qd[t])
 
 
 # ----------------------------------------------------------------- step 5
