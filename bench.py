@@ -272,11 +272,48 @@ def run_ours(args, rank, world, local_rank):
     ops_per_step = sum(2.0 * p.M * p.N * p.K for p in probs)
     value = ops_per_step * world * args.steps / (total_ms * 1e-3) / 1e12
 
+    next_rows = time_next_rows(args, w, torch, probs, flush, stream) if world == 1 else None
+
     # ---- end to end through the C ABI with host buffers
     e2e = None
     if args.e2e_steps > 0:
         e2e = run_e2e(args, w, wdist, torch, probs, run, flush, stream, ops_per_step, world)
-    return finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall1 - wall0)
+    return finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall1 - wall0, next_rows)
+
+
+def time_next_rows(args, w, torch, probs, flush, stream, reps=50):
+    """Kernels of the rows built beyond the five-step path, timed one launch
+    at a time like the path's kernels (L2 flushed before each, outside the
+    events), on the first linear of the workload:
+    - quant_act_static: codes at a static per-tensor scale (range calibrated
+      beforehand on the same activations)."""
+    p = probs[0]
+    peaks, _ = load_peaks()
+    out = {}
+    rng = torch.empty(1, device=p.x.device)
+    w.sq_static_range_update(p.ax, p.inv, rng, first=True)
+
+    def timed(fn):
+        ts = []
+        for i in range(reps + 3):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            if i >= 3:
+                ts.append(e0.elapsed_time(e1))
+        return statistics.mean(ts)
+
+    ms = timed(lambda: w.quant_act_static(p.x, p.inv, rng, p.qx, p.sx))
+    nbytes = p.x.element_size() * p.M * p.K + p.M * p.K + 4 * p.K + 4 * p.M + 4
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    out["quant_act_static"] = {"us": round(ms * 1e3, 2), "bound": "hbm", "achieved": round(gbs, 1),
+                               "peak": round(peaks["hbm_gbs"], 1), "unit": "GB/s",
+                               "frac": round(gbs / peaks["hbm_gbs"], 4), "algorithmic": {"bytes": nbytes},
+                               "shape": [p.M, p.K]}
+    return out
 
 
 def run_e2e(args, w, wdist, torch, probs, run, flush, stream, ops_per_step, world):
@@ -306,7 +343,7 @@ def run_e2e(args, w, wdist, torch, probs, run, flush, stream, ops_per_step, worl
             "ms_per_step": round(e2e_total / len(e2e_ms), 4)}
 
 
-def finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall_s):
+def finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall_s, next_rows=None):
     names = NAMES
     # ---- rooflines per kernel (algorithmic work summed over the workload's linears)
     peaks, src = load_peaks()
@@ -383,6 +420,8 @@ def finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall_s):
         "clocks": clk.result,
         "wall_s_timed_region": round(wall_s, 3),
     }
+    if next_rows:
+        result["next_rows"] = next_rows
     return result
 
 

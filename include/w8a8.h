@@ -152,6 +152,32 @@ sq_status quant_act_per_token(const void *x, sq_dtype xt, int64_t M, int64_t K,
                               const float *inv_s, int8_t *q_out, float *scale_out,
                               void *stream);
 
+/* ------------------------------------------- static activation scale (next)
+ * A per-tensor activation range calibrated offline instead of the per-token
+ * scales of step 4: the moving-average abs-max of "PaddleNLP GPT
+ * 量化感知训练（QAT）实战指南" section 六 (activation_quantize_type
+ * moving_average_abs_max) with the range calibration and saturation of [CQ]
+ * 2.1.  The pages give no moving rate; 0.9 is this library's default
+ * reading (the caller passes it).
+ *
+ * sq_static_range_update: one calibration batch.  x_absmax: [K] fp32, that
+ * batch's per-channel abs-max (sq_calib_absmax with accumulate = 0); inv_s:
+ * [K] fp32 or NULL.  With a = max_j fl(x_absmax[j] * inv_s[j]) (the batch's
+ * abs-max of x * inv_s):
+ *     *range = first ? a : fl(fl(rate * *range) + fl(fl(1 - rate) * a))
+ * range: one fp32 in device memory, in/out.  rate in [0,1]. */
+sq_status sq_static_range_update(const float *x_absmax, const float *inv_s, int64_t K,
+                                 float rate, int first, float *range, void *stream);
+
+/* quant_act_static: codes at the static scale S = fl(*range / 127):
+ *     q[t,j] = clamp(rint(x[t,j] * inv_s[j] / S), -127, 127)   (0 if S == 0)
+ * Values beyond the range saturate.  scale_out: [M] fp32 or NULL; if given,
+ * every entry receives S, so that w8a8_gemm_dequant applies the static
+ * scale unchanged.  Shapes, dtypes and alignment as quant_act_per_token. */
+sq_status quant_act_static(const void *x, sq_dtype xt, int64_t M, int64_t K,
+                           const float *inv_s, const float *range, int8_t *q_out,
+                           float *scale_out, void *stream);
+
 /* ------------------------------------------------------------------ step 5
  * INT8 x INT8 -> INT32 GEMM with fused per-token x per-channel dequant
  * [CQ] 3.2 and 4.2:

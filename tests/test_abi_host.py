@@ -121,6 +121,33 @@ def test_quant_act_rejects(lib, case, status):
     assert rc == status, _detail(lib)
 
 
+@pytest.mark.parametrize("case,status", [("null", 1), ("null_range", 1), ("k", 2), ("align_q", 4),
+                                         ("dtype", 3)])
+def test_quant_act_static_rejects(lib, case, status):
+    a = dict(x=P(), xt=1, M=4, K=64, inv=NULL, rng=P(4096), q=P(8192), sc=NULL)
+    if case == "null": a["q"] = NULL
+    if case == "null_range": a["rng"] = NULL
+    if case == "k": a["K"] = 65
+    if case == "align_q": a["q"] = P(8)
+    if case == "dtype": a["xt"] = 5
+    rc = lib.quant_act_static(a["x"], a["xt"], a["M"], a["K"], a["inv"], a["rng"], a["q"], a["sc"], None)
+    assert rc == status, _detail(lib)
+
+
+@pytest.mark.parametrize("case,status", [("null", 1), ("k", 2), ("rate_neg", 5), ("rate_big", 5),
+                                         ("rate_nan", 5), ("align", 4)])
+def test_static_range_update_rejects(lib, case, status):
+    a = dict(ax=P(), inv=NULL, K=64, rate=0.9, rng=P(4096))
+    if case == "null": a["rng"] = NULL
+    if case == "k": a["K"] = 0
+    if case == "rate_neg": a["rate"] = -0.1
+    if case == "rate_big": a["rate"] = 1.5
+    if case == "rate_nan": a["rate"] = float("nan")
+    if case == "align": a["ax"] = P(2)
+    rc = lib.sq_static_range_update(a["ax"], a["inv"], a["K"], a["rate"], 0, a["rng"], None)
+    assert rc == status, _detail(lib)
+
+
 @pytest.mark.parametrize("case,status", [
     ("null_sw", 1), ("k", 2), ("n_bf16", 2), ("n_f32", 2), ("align_y", 4), ("dtype", 3), ("k_huge", 2),
 ])
@@ -141,6 +168,7 @@ def test_gemm_rejects(lib, case, status):
 def test_empty_inputs_are_noops(lib):
     # M == 0 / N == 0 return OK without touching the device
     assert lib.quant_act_per_token(NULL, 1, 0, 64, NULL, NULL, NULL, None) == 0
+    assert lib.quant_act_static(NULL, 1, 0, 64, NULL, NULL, NULL, NULL, None) == 0
     assert lib.ssz_quant_weight(NULL, 1, 0, 64, NULL, 8, 20, NULL, NULL, NULL, NULL, None) == 0
     assert lib.w8a8_gemm_dequant(NULL, NULL, NULL, NULL, 0, 16, 64, NULL, 1, NULL, None) == 0
     assert lib.w8a8_gemm_dequant(NULL, NULL, NULL, NULL, 4, 0, 64, NULL, 1, NULL, None) == 0

@@ -26,7 +26,7 @@ STATUS = ["SQ_OK", "SQ_ERR_NULL", "SQ_ERR_SHAPE", "SQ_ERR_DTYPE", "SQ_ERR_ALIGN"
 EXPORTS = ["sq_status_string", "sq_last_error_detail", "sq_abi_version", "sq_device_fault",
            "sq_selftest_bounded_wait",
            "sq_calib_absmax", "sq_smooth_fold", "ssz_quant_weight", "quant_act_per_token",
-           "w8a8_gemm_dequant"]
+           "w8a8_gemm_dequant", "sq_static_range_update", "quant_act_static"]
 
 
 class W8A8Error(RuntimeError):
@@ -54,6 +54,8 @@ def _load() -> ctypes.CDLL:
         "ssz_quant_weight": ([P, I, I64, I64, P, I, I, P, P, P, P, P], I),
         "quant_act_per_token": ([P, I, I64, I64, P, P, P, P], I),
         "w8a8_gemm_dequant": ([P, P, P, P, I64, I64, I64, P, I, P, P], I),
+        "sq_static_range_update": ([P, P, I64, F, I, P, P], I),
+        "quant_act_static": ([P, I, I64, I64, P, P, P, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -160,6 +162,33 @@ def quant_act_per_token(x: torch.Tensor, inv_s: torch.Tensor | None, q_out: torc
     M, K = x.shape
     _check("quant_act_per_token", lib.quant_act_per_token(_ptr(x), _dtype(x), M, K, _ptr(inv_s), _ptr(q_out),
                                                            _ptr(scale_out), _stream(stream)))
+
+
+STATIC_RANGE_RATE = 0.9  # moving rate of the static activation range (not given by the pages)
+
+
+def sq_static_range_update(x_absmax: torch.Tensor, inv_s: torch.Tensor | None, range_: torch.Tensor,
+                           first: bool, rate: float = STATIC_RANGE_RATE, stream=None) -> None:
+    """Blend one calibration batch (its per-channel abs-max) into the static
+    activation range held in range_ (one fp32 on the device)."""
+    _need(x_absmax, torch.float32, "x_absmax")
+    _need(inv_s, torch.float32, "inv_s")
+    _need(range_, torch.float32, "range")
+    K = x_absmax.shape[0]
+    _check("sq_static_range_update", lib.sq_static_range_update(_ptr(x_absmax), _ptr(inv_s), K, float(rate),
+                                                                 1 if first else 0, _ptr(range_), _stream(stream)))
+
+
+def quant_act_static(x: torch.Tensor, inv_s: torch.Tensor | None, range_: torch.Tensor, q_out: torch.Tensor,
+                     scale_out: torch.Tensor | None = None, stream=None) -> None:
+    """int8 codes of x * inv_s at the static scale range_/127 (saturating)."""
+    _need(inv_s, torch.float32, "inv_s")
+    _need(range_, torch.float32, "range")
+    _need(q_out, torch.int8, "q_out")
+    _need(scale_out, torch.float32, "scale_out")
+    M, K = x.shape
+    _check("quant_act_static", lib.quant_act_static(_ptr(x), _dtype(x), M, K, _ptr(inv_s), _ptr(range_),
+                                                     _ptr(q_out), _ptr(scale_out), _stream(stream)))
 
 
 def w8a8_gemm_dequant(qx: torch.Tensor, sx: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor, y: torch.Tensor,

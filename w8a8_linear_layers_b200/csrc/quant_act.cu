@@ -81,10 +81,15 @@ __device__ __forceinline__ uint2 fast_codes_tied(const float (&v)[8], float s, f
 // Measured on B200: one row per CTA of one or two warps (E = 32 or 64) with
 // many CTAs per SM beats several rows per larger CTA and beats staging rows
 // in shared memory with bulk copies.
-template <typename T, int E, int ROWS>
+//
+// STATIC: one scale for the whole tensor, S = range[0] / 127 (a range
+// calibrated beforehand, see sq_static_range_update); no per-row reduction,
+// values beyond the range saturate, and scale[row] (if given) receives S so
+// that the GEMM's per-token dequant applies it unchanged.
+template <typename T, int E, int ROWS, bool STATIC>
 __global__ void __launch_bounds__(512)
 quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__restrict__ inv_s,
-                 int8_t *__restrict__ q, float *__restrict__ scale) {
+                 const float *__restrict__ range, int8_t *__restrict__ q, float *__restrict__ scale) {
     constexpr int C = E / 8;  // chunks per thread
     // inv_s is kept in registers across rows unless that would spill
     constexpr bool kCacheInvS = C * ROWS <= 4;
@@ -130,7 +135,7 @@ quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__r
                     raw[rr][c].zero();
             }
         }
-        float amax[ROWS];
+        float amax[ROWS];  // dynamic: the row's abs-max; static: this thread's
 #pragma unroll
         for (int rr = 0; rr < ROWS; ++rr) {
             amax[rr] = 0.0f;
@@ -141,23 +146,32 @@ quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__r
 #pragma unroll
                 for (int i = 0; i < 8; ++i) amax[rr] = fmaxf(amax[rr], fabsf(v[i]));
             }
-            amax[rr] = warp_max(amax[rr]);
-            if (lane == 0) red[parity][rr][warp] = amax[rr];
+            if (!STATIC) {
+                amax[rr] = warp_max(amax[rr]);
+                if (lane == 0) red[parity][rr][warp] = amax[rr];
+            }
         }
-        __syncthreads();  // red[parity] complete; red[parity^1] free for the next rows
+        if (!STATIC) __syncthreads();  // red[parity] complete; red[parity^1] free for the next rows
 #pragma unroll
         for (int rr = 0; rr < ROWS; ++rr) {
             const int64_t row = row0 + rr;
             if (row >= M) break;
-            float am = red[parity][rr][0];
-            for (int w = 1; w < nwarps; ++w) am = fmaxf(am, red[parity][rr][w]);
-            const float s = __fdiv_rn(am, 127.0f);
-            if (threadIdx.x == 0) scale[row] = s;
+            float am = amax[rr], s;
+            if (STATIC) {
+                s = __fdiv_rn(__ldg(range), 127.0f);
+                if (scale && threadIdx.x == 0) scale[row] = s;
+            } else {
+                am = red[parity][rr][0];
+                for (int w = 1; w < nwarps; ++w) am = fmaxf(am, red[parity][rr][w]);
+                s = __fdiv_rn(am, 127.0f);
+                if (threadIdx.x == 0) scale[row] = s;
+            }
             const float r = __fdiv_rn(1.0f, s);
             const bool exact_only = !(fabsf(r) <= 3.402823466e38f);  // 1/s overflowed (or s == 0)
-            // |v r| <= am r (about 127): the int16 clamp of fast_codes8 applies;
-            // a fast code can differ from the exact one only where |d| comes
-            // within |y| 2^-21 + 2^-22 of 0.5
+            // |v r| <= am r (about 127 in the dynamic case): below 2^14 the
+            // int16 clamp of fast_codes8 applies; a fast code can differ from
+            // the exact one only where |d| comes within |y| 2^-21 + 2^-22 of
+            // 0.5 (in the static case am is this thread's abs-max)
             const bool narrow = am * r < 16384.0f;
             const float tie_bound = 0.5f - fmaf(am * r, 4.76837158203125e-07f, 2.384185791015625e-07f);
             int8_t *qr = q + row * K;
@@ -183,14 +197,57 @@ quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__r
     }
 }
 
-template <typename T, int E, int ROWS>
-static void launch_quant_act(const void *x, int64_t M, int64_t K, const float *inv_s, int8_t *q,
-                             float *scale, int sms, cudaStream_t st) {
+template <typename T, int E, int ROWS, bool STATIC>
+static void launch_quant_act(const void *x, int64_t M, int64_t K, const float *inv_s, const float *range,
+                             int8_t *q, float *scale, int sms, cudaStream_t st) {
     int threads = (int)ceil_div(ceil_div(K, E), 32) * 32;
     // enough CTAs to fill the machine; each strides over groups of ROWS rows
     int per_sm = std::max(1, std::min(32, 2048 / threads));
     int64_t grid = std::min<int64_t>(ceil_div(M, ROWS), (int64_t)sms * per_sm);
-    quant_act_kernel<T, E, ROWS><<<(unsigned)grid, threads, 0, st>>>((const T *)x, M, K, inv_s, q, scale);
+    quant_act_kernel<T, E, ROWS, STATIC>
+        <<<(unsigned)grid, threads, 0, st>>>((const T *)x, M, K, inv_s, range, q, scale);
+}
+
+// E elements per thread: one warp per row up to K = 32 E, at most 64
+// elements per thread.
+template <bool STATIC>
+static void dispatch_quant(const void *x, bool bf, int64_t M, int64_t K, const float *inv_s, const float *range,
+                           int8_t *q, float *scale, int sms, cudaStream_t cs) {
+    if (K <= 256) {
+        if (bf) launch_quant_act<__nv_bfloat16, 8, 1, STATIC>(x, M, K, inv_s, range, q, scale, sms, cs);
+        else launch_quant_act<float, 8, 1, STATIC>(x, M, K, inv_s, range, q, scale, sms, cs);
+    } else if (K <= 512) {
+        if (bf) launch_quant_act<__nv_bfloat16, 16, 1, STATIC>(x, M, K, inv_s, range, q, scale, sms, cs);
+        else launch_quant_act<float, 16, 1, STATIC>(x, M, K, inv_s, range, q, scale, sms, cs);
+    } else if (K <= 1024) {
+        if (bf) launch_quant_act<__nv_bfloat16, 32, 1, STATIC>(x, M, K, inv_s, range, q, scale, sms, cs);
+        else launch_quant_act<float, 32, 1, STATIC>(x, M, K, inv_s, range, q, scale, sms, cs);
+    } else {
+        if (bf) launch_quant_act<__nv_bfloat16, 64, 1, STATIC>(x, M, K, inv_s, range, q, scale, sms, cs);
+        else launch_quant_act<float, 64, 1, STATIC>(x, M, K, inv_s, range, q, scale, sms, cs);
+    }
+}
+
+// range = first ? a : fl(fl(rate range) + fl(fl(1 - rate) a)) with
+// a = max_j fl(ax_j inv_s_j) -- the batch's abs-max of x * inv_s, since
+// |x| c is monotonic in |x| for c >= 0.  One CTA.
+__global__ void __launch_bounds__(1024)
+static_range_kernel(const float *__restrict__ ax, const float *__restrict__ inv_s, int64_t K, float rate,
+                    int first, float *__restrict__ range) {
+    __shared__ float red[32];
+    float a = 0.0f;
+    for (int64_t j = threadIdx.x; j < K; j += blockDim.x) {
+        const float v = inv_s ? __fmul_rn(ax[j], inv_s[j]) : ax[j];
+        a = fmaxf(a, fabsf(v));
+    }
+    a = warp_max(a);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) a = fmaxf(a, red[w]);
+        a = fmaxf(a, red[0]);
+        range[0] = first ? a : __fadd_rn(__fmul_rn(rate, range[0]), __fmul_rn(__fsub_rn(1.0f, rate), a));
+    }
 }
 
 }  // namespace w8a8
@@ -212,22 +269,39 @@ extern "C" sq_status quant_act_per_token(const void *x, sq_dtype xt, int64_t M, 
     sq_status st = check_device(&sms);
     if (st != SQ_OK) return st;
     cudaStream_t cs = (cudaStream_t)stream;
-    const bool bf = xt == SQ_BF16;
-    // E elements per thread: one warp per row up to K = 32 E, at most 64
-    // elements per thread
-    if (K <= 256) {
-        if (bf) launch_quant_act<__nv_bfloat16, 8, 1>(x, M, K, inv_s, q_out, scale_out, sms, cs);
-        else launch_quant_act<float, 8, 1>(x, M, K, inv_s, q_out, scale_out, sms, cs);
-    } else if (K <= 512) {
-        if (bf) launch_quant_act<__nv_bfloat16, 16, 1>(x, M, K, inv_s, q_out, scale_out, sms, cs);
-        else launch_quant_act<float, 16, 1>(x, M, K, inv_s, q_out, scale_out, sms, cs);
-    } else if (K <= 1024) {
-        if (bf) launch_quant_act<__nv_bfloat16, 32, 1>(x, M, K, inv_s, q_out, scale_out, sms, cs);
-        else launch_quant_act<float, 32, 1>(x, M, K, inv_s, q_out, scale_out, sms, cs);
-    } else if (bf) {
-        launch_quant_act<__nv_bfloat16, 64, 1>(x, M, K, inv_s, q_out, scale_out, sms, cs);
-    } else {
-        launch_quant_act<float, 64, 1>(x, M, K, inv_s, q_out, scale_out, sms, cs);
-    }
+    dispatch_quant<false>(x, xt == SQ_BF16, M, K, inv_s, nullptr, q_out, scale_out, sms, cs);
+    return launch_status("quant_act_kernel");
+}
+
+extern "C" sq_status sq_static_range_update(const float *x_absmax, const float *inv_s, int64_t K, float rate,
+                                            int first, float *range, void *stream) {
+    if (!x_absmax || !range) return fail(SQ_ERR_NULL, "sq_static_range_update: NULL pointer");
+    if (K <= 0) return fail(SQ_ERR_SHAPE, "sq_static_range_update: K=%lld", (long long)K);
+    if (!(rate >= 0.0f && rate <= 1.0f))
+        return fail(SQ_ERR_ARG, "sq_static_range_update: rate=%g outside [0,1]", (double)rate);
+    if (!aligned(x_absmax, 4) || !aligned(range, 4) || (inv_s && !aligned(inv_s, 4)))
+        return fail(SQ_ERR_ALIGN, "sq_static_range_update: misaligned pointer");
+    int sms;
+    sq_status st = check_device(&sms);
+    if (st != SQ_OK) return st;
+    static_range_kernel<<<1, 1024, 0, (cudaStream_t)stream>>>(x_absmax, inv_s, K, rate, first != 0, range);
+    return launch_status("static_range_kernel");
+}
+
+extern "C" sq_status quant_act_static(const void *x, sq_dtype xt, int64_t M, int64_t K, const float *inv_s,
+                                      const float *range, int8_t *q_out, float *scale_out, void *stream) {
+    if (M > 0 && (!x || !q_out || !range)) return fail(SQ_ERR_NULL, "quant_act_static: NULL pointer");
+    if (xt != SQ_F32 && xt != SQ_BF16) return fail(SQ_ERR_DTYPE, "quant_act_static: dtype %d", (int)xt);
+    if (M < 0 || K <= 0 || K % 16 != 0 || K > 32768)
+        return fail(SQ_ERR_SHAPE, "quant_act_static: M=%lld K=%lld (K must be a multiple of 16 in [16, 32768])",
+                    (long long)M, (long long)K);
+    if (M == 0) return SQ_OK;
+    if (!aligned(x, 16) || !aligned(q_out, 16) || !aligned(range, 4) || (scale_out && !aligned(scale_out, 4)) ||
+        (inv_s && !aligned(inv_s, 16)))
+        return fail(SQ_ERR_ALIGN, "quant_act_static: misaligned pointer (x, q_out, inv_s need 16 bytes)");
+    int sms;
+    sq_status st = check_device(&sms);
+    if (st != SQ_OK) return st;
+    dispatch_quant<true>(x, xt == SQ_BF16, M, K, inv_s, range, q_out, scale_out, sms, (cudaStream_t)stream);
     return launch_status("quant_act_kernel");
 }
