@@ -79,6 +79,10 @@ def _L():
             "oracle_gemm_i8": [P, P, I64, I64, I64, P],
             "oracle_dequant": [P, P, P, I64, I64, P, P],
             "oracle_static_batch_absmax": [P, I64, I64, P],
+            "oracle_ssz_quant_weight_asym": [P, I64, I64, I, P, P, P, P, P, P],
+            "oracle_channel_mse_asym": [P, I64, ctypes.c_float, ctypes.c_float],
+            "oracle_act_rowsum": [P, I64, I64, P],
+            "oracle_dequant_asym": [P, P, P, P, P, I64, I64, P, P],
             "oracle_static_ema": [ctypes.c_float, ctypes.c_float, ctypes.c_float, I],
             "oracle_quant_act_static": [P, I64, I64, P, ctypes.c_float, P],
             "oracle_to_bf16": [P, I64, P],
@@ -90,6 +94,8 @@ def _L():
         _lib.oracle_ssz_quant_weight.restype = ctypes.c_int
         _lib.oracle_channel_mse.restype = ctypes.c_double
         _lib.oracle_static_batch_absmax.restype = ctypes.c_float
+        _lib.oracle_ssz_quant_weight_asym.restype = ctypes.c_int
+        _lib.oracle_channel_mse_asym.restype = ctypes.c_double
         _lib.oracle_static_ema.restype = ctypes.c_float
     return _lib
 
@@ -192,6 +198,59 @@ def quant_act_per_token(x, inv_s=None):
     sx = np.empty(M, np.float32)
     _L().oracle_quant_act_per_token(_ptr(x), M, K, _ptr(inv), _ptr(q), _ptr(sx))
     return q, sx
+
+
+# ------------------------------------------------------ asymmetric int8 SSZ
+def ssz_quant_weight_asym(w, max_iters: int = SSZ_ITERS, s=None, trace: bool = False):
+    """Asymmetric per-channel int8 SSZ of w [N,K] (folded by s if given):
+    w ~ scale * (q + 128) + offset.  Returns dict(q, scale, offset, mse,
+    iters[, trace])."""
+    w = _f32(w)
+    if s is not None:
+        w = scale_columns(w, s)
+    N, K = w.shape
+    q = np.empty((N, K), np.int8)
+    scale = np.empty(N, np.float32)
+    offset = np.empty(N, np.float32)
+    mse = np.empty(N, np.float64)
+    iters = np.empty(N, np.int32)
+    tr = np.empty((N, max_iters + 1), np.float64) if trace else None
+    rc = _L().oracle_ssz_quant_weight_asym(_ptr(w), N, K, int(max_iters), _ptr(q), _ptr(scale), _ptr(offset),
+                                           _ptr(mse), _ptr(iters), _ptr(tr))
+    if rc != 0:
+        raise ValueError("asymmetric SSZ: unsupported arguments")
+    out = dict(q=q, scale=scale, offset=offset, mse=mse, iters=iters)
+    if trace:
+        out["trace"] = tr
+    return out
+
+
+def channel_mse_asym(w_row, S, m) -> float:
+    w_row = _f32(w_row)
+    return float(_L().oracle_channel_mse_asym(_ptr(w_row), w_row.shape[0], float(S), float(m)))
+
+
+def act_rowsum(qx) -> np.ndarray:
+    qx = np.ascontiguousarray(qx, dtype=np.int8)
+    M, K = qx.shape
+    R = np.empty(M, np.int32)
+    _L().oracle_act_rowsum(_ptr(qx), M, K, _ptr(R))
+    return R
+
+
+def dequant_asym(acc, R, sx, S, m, out: str = "bf16") -> np.ndarray:
+    """sx (S (acc + 128 R) + m R) in fp32; out as in dequant."""
+    acc = np.ascontiguousarray(acc, dtype=np.int32)
+    R = np.ascontiguousarray(R, dtype=np.int32)
+    sx, S, m = _f32(sx), _f32(S), _f32(m)
+    M, N = acc.shape
+    if out == "f32":
+        y = np.empty((M, N), np.float32)
+        _L().oracle_dequant_asym(_ptr(acc), _ptr(R), _ptr(sx), _ptr(S), _ptr(m), M, N, _ptr(y), None)
+    else:
+        y = np.empty((M, N), np.uint16)
+        _L().oracle_dequant_asym(_ptr(acc), _ptr(R), _ptr(sx), _ptr(S), _ptr(m), M, N, None, _ptr(y))
+    return y
 
 
 # ------------------------------------------------------ static activation scale

@@ -65,6 +65,7 @@
 #define SSZ_CONVERGE_THRESHOLD 1e-10 /* [SSZ] 算法参数 */
 #define SSZ_MIN_SCALE 1e-5f          /* [SSZ] 算法参数 */
 #define ACT_QMAX 127                 /* symmetric int8, narrow range */
+#define ASYM_UMAX 255                /* asymmetric int8: u in [0, 255] */
 
 /* ---------------------------------------------------------------- step 1 */
 /* Per-input-channel activation absmax, [SQ] max(|X_j|), gathered over the
@@ -260,6 +261,138 @@ double oracle_channel_mse(const float *w, int64_t K, float s, int bits)
     return channel_mse(w, K, s, (1 << (bits - 1)) - 1);
 }
 
+/* ------------------------------------------------- asymmetric int8 SSZ */
+/* Asymmetric code ([SSZ] 迭代优化阶段, 非对称量化: scale and offset both
+ * free; [CQ] 2.1 Q = round(R/S) + Z).  Reading: the offset m lives in the
+ * weight domain, w ~ S u + m with u = clamp(rint(fl(w - m) / S), 0, 255)
+ * (all 256 levels of int8; stored as q = u - 128). */
+static float asym_code(float w, float S, float m)
+{
+    float v = w - m;
+    float r = rintf(v / S);
+    if (r > (float)ASYM_UMAX)
+        r = (float)ASYM_UMAX;
+    if (r < 0.0f)
+        r = 0.0f;
+    return r;
+}
+
+/* mean over K of (w - (S u + m))^2 in fp64, index order, re-quantising at
+ * (S, m). */
+static double channel_mse_asym(const float *w, int64_t K, float S, float m)
+{
+    double acc = 0.0;
+    for (int64_t k = 0; k < K; ++k) {
+        double u = (double)asym_code(w[k], S, m);
+        double e = (double)w[k] - ((double)S * u + (double)m);
+        acc += e * e;
+    }
+    return acc / (double)K;
+}
+
+/* One channel: MinMax init (m = min w, S = (max w - min w) / 255, floored),
+ * then rounds of least squares for (S, m) given the codes of the kept pair,
+ *     den = K sum u^2 - (sum u)^2,  a = (K sum wu - sum w sum u) / den,
+ *     b = (sum w - a sum u) / K   (fp64; den == 0 keeps the pair),
+ * candidate S = max(fp32(a), 1e-5), m = fp32(b); the error, greedy keep and
+ * convergence tests are those of the symmetric search. */
+static int ssz_channel_asym(const float *w, int64_t K, int max_iters, float *scale, float *offset,
+                            double *mse, double *trace)
+{
+    float wmin = w[0], wmax = w[0];
+    for (int64_t k = 1; k < K; ++k) {
+        if (w[k] < wmin)
+            wmin = w[k];
+        if (w[k] > wmax)
+            wmax = w[k];
+    }
+    float s_best = (wmax - wmin) / (float)ASYM_UMAX;
+    if (s_best < SSZ_MIN_SCALE)
+        s_best = SSZ_MIN_SCALE;
+    float m_off = wmin;
+    double e_best = channel_mse_asym(w, K, s_best, m_off);
+    if (trace)
+        trace[0] = e_best;
+    int it = 0;
+    int done = 0;
+    while (it < max_iters && !done) {
+        ++it;
+        double sw = 0.0, swu = 0.0;
+        int64_t su = 0, suu = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            float u = asym_code(w[k], s_best, m_off);
+            sw += (double)w[k];
+            swu += (double)w[k] * (double)u;
+            su += (int64_t)u;
+            suu += (int64_t)u * (int64_t)u;
+        }
+        double den = (double)K * (double)suu - (double)su * (double)su;
+        float s_cand = s_best, m_cand = m_off;
+        if (den != 0.0) {
+            double a = ((double)K * swu - sw * (double)su) / den;
+            double b = (sw - a * (double)su) / (double)K;
+            s_cand = (float)a;
+            if (s_cand < SSZ_MIN_SCALE)
+                s_cand = SSZ_MIN_SCALE;
+            m_cand = (float)b;
+        }
+        double e_cand = channel_mse_asym(w, K, s_cand, m_cand);
+        double delta = e_best - e_cand;
+        done = (e_best == 0.0) || (delta / e_best < SSZ_CONVERGE_THRESHOLD) ||
+               (fabs(delta) < SSZ_CONVERGE_THRESHOLD);
+        if (e_cand < e_best) {
+            s_best = s_cand;
+            m_off = m_cand;
+            e_best = e_cand;
+        }
+        if (trace)
+            trace[it] = e_best;
+    }
+    if (trace)
+        for (int r = it + 1; r <= max_iters; ++r)
+            trace[r] = e_best;
+    *scale = s_best;
+    *offset = m_off;
+    *mse = e_best;
+    return it;
+}
+
+/* Per-output-channel asymmetric int8 weight quantization with the SSZ
+ * search (int4 asymmetric is unsupported on the SSZ page, 使用限制).
+ * w: smoothed [N,K] fp32.  Outputs: q [N,K] int8 = u - 128, scale [N],
+ * offset [N] (weight domain), mse/iters/trace nullable as in the symmetric
+ * search.  Returns 0, or -1 on a bad argument. */
+int oracle_ssz_quant_weight_asym(const float *w, int64_t N, int64_t K, int max_iters, int8_t *q,
+                                 float *scale, float *offset, double *mse, int32_t *iters,
+                                 double *trace)
+{
+    if (N < 0 || K <= 0 || max_iters < 0)
+        return -1;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t n = 0; n < N; ++n) {
+        const float *row = w + n * K;
+        float S, m;
+        double e;
+        int it = ssz_channel_asym(row, K, max_iters, &S, &m, &e,
+                                  trace ? trace + n * (int64_t)(max_iters + 1) : 0);
+        scale[n] = S;
+        offset[n] = m;
+        if (mse)
+            mse[n] = e;
+        if (iters)
+            iters[n] = it;
+        for (int64_t k = 0; k < K; ++k)
+            q[n * K + k] = (int8_t)((int)asym_code(row[k], S, m) - 128);
+    }
+    return 0;
+}
+
+/* The error of one channel at a given (S, m) (exposed for the pins). */
+double oracle_channel_mse_asym(const float *w, int64_t K, float S, float m)
+{
+    return channel_mse_asym(w, K, S, m);
+}
+
 /* ---------------------------------------------------------------- step 4 */
 /* Per-token symmetric activation quantization ([CQ] 2.1, Z = 0): with
  * x' = x * inv_s (inv_s nullable: no smoothing), sx_t = max_j|x'_tj| / 127
@@ -367,6 +500,38 @@ void oracle_dequant(const int32_t *acc, const float *sx, const float *sw,
     for (int64_t t = 0; t < M; ++t)
         for (int64_t n = 0; n < N; ++n) {
             float y = ((float)acc[t * N + n] * sx[t]) * sw[n];
+            if (y_f32)
+                y_f32[t * N + n] = y;
+            if (y_bf16)
+                y_bf16[t * N + n] = f32_to_bf16_rne(y);
+        }
+}
+
+/* Row sums R_t = sum_k qx[t,k] of the activation codes (exact). */
+void oracle_act_rowsum(const int8_t *qx, int64_t M, int64_t K, int32_t *R)
+{
+    for (int64_t t = 0; t < M; ++t) {
+        int64_t r = 0;
+        for (int64_t k = 0; k < K; ++k)
+            r += qx[t * K + k];
+        R[t] = (int32_t)r;
+    }
+}
+
+/* Dequant with asymmetric weights ([CQ] 4.2 with the zero point of 2.1):
+ * w ~ S_n u + m_n with u = q + 128, so
+ *     sum_k sx_t qx[t,k] (S_n u[n,k] + m_n) = sx_t (S_n A + m_n R_t),
+ *     A = acc[t,n] + 128 R_t  (exact int32; acc = sum qx q of the stored codes)
+ * in fp32: y = fl(sx_t * fl(fl(S_n * (float)A) + fl(m_n * (float)R_t))). */
+void oracle_dequant_asym(const int32_t *acc, const int32_t *R, const float *sx, const float *S,
+                         const float *m, int64_t M, int64_t N, float *y_f32, uint16_t *y_bf16)
+{
+    for (int64_t t = 0; t < M; ++t)
+        for (int64_t n = 0; n < N; ++n) {
+            int32_t A = acc[t * N + n] + 128 * R[t];
+            float p = S[n] * (float)A;
+            float o = m[n] * (float)R[t];
+            float y = sx[t] * (p + o);
             if (y_f32)
                 y_f32[t * N + n] = y;
             if (y_bf16)

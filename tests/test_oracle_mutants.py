@@ -54,6 +54,13 @@ MUTANTS = [
     ("static_range_drops_smoothing", "float v = inv_s ? x[t * K + j] * inv_s[j] : x[t * K + j];\n            float a",
      "float v = x[t * K + j];\n            float a"),
     ("static_scale_128", "float S = m / (float)ACT_QMAX;", "float S = m / 128.0f;"),
+    ("asym_code_ignores_offset", "float v = w - m;", "float v = w;"),
+    ("asym_ls_offset_sign", "double b = (sw - a * (double)su) / (double)K;",
+     "double b = (sw + a * (double)su) / (double)K;"),
+    ("asym_minmax_254_levels", "float s_best = (wmax - wmin) / (float)ASYM_UMAX;",
+     "float s_best = (wmax - wmin) / 254.0f;"),
+    ("asym_dequant_drops_128R", "int32_t A = acc[t * N + n] + 128 * R[t];", "int32_t A = acc[t * N + n];"),
+    ("asym_dequant_drops_offset", "float y = sx[t] * (p + o);", "float y = sx[t] * p;"),
 ]
 
 PIN_TESTS = []

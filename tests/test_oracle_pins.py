@@ -326,6 +326,100 @@ def test_act_quant_zero_row_and_identity_smoothing(orc):
     np.testing.assert_array_equal(sx, sx1)
 
 
+# ------------------------------------------------- asymmetric int8 SSZ
+# "SSZ：权重量化算法说明": 初始化阶段 (MinMax min/max), 迭代优化阶段 (asymmetric:
+# scale and offset by least squares), 收敛判断, 算法参数.
+def _asym_codes_np(w, S, m):
+    return np.clip(np.rint((w - np.float32(m)) / np.float32(S)), 0, 255)
+
+
+def test_ssz_asym_minmax_init(orc):
+    r = np.random.default_rng(40)
+    w = (r.standard_normal((6, 96)) * 0.3 + 0.2).astype(np.float32)
+    out = orc.ssz_quant_weight_asym(w, max_iters=0)
+    np.testing.assert_array_equal(out["offset"], w.min(1))
+    np.testing.assert_array_equal(out["scale"], (w.max(1) - w.min(1)) / np.float32(255))
+    u = out["q"].astype(np.int32) + 128
+    assert np.all(u[np.arange(6), w.argmin(1)] == 0) and np.all(u[np.arange(6), w.argmax(1)] == 255)
+    for n in range(6):
+        np.testing.assert_array_equal(u[n], _asym_codes_np(w[n], out["scale"][n], out["offset"][n]))
+
+
+def test_ssz_asym_one_round_is_least_squares(orc):
+    # one round by hand: codes at the MinMax pair, lstsq of w on [u, 1],
+    # re-quantise, keep if better (numpy throughout)
+    r = np.random.default_rng(41)
+    w = (r.standard_normal((8, 200)) + 3.0).astype(np.float32)
+    out = orc.ssz_quant_weight_asym(w, max_iters=1)
+    for n in range(8):
+        S0 = max((w[n].max() - w[n].min()) / np.float32(255), np.float32(1e-5))
+        m0 = w[n].min()
+        u = _asym_codes_np(w[n], S0, m0).astype(np.float64)
+        a, b = np.linalg.lstsq(np.stack([u, np.ones_like(u)], 1), w[n].astype(np.float64), rcond=None)[0]
+        Sc, mc = max(np.float32(a), np.float32(1e-5)), np.float32(b)
+
+        def err(S, m):
+            uu = _asym_codes_np(w[n], S, m).astype(np.float64)
+            return np.mean((w[n].astype(np.float64) - (np.float64(S) * uu + np.float64(m))) ** 2)
+        S_want, m_want = (Sc, mc) if err(Sc, mc) < err(S0, m0) else (S0, m0)
+        np.testing.assert_allclose(out["scale"][n], S_want, rtol=1e-6)
+        np.testing.assert_allclose(out["offset"][n], m_want, rtol=1e-6, atol=1e-6 * abs(m_want))
+
+
+def test_ssz_asym_error_trace_and_codes(orc):
+    r = np.random.default_rng(42)
+    w = (r.standard_normal((12, 160)) * np.linspace(0.1, 2.0, 12)[:, None] + 0.5).astype(np.float32)
+    out = orc.ssz_quant_weight_asym(w, trace=True)
+    mm = orc.ssz_quant_weight_asym(w, max_iters=0)
+    for n in range(12):
+        u = _asym_codes_np(w[n], out["scale"][n], out["offset"][n])
+        np.testing.assert_array_equal(out["q"][n].astype(np.int32) + 128, u)
+        e = np.mean((w[n].astype(np.float64) - (np.float64(out["scale"][n]) * u + np.float64(out["offset"][n]))) ** 2)
+        assert abs(out["mse"][n] - e) <= 1e-12 * e + 1e-30
+        assert out["mse"][n] <= mm["mse"][n]
+        assert np.all(np.diff(out["trace"][n]) <= 0)
+    assert np.mean(out["mse"] < mm["mse"]) > 0.5
+
+
+def test_ssz_asym_beats_symmetric_on_offset_rows(orc):
+    r = np.random.default_rng(43)
+    w = (r.standard_normal((16, 256)) + 10.0).astype(np.float32)  # far from zero
+    a = orc.ssz_quant_weight_asym(w)
+    sym = orc.ssz_quant_weight(w, bits=8)
+    assert np.all(a["mse"] < 0.2 * sym["mse"])
+
+
+def test_ssz_asym_scale_equivariance(orc):
+    # w -> 2 w scales every fp operation exactly: codes equal, (S, m) double
+    r = np.random.default_rng(44)
+    w = (r.standard_normal((6, 128)) + 1.0).astype(np.float32)
+    a = orc.ssz_quant_weight_asym(w, max_iters=3)
+    b = orc.ssz_quant_weight_asym(2 * w, max_iters=3)
+    np.testing.assert_array_equal(a["q"], b["q"])
+    np.testing.assert_array_equal(2 * a["scale"], b["scale"])
+    np.testing.assert_array_equal(2 * a["offset"], b["offset"])
+
+
+def test_act_rowsum_and_asym_dequant(orc):
+    r = np.random.default_rng(45)
+    qx = r.integers(-127, 128, (9, 64)).astype(np.int8)
+    qw = r.integers(-128, 128, (7, 64)).astype(np.int8)
+    sx = (r.random(9) * 0.1).astype(np.float32)
+    S = (r.random(7) * 0.01).astype(np.float32)
+    m = (r.standard_normal(7) * 0.1).astype(np.float32)
+    R = orc.act_rowsum(qx)
+    np.testing.assert_array_equal(R, qx.astype(np.int64).sum(1))
+    acc = orc.gemm_i8(qx, qw)
+    y = orc.dequant_asym(acc, R, sx, S, m, out="f32")
+    A = (acc + 128 * R[:, None]).astype(np.float32)
+    want = sx[:, None] * (S[None, :] * A + m[None, :] * R[:, None].astype(np.float32))
+    np.testing.assert_array_equal(y, want)
+    # the same as sum_k sx qx (S u + m) in fp64, up to fp32 rounding
+    u = qw.astype(np.float64) + 128
+    ref = sx[:, None].astype(np.float64) * (qx.astype(np.float64) @ (S[:, None] * u + m[:, None]).T)
+    np.testing.assert_allclose(y, ref, rtol=1e-5, atol=1e-6 * np.abs(ref).max())
+
+
 # ------------------------------------------------- static activation scale
 # "PaddleNLP GPT 量化感知训练（QAT）实战指南" section 六 (moving_average_abs_max)
 # and the CUDA INT8 notes section 2.1 (range calibration, saturation).
