@@ -33,14 +33,19 @@ MUTANTS = [
     ("round_half_away", "float r = rintf(w / s);", "float r = roundf(w / s);"),
     ("asymmetric_clamp", "if (r < -(float)qmax)\n        r = -(float)qmax;",
      "if (r < -(float)(qmax + 1))\n        r = -(float)(qmax + 1);"),
-    ("mse_is_sum_not_mean", "return acc / (double)K;", "return acc;"),
+    ("mse_is_sum_not_mean", "(double)sym_code(w[k], s, qmax);\n        acc += e * e;\n    }\n    return acc / (double)K;",
+     "(double)sym_code(w[k], s, qmax);\n        acc += e * e;\n    }\n    return acc;"),
+    ("asym_mse_is_sum_not_mean", "(double)m);\n        acc += e * e;\n    }\n    return acc / (double)K;",
+     "(double)m);\n        acc += e * e;\n    }\n    return acc;"),
     ("ls_inverted", "s_cand = (float)(num / (double)den);", "s_cand = (float)((double)den / num);"),
     ("ls_drops_square", "den += (int64_t)q * (int64_t)q;", "den += (int64_t)(q < 0 ? -q : q);"),
     ("convergence_sign_flipped", "(delta / m_best < SSZ_CONVERGE_THRESHOLD)",
      "(delta / m_best > SSZ_CONVERGE_THRESHOLD)"),
     ("minmax_uses_qmax_plus_one", "float s_best = amax / (float)qmax;",
      "float s_best = amax / (float)(qmax + 1);"),
-    ("candidate_not_floored", "if (s_cand < SSZ_MIN_SCALE)\n                s_cand = SSZ_MIN_SCALE;", ""),
+    ("candidate_not_floored",
+     "s_cand = (float)(num / (double)den);\n            if (s_cand < SSZ_MIN_SCALE)\n                s_cand = SSZ_MIN_SCALE;",
+     "s_cand = (float)(num / (double)den);"),
     ("act_scale_128", "float s = amax / (float)ACT_QMAX;", "float s = amax / 128.0f;"),
     ("act_divides_by_inv_s", "float v = inv_s ? row[j] * inv_s[j] : row[j];\n            q[",
      "float v = inv_s ? row[j] / inv_s[j] : row[j];\n            q["),
