@@ -286,7 +286,10 @@ def time_next_rows(args, w, torch, probs, flush, stream, reps=50):
     at a time like the path's kernels (L2 flushed before each, outside the
     events), on the first linear of the workload:
     - quant_act_static: codes at a static per-tensor scale (range calibrated
-      beforehand on the same activations)."""
+      beforehand on the same activations);
+    - ssz_quant_weight_asym, quant_act_per_token_rowsum and
+      w8a8_gemm_dequant_asym: the asymmetric int8 weight path.
+    Per-launch times include the launch gap that in-step events hide."""
     p = probs[0]
     peaks, _ = load_peaks()
     out = {}
@@ -313,6 +316,36 @@ def time_next_rows(args, w, torch, probs, flush, stream, reps=50):
                                "peak": round(peaks["hbm_gbs"], 1), "unit": "GB/s",
                                "frac": round(gbs / peaks["hbm_gbs"], 4), "algorithmic": {"bytes": nbytes},
                                "shape": [p.M, p.K]}
+
+    # asymmetric int8 weights: SSZ over (scale, offset), per-token codes with
+    # row sums, GEMM with the offset dequant
+    dev = p.x.device
+    qa, sa, ow = torch.empty_like(p.qw), torch.empty_like(p.sw), torch.empty(p.N, device=dev)
+    its = torch.empty(p.N, device=dev, dtype=torch.int32)
+    rs = torch.empty(p.M, device=dev, dtype=torch.int32)
+    ms = timed(lambda: w.ssz_quant_weight_asym(p.wt, p.s, p.max_iters, qa, sa, ow, iters_out=its))
+    iters = float(its.double().mean().item())
+    ops = SSZ_OPS_PER_ELEMENT_ROUND * p.N * p.K * (1.0 + iters)
+    sm_mhz = NOMINAL_SM_MHZ
+    alu_peak = B200_SMS * FP32_LANES_PER_SM * sm_mhz * 1e6 / 1e12
+    ach = ops / (ms * 1e-3) / 1e12
+    out["ssz_quant_weight_asym"] = {"us": round(ms * 1e3, 2), "bound": "alu", "achieved": round(ach, 2),
+                                    "peak": round(alu_peak, 2), "unit": "Tops/s", "frac": round(ach / alu_peak, 4),
+                                    "mean_iters": round(iters, 3), "peak_clock_mhz": sm_mhz,
+                                    "shape": [p.N, p.K]}
+    ms = timed(lambda: w.quant_act_per_token_rowsum(p.x, p.inv, p.qx, p.sx, rs))
+    nbytes = p.x.element_size() * p.M * p.K + p.M * p.K + 4 * p.K + 8 * p.M
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    out["quant_act_per_token_rowsum"] = {"us": round(ms * 1e3, 2), "bound": "hbm", "achieved": round(gbs, 1),
+                                         "peak": round(peaks["hbm_gbs"], 1), "unit": "GB/s",
+                                         "frac": round(gbs / peaks["hbm_gbs"], 4), "shape": [p.M, p.K]}
+    if p.bits == 8:
+        ms = timed(lambda: w.w8a8_gemm_dequant_asym(p.qx, p.sx, rs, qa, sa, ow, p.y))
+        tops = 2.0 * p.M * p.N * p.K / (ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+        out["w8a8_gemm_dequant_asym"] = {"us": round(ms * 1e3, 2), "bound": "tensor", "achieved": round(tops, 1),
+                                         "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(tops / peak, 4),
+                                         "shape": [p.M, p.N, p.K]}
     return out
 
 

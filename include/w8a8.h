@@ -152,6 +152,44 @@ sq_status quant_act_per_token(const void *x, sq_dtype xt, int64_t M, int64_t K,
                               const float *inv_s, int8_t *q_out, float *scale_out,
                               void *stream);
 
+/* Step 4 with the row sums R[t] = sum_j q_out[t,j] (exact int32) that the
+ * GEMM with asymmetric weights needs.  rowsum_out: [M] int32 or NULL (then
+ * this is quant_act_per_token).  Same op, codes and scales otherwise. */
+sq_status quant_act_per_token_rowsum(const void *x, sq_dtype xt, int64_t M, int64_t K,
+                                     const float *inv_s, int8_t *q_out, float *scale_out,
+                                     int32_t *rowsum_out, void *stream);
+
+/* --------------------------------------------- asymmetric int8 SSZ (next)
+ * [SSZ] 初始化阶段 / 迭代优化阶段 (asymmetric: scale and offset optimised
+ * together by least squares); int8 only (使用限制: asymmetric int4 is not
+ * supported).  Reading: w' ~ S u + m per channel, offset m in the weight
+ * domain, u = clamp(rint(fl(w' - m) / S), 0, 255), stored as q = u - 128.
+ *     MinMax: m = min_k w'[k], S = max((max_k w'[k] - m) / 255, 1e-5)
+ *     round: least squares of w' on (u, 1) for the kept codes (fp64):
+ *         den = K sum u^2 - (sum u)^2 (0: keep the pair),
+ *         a = (K sum w'u - sum w' sum u) / den, b = (sum w' - a sum u) / K,
+ *         candidate S = max(fp32(a), 1e-5), m = fp32(b);
+ *     error, greedy keep, convergence and max_iters as ssz_quant_weight.
+ * w: [N,K] of dtype wt; s: [K] fp32 fold or NULL.  q_out: [N,K] int8;
+ * scale_out, offset_out: [N] fp32; mse_out [N] fp64 / iters_out [N] int32
+ * or NULL.  K <= 32768, a multiple of 16. */
+sq_status ssz_quant_weight_asym(const void *w, sq_dtype wt, int64_t N, int64_t K, const float *s,
+                                int max_iters, int8_t *q_out, float *scale_out, float *offset_out,
+                                double *mse_out, int32_t *iters_out, void *stream);
+
+/* GEMM + dequant for asymmetric weights (scale sw, offset ow, codes
+ * q = u - 128 as written by ssz_quant_weight_asym) [CQ] 3.2 / 4.2:
+ *     acc[t,n] = sum_k qx[t,k] * qw[n,k]                (exact int32)
+ *     A        = acc[t,n] + 128 rowsum[t]               (exact: sum qx u)
+ *     y[t,n]   = yt( sx[t] * (sw[n] * (float)A + ow[n] * (float)rowsum[t]) )
+ * in fp32, each product and the sum rounded once.  rowsum: [M] int32 from
+ * quant_act_per_token_rowsum; ow: [N] fp32 (16-byte aligned).  Other
+ * arguments as w8a8_gemm_dequant; K <= 65792 (|A| < 2^31). */
+sq_status w8a8_gemm_dequant_asym(const int8_t *qx, const float *sx, const int32_t *rowsum,
+                                 const int8_t *qw, const float *sw, const float *ow, int64_t M,
+                                 int64_t N, int64_t K, void *y, sq_dtype yt, int32_t *acc_out,
+                                 void *stream);
+
 /* ------------------------------------------- static activation scale (next)
  * A per-tensor activation range calibrated offline instead of the per-token
  * scales of step 4: the moving-average abs-max of "PaddleNLP GPT

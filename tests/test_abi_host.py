@@ -121,6 +121,35 @@ def test_quant_act_rejects(lib, case, status):
     assert rc == status, _detail(lib)
 
 
+@pytest.mark.parametrize("case,status", [("null_off", 1), ("k", 2), ("iters", 5), ("align_off", 4), ("dtype", 3)])
+def test_ssz_asym_rejects(lib, case, status):
+    a = dict(w=P(), wt=1, N=4, K=64, s=NULL, it=20, q=P(8192), sc=P(12288), off=P(12544))
+    if case == "null_off": a["off"] = NULL
+    if case == "k": a["K"] = 40
+    if case == "iters": a["it"] = 300
+    if case == "align_off": a["off"] = P(2)
+    if case == "dtype": a["wt"] = 4
+    rc = lib.ssz_quant_weight_asym(a["w"], a["wt"], a["N"], a["K"], a["s"], a["it"], a["q"], a["sc"], a["off"],
+                                   NULL, NULL, None)
+    assert rc == status, _detail(lib)
+
+
+@pytest.mark.parametrize("case,status", [("null_rs", 1), ("null_ow", 1), ("k_asym_limit", 2), ("align_ow", 4)])
+def test_gemm_asym_rejects(lib, case, status):
+    a = dict(qx=P(), sx=P(4096), rs=P(4608), qw=P(8192), sw=P(12288), ow=P(12544), M=4, N=16, K=64, y=P(16384))
+    if case == "null_rs": a["rs"] = NULL
+    if case == "null_ow": a["ow"] = NULL
+    if case == "k_asym_limit": a["K"] = 65808
+    if case == "align_ow": a["ow"] = P(12548)
+    rc = lib.w8a8_gemm_dequant_asym(a["qx"], a["sx"], a["rs"], a["qw"], a["sw"], a["ow"], a["M"], a["N"], a["K"],
+                                    a["y"], 1, NULL, None)
+    assert rc == status, _detail(lib)
+
+
+def test_quant_rowsum_rejects_misaligned(lib):
+    assert lib.quant_act_per_token_rowsum(P(), 1, 4, 64, NULL, P(8192), P(12288), P(2), None) == 4
+
+
 @pytest.mark.parametrize("case,status", [("null", 1), ("null_range", 1), ("k", 2), ("align_q", 4),
                                          ("dtype", 3)])
 def test_quant_act_static_rejects(lib, case, status):

@@ -26,7 +26,8 @@ STATUS = ["SQ_OK", "SQ_ERR_NULL", "SQ_ERR_SHAPE", "SQ_ERR_DTYPE", "SQ_ERR_ALIGN"
 EXPORTS = ["sq_status_string", "sq_last_error_detail", "sq_abi_version", "sq_device_fault",
            "sq_selftest_bounded_wait",
            "sq_calib_absmax", "sq_smooth_fold", "ssz_quant_weight", "quant_act_per_token",
-           "w8a8_gemm_dequant", "sq_static_range_update", "quant_act_static"]
+           "w8a8_gemm_dequant", "sq_static_range_update", "quant_act_static", "quant_act_per_token_rowsum",
+           "ssz_quant_weight_asym", "w8a8_gemm_dequant_asym"]
 
 
 class W8A8Error(RuntimeError):
@@ -56,6 +57,9 @@ def _load() -> ctypes.CDLL:
         "w8a8_gemm_dequant": ([P, P, P, P, I64, I64, I64, P, I, P, P], I),
         "sq_static_range_update": ([P, P, I64, F, I, P, P], I),
         "quant_act_static": ([P, I, I64, I64, P, P, P, P, P], I),
+        "quant_act_per_token_rowsum": ([P, I, I64, I64, P, P, P, P, P], I),
+        "ssz_quant_weight_asym": ([P, I, I64, I64, P, I, P, P, P, P, P, P], I),
+        "w8a8_gemm_dequant_asym": ([P, P, P, P, P, P, I64, I64, I64, P, I, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -162,6 +166,54 @@ def quant_act_per_token(x: torch.Tensor, inv_s: torch.Tensor | None, q_out: torc
     M, K = x.shape
     _check("quant_act_per_token", lib.quant_act_per_token(_ptr(x), _dtype(x), M, K, _ptr(inv_s), _ptr(q_out),
                                                            _ptr(scale_out), _stream(stream)))
+
+
+def quant_act_per_token_rowsum(x: torch.Tensor, inv_s: torch.Tensor | None, q_out: torch.Tensor,
+                               scale_out: torch.Tensor, rowsum_out: torch.Tensor, stream=None) -> None:
+    """quant_act_per_token plus the exact row sums of the codes (int32)."""
+    _need(inv_s, torch.float32, "inv_s")
+    _need(q_out, torch.int8, "q_out")
+    _need(scale_out, torch.float32, "scale_out")
+    _need(rowsum_out, torch.int32, "rowsum_out")
+    M, K = x.shape
+    _check("quant_act_per_token_rowsum",
+           lib.quant_act_per_token_rowsum(_ptr(x), _dtype(x), M, K, _ptr(inv_s), _ptr(q_out), _ptr(scale_out),
+                                          _ptr(rowsum_out), _stream(stream)))
+
+
+def ssz_quant_weight_asym(w: torch.Tensor, s: torch.Tensor | None, max_iters: int, q_out: torch.Tensor,
+                          scale_out: torch.Tensor, offset_out: torch.Tensor, mse_out: torch.Tensor | None = None,
+                          iters_out: torch.Tensor | None = None, stream=None) -> None:
+    """Asymmetric per-channel int8 SSZ: w * s ~ scale * (q + 128) + offset."""
+    _need(s, torch.float32, "s")
+    _need(q_out, torch.int8, "q_out")
+    _need(scale_out, torch.float32, "scale_out")
+    _need(offset_out, torch.float32, "offset_out")
+    _need(mse_out, torch.float64, "mse_out")
+    _need(iters_out, torch.int32, "iters_out")
+    N, K = w.shape
+    _check("ssz_quant_weight_asym",
+           lib.ssz_quant_weight_asym(_ptr(w), _dtype(w), N, K, _ptr(s), int(max_iters), _ptr(q_out),
+                                     _ptr(scale_out), _ptr(offset_out), _ptr(mse_out), _ptr(iters_out),
+                                     _stream(stream)))
+
+
+def w8a8_gemm_dequant_asym(qx: torch.Tensor, sx: torch.Tensor, rowsum: torch.Tensor, qw: torch.Tensor,
+                           sw: torch.Tensor, ow: torch.Tensor, y: torch.Tensor, acc_out: torch.Tensor | None = None,
+                           stream=None) -> None:
+    """GEMM + dequant with asymmetric weights (scale sw, offset ow)."""
+    _need(qx, torch.int8, "qx")
+    _need(qw, torch.int8, "qw")
+    _need(sx, torch.float32, "sx")
+    _need(sw, torch.float32, "sw")
+    _need(ow, torch.float32, "ow")
+    _need(rowsum, torch.int32, "rowsum")
+    _need(acc_out, torch.int32, "acc_out")
+    M, K = qx.shape
+    N = qw.shape[0]
+    _check("w8a8_gemm_dequant_asym",
+           lib.w8a8_gemm_dequant_asym(_ptr(qx), _ptr(sx), _ptr(rowsum), _ptr(qw), _ptr(sw), _ptr(ow), M, N, K,
+                                      _ptr(y), _dtype(y), _ptr(acc_out), _stream(stream)))
 
 
 STATIC_RANGE_RATE = 0.9  # moving rate of the static activation range (not given by the pages)

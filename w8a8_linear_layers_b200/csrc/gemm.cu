@@ -202,64 +202,70 @@ struct Cfg {
     static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
 };
 
-template <typename OutT>
-__device__ __forceinline__ void store_row_chunk(OutT *yrow, const uint32_t (&acc)[32], float sxr,
-                                                const float *__restrict__ swc, int valid, bool vec_ok);
+// Dequant of one accumulator.  Symmetric weights: ((float)acc * sx) * sw.
+// Asymmetric weights (w ~ sw (q + 128) + ow): with R the row sum of the
+// activation codes and A = acc + 128 R (exact int32),
+// sx * (sw * (float)A + ow * (float)R).
+template <bool ASYM>
+__device__ __forceinline__ float dequant1(uint32_t acc, float sxr, int Rr, float swv, float owv) {
+    if (ASYM) {
+        const float p = swv * __int2float_rn((int)acc + 128 * Rr);
+        const float o = owv * __int2float_rn(Rr);
+        return sxr * (p + o);
+    }
+    return (__int2float_rn((int)acc) * sxr) * swv;
+}
 
-template <>
-__device__ __forceinline__ void store_row_chunk<__nv_bfloat16>(__nv_bfloat16 *yrow, const uint32_t (&acc)[32],
-                                                               float sxr, const float *__restrict__ swc,
-                                                               int valid, bool vec_ok) {
+template <typename OutT, bool ASYM>
+__device__ __forceinline__ void store_row_chunk(OutT *yrow, const uint32_t (&acc)[32], float sxr, int Rr,
+                                                const float *__restrict__ swc, const float *__restrict__ owc,
+                                                int valid, bool vec_ok) {
     if (vec_ok && valid >= 32) {
-        uint32_t packed[16];
+        float y[32];
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
-            float4 f = __ldg(reinterpret_cast<const float4 *>(swc + j));
-            float sv[4] = {f.x, f.y, f.z, f.w};
-            float y[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) y[i] = (__int2float_rn((int)acc[j + i]) * sxr) * sv[i];
-            __nv_bfloat162 lo = __floats2bfloat162_rn(y[0], y[1]);
-            __nv_bfloat162 hi = __floats2bfloat162_rn(y[2], y[3]);
-            packed[j / 2] = *reinterpret_cast<uint32_t *>(&lo);
-            packed[j / 2 + 1] = *reinterpret_cast<uint32_t *>(&hi);
+            const float4 f = __ldg(reinterpret_cast<const float4 *>(swc + j));
+            const float4 o = ASYM ? __ldg(reinterpret_cast<const float4 *>(owc + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            y[j] = dequant1<ASYM>(acc[j], sxr, Rr, f.x, o.x);
+            y[j + 1] = dequant1<ASYM>(acc[j + 1], sxr, Rr, f.y, o.y);
+            y[j + 2] = dequant1<ASYM>(acc[j + 2], sxr, Rr, f.z, o.z);
+            y[j + 3] = dequant1<ASYM>(acc[j + 3], sxr, Rr, f.w, o.w);
         }
-        uint4 *dst = reinterpret_cast<uint4 *>(yrow);
+        if (sizeof(OutT) == 2) {
+            uint32_t packed[16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+            for (int j = 0; j < 32; j += 2) {
+                __nv_bfloat162 h = __floats2bfloat162_rn(y[j], y[j + 1]);
+                packed[j / 2] = *reinterpret_cast<uint32_t *>(&h);
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(yrow);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+        } else {
+            float4 *dst = reinterpret_cast<float4 *>(yrow);
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) dst[j / 4] = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
+        }
     } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-            if (j < valid) yrow[j] = __float2bfloat16_rn((__int2float_rn((int)acc[j]) * sxr) * swc[j]);
+            if (j < valid) {
+                const float v = dequant1<ASYM>(acc[j], sxr, Rr, swc[j], ASYM ? owc[j] : 0.0f);
+                if (sizeof(OutT) == 2)
+                    reinterpret_cast<__nv_bfloat16 *>(yrow)[j] = __float2bfloat16_rn(v);
+                else
+                    reinterpret_cast<float *>(yrow)[j] = v;
+            }
     }
 }
 
-template <>
-__device__ __forceinline__ void store_row_chunk<float>(float *yrow, const uint32_t (&acc)[32], float sxr,
-                                                       const float *__restrict__ swc, int valid, bool vec_ok) {
-    if (vec_ok && valid >= 32) {
-        float4 *dst = reinterpret_cast<float4 *>(yrow);
-#pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-            float4 f = __ldg(reinterpret_cast<const float4 *>(swc + j));
-            dst[j / 4] = make_float4((__int2float_rn((int)acc[j]) * sxr) * f.x,
-                                     (__int2float_rn((int)acc[j + 1]) * sxr) * f.y,
-                                     (__int2float_rn((int)acc[j + 2]) * sxr) * f.z,
-                                     (__int2float_rn((int)acc[j + 3]) * sxr) * f.w);
-        }
-    } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-            if (j < valid) yrow[j] = (__int2float_rn((int)acc[j]) * sxr) * swc[j];
-    }
-}
-
-template <int BN, typename OutT>
+template <int BN, typename OutT, bool ASYM>
 __global__ void __launch_bounds__(kThreads, 1)
 w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                 const float *__restrict__ sx, const float *__restrict__ sw, OutT *__restrict__ y,
-                 int32_t *__restrict__ acc_out, int M, int N, int K) {
+                 const float *__restrict__ sx, const float *__restrict__ sw, const int32_t *__restrict__ rs,
+                 const float *__restrict__ ow, OutT *__restrict__ y, int32_t *__restrict__ acc_out, int M, int N,
+                 int K) {
     using C = Cfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full_bar[C::STAGES];
@@ -404,6 +410,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             const int m0 = (tile % tiles_m) * BM, n0 = (tile / tiles_m) * BN;
             const int row = m0 + row_in_tile;
             const float sxr = row < M ? sx[row] : 0.0f;
+            const int Rr = (ASYM && row < M) ? rs[row] : 0;
             // the TMEM loads below are warp-collective: leave together or not at all
             const bool ok = wait_bounded(smem_u32(&tfull_bar[buf]), buf_phase, &abort_flag, kFaultEpilogue);
             if (!__all_sync(0xffffffffu, ok)) break;
@@ -417,7 +424,8 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
                 if (row < M && col < N) {
                     const int valid = N - col;
                     OutT *yrow = y + (int64_t)row * N + col;
-                    store_row_chunk<OutT>(yrow, acc, sxr, sw + col, valid, vec_ok);
+                    store_row_chunk<OutT, ASYM>(yrow, acc, sxr, Rr, sw + col, ASYM ? ow + col : nullptr, valid,
+                                                vec_ok);
                     if (acc_out) {
                         int32_t *arow = acc_out + (int64_t)row * N + col;
                         if (acc_vec_ok && valid >= 32) {
@@ -536,10 +544,10 @@ __device__ __forceinline__ void mbar_arrive_leader(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar & kPeerMask) : "memory");
 }
 
-template <typename OutT>
+template <typename OutT, bool ASYM>
 __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int row, int M, int n0, int N, const float sxr,
-                                              const float *__restrict__ sw, OutT *__restrict__ y,
-                                              int32_t *__restrict__ acc_out, int BNc) {
+                                              int Rr, const float *__restrict__ sw, const float *__restrict__ ow,
+                                              OutT *__restrict__ y, int32_t *__restrict__ acc_out, int BNc) {
     const bool vec_ok = (N % (16 / (int)sizeof(OutT))) == 0;
     const bool acc_vec_ok = (N % 4) == 0;
 #pragma unroll 1
@@ -549,7 +557,8 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int row, int M, in
         const int col = n0 + c0;
         if (row < M && col < N) {
             const int valid = N - col;
-            store_row_chunk<OutT>(y + (int64_t)row * N + col, acc, sxr, sw + col, valid, vec_ok);
+            store_row_chunk<OutT, ASYM>(y + (int64_t)row * N + col, acc, sxr, Rr, sw + col,
+                                        ASYM ? ow + col : nullptr, valid, vec_ok);
             if (acc_out) {
                 int32_t *arow = acc_out + (int64_t)row * N + col;
                 if (acc_vec_ok && valid >= 32) {
@@ -582,11 +591,12 @@ struct Cfg2 {
     static constexpr int SMEM = STAGES * STAGE_BYTES + 1024;
 };
 
-template <typename OutT>
+template <typename OutT, bool ASYM>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 w8a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                      const float *__restrict__ sx, const float *__restrict__ sw, OutT *__restrict__ y,
-                      int32_t *__restrict__ acc_out, int M, int N, int K) {
+                      const float *__restrict__ sx, const float *__restrict__ sw, const int32_t *__restrict__ rs,
+                      const float *__restrict__ ow, OutT *__restrict__ y, int32_t *__restrict__ acc_out, int M,
+                      int N, int K) {
     using C = Cfg2;
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full_bar[C::STAGES];
@@ -736,11 +746,12 @@ w8a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_c
             const int m0 = tm * C::PM, n0 = tn * C::BN;
             const int row = m0 + row_in_tile;
             const float sxr = row < M ? sx[row] : 0.0f;
+            const int Rr = (ASYM && row < M) ? rs[row] : 0;
             const bool ok = wait_bounded(smem_u32(&tfull_bar[buf]), buf_phase, &abort_flag, kFaultEpilogue);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
             const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * C::BN);
-            epilogue_tile<OutT>(tbase, row, M, n0, N, sxr, sw, y, acc_out, C::BN);
+            epilogue_tile<OutT, ASYM>(tbase, row, M, n0, N, sxr, Rr, sw, ow, y, acc_out, C::BN);
             tc_fence_before();
             mbar_arrive_leader(smem_u32(&tempty_bar[buf]));
             buf ^= 1;
@@ -799,14 +810,14 @@ static bool make_map(CUtensorMap *map, const void *base, int64_t rows, int64_t K
     return r == CUDA_SUCCESS;
 }
 
-template <int BN, typename OutT>
-static sq_status launch(const int8_t *qx, const float *sx, const int8_t *qw, const float *sw, int M, int N,
-                        int K, void *y, int32_t *acc_out, int sms, cudaStream_t st) {
+template <int BN, typename OutT, bool ASYM>
+static sq_status launch(const int8_t *qx, const float *sx, const int32_t *rs, const int8_t *qw, const float *sw,
+                        const float *ow, int M, int N, int K, void *y, int32_t *acc_out, int sms, cudaStream_t st) {
     using C = Cfg<BN>;
     CUtensorMap ma, mb;
     if (!make_map(&ma, qx, M, K, BM) || !make_map(&mb, qw, N, K, BN))
         return fail(SQ_ERR_CUDA, "w8a8_gemm_dequant: cuTensorMapEncodeTiled failed");
-    auto kern = w8a8_gemm_kernel<BN, OutT>;
+    auto kern = w8a8_gemm_kernel<BN, OutT, ASYM>;
     static int configured_dev[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -817,18 +828,19 @@ static sq_status launch(const int8_t *qx, const float *sx, const int8_t *qw, con
     }
     const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int grid = std::min(tiles, sms);
-    kern<<<grid, kThreads, C::SMEM, st>>>(ma, mb, sx, sw, (OutT *)y, acc_out, M, N, K);
+    kern<<<grid, kThreads, C::SMEM, st>>>(ma, mb, sx, sw, rs, ow, (OutT *)y, acc_out, M, N, K);
     return launch_status("w8a8_gemm_kernel");
 }
 
-template <typename OutT>
-static sq_status launch_pair(const int8_t *qx, const float *sx, const int8_t *qw, const float *sw, int M, int N,
-                             int K, void *y, int32_t *acc_out, int sms, cudaStream_t st) {
+template <typename OutT, bool ASYM>
+static sq_status launch_pair(const int8_t *qx, const float *sx, const int32_t *rs, const int8_t *qw,
+                             const float *sw, const float *ow, int M, int N, int K, void *y, int32_t *acc_out,
+                             int sms, cudaStream_t st) {
     using C = Cfg2;
     CUtensorMap ma, mb;
     if (!make_map(&ma, qx, M, K, BM) || !make_map(&mb, qw, N, K, C::BN / 2))
         return fail(SQ_ERR_CUDA, "w8a8_gemm_dequant: cuTensorMapEncodeTiled failed");
-    auto kern = w8a8_gemm_pair_kernel<OutT>;
+    auto kern = w8a8_gemm_pair_kernel<OutT, ASYM>;
     static int configured_dev[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -839,7 +851,7 @@ static sq_status launch_pair(const int8_t *qx, const float *sx, const int8_t *qw
     }
     const int tiles = ((M + C::PM - 1) / C::PM) * ((N + C::BN - 1) / C::BN);
     const int pairs = std::min(tiles, sms / 2);
-    kern<<<2 * pairs, kThreads, C::SMEM, st>>>(ma, mb, sx, sw, (OutT *)y, acc_out, M, N, K);
+    kern<<<2 * pairs, kThreads, C::SMEM, st>>>(ma, mb, sx, sw, rs, ow, (OutT *)y, acc_out, M, N, K);
     return launch_status("w8a8_gemm_pair_kernel");
 }
 
@@ -848,37 +860,59 @@ static sq_status launch_pair(const int8_t *qx, const float *sx, const int8_t *qw
 
 using namespace w8a8;
 
-extern "C" sq_status w8a8_gemm_dequant(const int8_t *qx, const float *sx, const int8_t *qw, const float *sw,
-                                       int64_t M, int64_t N, int64_t K, void *y, sq_dtype yt, int32_t *acc_out,
-                                       void *stream) {
-    if (M > 0 && N > 0 && (!qx || !sx || !qw || !sw || !y))
-        return fail(SQ_ERR_NULL, "w8a8_gemm_dequant: NULL pointer");
-    if (yt != SQ_F32 && yt != SQ_BF16) return fail(SQ_ERR_DTYPE, "w8a8_gemm_dequant: output dtype %d", (int)yt);
-    if (M < 0 || N < 0 || K <= 0 || K % 16 != 0 || K > 133144 || M > INT32_MAX || N > INT32_MAX)
-        return fail(SQ_ERR_SHAPE, "w8a8_gemm_dequant: M=%lld N=%lld K=%lld (K a multiple of 16 in [16, 133144])",
-                    (long long)M, (long long)N, (long long)K);
+// Argument checks and dispatch shared by the symmetric and asymmetric
+// entry points (rs/ow non-NULL: asymmetric weights).
+static sq_status gemm_entry(const char *fn, const int8_t *qx, const float *sx, const int32_t *rs, const int8_t *qw,
+                            const float *sw, const float *ow, int64_t M, int64_t N, int64_t K, void *y,
+                            sq_dtype yt, int32_t *acc_out, void *stream) {
+    const bool asym = rs != nullptr;
+    if (M > 0 && N > 0 && (!qx || !sx || !qw || !sw || !y || (asym && !ow)))
+        return fail(SQ_ERR_NULL, "%s: NULL pointer", fn);
+    if (yt != SQ_F32 && yt != SQ_BF16) return fail(SQ_ERR_DTYPE, "%s: output dtype %d", fn, (int)yt);
+    if (M < 0 || N < 0 || K <= 0 || K % 16 != 0 || K > (asym ? 65792 : 133144) || M > INT32_MAX || N > INT32_MAX)
+        return fail(SQ_ERR_SHAPE, "%s: M=%lld N=%lld K=%lld (K a multiple of 16 in [16, %d])", fn, (long long)M,
+                    (long long)N, (long long)K, asym ? 65792 : 133144);
     if (M == 0 || N == 0) return SQ_OK;
     const int out_vec = (yt == SQ_BF16) ? 8 : 4;
     if (N % out_vec != 0)
-        return fail(SQ_ERR_SHAPE, "w8a8_gemm_dequant: N=%lld must be a multiple of %d for this output dtype",
-                    (long long)N, out_vec);
-    if (acc_out && N % 4 != 0) return fail(SQ_ERR_SHAPE, "w8a8_gemm_dequant: acc_out needs N %% 4 == 0");
+        return fail(SQ_ERR_SHAPE, "%s: N=%lld must be a multiple of %d for this output dtype", fn, (long long)N,
+                    out_vec);
+    if (acc_out && N % 4 != 0) return fail(SQ_ERR_SHAPE, "%s: acc_out needs N %% 4 == 0", fn);
     if (!aligned(qx, 16) || !aligned(qw, 16) || !aligned(y, 16) || !aligned(sw, 16) || !aligned(sx, 4) ||
-        (acc_out && !aligned(acc_out, 16)))
-        return fail(SQ_ERR_ALIGN, "w8a8_gemm_dequant: misaligned pointer (qx, qw, y, sw, acc_out need 16 bytes)");
+        (acc_out && !aligned(acc_out, 16)) || (asym && (!aligned(ow, 16) || !aligned(rs, 4))))
+        return fail(SQ_ERR_ALIGN, "%s: misaligned pointer (qx, qw, y, sw, ow, acc_out need 16 bytes)", fn);
     int sms;
     sq_status st = check_device(&sms);
     if (st != SQ_OK) return st;
     cudaStream_t cs = (cudaStream_t)stream;
+    const int m = (int)M, n = (int)N, k = (int)K;
     // M > 128: 256-row tiles on CTA pairs; otherwise one CTA per 128 x 256 tile
     if (M > gemm::BM) {
         if (yt == SQ_BF16)
-            return gemm::launch_pair<__nv_bfloat16>(qx, sx, qw, sw, (int)M, (int)N, (int)K, y, acc_out, sms, cs);
-        return gemm::launch_pair<float>(qx, sx, qw, sw, (int)M, (int)N, (int)K, y, acc_out, sms, cs);
+            return asym ? gemm::launch_pair<__nv_bfloat16, true>(qx, sx, rs, qw, sw, ow, m, n, k, y, acc_out, sms, cs)
+                        : gemm::launch_pair<__nv_bfloat16, false>(qx, sx, rs, qw, sw, ow, m, n, k, y, acc_out, sms, cs);
+        return asym ? gemm::launch_pair<float, true>(qx, sx, rs, qw, sw, ow, m, n, k, y, acc_out, sms, cs)
+                    : gemm::launch_pair<float, false>(qx, sx, rs, qw, sw, ow, m, n, k, y, acc_out, sms, cs);
     }
     if (yt == SQ_BF16)
-        return gemm::launch<256, __nv_bfloat16>(qx, sx, qw, sw, (int)M, (int)N, (int)K, y, acc_out, sms, cs);
-    return gemm::launch<256, float>(qx, sx, qw, sw, (int)M, (int)N, (int)K, y, acc_out, sms, cs);
+        return asym ? gemm::launch<256, __nv_bfloat16, true>(qx, sx, rs, qw, sw, ow, m, n, k, y, acc_out, sms, cs)
+                    : gemm::launch<256, __nv_bfloat16, false>(qx, sx, rs, qw, sw, ow, m, n, k, y, acc_out, sms, cs);
+    return asym ? gemm::launch<256, float, true>(qx, sx, rs, qw, sw, ow, m, n, k, y, acc_out, sms, cs)
+                : gemm::launch<256, float, false>(qx, sx, rs, qw, sw, ow, m, n, k, y, acc_out, sms, cs);
+}
+
+extern "C" sq_status w8a8_gemm_dequant(const int8_t *qx, const float *sx, const int8_t *qw, const float *sw,
+                                       int64_t M, int64_t N, int64_t K, void *y, sq_dtype yt, int32_t *acc_out,
+                                       void *stream) {
+    return gemm_entry("w8a8_gemm_dequant", qx, sx, nullptr, qw, sw, nullptr, M, N, K, y, yt, acc_out, stream);
+}
+
+extern "C" sq_status w8a8_gemm_dequant_asym(const int8_t *qx, const float *sx, const int32_t *rowsum,
+                                            const int8_t *qw, const float *sw, const float *ow, int64_t M,
+                                            int64_t N, int64_t K, void *y, sq_dtype yt, int32_t *acc_out,
+                                            void *stream) {
+    if (M > 0 && N > 0 && !rowsum) return fail(SQ_ERR_NULL, "w8a8_gemm_dequant_asym: NULL pointer");
+    return gemm_entry("w8a8_gemm_dequant_asym", qx, sx, rowsum, qw, sw, ow, M, N, K, y, yt, acc_out, stream);
 }
 
 extern "C" sq_status sq_selftest_bounded_wait(uint32_t limit_ms, void *stream) {

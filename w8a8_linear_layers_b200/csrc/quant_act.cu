@@ -86,14 +86,19 @@ __device__ __forceinline__ uint2 fast_codes_tied(const float (&v)[8], float s, f
 // calibrated beforehand, see sq_static_range_update); no per-row reduction,
 // values beyond the range saturate, and scale[row] (if given) receives S so
 // that the GEMM's per-token dequant applies it unchanged.
+//
+// rowsum (nullable): R[row] = sum of the row's codes (exact), which the GEMM
+// with asymmetric weights needs.
 template <typename T, int E, int ROWS, bool STATIC>
 __global__ void __launch_bounds__(512)
 quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__restrict__ inv_s,
-                 const float *__restrict__ range, int8_t *__restrict__ q, float *__restrict__ scale) {
+                 const float *__restrict__ range, int8_t *__restrict__ q, float *__restrict__ scale,
+                 int32_t *__restrict__ rowsum) {
     constexpr int C = E / 8;  // chunks per thread
     // inv_s is kept in registers across rows unless that would spill
     constexpr bool kCacheInvS = C * ROWS <= 4;
     __shared__ float red[2][ROWS][32];
+    __shared__ int rsum_red[2][ROWS][32];
     const int T_ = blockDim.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = T_ >> 5;
 
@@ -175,6 +180,7 @@ quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__r
             const bool narrow = am * r < 16384.0f;
             const float tie_bound = 0.5f - fmaf(am * r, 4.76837158203125e-07f, 2.384185791015625e-07f);
             int8_t *qr = q + row * K;
+            int rsum = 0;
 #pragma unroll
             for (int c = 0; c < C; ++c) {
                 if (!live[c]) continue;
@@ -192,6 +198,22 @@ quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__r
                     code = fast_codes_tied(v, s, r, narrow, tie_bound);
                 }
                 *reinterpret_cast<uint2 *>(qr + ((int64_t)c * T_ + threadIdx.x) * 8) = code;
+                if (rowsum) rsum = __dp4a((int)code.y, 0x01010101, __dp4a((int)code.x, 0x01010101, rsum));
+            }
+            if (rowsum) {  // uniform: every thread of the CTA takes this branch
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) rsum += __shfl_xor_sync(0xffffffffu, rsum, o);
+                if (nwarps == 1) {
+                    if (lane == 0) rowsum[row] = rsum;
+                } else {
+                    if (lane == 0) rsum_red[parity][rr][warp] = rsum;
+                    __syncthreads();
+                    if (threadIdx.x == 0) {
+                        int t = 0;
+                        for (int w = 0; w < nwarps; ++w) t += rsum_red[parity][rr][w];
+                        rowsum[row] = t;
+                    }
+                }
             }
         }
     }
@@ -199,32 +221,32 @@ quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__r
 
 template <typename T, int E, int ROWS, bool STATIC>
 static void launch_quant_act(const void *x, int64_t M, int64_t K, const float *inv_s, const float *range,
-                             int8_t *q, float *scale, int sms, cudaStream_t st) {
+                             int8_t *q, float *scale, int32_t *rowsum, int sms, cudaStream_t st) {
     int threads = (int)ceil_div(ceil_div(K, E), 32) * 32;
     // enough CTAs to fill the machine; each strides over groups of ROWS rows
     int per_sm = std::max(1, std::min(32, 2048 / threads));
     int64_t grid = std::min<int64_t>(ceil_div(M, ROWS), (int64_t)sms * per_sm);
     quant_act_kernel<T, E, ROWS, STATIC>
-        <<<(unsigned)grid, threads, 0, st>>>((const T *)x, M, K, inv_s, range, q, scale);
+        <<<(unsigned)grid, threads, 0, st>>>((const T *)x, M, K, inv_s, range, q, scale, rowsum);
 }
 
 // E elements per thread: one warp per row up to K = 32 E, at most 64
 // elements per thread.
 template <bool STATIC>
 static void dispatch_quant(const void *x, bool bf, int64_t M, int64_t K, const float *inv_s, const float *range,
-                           int8_t *q, float *scale, int sms, cudaStream_t cs) {
+                           int8_t *q, float *scale, int32_t *rowsum, int sms, cudaStream_t cs) {
     if (K <= 256) {
-        if (bf) launch_quant_act<__nv_bfloat16, 8, 1, STATIC>(x, M, K, inv_s, range, q, scale, sms, cs);
-        else launch_quant_act<float, 8, 1, STATIC>(x, M, K, inv_s, range, q, scale, sms, cs);
+        if (bf) launch_quant_act<__nv_bfloat16, 8, 1, STATIC>(x, M, K, inv_s, range, q, scale, rowsum, sms, cs);
+        else launch_quant_act<float, 8, 1, STATIC>(x, M, K, inv_s, range, q, scale, rowsum, sms, cs);
     } else if (K <= 512) {
-        if (bf) launch_quant_act<__nv_bfloat16, 16, 1, STATIC>(x, M, K, inv_s, range, q, scale, sms, cs);
-        else launch_quant_act<float, 16, 1, STATIC>(x, M, K, inv_s, range, q, scale, sms, cs);
+        if (bf) launch_quant_act<__nv_bfloat16, 16, 1, STATIC>(x, M, K, inv_s, range, q, scale, rowsum, sms, cs);
+        else launch_quant_act<float, 16, 1, STATIC>(x, M, K, inv_s, range, q, scale, rowsum, sms, cs);
     } else if (K <= 1024) {
-        if (bf) launch_quant_act<__nv_bfloat16, 32, 1, STATIC>(x, M, K, inv_s, range, q, scale, sms, cs);
-        else launch_quant_act<float, 32, 1, STATIC>(x, M, K, inv_s, range, q, scale, sms, cs);
+        if (bf) launch_quant_act<__nv_bfloat16, 32, 1, STATIC>(x, M, K, inv_s, range, q, scale, rowsum, sms, cs);
+        else launch_quant_act<float, 32, 1, STATIC>(x, M, K, inv_s, range, q, scale, rowsum, sms, cs);
     } else {
-        if (bf) launch_quant_act<__nv_bfloat16, 64, 1, STATIC>(x, M, K, inv_s, range, q, scale, sms, cs);
-        else launch_quant_act<float, 64, 1, STATIC>(x, M, K, inv_s, range, q, scale, sms, cs);
+        if (bf) launch_quant_act<__nv_bfloat16, 64, 1, STATIC>(x, M, K, inv_s, range, q, scale, rowsum, sms, cs);
+        else launch_quant_act<float, 64, 1, STATIC>(x, M, K, inv_s, range, q, scale, rowsum, sms, cs);
     }
 }
 
@@ -257,7 +279,15 @@ using namespace w8a8;
 extern "C" sq_status quant_act_per_token(const void *x, sq_dtype xt, int64_t M, int64_t K,
                                          const float *inv_s, int8_t *q_out, float *scale_out,
                                          void *stream) {
+    return quant_act_per_token_rowsum(x, xt, M, K, inv_s, q_out, scale_out, nullptr, stream);
+}
+
+extern "C" sq_status quant_act_per_token_rowsum(const void *x, sq_dtype xt, int64_t M, int64_t K,
+                                                const float *inv_s, int8_t *q_out, float *scale_out,
+                                                int32_t *rowsum_out, void *stream) {
     if (M > 0 && (!x || !q_out || !scale_out)) return fail(SQ_ERR_NULL, "quant_act_per_token: NULL pointer");
+    if (rowsum_out && !aligned(rowsum_out, 4))
+        return fail(SQ_ERR_ALIGN, "quant_act_per_token: misaligned rowsum_out");
     if (xt != SQ_F32 && xt != SQ_BF16) return fail(SQ_ERR_DTYPE, "quant_act_per_token: dtype %d", (int)xt);
     if (M < 0 || K <= 0 || K % 16 != 0 || K > 32768)
         return fail(SQ_ERR_SHAPE, "quant_act_per_token: M=%lld K=%lld (K must be a multiple of 16 in [16, 32768])",
@@ -269,7 +299,7 @@ extern "C" sq_status quant_act_per_token(const void *x, sq_dtype xt, int64_t M, 
     sq_status st = check_device(&sms);
     if (st != SQ_OK) return st;
     cudaStream_t cs = (cudaStream_t)stream;
-    dispatch_quant<false>(x, xt == SQ_BF16, M, K, inv_s, nullptr, q_out, scale_out, sms, cs);
+    dispatch_quant<false>(x, xt == SQ_BF16, M, K, inv_s, nullptr, q_out, scale_out, rowsum_out, sms, cs);
     return launch_status("quant_act_kernel");
 }
 
@@ -302,6 +332,7 @@ extern "C" sq_status quant_act_static(const void *x, sq_dtype xt, int64_t M, int
     int sms;
     sq_status st = check_device(&sms);
     if (st != SQ_OK) return st;
-    dispatch_quant<true>(x, xt == SQ_BF16, M, K, inv_s, range, q_out, scale_out, sms, (cudaStream_t)stream);
+    dispatch_quant<true>(x, xt == SQ_BF16, M, K, inv_s, range, q_out, scale_out, nullptr, sms,
+                         (cudaStream_t)stream);
     return launch_status("quant_act_kernel");
 }

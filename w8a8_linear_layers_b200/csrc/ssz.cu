@@ -44,50 +44,12 @@
 // codes did not move, every warp takes the (identical) decision itself after
 // one barrier, and the next candidate is computed alongside the error.
 #include "common.cuh"
+#include "dd.cuh"
 
 namespace w8a8 {
 
 constexpr double kSszThreshold = 1e-10;
 constexpr float kSszMinScale = 1e-5f;
-
-// ------------------------------------------------------------ double-double
-struct dd {
-    double hi, lo;
-};
-
-__device__ __forceinline__ dd two_sum(double a, double b) {
-    const double s = a + b;
-    const double bb = s - a;
-    return {s, (a - (s - bb)) + (b - bb)};
-}
-
-// a += b (b a double-double), cascaded: exact in hi/lo pairs up to the
-// rounding of the small lo sum.  TwoSum's error term is exact and symmetric
-// in its arguments, so butterfly reductions give identical results on all
-// lanes.
-__device__ __forceinline__ dd dd_add_cascade(dd a, dd b) {
-    const dd s = two_sum(a.hi, b.hi);
-    return {s.hi, (a.lo + b.lo) + s.lo};
-}
-
-__device__ __forceinline__ void dd_acc(dd &a, double t) {
-    const dd s = two_sum(a.hi, t);
-    a.hi = s.hi;
-    a.lo += s.lo;
-}
-
-__device__ __forceinline__ dd warp_sum_dd(dd a) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        a = dd_add_cascade(a, {__shfl_xor_sync(0xffffffffu, a.hi, o), __shfl_xor_sync(0xffffffffu, a.lo, o)});
-    return a;
-}
-
-__device__ __forceinline__ int warp_sum_i(int v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
 
 // K e(c) = W2 - 2 c NUM + c^2 DEN, exact up to one final rounding.  The
 // search compares these K-scaled errors directly (K > 0 cancels), and
