@@ -82,6 +82,8 @@ def _L():
             "oracle_ssz_quant_weight_asym": [P, I64, I64, I, P, P, P, P, P, P],
             "oracle_channel_mse_asym": [P, I64, ctypes.c_float, ctypes.c_float],
             "oracle_act_rowsum": [P, I64, I64, P],
+            "oracle_pack_int4": [P, I64, I64, P],
+            "oracle_unpack_int4": [P, I64, I64, P],
             "oracle_dequant_asym": [P, P, P, P, P, I64, I64, P, P],
             "oracle_static_ema": [ctypes.c_float, ctypes.c_float, ctypes.c_float, I],
             "oracle_quant_act_static": [P, I64, I64, P, ctypes.c_float, P],
@@ -228,6 +230,23 @@ def ssz_quant_weight_asym(w, max_iters: int = SSZ_ITERS, s=None, trace: bool = F
 def channel_mse_asym(w_row, S, m) -> float:
     w_row = _f32(w_row)
     return float(_L().oracle_channel_mse_asym(_ptr(w_row), w_row.shape[0], float(S), float(m)))
+
+
+def pack_int4(q) -> np.ndarray:
+    """Two int4 codes per byte: element 2i low nibble, 2i+1 high nibble."""
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    N, K = q.shape
+    out = np.empty((N, K // 2), np.uint8)
+    _L().oracle_pack_int4(_ptr(q), N, K, _ptr(out))
+    return out
+
+
+def unpack_int4(packed, K: int) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    N = packed.shape[0]
+    out = np.empty((N, K), np.int8)
+    _L().oracle_unpack_int4(_ptr(packed), N, K, _ptr(out))
+    return out
 
 
 def act_rowsum(qx) -> np.ndarray:

@@ -507,6 +507,33 @@ void oracle_dequant(const int32_t *acc, const float *sx, const float *sw,
         }
 }
 
+/* ------------------------------------------------------- packed int4 */
+/* Two int4 codes per byte (SURVEY next row: packed int4 weights; the int4
+ * codes themselves are the SSZ page's int4 per-channel symmetric case).
+ * Reading: element 2i in the low nibble, 2i+1 in the high nibble, each in
+ * 4-bit two's complement; codes must lie in [-8, 7].  K is even. */
+void oracle_pack_int4(const int8_t *q, int64_t N, int64_t K, uint8_t *packed)
+{
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t i = 0; i < K / 2; ++i) {
+            unsigned lo = (unsigned)(q[n * K + 2 * i] & 0x0F);
+            unsigned hi = (unsigned)(q[n * K + 2 * i + 1] & 0x0F);
+            packed[n * (K / 2) + i] = (uint8_t)(lo | (hi << 4));
+        }
+}
+
+/* The inverse: sign-extend each nibble back to an int8 code. */
+void oracle_unpack_int4(const uint8_t *packed, int64_t N, int64_t K, int8_t *q)
+{
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t i = 0; i < K / 2; ++i) {
+            int b = packed[n * (K / 2) + i];
+            int lo = b & 0x0F, hi = (b >> 4) & 0x0F;
+            q[n * K + 2 * i] = (int8_t)(lo >= 8 ? lo - 16 : lo);
+            q[n * K + 2 * i + 1] = (int8_t)(hi >= 8 ? hi - 16 : hi);
+        }
+}
+
 /* Row sums R_t = sum_k qx[t,k] of the activation codes (exact). */
 void oracle_act_rowsum(const int8_t *qx, int64_t M, int64_t K, int32_t *R)
 {

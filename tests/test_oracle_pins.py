@@ -420,6 +420,32 @@ def test_act_rowsum_and_asym_dequant(orc):
     np.testing.assert_allclose(y, ref, rtol=1e-5, atol=1e-6 * np.abs(ref).max())
 
 
+# ------------------------------------------------- packed int4
+def test_pack_int4_layout_and_round_trip(orc):
+    # golden nibble layout: element 2i low, 2i+1 high, two's complement
+    q = np.array([[1, -1, 7, -8, 0, 3, -2, 5]], np.int8)
+    np.testing.assert_array_equal(orc.pack_int4(q)[0], np.array([0xF1, 0x87, 0x30, 0x5E], np.uint8))
+    r = np.random.default_rng(50)
+    q = r.integers(-8, 8, (13, 96)).astype(np.int8)
+    p = orc.pack_int4(q)
+    np.testing.assert_array_equal(p, ((q[:, 0::2].astype(np.int32) & 15) | ((q[:, 1::2].astype(np.int32) & 15) << 4)))
+    np.testing.assert_array_equal(orc.unpack_int4(p, 96), q)
+    # every byte value unpacks to a pair in [-8, 7] and packs back to itself
+    allb = np.arange(256, dtype=np.uint8)[None, :]
+    u = orc.unpack_int4(allb, 512)
+    assert u.min() == -8 and u.max() == 7
+    np.testing.assert_array_equal(orc.pack_int4(u), allb)
+
+
+def test_w4a8_product_equals_int8_product_of_the_codes(orc):
+    # the W4A8 GEMM is the int8 GEMM of the unpacked codes
+    r = np.random.default_rng(51)
+    qx = r.integers(-127, 128, (5, 64)).astype(np.int8)
+    q4 = r.integers(-7, 8, (9, 64)).astype(np.int8)
+    acc = orc.gemm_i8(qx, orc.unpack_int4(orc.pack_int4(q4), 64))
+    np.testing.assert_array_equal(acc, qx.astype(np.int64) @ q4.astype(np.int64).T)
+
+
 # ------------------------------------------------- static activation scale
 # "PaddleNLP GPT 量化感知训练（QAT）实战指南" section 六 (moving_average_abs_max)
 # and the CUDA INT8 notes section 2.1 (range calibration, saturation).
