@@ -288,7 +288,9 @@ def time_next_rows(args, w, torch, probs, flush, stream, reps=50):
     - quant_act_static: codes at a static per-tensor scale (range calibrated
       beforehand on the same activations);
     - ssz_quant_weight_asym, quant_act_per_token_rowsum and
-      w8a8_gemm_dequant_asym: the asymmetric int8 weight path.
+      w8a8_gemm_dequant_asym: the asymmetric int8 weight path;
+    - sq_pack_int4 and w4a8_gemm_dequant (packed int4 weights) against
+      w8a8_gemm_dequant on the 16 x 8192 -> 28672 decode shape.
     Per-launch times include the launch gap that in-step events hide."""
     p = probs[0]
     peaks, _ = load_peaks()
@@ -346,6 +348,35 @@ def time_next_rows(args, w, torch, probs, flush, stream, reps=50):
         out["w8a8_gemm_dequant_asym"] = {"us": round(ms * 1e3, 2), "bound": "tensor", "achieved": round(tops, 1),
                                          "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(tops / peak, 4),
                                          "shape": [p.M, p.N, p.K]}
+
+    # packed int4 weights on the decode shape (16 tokens, 8192 -> 28672),
+    # where the GEMM is bound by the weight bytes: W4A8 against W8A8 on the
+    # same codes (random codes, the kernels' speed does not depend on them)
+    Md, Kd, Nd = 16, 8192, 28672
+    g = torch.Generator(device=dev).manual_seed(0)
+    qxd = torch.randint(-127, 128, (Md, Kd), device=dev, dtype=torch.int8, generator=g)
+    q4 = torch.randint(-7, 8, (Nd, Kd), device=dev, dtype=torch.int8, generator=g)
+    sxd = torch.rand(Md, device=dev, generator=g) * 1e-2
+    swd = torch.rand(Nd, device=dev, generator=g) * 1e-2
+    packed = torch.empty(Nd, Kd // 2, device=dev, dtype=torch.uint8)
+    w.sq_pack_int4(q4, packed)
+    yd = torch.empty(Md, Nd, device=dev, dtype=torch.bfloat16)
+    for name, fn, wbytes in (("w8a8_gemm_dequant_decode", lambda: w.w8a8_gemm_dequant(qxd, sxd, q4, swd, yd), Nd * Kd),
+                             ("w4a8_gemm_dequant_decode", lambda: w.w4a8_gemm_dequant(qxd, sxd, packed, swd, yd),
+                              Nd * Kd // 2)):
+        ms = timed(fn)
+        nbytes = Md * Kd + wbytes + 2 * Md * Nd + 4 * Md + 4 * Nd
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[name] = {"us": round(ms * 1e3, 2), "bound": "hbm", "achieved": round(gbs, 1),
+                     "peak": round(peaks["hbm_gbs"], 1), "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                     "algorithmic": {"bytes": nbytes, "ops": 2 * Md * Nd * Kd}, "shape": [Md, Nd, Kd]}
+    ms = timed(lambda: w.sq_pack_int4(q4, packed))
+    nbytes = Nd * Kd + Nd * Kd // 2
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    out["sq_pack_int4"] = {"us": round(ms * 1e3, 2), "bound": "hbm", "achieved": round(gbs, 1),
+                           "peak": round(peaks["hbm_gbs"], 1), "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                           "shape": [Nd, Kd]}
+    del q4, packed, qxd, yd
     return out
 
 

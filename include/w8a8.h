@@ -83,7 +83,7 @@ int sq_abi_version(void);
  * naming the wait.  Synchronizes `stream`.  Kernels never trap: a wait that
  * runs out of time records its code here and the kernel returns.  Codes:
  * 1 GEMM producer, 2 GEMM MMA (operands), 3 GEMM MMA (accumulator buffer),
- * 4 GEMM epilogue, 6 sq_selftest_bounded_wait. */
+ * 4 GEMM epilogue, 6 sq_selftest_bounded_wait, 7 W4A8 GEMM unpacking. */
 sq_status sq_device_fault(void *stream, uint32_t *fault_out /* host */);
 
 /* Test hook for the bounded waits: launches one CTA that waits, with the same
@@ -189,6 +189,24 @@ sq_status w8a8_gemm_dequant_asym(const int8_t *qx, const float *sx, const int32_
                                  const int8_t *qw, const float *sw, const float *ow, int64_t M,
                                  int64_t N, int64_t K, void *y, sq_dtype yt, int32_t *acc_out,
                                  void *stream);
+
+/* ------------------------------------------ packed int4 weights (next)
+ * int4 codes (ssz_quant_weight with bits = 4, range [-7, 7]) stored two per
+ * byte, and a GEMM that reads them packed: half the weight bytes.  The pages
+ * have int4 per-channel SSZ but no int4 GEMM; this row is this library's.
+ *
+ * sq_pack_int4: packed[n, i] = (q[n,2i] & 15) | (q[n,2i+1] & 15) << 4
+ * (element 2i in the low nibble, 4-bit two's complement; codes must lie in
+ * [-8, 7]).  q: [N,K] int8; packed: [N, K/2] bytes; K a multiple of 32. */
+sq_status sq_pack_int4(const int8_t *q, int64_t N, int64_t K, uint8_t *packed, void *stream);
+
+/* w4a8_gemm_dequant: w8a8_gemm_dequant with the weight codes packed by
+ * sq_pack_int4 (qw4: [N, K/2] bytes, 16-byte aligned).  The codes are
+ * unpacked on chip; acc and y are exactly those of w8a8_gemm_dequant on
+ * the unpacked codes.  K a multiple of 32. */
+sq_status w4a8_gemm_dequant(const int8_t *qx, const float *sx, const uint8_t *qw4, const float *sw,
+                            int64_t M, int64_t N, int64_t K, void *y, sq_dtype yt, int32_t *acc_out,
+                            void *stream);
 
 /* ------------------------------------------- static activation scale (next)
  * A per-tensor activation range calibrated offline instead of the per-token

@@ -26,7 +26,7 @@ def lib():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(sq_\w+|ssz_\w+|quant_\w+|w8a8_\w+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(sq_\w+|ssz_\w+|quant_\w+|w8a8_\w+|w4a8_\w+)\s*\(", text)))
 
 
 def test_header_declares_the_five_steps():
@@ -144,6 +144,20 @@ def test_gemm_asym_rejects(lib, case, status):
     rc = lib.w8a8_gemm_dequant_asym(a["qx"], a["sx"], a["rs"], a["qw"], a["sw"], a["ow"], a["M"], a["N"], a["K"],
                                     a["y"], 1, NULL, None)
     assert rc == status, _detail(lib)
+
+
+@pytest.mark.parametrize("case,status", [("null", 1), ("k16", 2), ("align", 4), ("dtype", 3)])
+def test_w4a8_rejects(lib, case, status):
+    a = dict(qx=P(), sx=P(4096), qw=P(8192), sw=P(12288), M=4, N=16, K=64, y=P(16384), yt=1)
+    if case == "null": a["qw"] = NULL
+    if case == "k16": a["K"] = 48
+    if case == "align": a["qw"] = P(8200)
+    if case == "dtype": a["yt"] = 2
+    rc = lib.w4a8_gemm_dequant(a["qx"], a["sx"], a["qw"], a["sw"], a["M"], a["N"], a["K"], a["y"], a["yt"], NULL,
+                               None)
+    assert rc == status, _detail(lib)
+    assert lib.sq_pack_int4(P(), 4, 48, P(4096), None) == 2
+    assert lib.sq_pack_int4(P(), 4, 64, NULL, None) == 1
 
 
 def test_quant_rowsum_rejects_misaligned(lib):

@@ -27,7 +27,7 @@ EXPORTS = ["sq_status_string", "sq_last_error_detail", "sq_abi_version", "sq_dev
            "sq_selftest_bounded_wait",
            "sq_calib_absmax", "sq_smooth_fold", "ssz_quant_weight", "quant_act_per_token",
            "w8a8_gemm_dequant", "sq_static_range_update", "quant_act_static", "quant_act_per_token_rowsum",
-           "ssz_quant_weight_asym", "w8a8_gemm_dequant_asym"]
+           "ssz_quant_weight_asym", "w8a8_gemm_dequant_asym", "sq_pack_int4", "w4a8_gemm_dequant"]
 
 
 class W8A8Error(RuntimeError):
@@ -60,6 +60,8 @@ def _load() -> ctypes.CDLL:
         "quant_act_per_token_rowsum": ([P, I, I64, I64, P, P, P, P, P], I),
         "ssz_quant_weight_asym": ([P, I, I64, I64, P, I, P, P, P, P, P, P], I),
         "w8a8_gemm_dequant_asym": ([P, P, P, P, P, P, I64, I64, I64, P, I, P, P], I),
+        "sq_pack_int4": ([P, I64, I64, P, P], I),
+        "w4a8_gemm_dequant": ([P, P, P, P, I64, I64, I64, P, I, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -214,6 +216,28 @@ def w8a8_gemm_dequant_asym(qx: torch.Tensor, sx: torch.Tensor, rowsum: torch.Ten
     _check("w8a8_gemm_dequant_asym",
            lib.w8a8_gemm_dequant_asym(_ptr(qx), _ptr(sx), _ptr(rowsum), _ptr(qw), _ptr(sw), _ptr(ow), M, N, K,
                                       _ptr(y), _dtype(y), _ptr(acc_out), _stream(stream)))
+
+
+def sq_pack_int4(q: torch.Tensor, packed: torch.Tensor, stream=None) -> None:
+    """Two int4 codes per byte (element 2i in the low nibble)."""
+    _need(q, torch.int8, "q")
+    _need(packed, torch.uint8, "packed")
+    N, K = q.shape
+    _check("sq_pack_int4", lib.sq_pack_int4(_ptr(q), N, K, _ptr(packed), _stream(stream)))
+
+
+def w4a8_gemm_dequant(qx: torch.Tensor, sx: torch.Tensor, qw4: torch.Tensor, sw: torch.Tensor, y: torch.Tensor,
+                      acc_out: torch.Tensor | None = None, stream=None) -> None:
+    """GEMM + dequant with packed int4 weight codes qw4 [N, K/2]."""
+    _need(qx, torch.int8, "qx")
+    _need(qw4, torch.uint8, "qw4")
+    _need(sx, torch.float32, "sx")
+    _need(sw, torch.float32, "sw")
+    _need(acc_out, torch.int32, "acc_out")
+    M, K = qx.shape
+    N = qw4.shape[0]
+    _check("w4a8_gemm_dequant", lib.w4a8_gemm_dequant(_ptr(qx), _ptr(sx), _ptr(qw4), _ptr(sw), M, N, K, _ptr(y),
+                                                       _dtype(y), _ptr(acc_out), _stream(stream)))
 
 
 STATIC_RANGE_RATE = 0.9  # moving rate of the static activation range (not given by the pages)

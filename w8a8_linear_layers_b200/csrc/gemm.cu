@@ -56,6 +56,7 @@ enum : unsigned {
     kFaultEpilogue = 4,
     kFaultDrain = 5,
     kFaultSelftest = 6,
+    kFaultConvert = 7,
 };
 
 // ------------------------------------------------------------ PTX wrappers
@@ -768,6 +769,305 @@ w8a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_c
     }
 }
 
+// ============================================================ W4A8 kernel
+// Weights as packed int4 (two codes per byte, element 2i in the low nibble,
+// 4-bit two's complement).  Per stage TMA brings the A tile (int8, 128-byte
+// swizzle) and the packed B tile (256 rows x 64 bytes, no swizzle); eight
+// converter warps unpack B into int8 codes in the 128B-swizzled K-major layout
+// the MMA reads (16-byte chunk c of row r at chunk c ^ (r & 7) of its
+// 1024-byte row group), fence their writes to the async proxy and arrive on
+// conv[s]; the MMA warp then runs the int8 MMAs of w8a8_gemm_kernel.  The
+// weight bytes read from HBM are halved; the tensor-core work is the same.
+constexpr int kConvWarps = 8;
+constexpr int kThreadsW4 = (6 + kConvWarps) * 32;  // TMA, MMA, 4 epilogue and 8 converter warps
+
+// Two rings: IN_STAGES input stages (A by TMA, 128-byte swizzle, and the
+// packed B tile, 32 KB together) run ahead of OP_STAGES unpacked B buffers
+// (32 KB each), so that loads from HBM do not wait on the conversion; the MMA
+// reads A from the input stage and B from the operand buffer and releases
+// both.
+struct CfgW4 {
+    static constexpr int BN = 256;
+    static constexpr int IN_STAGES = 5;
+    static constexpr int OP_STAGES = 2;
+    static constexpr int A_BYTES = BM * BK;        // 16 KB int8 activations
+    static constexpr int B_BYTES = BN * BK;        // 32 KB unpacked int8 weights
+    static constexpr int RAW_BYTES = BN * BK / 2;  // 16 KB packed int4 weights
+    static constexpr int IN_BYTES = A_BYTES + RAW_BYTES;
+    static constexpr int IN_OFFSET = OP_STAGES * B_BYTES;
+    static constexpr int TMEM_COLS = 2 * BN;
+    static constexpr int SMEM = IN_OFFSET + IN_STAGES * IN_BYTES + 1024;
+};
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 8 int4 codes (one 32-bit word, element 2i in the low nibble of byte i) to
+// 8 int8 codes.  A nibble x sign-extends as ((x ^ 8) + 0x78) ^ 0x80: every
+// byte stays below 0x88 before the last step, so one 32-bit add serves four
+// bytes without carries.  Low and high nibble values are then interleaved.
+__device__ __forceinline__ void unpack_int4x8(uint32_t w, uint32_t &o0, uint32_t &o1) {
+    const uint32_t lo = (((w & 0x0F0F0F0Fu) ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
+    const uint32_t hi = ((((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
+    o0 = __byte_perm(lo, hi, 0x5140);
+    o1 = __byte_perm(lo, hi, 0x7362);
+}
+
+// Synchronisation (no block-level barrier in the main loop):
+//   in_full[s]  : producer's expect_tx; the A and packed-B TMAs complete it.
+//   in_empty[s] : MMA commit (the MMA is the last reader of A; the
+//                 converters are done with the packed tile before op_full).
+//   op_full[p]  : one arrival per converter thread after its fenced writes.
+//   op_empty[p] : MMA commit.
+template <typename OutT>
+__global__ void __launch_bounds__(kThreadsW4, 1)
+w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b4,
+                 const float *__restrict__ sx, const float *__restrict__ sw, OutT *__restrict__ y,
+                 int32_t *__restrict__ acc_out, int M, int N, int K) {
+    using C = CfgW4;
+    constexpr int BNw = C::BN;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t in_full[C::IN_STAGES];
+    __shared__ __align__(8) uint64_t in_empty[C::IN_STAGES];
+    __shared__ __align__(8) uint64_t op_full[C::OP_STAGES];
+    __shared__ __align__(8) uint64_t op_empty[C::OP_STAGES];
+    __shared__ __align__(8) uint64_t tfull_bar[2];
+    __shared__ __align__(8) uint64_t tempty_bar[2];
+    __shared__ __align__(8) uint64_t drain_bar;
+    __shared__ uint32_t tmem_slot;
+    __shared__ volatile int abort_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;  // 1024-aligned for 128B swizzle
+    uint8_t *gbase = smem_raw + (smem_base - smem_u32(smem_raw));      // the same bytes, generic address
+
+    const int tiles_m = (M + BM - 1) / BM;
+    const int tiles_n = (N + BNw - 1) / BNw;
+    const int num_tiles = tiles_m * tiles_n;
+    const int num_kb = (K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::IN_STAGES; ++s) {
+            mbar_init(smem_u32(&in_full[s]), 1);
+            mbar_init(smem_u32(&in_empty[s]), 1);
+        }
+        for (int s = 0; s < C::OP_STAGES; ++s) {
+            mbar_init(smem_u32(&op_full[s]), kConvWarps * 32);
+            mbar_init(smem_u32(&op_empty[s]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&tfull_bar[b]), 1);
+            mbar_init(smem_u32(&tempty_bar[b]), 4 * 32);
+        }
+        mbar_init(smem_u32(&drain_bar), 1);
+        abort_flag = 0;
+        fence_barrier_init();
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tmap_a) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tmap_b4) : "memory");
+    }
+    if (warp == 1) tmem_alloc(smem_u32(&tmem_slot), C::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (A + packed B)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int m0 = (tile % tiles_m) * BM, n0 = (tile / tiles_m) * BNw;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!wait_bounded(smem_u32(&in_empty[stage]), phase ^ 1u, &abort_flag, kFaultProducer)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t a_dst = smem_base + C::IN_OFFSET + stage * C::IN_BYTES;
+                    const uint32_t fb = smem_u32(&in_full[stage]);
+                    mbar_arrive_expect_tx(fb, C::IN_BYTES);
+                    tma_load_2d(a_dst, &tmap_a, fb, kb * BK, m0);
+                    tma_load_2d(a_dst + C::A_BYTES, &tmap_b4, fb, kb * (BK / 2), n0);
+                    ++issued;
+                    if (++stage == C::IN_STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                int outstanding = issued < C::IN_STAGES ? issued : C::IN_STAGES;
+                int s = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < outstanding; ++i) {
+                    if (--s < 0) {
+                        s = C::IN_STAGES - 1;
+                        ph ^= 1u;
+                    }
+                    const unsigned long long t0 = globaltimer();
+                    while (!mbar_try_wait(smem_u32(&in_full[s]), ph) && globaltimer() - t0 < kWaitNs) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_i8(BM, BNw);
+            int stage = 0, istage = 0;
+            uint32_t phase = 0;
+            int buf = 0;
+            uint32_t buf_phase = 0;
+            bool ok = true;
+            bool issued_any = false;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                if (!wait_bounded(smem_u32(&tempty_bar[buf]), buf_phase ^ 1u, &abort_flag, kFaultMmaTmemEmpty)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BNw);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    // op_full implies in_full: the converters waited for it
+                    if (!wait_bounded(smem_u32(&op_full[stage]), phase, &abort_flag, kFaultMmaFull)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_base + C::IN_OFFSET + istage * C::IN_BYTES;
+                    const uint32_t b_addr = smem_base + stage * C::B_BYTES;
+#pragma unroll
+                    for (int k = 0; k < BK / UMMA_K; ++k) {
+                        mma_i8(d_tmem, smem_desc_sw128(a_addr + k * UMMA_K), smem_desc_sw128(b_addr + k * UMMA_K),
+                               idesc, (kb | k) != 0 ? 1u : 0u);
+                    }
+                    issued_any = true;
+                    mma_commit(smem_u32(&op_empty[stage]));
+                    mma_commit(smem_u32(&in_empty[istage]));
+                    if (++stage == C::OP_STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                    if (++istage == C::IN_STAGES) istage = 0;
+                }
+                if (!ok) break;
+                mma_commit(smem_u32(&tfull_bar[buf]));
+                buf ^= 1;
+                if (buf == 0) buf_phase ^= 1u;
+            }
+            if (!ok && issued_any) {
+                mma_commit(smem_u32(&drain_bar));
+                const unsigned long long t0 = globaltimer();
+                while (!mbar_try_wait(smem_u32(&drain_bar), 0) && globaltimer() - t0 < kWaitNs) {
+                }
+            }
+        }
+    } else if (warp >= 6) {
+        // ------------------------------------------------ converters (warps 6..13)
+        // Per k-block every converter thread waits for a free operand buffer
+        // and for the input stage, unpacks its share of the packed tile into
+        // the buffer, fences the writes to the async proxy and arrives on
+        // op_full.
+        const int cw = warp - 6;
+        const int rsub = lane >> 2, sub = lane & 3;   // 8 rows x 4 lanes of 16 packed bytes per warp step
+        int rs = 0, os = 0;
+        uint32_t rph = 0, oph = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            for (int kb = 0; kb < num_kb; ++kb) {
+                if (!wait_bounded(smem_u32(&op_empty[os]), oph ^ 1u, &abort_flag, kFaultConvert)) {
+                    ok = false;
+                    break;
+                }
+                if (!wait_bounded(smem_u32(&in_full[rs]), rph, &abort_flag, kFaultConvert)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t *raw = gbase + C::IN_OFFSET + rs * C::IN_BYTES + C::A_BYTES;
+                uint8_t *bdst = gbase + os * C::B_BYTES;
+#pragma unroll 2
+                for (int it = 0; it < BNw / (8 * kConvWarps); ++it) {
+                    const int r = (it * kConvWarps + cw) * 8 + rsub;
+                    const uint4 p = *reinterpret_cast<const uint4 *>(raw + r * (BK / 2) + sub * 16);
+                    uint32_t o[8];
+                    unpack_int4x8(p.x, o[0], o[1]);
+                    unpack_int4x8(p.y, o[2], o[3]);
+                    unpack_int4x8(p.z, o[4], o[5]);
+                    unpack_int4x8(p.w, o[6], o[7]);
+                    uint8_t *rowp = bdst + (r >> 3) * 1024 + (r & 7) * 128;
+                    const int c0 = 2 * sub, c1 = 2 * sub + 1;
+                    *reinterpret_cast<uint4 *>(rowp + ((c0 ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<uint4 *>(rowp + ((c1 ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+                }
+                fence_proxy_async_smem();  // the MMA reads these bytes through the async proxy
+                mbar_arrive(smem_u32(&op_full[os]));
+                if (++rs == C::IN_STAGES) {
+                    rs = 0;
+                    rph ^= 1u;
+                }
+                if (++os == C::OP_STAGES) {
+                    os = 0;
+                    oph ^= 1u;
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue (warps 2..5)
+        const int quarter = warp & 3;
+        const int row_in_tile = quarter * 32 + lane;
+        int buf = 0;
+        uint32_t buf_phase = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+            const int m0 = (tile % tiles_m) * BM, n0 = (tile / tiles_m) * BNw;
+            const int row = m0 + row_in_tile;
+            const float sxr = row < M ? sx[row] : 0.0f;
+            const bool ok = wait_bounded(smem_u32(&tfull_bar[buf]), buf_phase, &abort_flag, kFaultEpilogue);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BNw);
+            epilogue_tile<OutT, false>(tbase, row, M, n0, N, sxr, 0, sw, nullptr, y, acc_out, BNw);
+            tc_fence_before();
+            mbar_arrive(smem_u32(&tempty_bar[buf]));
+            buf ^= 1;
+            if (buf == 0) buf_phase ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// Packs int8 codes in [-8, 7] two per byte (element 2i in the low nibble);
+// one thread per 8 output bytes.
+__global__ void pack_int4_kernel(const int8_t *__restrict__ q, int64_t total_out8, uint8_t *__restrict__ out) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total_out8;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const uint4 c = __ldg(reinterpret_cast<const uint4 *>(q) + i);  // 16 codes
+        const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+        uint32_t p[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t v = 0;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const uint32_t word = w[2 * h + (b >> 1)];
+                const uint32_t lo = (word >> (16 * (b & 1))) & 0xFu;
+                const uint32_t hi = (word >> (16 * (b & 1) + 8)) & 0xFu;
+                v |= (lo | (hi << 4)) << (8 * b);
+            }
+            p[h] = v;
+        }
+        reinterpret_cast<uint2 *>(out)[i] = make_uint2(p[0], p[1]);
+    }
+}
+
 // One CTA waits, with the same bounded wait the GEMM uses, on an mbarrier
 // that nothing ever arrives at: the wait must run out, record
 // kFaultSelftest and return, leaving the context usable.
@@ -808,6 +1108,43 @@ static bool make_map(CUtensorMap *map, const void *base, int64_t rows, int64_t K
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// Packed int4 weights [rows, K/2 bytes]: box [box_rows, 64 bytes] (BK codes),
+// no swizzle (the converter warps read it with plain loads).
+static bool make_map_int4(CUtensorMap *map, const void *base, int64_t rows, int64_t K, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+    cuuint32_t box[2] = {(cuuint32_t)(BK / 2), (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <typename OutT>
+static sq_status launch_w4(const int8_t *qx, const float *sx, const uint8_t *qw4, const float *sw, int M, int N,
+                           int K, void *y, int32_t *acc_out, int sms, cudaStream_t st) {
+    using C = CfgW4;
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, qx, M, K, BM) || !make_map_int4(&mb, qw4, N, K, C::BN))
+        return fail(SQ_ERR_CUDA, "w4a8_gemm_dequant: cuTensorMapEncodeTiled failed");
+    auto kern = w4a8_gemm_kernel<OutT>;
+    static int configured_dev[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !configured_dev[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e != cudaSuccess) return fail(SQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        configured_dev[dev] = 1;
+    }
+    const int tiles = ((M + BM - 1) / BM) * ((N + C::BN - 1) / C::BN);
+    const int grid = std::min(tiles, sms);
+    kern<<<grid, kThreadsW4, C::SMEM, st>>>(ma, mb, sx, sw, (OutT *)y, acc_out, M, N, K);
+    return launch_status("w4a8_gemm_kernel");
 }
 
 template <int BN, typename OutT, bool ASYM>
@@ -913,6 +1250,49 @@ extern "C" sq_status w8a8_gemm_dequant_asym(const int8_t *qx, const float *sx, c
                                             void *stream) {
     if (M > 0 && N > 0 && !rowsum) return fail(SQ_ERR_NULL, "w8a8_gemm_dequant_asym: NULL pointer");
     return gemm_entry("w8a8_gemm_dequant_asym", qx, sx, rowsum, qw, sw, ow, M, N, K, y, yt, acc_out, stream);
+}
+
+extern "C" sq_status w4a8_gemm_dequant(const int8_t *qx, const float *sx, const uint8_t *qw4, const float *sw,
+                                       int64_t M, int64_t N, int64_t K, void *y, sq_dtype yt, int32_t *acc_out,
+                                       void *stream) {
+    const char *fn = "w4a8_gemm_dequant";
+    if (M > 0 && N > 0 && (!qx || !sx || !qw4 || !sw || !y)) return fail(SQ_ERR_NULL, "%s: NULL pointer", fn);
+    if (yt != SQ_F32 && yt != SQ_BF16) return fail(SQ_ERR_DTYPE, "%s: output dtype %d", fn, (int)yt);
+    if (M < 0 || N < 0 || K <= 0 || K % 32 != 0 || K > 133144 || M > INT32_MAX || N > INT32_MAX)
+        return fail(SQ_ERR_SHAPE, "%s: M=%lld N=%lld K=%lld (K a multiple of 32 in [32, 133144])", fn, (long long)M,
+                    (long long)N, (long long)K);
+    if (M == 0 || N == 0) return SQ_OK;
+    const int out_vec = (yt == SQ_BF16) ? 8 : 4;
+    if (N % out_vec != 0)
+        return fail(SQ_ERR_SHAPE, "%s: N=%lld must be a multiple of %d for this output dtype", fn, (long long)N,
+                    out_vec);
+    if (acc_out && N % 4 != 0) return fail(SQ_ERR_SHAPE, "%s: acc_out needs N %% 4 == 0", fn);
+    if (!aligned(qx, 16) || !aligned(qw4, 16) || !aligned(y, 16) || !aligned(sw, 16) || !aligned(sx, 4) ||
+        (acc_out && !aligned(acc_out, 16)))
+        return fail(SQ_ERR_ALIGN, "%s: misaligned pointer (qx, qw4, y, sw, acc_out need 16 bytes)", fn);
+    int sms;
+    sq_status st = check_device(&sms);
+    if (st != SQ_OK) return st;
+    cudaStream_t cs = (cudaStream_t)stream;
+    if (yt == SQ_BF16)
+        return gemm::launch_w4<__nv_bfloat16>(qx, sx, qw4, sw, (int)M, (int)N, (int)K, y, acc_out, sms, cs);
+    return gemm::launch_w4<float>(qx, sx, qw4, sw, (int)M, (int)N, (int)K, y, acc_out, sms, cs);
+}
+
+extern "C" sq_status sq_pack_int4(const int8_t *q, int64_t N, int64_t K, uint8_t *packed, void *stream) {
+    if (N > 0 && (!q || !packed)) return fail(SQ_ERR_NULL, "sq_pack_int4: NULL pointer");
+    if (N < 0 || K <= 0 || K % 32 != 0)
+        return fail(SQ_ERR_SHAPE, "sq_pack_int4: N=%lld K=%lld (K a positive multiple of 32)", (long long)N,
+                    (long long)K);
+    if (N == 0) return SQ_OK;
+    if (!aligned(q, 16) || !aligned(packed, 16)) return fail(SQ_ERR_ALIGN, "sq_pack_int4: misaligned pointer");
+    int sms;
+    sq_status st = check_device(&sms);
+    if (st != SQ_OK) return st;
+    const int64_t units = N * K / 16;
+    const unsigned blocks = (unsigned)std::min<int64_t>(ceil_div(units, 256), 8LL * sms);
+    gemm::pack_int4_kernel<<<blocks, 256, 0, (cudaStream_t)stream>>>(q, units, packed);
+    return launch_status("pack_int4_kernel");
 }
 
 extern "C" sq_status sq_selftest_bounded_wait(uint32_t limit_ms, void *stream) {
