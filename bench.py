@@ -47,6 +47,8 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=20)
+    p.add_argument("--no-next-rows", action="store_true",
+                   help="skip the per-kernel timings of the rows beyond the five-step path")
     p.add_argument("--record-traffic", metavar="NCU_CSV",
                    help="read an ncu --csv capture (gpu__time_duration.sum, dram__bytes_read.sum, "
                         "dram__bytes_write.sum) of this workload and write profiles/dram_traffic.json")
@@ -272,7 +274,8 @@ def run_ours(args, rank, world, local_rank):
     ops_per_step = sum(2.0 * p.M * p.N * p.K for p in probs)
     value = ops_per_step * world * args.steps / (total_ms * 1e-3) / 1e12
 
-    next_rows = time_next_rows(args, w, torch, probs, flush, stream) if world == 1 else None
+    next_rows = (time_next_rows(args, w, torch, probs, flush, stream)
+                 if world == 1 and not args.no_next_rows else None)
 
     # ---- end to end through the C ABI with host buffers
     e2e = None
@@ -581,7 +584,8 @@ def run_reference(args, rank):
 
 # kernel name prefix in an ncu capture -> step of the path
 NCU_KERNELS = [("col_absmax_kernel", None), ("smooth_factor_kernel", "smooth_fold"), ("ssz_kernel", "ssz_quant_weight"),
-               ("quant_act_kernel", "quant_act_per_token"), ("w8a8_gemm_kernel", "w8a8_gemm_dequant")]
+               ("quant_act_kernel", "quant_act_per_token"), ("w8a8_gemm_kernel", "w8a8_gemm_dequant"),
+               ("w8a8_gemm_pair_kernel", "w8a8_gemm_dequant")]
 
 
 def record_traffic(csv_path, workload):
