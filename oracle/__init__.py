@@ -83,6 +83,7 @@ def _L():
             "oracle_channel_mse_asym": [P, I64, ctypes.c_float, ctypes.c_float],
             "oracle_act_rowsum": [P, I64, I64, P],
             "oracle_pack_int4": [P, I64, I64, P],
+            "oracle_layernorm_quant": [P, I64, I64, P, P, ctypes.c_float, P, P, P, P],
             "oracle_unpack_int4": [P, I64, I64, P],
             "oracle_dequant_asym": [P, P, P, P, P, I64, I64, P, P],
             "oracle_static_ema": [ctypes.c_float, ctypes.c_float, ctypes.c_float, I],
@@ -230,6 +231,21 @@ def ssz_quant_weight_asym(w, max_iters: int = SSZ_ITERS, s=None, trace: bool = F
 def channel_mse_asym(w_row, S, m) -> float:
     w_row = _f32(w_row)
     return float(_L().oracle_channel_mse_asym(_ptr(w_row), w_row.shape[0], float(S), float(m)))
+
+
+def layernorm_quant(h, gamma=None, beta=None, eps: float = 1e-5, inv_s=None):
+    """LayerNorm (fp64 statistics, fp32 output) of h [M,K] times inv_s, then
+    per-token int8 codes.  Returns (q, sx, y) with y the LayerNorm output."""
+    h = _f32(h)
+    M, K = h.shape
+    g = None if gamma is None else _f32(gamma)
+    b = None if beta is None else _f32(beta)
+    inv = None if inv_s is None else _f32(inv_s)
+    q = np.empty((M, K), np.int8)
+    sx = np.empty(M, np.float32)
+    y = np.empty((M, K), np.float32)
+    _L().oracle_layernorm_quant(_ptr(h), M, K, _ptr(g), _ptr(b), float(eps), _ptr(inv), _ptr(q), _ptr(sx), _ptr(y))
+    return q, sx, y
 
 
 def pack_int4(q) -> np.ndarray:

@@ -420,6 +420,57 @@ void oracle_quant_act_per_token(const float *x, int64_t M, int64_t K,
     }
 }
 
+/* ------------------------------------------- LayerNorm fused with step 4 */
+/* Activation quantization fused upstream: the smoothing 1/s folded into the
+ * LayerNorm that produces X (SmoothQuant page, section 1: the scaling is an
+ * equivalent transform; CUDA INT8 notes 4.2: fuse quantization with the
+ * neighbouring op so the intermediate never goes to memory).  Per row t of
+ * h [M,K]:
+ *     mu  = sum_j h_j / K,  var = sum_j (h_j - mu)^2 / K      (fp64, index order)
+ *     y_j = fp32(((h_j - mu) * (1 / sqrt(var + eps))) * gamma_j + beta_j)  (fp64)
+ *     x'_j = y_j * inv_s_j (fp32), then the per-token codes and scale of step 4.
+ * gamma, beta, inv_s nullable (1, 0, 1).  Also writes y (the LayerNorm
+ * output, nullable) so the pins can check it. */
+void oracle_layernorm_quant(const float *h, int64_t M, int64_t K, const float *gamma,
+                            const float *beta, float eps, const float *inv_s, int8_t *q,
+                            float *sx, float *y_out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < M; ++t) {
+        const float *row = h + t * K;
+        double sum = 0.0;
+        for (int64_t j = 0; j < K; ++j)
+            sum += (double)row[j];
+        double mu = sum / (double)K;
+        double ss = 0.0;
+        for (int64_t j = 0; j < K; ++j) {
+            double d = (double)row[j] - mu;
+            ss += d * d;
+        }
+        double rstd = 1.0 / sqrt(ss / (double)K + (double)eps);
+        float *y = (float *)malloc((size_t)K * sizeof(float));
+        float amax = 0.0f;
+        for (int64_t j = 0; j < K; ++j) {
+            double g = gamma ? (double)gamma[j] : 1.0;
+            double b = beta ? (double)beta[j] : 0.0;
+            double n = ((double)row[j] - mu) * rstd;
+            float yj = (float)(n * g + b);
+            if (y_out)
+                y_out[t * K + j] = yj;
+            float v = inv_s ? yj * inv_s[j] : yj;
+            y[j] = v;
+            float a = fabsf(v);
+            if (a > amax)
+                amax = a;
+        }
+        float s = amax / (float)ACT_QMAX;
+        sx[t] = s;
+        for (int64_t j = 0; j < K; ++j)
+            q[t * K + j] = (s == 0.0f) ? (int8_t)0 : (int8_t)sym_code(y[j], s, ACT_QMAX);
+        free(y);
+    }
+}
+
 /* ------------------------------------------------- static activation scale */
 /* Abs-max of the smoothed activations x' = x * inv_s over one calibration
  * batch x [M,K] (inv_s nullable): the per-tensor range [CQ] 2.1 "范围校准". */

@@ -66,6 +66,12 @@ MUTANTS = [
      "float s_best = (wmax - wmin) / 254.0f;"),
     ("asym_dequant_drops_128R", "int32_t A = acc[t * N + n] + 128 * R[t];", "int32_t A = acc[t * N + n];"),
     ("asym_dequant_drops_offset", "float y = sx[t] * (p + o);", "float y = sx[t] * p;"),
+    ("ln_drops_eps", "double rstd = 1.0 / sqrt(ss / (double)K + (double)eps);",
+     "double rstd = 1.0 / sqrt(ss / (double)K);"),
+    ("ln_unbiased_variance", "double rstd = 1.0 / sqrt(ss / (double)K + (double)eps);",
+     "double rstd = 1.0 / sqrt(ss / (double)(K - 1) + (double)eps);"),
+    ("ln_drops_beta", "double b = beta ? (double)beta[j] : 0.0;", "double b = 0.0;"),
+    ("ln_smooths_before_norm", "float v = inv_s ? yj * inv_s[j] : yj;", "float v = yj;"),
     ("int4_nibbles_swapped", "packed[n * (K / 2) + i] = (uint8_t)(lo | (hi << 4));",
      "packed[n * (K / 2) + i] = (uint8_t)(hi | (lo << 4));"),
     ("int4_unpack_no_sign", "q[n * K + 2 * i] = (int8_t)(lo >= 8 ? lo - 16 : lo);", "q[n * K + 2 * i] = (int8_t)lo;"),

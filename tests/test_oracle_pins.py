@@ -420,6 +420,52 @@ def test_act_rowsum_and_asym_dequant(orc):
     np.testing.assert_allclose(y, ref, rtol=1e-5, atol=1e-6 * np.abs(ref).max())
 
 
+# ------------------------------------------------- LayerNorm fused with step 4
+# SmoothQuant page section 1 (the scaling moves into the op that produces X);
+# CUDA INT8 notes 4.2 (fuse quantization with the neighbouring kernel).
+def test_layernorm_matches_torch_fp64(orc):
+    r = np.random.default_rng(60)
+    for scale, eps in ((3.0, 1e-5), (0.01, 1e-5), (1.0, 0.0)):
+        h = (r.standard_normal((9, 96)) * scale + 0.5 * scale).astype(np.float32)
+        g = (r.random(96) + 0.5).astype(np.float32)
+        b = (r.standard_normal(96) * 0.1).astype(np.float32)
+        _, _, y = orc.layernorm_quant(h, g, b, eps)
+        want = torch.nn.functional.layer_norm(torch.from_numpy(h).double(), (96,), torch.from_numpy(g).double(),
+                                              torch.from_numpy(b).double(), eps).numpy()
+        np.testing.assert_allclose(y, want.astype(np.float32), rtol=2e-7, atol=2e-7 * np.abs(want).max())
+
+
+def test_layernorm_quant_composes_with_per_token_quant(orc):
+    r = np.random.default_rng(61)
+    h = _llm_like(20, 128, seed=62)
+    g = (r.random(128) + 0.5).astype(np.float32)
+    b = (r.standard_normal(128) * 0.1).astype(np.float32)
+    inv = (r.random(128) + 0.25).astype(np.float32)
+    q, sx, y = orc.layernorm_quant(h, g, b, 1e-5, inv)
+    q2, sx2 = orc.quant_act_per_token(y, inv)
+    np.testing.assert_array_equal(q, q2)
+    np.testing.assert_array_equal(sx, sx2)
+
+
+def test_layernorm_fold_of_smoothing_is_equivalent(orc):
+    # diag(1/s) folded into gamma and beta gives the same codes up to rounding
+    r = np.random.default_rng(63)
+    h = _llm_like(32, 256, seed=64)
+    g = (r.random(256) + 0.5).astype(np.float32)
+    b = (r.standard_normal(256) * 0.1).astype(np.float32)
+    inv = (r.random(256) * 2 + 0.1).astype(np.float32)
+    q, sx, _ = orc.layernorm_quant(h, g, b, 1e-5, inv)
+    qf, sxf, _ = orc.layernorm_quant(h, g * inv, b * inv, 1e-5)
+    np.testing.assert_allclose(sxf, sx, rtol=1e-6)
+    assert np.mean(q == qf) > 0.999 and np.abs(q.astype(int) - qf).max() <= 1
+
+
+def test_layernorm_quant_constant_row(orc):
+    h = np.full((2, 64), 3.25, np.float32)
+    q, sx, y = orc.layernorm_quant(h, None, None, 1e-5)
+    assert not y.any() and not q.any() and not sx.any()
+
+
 # ------------------------------------------------- packed int4
 def test_pack_int4_layout_and_round_trip(orc):
     # golden nibble layout: element 2i low, 2i+1 high, two's complement
