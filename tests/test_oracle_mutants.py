@@ -46,7 +46,10 @@ MUTANTS = [
     ("candidate_not_floored",
      "s_cand = (float)(num / (double)den);\n            if (s_cand < SSZ_MIN_SCALE)\n                s_cand = SSZ_MIN_SCALE;",
      "s_cand = (float)(num / (double)den);"),
-    ("act_scale_128", "float s = amax / (float)ACT_QMAX;", "float s = amax / 128.0f;"),
+    ("act_scale_128", "float s = amax / (float)ACT_QMAX;\n        sx[t] = s;\n        for (int64_t j = 0; j < K; ++j) {\n            float v = inv_s",
+     "float s = amax / 128.0f;\n        sx[t] = s;\n        for (int64_t j = 0; j < K; ++j) {\n            float v = inv_s"),
+    ("ln_act_scale_128", "float s = amax / (float)ACT_QMAX;\n        sx[t] = s;\n        for (int64_t j = 0; j < K; ++j)\n            q[t * K + j] = (s == 0.0f) ? (int8_t)0 : (int8_t)sym_code(y[j]",
+     "float s = amax / 128.0f;\n        sx[t] = s;\n        for (int64_t j = 0; j < K; ++j)\n            q[t * K + j] = (s == 0.0f) ? (int8_t)0 : (int8_t)sym_code(y[j]"),
     ("act_divides_by_inv_s", "float v = inv_s ? row[j] * inv_s[j] : row[j];\n            q[",
      "float v = inv_s ? row[j] / inv_s[j] : row[j];\n            q["),
     ("gemm_transposed_weight", "(int64_t)qw[n * K + k]", "(int64_t)qw[k * N + n]"),
