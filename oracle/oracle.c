@@ -427,7 +427,8 @@ void oracle_quant_act_per_token(const float *x, int64_t M, int64_t K,
  * neighbouring op so the intermediate never goes to memory).  Per row t of
  * h [M,K]:
  *     mu  = sum_j h_j / K,  var = sum_j (h_j - mu)^2 / K      (fp64, index order)
- *     y_j = fp32(((h_j - mu) * (1 / sqrt(var + eps))) * gamma_j + beta_j)  (fp64)
+ *     m = fp32(mu), r = fp32(1 / sqrt(var + eps))
+ *     y_j = ((h_j - m) * r) * gamma_j + beta_j                  (fp32, each op rounded)
  *     x'_j = y_j * inv_s_j (fp32), then the per-token codes and scale of step 4.
  * gamma, beta, inv_s nullable (1, 0, 1).  Also writes y (the LayerNorm
  * output, nullable) so the pins can check it. */
@@ -448,13 +449,14 @@ void oracle_layernorm_quant(const float *h, int64_t M, int64_t K, const float *g
             ss += d * d;
         }
         double rstd = 1.0 / sqrt(ss / (double)K + (double)eps);
+        float m32 = (float)mu, r32 = (float)rstd;
         float *y = (float *)malloc((size_t)K * sizeof(float));
         float amax = 0.0f;
         for (int64_t j = 0; j < K; ++j) {
-            double g = gamma ? (double)gamma[j] : 1.0;
-            double b = beta ? (double)beta[j] : 0.0;
-            double n = ((double)row[j] - mu) * rstd;
-            float yj = (float)(n * g + b);
+            float g = gamma ? gamma[j] : 1.0f;
+            float b = beta ? beta[j] : 0.0f;
+            float n = (row[j] - m32) * r32;
+            float yj = n * g + b;
             if (y_out)
                 y_out[t * K + j] = yj;
             float v = inv_s ? yj * inv_s[j] : yj;

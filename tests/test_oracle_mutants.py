@@ -73,7 +73,7 @@ MUTANTS = [
      "double rstd = 1.0 / sqrt(ss / (double)K);"),
     ("ln_unbiased_variance", "double rstd = 1.0 / sqrt(ss / (double)K + (double)eps);",
      "double rstd = 1.0 / sqrt(ss / (double)(K - 1) + (double)eps);"),
-    ("ln_drops_beta", "double b = beta ? (double)beta[j] : 0.0;", "double b = 0.0;"),
+    ("ln_drops_beta", "float b = beta ? beta[j] : 0.0f;", "float b = 0.0f;"),
     ("ln_smooths_before_norm", "float v = inv_s ? yj * inv_s[j] : yj;", "float v = yj;"),
     ("int4_nibbles_swapped", "packed[n * (K / 2) + i] = (uint8_t)(lo | (hi << 4));",
      "packed[n * (K / 2) + i] = (uint8_t)(hi | (lo << 4));"),

@@ -432,7 +432,8 @@ def test_layernorm_matches_torch_fp64(orc):
         _, _, y = orc.layernorm_quant(h, g, b, eps)
         want = torch.nn.functional.layer_norm(torch.from_numpy(h).double(), (96,), torch.from_numpy(g).double(),
                                               torch.from_numpy(b).double(), eps).numpy()
-        np.testing.assert_allclose(y, want.astype(np.float32), rtol=2e-7, atol=2e-7 * np.abs(want).max())
+        # fp32 elementwise arithmetic after fp64 statistics: a few ulp of the fp64 result
+        np.testing.assert_allclose(y, want.astype(np.float32), rtol=1e-6, atol=1e-6 * np.abs(want).max())
 
 
 def test_layernorm_quant_composes_with_per_token_quant(orc):
