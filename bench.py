@@ -290,6 +290,8 @@ def time_next_rows(args, w, torch, probs, flush, stream, reps=50):
     events), on the first linear of the workload:
     - quant_act_static: codes at a static per-tensor scale (range calibrated
       beforehand on the same activations);
+    - sq_layernorm_quant: LayerNorm, smoothing and per-token codes in one
+      pass (unfused_bytes: what a separate LayerNorm output would add);
     - ssz_quant_weight_asym, quant_act_per_token_rowsum and
       w8a8_gemm_dequant_asym: the asymmetric int8 weight path;
     - sq_pack_int4 and w4a8_gemm_dequant (packed int4 weights) against
@@ -321,6 +323,19 @@ def time_next_rows(args, w, torch, probs, flush, stream, reps=50):
                                "peak": round(peaks["hbm_gbs"], 1), "unit": "GB/s",
                                "frac": round(gbs / peaks["hbm_gbs"], 4), "algorithmic": {"bytes": nbytes},
                                "shape": [p.M, p.K]}
+
+    # activation quantization fused upstream: LayerNorm + smoothing + codes
+    # in one pass over the layer input (the X of this linear serves as h)
+    g_ln = torch.ones(p.K, device=p.x.device)
+    b_ln = torch.zeros(p.K, device=p.x.device)
+    ms = timed(lambda: w.sq_layernorm_quant(p.x, g_ln, b_ln, 1e-5, p.inv, p.qx, p.sx))
+    nbytes = p.x.element_size() * p.M * p.K + p.M * p.K + 12 * p.K + 4 * p.M
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    out["sq_layernorm_quant"] = {"us": round(ms * 1e3, 2), "bound": "hbm", "achieved": round(gbs, 1),
+                                 "peak": round(peaks["hbm_gbs"], 1), "unit": "GB/s",
+                                 "frac": round(gbs / peaks["hbm_gbs"], 4), "algorithmic": {"bytes": nbytes},
+                                 "shape": [p.M, p.K],
+                                 "unfused_bytes": 2 * p.x.element_size() * p.M * p.K + nbytes}
 
     # asymmetric int8 weights: SSZ over (scale, offset), per-token codes with
     # row sums, GEMM with the offset dequant

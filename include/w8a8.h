@@ -208,6 +208,25 @@ sq_status w4a8_gemm_dequant(const int8_t *qx, const float *sx, const uint8_t *qw
                             int64_t M, int64_t N, int64_t K, void *y, sq_dtype yt, int32_t *acc_out,
                             void *stream);
 
+/* -------------------------------- LayerNorm fused with step 4 (next)
+ * Activation quantization fused upstream: the smoothing 1/s folded into the
+ * LayerNorm that produces X ("SmoothQuant大模型量化技术深度解析" section 1: an
+ * equivalent rescaling) and the quantization fused with it so that X never
+ * goes to memory (CUDA INT8 notes 4.2, kernel fusion).  Per row t of
+ * h [M,K] (dtype ht):
+ *     mu = sum_j h_j / K, var = sum_j (h_j - mu)^2 / K          (fp64)
+ *     m = fp32(mu), r = fp32(1 / sqrt(var + eps))
+ *     y_j = ((h_j - m) * r) * gamma_j + beta_j                   (fp32, each op rounded)
+ *     x'_j = y_j * inv_s_j (fp32); codes and scale as quant_act_per_token.
+ * gamma, beta, inv_s: [K] fp32 or NULL (1, 0, 1), 16-byte aligned.  eps >= 0.
+ * K: a multiple of 16 up to 16384 (one row is held in registers).
+ * The fp64 sums are taken in tree order; they equal a sequential sum
+ * whenever they are exact (bf16 inputs of moderate range), otherwise they
+ * may differ in the last bit. */
+sq_status sq_layernorm_quant(const void *h, sq_dtype ht, int64_t M, int64_t K, const float *gamma,
+                             const float *beta, float eps, const float *inv_s, int8_t *q_out,
+                             float *scale_out, void *stream);
+
 /* ------------------------------------------- static activation scale (next)
  * A per-tensor activation range calibrated offline instead of the per-token
  * scales of step 4: the moving-average abs-max of "PaddleNLP GPT

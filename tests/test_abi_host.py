@@ -160,6 +160,21 @@ def test_w4a8_rejects(lib, case, status):
     assert lib.sq_pack_int4(P(), 4, 64, NULL, None) == 1
 
 
+@pytest.mark.parametrize("case,status", [("null", 1), ("k", 2), ("k_big", 2), ("eps", 5), ("align_g", 4),
+                                         ("dtype", 3)])
+def test_layernorm_quant_rejects(lib, case, status):
+    a = dict(h=P(), ht=1, M=4, K=64, g=NULL, b=NULL, eps=1e-5, inv=NULL, q=P(8192), sc=P(12288))
+    if case == "null": a["sc"] = NULL
+    if case == "k": a["K"] = 40
+    if case == "k_big": a["K"] = 16400
+    if case == "eps": a["eps"] = -1.0
+    if case == "align_g": a["g"] = P(4)
+    if case == "dtype": a["ht"] = 6
+    rc = lib.sq_layernorm_quant(a["h"], a["ht"], a["M"], a["K"], a["g"], a["b"], a["eps"], a["inv"], a["q"], a["sc"],
+                                None)
+    assert rc == status, _detail(lib)
+
+
 def test_quant_rowsum_rejects_misaligned(lib):
     assert lib.quant_act_per_token_rowsum(P(), 1, 4, 64, NULL, P(8192), P(12288), P(2), None) == 4
 

@@ -27,7 +27,8 @@ EXPORTS = ["sq_status_string", "sq_last_error_detail", "sq_abi_version", "sq_dev
            "sq_selftest_bounded_wait",
            "sq_calib_absmax", "sq_smooth_fold", "ssz_quant_weight", "quant_act_per_token",
            "w8a8_gemm_dequant", "sq_static_range_update", "quant_act_static", "quant_act_per_token_rowsum",
-           "ssz_quant_weight_asym", "w8a8_gemm_dequant_asym", "sq_pack_int4", "w4a8_gemm_dequant"]
+           "ssz_quant_weight_asym", "w8a8_gemm_dequant_asym", "sq_pack_int4", "w4a8_gemm_dequant",
+           "sq_layernorm_quant"]
 
 
 class W8A8Error(RuntimeError):
@@ -61,6 +62,7 @@ def _load() -> ctypes.CDLL:
         "ssz_quant_weight_asym": ([P, I, I64, I64, P, I, P, P, P, P, P, P], I),
         "w8a8_gemm_dequant_asym": ([P, P, P, P, P, P, I64, I64, I64, P, I, P, P], I),
         "sq_pack_int4": ([P, I64, I64, P, P], I),
+        "sq_layernorm_quant": ([P, I, I64, I64, P, P, F, P, P, P, P], I),
         "w4a8_gemm_dequant": ([P, P, P, P, I64, I64, I64, P, I, P, P], I),
     }
     for name, (args, res) in sig.items():
@@ -216,6 +218,20 @@ def w8a8_gemm_dequant_asym(qx: torch.Tensor, sx: torch.Tensor, rowsum: torch.Ten
     _check("w8a8_gemm_dequant_asym",
            lib.w8a8_gemm_dequant_asym(_ptr(qx), _ptr(sx), _ptr(rowsum), _ptr(qw), _ptr(sw), _ptr(ow), M, N, K,
                                       _ptr(y), _dtype(y), _ptr(acc_out), _stream(stream)))
+
+
+def sq_layernorm_quant(h: torch.Tensor, gamma: torch.Tensor | None, beta: torch.Tensor | None, eps: float,
+                       inv_s: torch.Tensor | None, q_out: torch.Tensor, scale_out: torch.Tensor, stream=None) -> None:
+    """LayerNorm of h, times inv_s, as per-token int8 codes and scales."""
+    _need(gamma, torch.float32, "gamma")
+    _need(beta, torch.float32, "beta")
+    _need(inv_s, torch.float32, "inv_s")
+    _need(q_out, torch.int8, "q_out")
+    _need(scale_out, torch.float32, "scale_out")
+    M, K = h.shape
+    _check("sq_layernorm_quant", lib.sq_layernorm_quant(_ptr(h), _dtype(h), M, K, _ptr(gamma), _ptr(beta),
+                                                         float(eps), _ptr(inv_s), _ptr(q_out), _ptr(scale_out),
+                                                         _stream(stream)))
 
 
 def sq_pack_int4(q: torch.Tensor, packed: torch.Tensor, stream=None) -> None:

@@ -230,6 +230,136 @@ static void launch_quant_act(const void *x, int64_t M, int64_t K, const float *i
         <<<(unsigned)grid, threads, 0, st>>>((const T *)x, M, K, inv_s, range, q, scale, rowsum);
 }
 
+// ------------------------------------------------ LayerNorm fused with step 4
+// One CTA per row (as quant_act_kernel), the raw row in registers for the
+// whole computation: fp64 mean, then fp64 sum of squared deviations (two
+// passes over registers), rstd = 1 / sqrt(var + eps) (IEEE fp64); m and r
+// rounded to fp32, then per element y = ((h - m) r) gamma + beta and
+// x' = y inv_s in fp32 with no fused multiply-add (the build contracts
+// nothing), the row abs-max and the packed per-token codes.  X' never goes
+// to memory.
+__device__ __forceinline__ double block_sum_d(double v, double (&red)[32], int lane, int warp, int nwarps) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    double t = red[0];
+    for (int w = 1; w < nwarps; ++w) t += red[w];
+    __syncthreads();  // red is reused by the next reduction
+    return t;
+}
+
+template <typename T, int E>
+__global__ void __launch_bounds__(512)
+ln_quant_kernel(const T *__restrict__ h, int64_t M, int64_t K, const float *__restrict__ gamma,
+                const float *__restrict__ beta, float eps, const float *__restrict__ inv_s, int8_t *__restrict__ q,
+                float *__restrict__ scale) {
+    constexpr int C = E / 8;
+    __shared__ double redd[32];
+    __shared__ float redf[32];
+    const int T_ = blockDim.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = T_ >> 5;
+    bool live[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) live[c] = ((int64_t)c * T_ + threadIdx.x) * 8 < K;
+    const double kd = (double)K;
+
+    for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
+        Raw8<T> raw[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            if (live[c]) raw[c].load(h + row * K + ((int64_t)c * T_ + threadIdx.x) * 8);
+            else raw[c].zero();
+        }
+        double sum = 0.0;
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            float v[8];
+            raw[c].widen(v);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) sum += (double)v[i];
+        }
+        const double mu = block_sum_d(sum, redd, lane, warp, nwarps) / kd;
+        double ss = 0.0;
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            if (!live[c]) continue;
+            float v[8];
+            raw[c].widen(v);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const double d = (double)v[i] - mu;
+                ss += d * d;
+            }
+        }
+        const double rstd = 1.0 / sqrt(block_sum_d(ss, redd, lane, warp, nwarps) / kd + (double)eps);
+        const float m32 = (float)mu, r32 = (float)rstd;
+        // x' of chunk c: ((h - m) r) gamma + beta, times inv_s, each op in fp32
+        auto xs = [&](int c, float (&x)[8]) {
+            const int64_t j = ((int64_t)c * T_ + threadIdx.x) * 8;
+            float v[8], g[8], b[8], f[8];
+            raw[c].widen(v);
+            if (gamma) load8_f32(gamma + j, g);
+            if (beta) load8_f32(beta + j, b);
+            if (inv_s) load8_f32(inv_s + j, f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float n = (v[i] - m32) * r32;
+                const float gn = gamma ? n * g[i] : n;
+                const float y = beta ? gn + b[i] : gn;
+                x[i] = inv_s ? y * f[i] : y;
+            }
+        };
+        float amax = 0.0f;
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            if (!live[c]) continue;
+            float x[8];
+            xs(c, x);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
+        }
+        amax = warp_max(amax);
+        if (lane == 0) redf[warp] = amax;
+        __syncthreads();
+        float am = redf[0];
+        for (int w = 1; w < nwarps; ++w) am = fmaxf(am, redf[w]);
+        __syncthreads();  // redf is rewritten for the next row
+        const float s = __fdiv_rn(am, 127.0f);
+        if (threadIdx.x == 0) scale[row] = s;
+        const float r = __fdiv_rn(1.0f, s);
+        const bool exact_only = !(fabsf(r) <= 3.402823466e38f);
+        const bool narrow = am * r < 16384.0f;
+        const float tie_bound = 0.5f - fmaf(am * r, 4.76837158203125e-07f, 2.384185791015625e-07f);
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            if (!live[c]) continue;
+            float x[8];
+            xs(c, x);
+            uint2 code = make_uint2(0u, 0u);
+            if (s == 0.0f) {
+            } else if (exact_only) {
+                int e[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) e[i] = (int)sym_code(x[i], s, r, 127.0f, true);
+                code = pack8_codes(e);
+            } else {
+                code = fast_codes_tied(x, s, r, narrow, tie_bound);
+            }
+            *reinterpret_cast<uint2 *>(q + row * K + ((int64_t)c * T_ + threadIdx.x) * 8) = code;
+        }
+    }
+}
+
+template <typename T, int E>
+static void launch_ln_quant(const void *h, int64_t M, int64_t K, const float *gamma, const float *beta, float eps,
+                            const float *inv_s, int8_t *q, float *scale, int sms, cudaStream_t st) {
+    const int threads = (int)ceil_div(ceil_div(K, E), 32) * 32;
+    const int per_sm = std::max(1, std::min(32, 2048 / threads));
+    const int64_t grid = std::min<int64_t>(M, (int64_t)sms * per_sm);
+    ln_quant_kernel<T, E><<<(unsigned)grid, threads, 0, st>>>((const T *)h, M, K, gamma, beta, eps, inv_s, q, scale);
+}
+
 // E elements per thread: one warp per row up to K = 32 E, at most 64
 // elements per thread.
 template <bool STATIC>
@@ -335,4 +465,41 @@ extern "C" sq_status quant_act_static(const void *x, sq_dtype xt, int64_t M, int
     dispatch_quant<true>(x, xt == SQ_BF16, M, K, inv_s, range, q_out, scale_out, nullptr, sms,
                          (cudaStream_t)stream);
     return launch_status("quant_act_kernel");
+}
+
+extern "C" sq_status sq_layernorm_quant(const void *h, sq_dtype ht, int64_t M, int64_t K, const float *gamma,
+                                        const float *beta, float eps, const float *inv_s, int8_t *q_out,
+                                        float *scale_out, void *stream) {
+    if (M > 0 && (!h || !q_out || !scale_out)) return fail(SQ_ERR_NULL, "sq_layernorm_quant: NULL pointer");
+    if (ht != SQ_F32 && ht != SQ_BF16) return fail(SQ_ERR_DTYPE, "sq_layernorm_quant: dtype %d", (int)ht);
+    if (M < 0 || K <= 0 || K % 16 != 0 || K > 16384)
+        return fail(SQ_ERR_SHAPE, "sq_layernorm_quant: M=%lld K=%lld (K must be a multiple of 16 in [16, 16384])",
+                    (long long)M, (long long)K);
+    if (!(eps >= 0.0f) || isinf(eps)) return fail(SQ_ERR_ARG, "sq_layernorm_quant: eps=%g", (double)eps);
+    if (M == 0) return SQ_OK;
+    if (!aligned(h, 16) || !aligned(q_out, 16) || !aligned(scale_out, 4) || (gamma && !aligned(gamma, 16)) ||
+        (beta && !aligned(beta, 16)) || (inv_s && !aligned(inv_s, 16)))
+        return fail(SQ_ERR_ALIGN, "sq_layernorm_quant: misaligned pointer (h, q_out, gamma, beta, inv_s need 16 bytes)");
+    int sms;
+    sq_status st = check_device(&sms);
+    if (st != SQ_OK) return st;
+    cudaStream_t cs = (cudaStream_t)stream;
+    const bool bf = ht == SQ_BF16;
+    // E elements per thread: one warp per row up to K = 32 E, at most 32
+    // (measured faster than 64, which spills); K <= 16384 keeps a row within
+    // 512 threads
+    if (K <= 256) {
+        if (bf) launch_ln_quant<__nv_bfloat16, 8>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);
+        else launch_ln_quant<float, 8>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);
+    } else if (K <= 512) {
+        if (bf) launch_ln_quant<__nv_bfloat16, 16>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);
+        else launch_ln_quant<float, 16>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);
+    } else if (K <= 1024) {
+        if (bf) launch_ln_quant<__nv_bfloat16, 32>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);
+        else launch_ln_quant<float, 32>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);
+    } else {
+        if (bf) launch_ln_quant<__nv_bfloat16, 32>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);
+        else launch_ln_quant<float, 32>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);
+    }
+    return launch_status("ln_quant_kernel");
 }
