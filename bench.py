@@ -77,8 +77,12 @@ def algorithmic_work_mnk(M, K, N, xb, yb, bits=8):
         "smooth_fold": {"bytes": xb * N * K + 3 * 4 * K},
         "ssz_quant_weight": {"bytes": xb * N * K + N * K + 4 * K + 4 * N + 8 * N + 4 * N},
         "quant_act_per_token": {"bytes": xb * M * K + M * K + 4 * K + 4 * M},
+        # int4: the step packs the codes (N K read, N K / 2 written) and the
+        # W4A8 GEMM reads them packed
         "w8a8_gemm_dequant": ({"ops": 2 * M * N * K, "bytes": M * K + N * K + 4 * M + 4 * N + yb * M * N}
-                              if bits == 8 else {"ops": 0, "bytes": 0}),
+                              if bits == 8 else
+                              {"ops": 2 * M * N * K,
+                               "bytes": N * K + N * K // 2 + M * K + N * K // 2 + 4 * M + 4 * N + yb * M * N}),
     }
 
 
@@ -185,6 +189,7 @@ class Problem:
         self.ax, self.aw, self.s, self.inv = (torch.empty(K, **f32) for _ in range(4))
         self.qw = torch.empty(N, K, device=dev, dtype=torch.int8)
         self.sw = torch.empty(N, **f32)
+        self.qw4 = torch.empty(N, K // 2, device=dev, dtype=torch.uint8) if bits == 4 else None
         self.iters = torch.empty(N, device=dev, dtype=torch.int32)  # SSZ rounds per channel (ALU work)
         self.qx = torch.empty(M, K, device=dev, dtype=torch.int8)
         self.sx = torch.empty(M, **f32)
@@ -238,6 +243,9 @@ def run_ours(args, rank, world, local_rank):
         mark(4)
         if p.bits == 8:
             w.w8a8_gemm_dequant(p.qx, p.sx, p.qw, p.sw, p.y)
+        else:  # int4 weights: packed two per byte, W4A8 GEMM
+            w.sq_pack_int4(p.qw, p.qw4)
+            w.w4a8_gemm_dequant(p.qx, p.sx, p.qw4, p.sw, p.y)
         mark(5)
 
     def step(evs=None):
@@ -454,7 +462,9 @@ def finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall_s, next_
                          hbm={"achieved": round(hbm, 1), "peak": round(peaks["hbm_gbs"], 1), "unit": "GB/s",
                               "frac": round(hbm / peaks["hbm_gbs"], 4)})
             work[n] = dict(work[n], ops=ssz_ops)
-        elif "ops" in work[n]:
+        elif "ops" in work[n] and (work[n]["ops"] / max(work[n]["bytes"], 1)
+                                   >= peaks["bf16_tflops"] * INT8_OVER_BF16 * 1e12 / (peaks["hbm_gbs"] * 1e9)):
+            # at or above the ridge point: bound by the tensor cores
             ach = work[n]["ops"] / t_s / 1e12
             peak = peaks["bf16_tflops"] * INT8_OVER_BF16
             entry.update(bound="tensor", achieved=round(ach, 1), peak=round(peak, 1), unit="TFLOP/s",
@@ -474,9 +484,9 @@ def finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall_s, next_
                            "alu": "derived: %d SMs x %d FP32 lanes x sampled SM clock" % (B200_SMS, FP32_LANES_PER_SM)
                            }[roof["bound"]]
 
-    launches_per_step = {"calib_absmax": 1, "smooth_fold": 2, "ssz_quant_weight": 1, "quant_act_per_token": 1,
-                         "w8a8_gemm_dequant": 1}
     p0 = probs[0]
+    launches_per_step = {"calib_absmax": 1, "smooth_fold": 2, "ssz_quant_weight": 1, "quant_act_per_token": 1,
+                         "w8a8_gemm_dequant": 1 if p0.bits == 8 else 2}
     M, K, N = p0.M, p0.K, p0.N
     result = {
         "metric": "W8A8 linear INT8 TOPS (% of peak); quant/SSZ GB/s (% of HBM) on 1 B200",
