@@ -581,6 +581,15 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int row, int M, in
 #define W8A8_PAIR_STAGES 6
 #endif
 
+#ifndef W8A8_PAIR_EPI_WARPS
+#define W8A8_PAIR_EPI_WARPS 8
+#endif
+// Epilogue warps of the pair kernel: 4 cover the 128 TMEM lanes once; 8 split
+// each tile's 256 columns between two warps per lane quarter, so that a short
+// main loop (small K) does not wait on the epilogue.
+constexpr int kPairEpiWarps = W8A8_PAIR_EPI_WARPS;
+constexpr int kThreadsPair = 64 + 32 * kPairEpiWarps;
+
 struct Cfg2 {
     static constexpr int BN = 256;              // pair tile N (each CTA stages BN/2 rows of B)
     static constexpr int PM = 2 * BM;           // pair tile M
@@ -593,7 +602,7 @@ struct Cfg2 {
 };
 
 template <typename OutT, bool ASYM>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
 w8a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                       const float *__restrict__ sx, const float *__restrict__ sw, const int32_t *__restrict__ rs,
                       const float *__restrict__ ow, OutT *__restrict__ y, int32_t *__restrict__ acc_out, int M,
@@ -626,7 +635,7 @@ w8a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_c
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&tfull_bar[b]), 1);
-            mbar_init(smem_u32(&tempty_bar[b]), 2 * 4 * 32);
+            mbar_init(smem_u32(&tempty_bar[b]), 2 * kPairEpiWarps * 32);
         }
         mbar_init(smem_u32(&drain_bar), 1);
         abort_flag = 0;
@@ -736,9 +745,11 @@ w8a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_c
             }
         }
     } else {
-        // ------------------------------------------------ epilogue (warps 2..5, both CTAs)
-        const int quarter = warp & 3;
+        // ------------------------------------------------ epilogue (warps 2.., both CTAs)
+        const int quarter = warp & 3;  // TMEM lanes this warp may access
         const int row_in_tile = (int)rank * BM + quarter * 32 + lane;
+        constexpr int kCols = C::BN * 4 / kPairEpiWarps;   // columns of a tile per warp
+        const int col0 = ((warp - 2) / 4) * kCols;
         int buf = 0;
         uint32_t buf_phase = 0;
         for (int tile = pair; tile < num_tiles; tile += num_pairs) {
@@ -751,8 +762,9 @@ w8a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_c
             const bool ok = wait_bounded(smem_u32(&tfull_bar[buf]), buf_phase, &abort_flag, kFaultEpilogue);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
-            const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * C::BN);
-            epilogue_tile<OutT, ASYM>(tbase, row, M, n0, N, sxr, Rr, sw, ow, y, acc_out, C::BN);
+            const uint32_t tbase =
+                tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * C::BN + col0);
+            epilogue_tile<OutT, ASYM>(tbase, row, M, n0 + col0, N, sxr, Rr, sw, ow, y, acc_out, kCols);
             tc_fence_before();
             mbar_arrive_leader(smem_u32(&tempty_bar[buf]));
             buf ^= 1;
@@ -1188,7 +1200,7 @@ static sq_status launch_pair(const int8_t *qx, const float *sx, const int32_t *r
     }
     const int tiles = ((M + C::PM - 1) / C::PM) * ((N + C::BN - 1) / C::BN);
     const int pairs = std::min(tiles, sms / 2);
-    kern<<<2 * pairs, kThreads, C::SMEM, st>>>(ma, mb, sx, sw, rs, ow, (OutT *)y, acc_out, M, N, K);
+    kern<<<2 * pairs, kThreadsPair, C::SMEM, st>>>(ma, mb, sx, sw, rs, ow, (OutT *)y, acc_out, M, N, K);
     return launch_status("w8a8_gemm_pair_kernel");
 }
 
