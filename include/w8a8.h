@@ -248,10 +248,12 @@ sq_status sq_static_range_update(const float *x_absmax, const float *inv_s, int6
  *     q[t,j] = clamp(rint(x[t,j] * inv_s[j] / S), -127, 127)   (0 if S == 0)
  * Values beyond the range saturate.  scale_out: [M] fp32 or NULL; if given,
  * every entry receives S, so that w8a8_gemm_dequant applies the static
- * scale unchanged.  Shapes, dtypes and alignment as quant_act_per_token. */
+ * scale unchanged.  rowsum_out: [M] int32 or NULL, the exact row sums of the
+ * codes (for w8a8_gemm_dequant_asym).  Shapes, dtypes and alignment as
+ * quant_act_per_token. */
 sq_status quant_act_static(const void *x, sq_dtype xt, int64_t M, int64_t K,
                            const float *inv_s, const float *range, int8_t *q_out,
-                           float *scale_out, void *stream);
+                           float *scale_out, int32_t *rowsum_out, void *stream);
 
 /* ------------------------------------------------------------------ step 5
  * INT8 x INT8 -> INT32 GEMM with fused per-token x per-channel dequant

@@ -188,7 +188,7 @@ def test_quant_act_static_rejects(lib, case, status):
     if case == "k": a["K"] = 65
     if case == "align_q": a["q"] = P(8)
     if case == "dtype": a["xt"] = 5
-    rc = lib.quant_act_static(a["x"], a["xt"], a["M"], a["K"], a["inv"], a["rng"], a["q"], a["sc"], None)
+    rc = lib.quant_act_static(a["x"], a["xt"], a["M"], a["K"], a["inv"], a["rng"], a["q"], a["sc"], NULL, None)
     assert rc == status, _detail(lib)
 
 
@@ -226,7 +226,7 @@ def test_gemm_rejects(lib, case, status):
 def test_empty_inputs_are_noops(lib):
     # M == 0 / N == 0 return OK without touching the device
     assert lib.quant_act_per_token(NULL, 1, 0, 64, NULL, NULL, NULL, None) == 0
-    assert lib.quant_act_static(NULL, 1, 0, 64, NULL, NULL, NULL, NULL, None) == 0
+    assert lib.quant_act_static(NULL, 1, 0, 64, NULL, NULL, NULL, NULL, NULL, None) == 0
     assert lib.ssz_quant_weight(NULL, 1, 0, 64, NULL, 8, 20, NULL, NULL, NULL, NULL, None) == 0
     assert lib.w8a8_gemm_dequant(NULL, NULL, NULL, NULL, 0, 16, 64, NULL, 1, NULL, None) == 0
     assert lib.w8a8_gemm_dequant(NULL, NULL, NULL, NULL, 4, 0, 64, NULL, 1, NULL, None) == 0

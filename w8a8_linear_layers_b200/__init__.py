@@ -57,7 +57,7 @@ def _load() -> ctypes.CDLL:
         "quant_act_per_token": ([P, I, I64, I64, P, P, P, P], I),
         "w8a8_gemm_dequant": ([P, P, P, P, I64, I64, I64, P, I, P, P], I),
         "sq_static_range_update": ([P, P, I64, F, I, P, P], I),
-        "quant_act_static": ([P, I, I64, I64, P, P, P, P, P], I),
+        "quant_act_static": ([P, I, I64, I64, P, P, P, P, P, P], I),
         "quant_act_per_token_rowsum": ([P, I, I64, I64, P, P, P, P, P], I),
         "ssz_quant_weight_asym": ([P, I, I64, I64, P, I, P, P, P, P, P, P], I),
         "w8a8_gemm_dequant_asym": ([P, P, P, P, P, P, I64, I64, I64, P, I, P, P], I),
@@ -272,15 +272,18 @@ def sq_static_range_update(x_absmax: torch.Tensor, inv_s: torch.Tensor | None, r
 
 
 def quant_act_static(x: torch.Tensor, inv_s: torch.Tensor | None, range_: torch.Tensor, q_out: torch.Tensor,
-                     scale_out: torch.Tensor | None = None, stream=None) -> None:
+                     scale_out: torch.Tensor | None = None, rowsum_out: torch.Tensor | None = None,
+                     stream=None) -> None:
     """int8 codes of x * inv_s at the static scale range_/127 (saturating)."""
     _need(inv_s, torch.float32, "inv_s")
     _need(range_, torch.float32, "range")
     _need(q_out, torch.int8, "q_out")
     _need(scale_out, torch.float32, "scale_out")
+    _need(rowsum_out, torch.int32, "rowsum_out")
     M, K = x.shape
     _check("quant_act_static", lib.quant_act_static(_ptr(x), _dtype(x), M, K, _ptr(inv_s), _ptr(range_),
-                                                     _ptr(q_out), _ptr(scale_out), _stream(stream)))
+                                                     _ptr(q_out), _ptr(scale_out), _ptr(rowsum_out),
+                                                     _stream(stream)))
 
 
 def w8a8_gemm_dequant(qx: torch.Tensor, sx: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor, y: torch.Tensor,
@@ -300,18 +303,35 @@ def w8a8_gemm_dequant(qx: torch.Tensor, sx: torch.Tensor, qw: torch.Tensor, sw: 
 
 
 class W8A8Linear:
-    """A calibrated SmoothQuant W8A8 linear layer built from the five calls.
+    """A calibrated SmoothQuant W8A8 linear layer built from the library calls.
 
     calibrate(x) accumulates the activation absmax; quantize() smooths and
-    SSZ-quantizes the weight; forward(x) quantizes x per token and runs the
-    integer GEMM with the fused dequant.  Buffers are torch tensors on the
-    weight's device (memory plumbing only)."""
+    SSZ-quantizes the weight; forward(x) quantizes x and runs the integer GEMM
+    with the fused dequant.  Options (the next rows of the path):
+      weights="sym8"  symmetric int8 SSZ (default), "asym8" asymmetric int8
+                      SSZ (scale and offset), "int4" int4 SSZ packed two per
+                      byte with the W4A8 GEMM;
+      act_scales="dynamic" per-token scales (default) or "static": a
+                      per-tensor range, the moving average of each
+                      calibration batch's abs-max (calibrate_static(x) after
+                      quantize()).
+    forward_ln(h, gamma, beta, eps) applies the LayerNorm that produces x,
+    the smoothing and the per-token quantization in one kernel.  Buffers are
+    torch tensors on the weight's device (memory plumbing only)."""
 
     def __init__(self, w: torch.Tensor, alpha: float = 0.5, bits: int = 8, max_iters: int = 20,
-                 out_dtype: torch.dtype | None = None):
+                 out_dtype: torch.dtype | None = None, weights: str = "sym8", act_scales: str = "dynamic",
+                 static_rate: float = 0.9):
+        if weights not in ("sym8", "asym8", "int4"):
+            raise ValueError("weights must be sym8, asym8 or int4")
+        if act_scales not in ("dynamic", "static"):
+            raise ValueError("act_scales must be dynamic or static")
+        if weights == "int4":
+            bits = 4
         self.w = w.contiguous()
         self.N, self.K = w.shape
         self.alpha, self.bits, self.max_iters = alpha, bits, max_iters
+        self.weights, self.act_scales, self.static_rate = weights, act_scales, static_rate
         self.out_dtype = out_dtype or w.dtype
         dev = w.device
         f32 = dict(device=dev, dtype=torch.float32)
@@ -321,9 +341,13 @@ class W8A8Linear:
         self.inv_s = torch.empty(self.K, **f32)
         self.qw = torch.empty(self.N, self.K, device=dev, dtype=torch.int8)
         self.sw = torch.empty(self.N, **f32)
+        self.ow = torch.empty(self.N, **f32) if weights == "asym8" else None
+        self.qw4 = torch.empty(self.N, self.K // 2, device=dev, dtype=torch.uint8) if weights == "int4" else None
         self.mse = torch.empty(self.N, device=dev, dtype=torch.float64)
         self.iters = torch.empty(self.N, device=dev, dtype=torch.int32)
+        self.range = torch.zeros(1, **f32)
         self._calibrated = False
+        self._static_batches = 0
 
     def calibrate(self, x: torch.Tensor) -> None:
         sq_calib_absmax(x, self.ax, accumulate=self._calibrated)
@@ -331,14 +355,56 @@ class W8A8Linear:
 
     def quantize(self) -> None:
         sq_smooth_fold(self.ax, self.w, self.alpha, self.aw, self.s, self.inv_s)
-        ssz_quant_weight(self.w, self.s, self.bits, self.max_iters, self.qw, self.sw, self.mse, self.iters)
+        if self.weights == "asym8":
+            ssz_quant_weight_asym(self.w, self.s, self.max_iters, self.qw, self.sw, self.ow, self.mse, self.iters)
+        else:
+            ssz_quant_weight(self.w, self.s, self.bits, self.max_iters, self.qw, self.sw, self.mse, self.iters)
+        if self.weights == "int4":
+            sq_pack_int4(self.qw, self.qw4)
+
+    def calibrate_static(self, x: torch.Tensor) -> None:
+        """Blend one calibration batch into the static activation range
+        (after quantize(): the range is of x * inv_s)."""
+        axb = torch.empty(self.K, device=x.device, dtype=torch.float32)
+        sq_calib_absmax(x, axb)
+        sq_static_range_update(axb, self.inv_s, self.range, first=self._static_batches == 0, rate=self.static_rate)
+        self._static_batches += 1
+
+    def _gemm(self, qx, sx, rs, y):
+        if self.weights == "asym8":
+            w8a8_gemm_dequant_asym(qx, sx, rs, self.qw, self.sw, self.ow, y)
+        elif self.weights == "int4":
+            w4a8_gemm_dequant(qx, sx, self.qw4, self.sw, y)
+        else:
+            w8a8_gemm_dequant(qx, sx, self.qw, self.sw, y)
 
     def forward(self, x: torch.Tensor, y: torch.Tensor | None = None) -> torch.Tensor:
         M = x.shape[0]
         qx = torch.empty(M, self.K, device=x.device, dtype=torch.int8)
         sx = torch.empty(M, device=x.device, dtype=torch.float32)
-        quant_act_per_token(x, self.inv_s, qx, sx)
+        rs = torch.empty(M, device=x.device, dtype=torch.int32) if self.weights == "asym8" else None
+        if self.act_scales == "static":
+            if self._static_batches == 0:
+                raise RuntimeError("static activation scales need calibrate_static() first")
+            quant_act_static(x, self.inv_s, self.range, qx, sx, rs)
+        else:
+            quant_act_per_token_rowsum(x, self.inv_s, qx, sx, rs)
         if y is None:
             y = torch.empty(M, self.N, device=x.device, dtype=self.out_dtype)
-        w8a8_gemm_dequant(qx, sx, self.qw, self.sw, y)
+        self._gemm(qx, sx, rs, y)
+        return y
+
+    def forward_ln(self, h: torch.Tensor, gamma: torch.Tensor | None, beta: torch.Tensor | None,
+                   eps: float = 1e-5, y: torch.Tensor | None = None) -> torch.Tensor:
+        """forward(LayerNorm(h)) with the LayerNorm, the smoothing and the
+        per-token quantization fused (dynamic scales, sym8 or int4 weights)."""
+        if self.weights == "asym8" or self.act_scales == "static":
+            raise ValueError("forward_ln supports dynamic scales with sym8 or int4 weights")
+        M = h.shape[0]
+        qx = torch.empty(M, self.K, device=h.device, dtype=torch.int8)
+        sx = torch.empty(M, device=h.device, dtype=torch.float32)
+        sq_layernorm_quant(h, gamma, beta, eps, self.inv_s, qx, sx)
+        if y is None:
+            y = torch.empty(M, self.N, device=h.device, dtype=self.out_dtype)
+        self._gemm(qx, sx, None, y)
         return y

@@ -449,7 +449,8 @@ extern "C" sq_status sq_static_range_update(const float *x_absmax, const float *
 }
 
 extern "C" sq_status quant_act_static(const void *x, sq_dtype xt, int64_t M, int64_t K, const float *inv_s,
-                                      const float *range, int8_t *q_out, float *scale_out, void *stream) {
+                                      const float *range, int8_t *q_out, float *scale_out, int32_t *rowsum_out,
+                                      void *stream) {
     if (M > 0 && (!x || !q_out || !range)) return fail(SQ_ERR_NULL, "quant_act_static: NULL pointer");
     if (xt != SQ_F32 && xt != SQ_BF16) return fail(SQ_ERR_DTYPE, "quant_act_static: dtype %d", (int)xt);
     if (M < 0 || K <= 0 || K % 16 != 0 || K > 32768)
@@ -457,12 +458,12 @@ extern "C" sq_status quant_act_static(const void *x, sq_dtype xt, int64_t M, int
                     (long long)M, (long long)K);
     if (M == 0) return SQ_OK;
     if (!aligned(x, 16) || !aligned(q_out, 16) || !aligned(range, 4) || (scale_out && !aligned(scale_out, 4)) ||
-        (inv_s && !aligned(inv_s, 16)))
+        (inv_s && !aligned(inv_s, 16)) || (rowsum_out && !aligned(rowsum_out, 4)))
         return fail(SQ_ERR_ALIGN, "quant_act_static: misaligned pointer (x, q_out, inv_s need 16 bytes)");
     int sms;
     sq_status st = check_device(&sms);
     if (st != SQ_OK) return st;
-    dispatch_quant<true>(x, xt == SQ_BF16, M, K, inv_s, range, q_out, scale_out, nullptr, sms,
+    dispatch_quant<true>(x, xt == SQ_BF16, M, K, inv_s, range, q_out, scale_out, rowsum_out, sms,
                          (cudaStream_t)stream);
     return launch_status("quant_act_kernel");
 }
