@@ -18,12 +18,19 @@
 //     accumulator buffers so the epilogue of one tile overlaps the main loop
 //     of the next;
 //   * warp roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
-//     warps 2..5 epilogue (TMEM lanes 32*(warp%4) .. +31 each).
+//     then epilogue warps (TMEM lanes 32*(warp%4) .. +31 each).
+//
+// Three kernels share these pieces: w8a8_gemm_kernel (one CTA per 128 x 256
+// tile, M <= 128), w8a8_gemm_pair_kernel (CTA pairs, cta_group::2, 256 x 256
+// tiles, 8 epilogue warps, M > 128) and w4a8_gemm_kernel (packed int4
+// weights unpacked on chip by converter warps).
 //
 // Epilogue: tcgen05.ld of 32 accumulator columns per thread (thread = output
 // row), y = ((float)acc * sx[row]) * sw[col] (two fp32 multiplies, int->fp32
-// round-to-nearest-even), converted to bf16 (RNE) or kept fp32, stored with
-// 16-byte stores.  Optionally the raw int32 accumulators are stored too.
+// round-to-nearest-even), or with asymmetric weights
+// sx * (sw * (float)(acc + 128 R) + ow * (float)R), converted to bf16 (RNE) or
+// kept fp32, stored with 16-byte stores.  Optionally the raw int32
+// accumulators are stored too.
 //
 // No TMA multicast is used anywhere (each CTA loads its own tiles).
 //

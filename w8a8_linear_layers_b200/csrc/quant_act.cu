@@ -1,4 +1,8 @@
-// quant_act.cu -- step 4: per-token symmetric int8 activation quantization.
+// quant_act.cu -- step 4: per-token symmetric int8 activation quantization,
+// and its variants: static per-tensor scales (quant_act_static with
+// sq_static_range_update), row sums of the codes for asymmetric weights, and
+// the LayerNorm fused with the smoothing and the quantization
+// (sq_layernorm_quant).
 //
 // Source: CUDA INT8 quantization notes (aicoding.csdn.net), section 2.1
 // ("量化基础理论"): Q = round(R/S) + Z with range calibration, parameter
