@@ -41,8 +41,9 @@
 // The search is a chain of rounds per channel, so the kernel is latency
 // bound; it keeps many channels in flight (small CTAs, shared-memory rows)
 // and keeps each round's serial tail short: warp trees skip warps whose
-// codes did not move, every warp takes the (identical) decision itself after
-// one barrier, and the next candidate is computed alongside the error.
+// codes did not move, warp 0 alone takes the decision (the exact error in
+// fp64 and the next candidate) and shares it through shared memory, so the
+// other warps skip that fp64 work.
 #include "common.cuh"
 #include "dd.cuh"
 
@@ -276,7 +277,12 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
     extern __shared__ __align__(16) uint8_t smem[];
     float *wrow = reinterpret_cast<float *>(smem);            // K floats: the folded row
     int8_t *q = reinterpret_cast<int8_t *>(wrow + K);         // K codes: the kept codes
-    __shared__ WarpPart part[2][16];                          // per-warp partials, by round parity
+    __shared__ WarpPart part[2][16];
+    struct Decision {
+        float c_next;
+        int keep, done;
+    };
+    __shared__ Decision decision[2];  // warp 0's decision of a round, by parity                          // per-warp partials, by round parity
     __shared__ float redmax[16];
     const int T_ = blockDim.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = T_ >> 5;
@@ -353,29 +359,37 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
             if (lane == 0) part[par][warp] = {p.num, {0.0, 0.0}, p.den};
             __syncthreads();  // the candidate codes and all partials are in place
             ++it;
-            dd num_c = NUM;
-            int den_c = DEN;
-            for (int i = 0; i < nwarps; ++i) {
-                num_c = dd_add_cascade(num_c, part[par][i].num);
-                den_c += part[par][i].den;
+            if (warp == 0) {  // warp 0 decides; the others read the decision
+                dd num_c = NUM;
+                int den_c = DEN;
+                for (int i = 0; i < nwarps; ++i) {
+                    num_c = dd_add_cascade(num_c, part[par][i].num);
+                    den_c += part[par][i].den;
+                }
+                const double m_c = exact_error_k(W2, num_c, den_c, c);
+                const float c_next = ls_candidate(num_c, den_c, c);
+                const double delta = m_best - m_c;
+                bool dn = (m_best == 0.0) || (delta < kSszThreshold * m_best) || (fabs(delta) < thr_k) ||
+                          it == max_iters;
+                const bool keep = m_c < m_best;
+                if (keep) {
+                    m_best = m_c;
+                    NUM = num_c;
+                    DEN = den_c;
+                } else {
+                    dn = true;
+                }
+                if (lane == 0) decision[par] = {c_next, keep ? 1 : 0, dn ? 1 : 0};
             }
-            const double m_c = exact_error_k(W2, num_c, den_c, c);
-            const float c_next = ls_candidate(num_c, den_c, c);  // used only if c is kept
-            // on K-scaled errors: d/e < thr  <=>  dK < thr eK (eK > 0), |d| < thr  <=>  |dK| < thr K
-            const double delta = m_best - m_c;
-            done = (m_best == 0.0) || (delta < kSszThreshold * m_best) || (fabs(delta) < thr_k) ||
-                   it == max_iters;
-            if (m_c < m_best) {  // keep c: its codes are now the kept codes
+            __syncthreads();
+            const Decision dcs = decision[par];
+            done = dcs.done != 0;
+            if (dcs.keep) {
                 s_best = c;
-                m_best = m_c;
-                NUM = num_c;
-                DEN = den_c;
-                c = c_next;
+                c = dcs.c_next;
             } else {
                 rejected = true;
-                done = true;  // implied by the tests above (m_best >= 0); stated for the restore below
             }
-            // part[par] is rewritten two rounds from now, after another barrier
         }
         if (rejected) restore_chunks(wrow, touched, s_best, qmax, wmax, q);
 
