@@ -366,7 +366,7 @@ static void launch_ln_quant(const void *h, int64_t M, int64_t K, const float *ga
 
 // E elements per thread: one warp per row up to K = 1024, then 32 elements
 // per thread (measured faster than 64 at K = 4096: fewer registers, more
-// rows in flight per SM).
+// rows in flight per SM), 64 past K = 16384 (at most 512 threads a row).
 template <bool STATIC>
 static void dispatch_quant(const void *x, bool bf, int64_t M, int64_t K, const float *inv_s, const float *range,
                            int8_t *q, float *scale, int32_t *rowsum, int sms, cudaStream_t cs) {
@@ -379,9 +379,12 @@ static void dispatch_quant(const void *x, bool bf, int64_t M, int64_t K, const f
     } else if (K <= 1024) {
         if (bf) launch_quant_act<__nv_bfloat16, 32, 1, STATIC>(x, M, K, inv_s, range, q, scale, rowsum, sms, cs);
         else launch_quant_act<float, 32, 1, STATIC>(x, M, K, inv_s, range, q, scale, rowsum, sms, cs);
-    } else {
+    } else if (K <= 16384) {
         if (bf) launch_quant_act<__nv_bfloat16, 32, 1, STATIC>(x, M, K, inv_s, range, q, scale, rowsum, sms, cs);
         else launch_quant_act<float, 32, 1, STATIC>(x, M, K, inv_s, range, q, scale, rowsum, sms, cs);
+    } else {  // at most 512 threads a row
+        if (bf) launch_quant_act<__nv_bfloat16, 64, 1, STATIC>(x, M, K, inv_s, range, q, scale, rowsum, sms, cs);
+        else launch_quant_act<float, 64, 1, STATIC>(x, M, K, inv_s, range, q, scale, rowsum, sms, cs);
     }
 }
 
