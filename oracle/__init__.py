@@ -84,6 +84,7 @@ def _L():
             "oracle_act_rowsum": [P, I64, I64, P],
             "oracle_pack_int4": [P, I64, I64, P],
             "oracle_layernorm_quant": [P, I64, I64, P, P, ctypes.c_float, P, P, P, P],
+            "oracle_quant_act_given_scale": [P, I64, I64, P, P, P],
             "oracle_unpack_int4": [P, I64, I64, P],
             "oracle_dequant_asym": [P, P, P, P, P, I64, I64, P, P],
             "oracle_static_ema": [ctypes.c_float, ctypes.c_float, ctypes.c_float, I],
@@ -231,6 +232,17 @@ def ssz_quant_weight_asym(w, max_iters: int = SSZ_ITERS, s=None, trace: bool = F
 def channel_mse_asym(w_row, S, m) -> float:
     w_row = _f32(w_row)
     return float(_L().oracle_channel_mse_asym(_ptr(w_row), w_row.shape[0], float(S), float(m)))
+
+
+def quant_act_given_scale(x, inv_s, sx):
+    """Codes of x [M,K] (times inv_s) at the given per-row scales sx [M]."""
+    x = _f32(x)
+    M, K = x.shape
+    inv = None if inv_s is None else _f32(inv_s)
+    sx = _f32(sx)
+    q = np.empty((M, K), np.int8)
+    _L().oracle_quant_act_given_scale(_ptr(x), M, K, _ptr(inv), _ptr(sx), _ptr(q))
+    return q
 
 
 def layernorm_quant(h, gamma=None, beta=None, eps: float = 1e-5, inv_s=None):

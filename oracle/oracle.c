@@ -473,6 +473,22 @@ void oracle_layernorm_quant(const float *h, int64_t M, int64_t K, const float *g
     }
 }
 
+/* ---------------------------------------- row-parallel (K-sharded) linear */
+/* Codes of x' = x * inv_s at given per-row scales sx[t] (sx[t] == 0: zero
+ * codes).  With K split across ranks, each rank's per-token scale is
+ * fl(max_local / 127); the MAX over ranks of those equals the unsharded
+ * scale (x -> fl(x / 127) is monotonic), and every rank then quantizes its
+ * slice at that scale ([CQ] 2.1), so the codes are the unsharded codes. */
+void oracle_quant_act_given_scale(const float *x, int64_t M, int64_t K, const float *inv_s,
+                                  const float *sx, int8_t *q)
+{
+    for (int64_t t = 0; t < M; ++t)
+        for (int64_t j = 0; j < K; ++j) {
+            float v = inv_s ? x[t * K + j] * inv_s[j] : x[t * K + j];
+            q[t * K + j] = (sx[t] == 0.0f) ? (int8_t)0 : (int8_t)sym_code(v, sx[t], ACT_QMAX);
+        }
+}
+
 /* ------------------------------------------------- static activation scale */
 /* Abs-max of the smoothed activations x' = x * inv_s over one calibration
  * batch x [M,K] (inv_s nullable): the per-tensor range [CQ] 2.1 "范围校准". */

@@ -69,6 +69,8 @@ MUTANTS = [
      "float s_best = (wmax - wmin) / 254.0f;"),
     ("asym_dequant_drops_128R", "int32_t A = acc[t * N + n] + 128 * R[t];", "int32_t A = acc[t * N + n];"),
     ("asym_dequant_drops_offset", "float y = sx[t] * (p + o);", "float y = sx[t] * p;"),
+    ("given_scale_ignores_smoothing", "float v = inv_s ? x[t * K + j] * inv_s[j] : x[t * K + j];\n            q[t * K + j] = (sx[t] == 0.0f)",
+     "float v = x[t * K + j];\n            q[t * K + j] = (sx[t] == 0.0f)"),
     ("ln_drops_eps", "double rstd = 1.0 / sqrt(ss / (double)K + (double)eps);",
      "double rstd = 1.0 / sqrt(ss / (double)K);"),
     ("ln_unbiased_variance", "double rstd = 1.0 / sqrt(ss / (double)K + (double)eps);",

@@ -420,6 +420,36 @@ def test_act_rowsum_and_asym_dequant(orc):
     np.testing.assert_allclose(y, ref, rtol=1e-5, atol=1e-6 * np.abs(ref).max())
 
 
+# ------------------------------------------------- row-parallel (K-sharded) linear
+def test_given_scale_codes_match_numpy_and_per_token(orc):
+    x = _llm_like(24, 96, seed=70)
+    inv = (np.random.default_rng(71).random(96) + 0.5).astype(np.float32)
+    q, sx = orc.quant_act_per_token(x, inv)
+    np.testing.assert_array_equal(orc.quant_act_given_scale(x, inv, sx), q)
+    sx2 = (sx * np.float32(0.6)).astype(np.float32)
+    sx2[3] = 0.0
+    want = np.clip(np.rint((x * inv[None, :]) / sx2[:, None]), -127, 127)
+    want[3] = 0
+    np.testing.assert_array_equal(orc.quant_act_given_scale(x, inv, sx2), want.astype(np.int8))
+
+
+def test_k_sharded_linear_equals_unsharded(orc):
+    # per-shard scales, MAX, codes at the global scale, int32 SUM, dequant:
+    # bit for bit the unsharded per-token path
+    x = _llm_like(16, 128, seed=72)
+    inv = (np.random.default_rng(73).random(128) + 0.5).astype(np.float32)
+    qw = np.random.default_rng(74).integers(-127, 128, (40, 128)).astype(np.int8)
+    sw = (np.random.default_rng(75).random(40) * 0.01).astype(np.float32)
+    q, sx = orc.quant_act_per_token(x, inv)
+    y_full = orc.dequant(orc.gemm_i8(q, qw), sx, sw, out="f32")
+    cuts = [0, 48, 80, 128]
+    sx_g = np.max([orc.quant_act_per_token(x[:, a:b], inv[a:b])[1] for a, b in zip(cuts, cuts[1:])], axis=0)
+    np.testing.assert_array_equal(sx_g, sx)
+    acc = sum(orc.gemm_i8(orc.quant_act_given_scale(x[:, a:b], inv[a:b], sx_g), qw[:, a:b])
+              for a, b in zip(cuts, cuts[1:]))
+    np.testing.assert_array_equal(orc.dequant(acc, sx_g, sw, out="f32"), y_full)
+
+
 # ------------------------------------------------- LayerNorm fused with step 4
 # SmoothQuant page section 1 (the scaling moves into the op that produces X);
 # CUDA INT8 notes 4.2 (fuse quantization with the neighbouring kernel).
