@@ -227,6 +227,28 @@ sq_status sq_layernorm_quant(const void *h, sq_dtype ht, int64_t M, int64_t K, c
                              const float *beta, float eps, const float *inv_s, int8_t *q_out,
                              float *scale_out, void *stream);
 
+/* ---------------------------------------- row-parallel (K-sharded) linear
+ * The exchange of a linear whose K is split across ranks: each rank takes
+ * its slice's per-token scales (quant_act_per_token), the ranks all-reduce
+ * them with MAX (x -> fl(x / 127) is monotonic, so this is the unsharded
+ * scale), quantize their slices at that scale, multiply (w8a8_gemm_dequant
+ * with acc_out), all-reduce the int32 accumulators with SUM (exact) and
+ * dequantize the sum.  The result equals the unsharded path bit for bit.
+ *
+ * quant_act_given_scale: q[t,j] = clamp(rint(x[t,j] * inv_s[j] / sx[t]),
+ * -127, 127), 0 where sx[t] == 0 ([CQ] 2.1).  sx: [M] fp32 (device).  Shapes,
+ * dtypes and alignment as quant_act_per_token (K a multiple of 16). */
+sq_status quant_act_given_scale(const void *x, sq_dtype xt, int64_t M, int64_t K,
+                                const float *inv_s, const float *sx, int8_t *q_out,
+                                void *stream);
+
+/* sq_dequant: y[t,n] = yt(((float)acc[t,n] * sx[t]) * sw[n]), the epilogue of
+ * w8a8_gemm_dequant as its own kernel ([CQ] 4.2).  acc: [M,N] int32 and sw
+ * 16-byte aligned; N a multiple of 4; y 8-byte (bf16) or 16-byte (fp32)
+ * aligned. */
+sq_status sq_dequant(const int32_t *acc, const float *sx, const float *sw, int64_t M, int64_t N,
+                     void *y, sq_dtype yt, void *stream);
+
 /* ------------------------------------------- static activation scale (next)
  * A per-tensor activation range calibrated offline instead of the per-token
  * scales of step 4: the moving-average abs-max of "PaddleNLP GPT

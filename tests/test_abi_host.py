@@ -175,6 +175,17 @@ def test_layernorm_quant_rejects(lib, case, status):
     assert rc == status, _detail(lib)
 
 
+def test_sharded_helpers_reject(lib):
+    assert lib.quant_act_given_scale(P(), 1, 4, 64, NULL, NULL, P(8192), None) == 1
+    assert lib.quant_act_given_scale(P(), 1, 4, 40, NULL, P(4096), P(8192), None) == 2
+    assert lib.quant_act_given_scale(P(), 1, 4, 64, NULL, P(4096), P(8200), None) == 4
+    assert lib.quant_act_given_scale(NULL, 1, 0, 64, NULL, NULL, NULL, None) == 0
+    assert lib.sq_dequant(P(), P(4096), P(8192), 4, 16, NULL, 1, None) == 1
+    assert lib.sq_dequant(P(), P(4096), P(8192), 4, 18, P(12288), 1, None) == 2
+    assert lib.sq_dequant(P(4), P(4096), P(8192), 4, 16, P(12288), 1, None) == 4
+    assert lib.sq_dequant(P(), P(4096), P(8192), 4, 16, P(12288), 7, None) == 3
+
+
 def test_quant_rowsum_rejects_misaligned(lib):
     assert lib.quant_act_per_token_rowsum(P(), 1, 4, 64, NULL, P(8192), P(12288), P(2), None) == 4
 

@@ -103,3 +103,64 @@ def test_single_rank_helpers_are_noops():
     assert torch.equal(ax, torch.arange(8, dtype=torch.float32))
     assert wdist.max_over_ranks(3.5) == 3.5
     assert wdist.world_size() == 1
+
+
+# ------------------------------------------------------------ K-sharded linear
+class _OracleOps:
+    """The kernels of the K-sharded linear, computed by the CPU oracle (this
+    checks the exchange itself: MAX of scales, exact SUM of products)."""
+
+    def __init__(self, oracle):
+        self.o = oracle
+
+    def per_token_scales(self, x, inv_s):
+        return torch.from_numpy(self.o.quant_act_per_token(x.numpy(), inv_s.numpy())[1].copy())
+
+    def quant_given(self, x, inv_s, sx):
+        return torch.from_numpy(self.o.quant_act_given_scale(x.numpy(), inv_s.numpy(), sx.numpy()))
+
+    def gemm_acc(self, qx, qw, sx, sw):
+        return torch.from_numpy(self.o.gemm_i8(qx.numpy(), qw.numpy()))
+
+    def dequant(self, acc, sx, sw, y):
+        y.copy_(torch.from_numpy(self.o.dequant(acc.numpy(), sx.numpy(), sw.numpy(), out="f32")))
+
+
+def _row_parallel_worker(rank, world, port, outdir):
+    _init(rank, world, port)
+    try:
+        import oracle
+        from w8a8_linear_layers_b200 import distributed as wdist
+        r = np.random.default_rng(0)
+        K = 96
+        x = (r.standard_normal((12, K)) * np.where(np.arange(K) % 17 == 0, 30.0, 1.0)).astype(np.float32)
+        inv = (r.random(K) + 0.5).astype(np.float32)
+        qw = r.integers(-127, 128, (24, K)).astype(np.int8)
+        sw = (r.random(24) * 0.01).astype(np.float32)
+        cut = [0, 48, 96][rank:rank + 2]
+        sl = slice(cut[0], cut[1])
+        y = torch.empty(12, 24)
+        wdist.row_parallel_linear(torch.from_numpy(x[:, sl].copy()), torch.from_numpy(inv[sl].copy()),
+                                  torch.from_numpy(qw[:, sl].copy()), torch.from_numpy(sw), y,
+                                  ops=_OracleOps(oracle))
+        np.save(os.path.join(outdir, "y%d.npy" % rank), y.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_row_parallel_linear_equals_unsharded():
+    import oracle
+    port = _free_port()
+    with tempfile.TemporaryDirectory() as d:
+        mp.spawn(_row_parallel_worker, args=(2, port, d), nprocs=2, join=True)
+        ys = [np.load(os.path.join(d, "y%d.npy" % r)) for r in range(2)]
+    r = np.random.default_rng(0)
+    K = 96
+    x = (r.standard_normal((12, K)) * np.where(np.arange(K) % 17 == 0, 30.0, 1.0)).astype(np.float32)
+    inv = (r.random(K) + 0.5).astype(np.float32)
+    qw = r.integers(-127, 128, (24, K)).astype(np.int8)
+    sw = (r.random(24) * 0.01).astype(np.float32)
+    q, sx = oracle.quant_act_per_token(x, inv)
+    want = oracle.dequant(oracle.gemm_i8(q, qw), sx, sw, out="f32")
+    for y in ys:
+        np.testing.assert_array_equal(y, want)

@@ -1,0 +1,64 @@
+"""GPU pieces of the K-sharded (row-parallel) linear, against the oracle and
+against the unsharded path (ranks emulated on one GPU: each shard's kernels
+run in turn and the MAX / SUM exchange is taken on the device between them;
+no kernel waits on another)."""
+import numpy as np
+import pytest
+import torch
+
+from tests.test_parity_gpu import Guarded, make_x, np32, w  # noqa: F401  (w: module fixture)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("M,K,dtype", [(1, 16, torch.float32), (77, 528, torch.bfloat16), (300, 4096, torch.bfloat16)])
+def test_quant_act_given_scale_bit_exact(w, orc, M, K, dtype):
+    x = make_x(M, K, dtype, seed=M + K)
+    inv = (np.random.default_rng(K).random(K) + 0.5).astype(np.float32)
+    _, sx = orc.quant_act_per_token(np32(x), inv)
+    sx = (sx * np.float32(0.7)).astype(np.float32)  # narrower than each row: saturation
+    sx[0] = 0.0
+    q = Guarded((M, K), torch.int8)
+    w.quant_act_given_scale(x.cuda(), torch.from_numpy(inv).cuda(), torch.from_numpy(sx).cuda(), q.t)
+    np.testing.assert_array_equal(q.t.cpu().numpy(), orc.quant_act_given_scale(np32(x), inv, sx))
+    assert q.intact()
+
+
+@pytest.mark.parametrize("M,N,ydt", [(1, 4, torch.float32), (77, 264, torch.bfloat16), (300, 1028, torch.float32)])
+def test_dequant_bit_exact(w, orc, M, N, ydt):
+    r = np.random.default_rng(M * N)
+    acc = r.integers(-2**30, 2**30, (M, N)).astype(np.int32)
+    sx = (r.random(M) * 1e-3).astype(np.float32)
+    sw = (r.random(N) * 1e-3).astype(np.float32)
+    y = Guarded((M, N), ydt)
+    w.sq_dequant(torch.from_numpy(acc).cuda(), torch.from_numpy(sx).cuda(), torch.from_numpy(sw).cuda(), y.t)
+    if ydt == torch.bfloat16:
+        np.testing.assert_array_equal(y.t.cpu().view(torch.int16).numpy().view(np.uint16), orc.dequant(acc, sx, sw))
+    else:
+        np.testing.assert_array_equal(y.t.cpu().numpy(), orc.dequant(acc, sx, sw, out="f32"))
+    assert y.intact()
+
+
+def test_row_parallel_emulated_equals_unsharded(w):
+    from w8a8_linear_layers_b200.distributed import KernelOps
+    ops = KernelOps(w)
+    M, K, N = 256, 4096, 1024
+    x = make_x(M, K, torch.bfloat16, seed=9).cuda()
+    inv = torch.rand(K, device="cuda") + 0.5
+    qw = torch.randint(-127, 128, (N, K), dtype=torch.int8, device="cuda")
+    sw = torch.rand(N, device="cuda") * 1e-3
+    # unsharded
+    qx = torch.empty(M, K, dtype=torch.int8, device="cuda")
+    sx = torch.empty(M, device="cuda")
+    w.quant_act_per_token(x, inv, qx, sx)
+    y_full = torch.empty(M, N, device="cuda")
+    w.w8a8_gemm_dequant(qx, sx, qw, sw, y_full)
+    # four shards of K
+    cuts = [0, 1024, 1536, 3072, 4096]
+    parts = [(x[:, a:b].contiguous(), inv[a:b].contiguous(), qw[:, a:b].contiguous()) for a, b in zip(cuts, cuts[1:])]
+    sx_g = torch.stack([ops.per_token_scales(xs, iv) for xs, iv, _ in parts]).amax(0)
+    assert torch.equal(sx_g, sx)
+    acc = sum(ops.gemm_acc(ops.quant_given(xs, iv, sx_g), q, sx_g, sw) for xs, iv, q in parts)
+    y = torch.empty(M, N, device="cuda")
+    ops.dequant(acc.to(torch.int32), sx_g, sw, y)
+    assert torch.equal(y, y_full)

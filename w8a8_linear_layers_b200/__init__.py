@@ -28,7 +28,7 @@ EXPORTS = ["sq_status_string", "sq_last_error_detail", "sq_abi_version", "sq_dev
            "sq_calib_absmax", "sq_smooth_fold", "ssz_quant_weight", "quant_act_per_token",
            "w8a8_gemm_dequant", "sq_static_range_update", "quant_act_static", "quant_act_per_token_rowsum",
            "ssz_quant_weight_asym", "w8a8_gemm_dequant_asym", "sq_pack_int4", "w4a8_gemm_dequant",
-           "sq_layernorm_quant"]
+           "sq_layernorm_quant", "quant_act_given_scale", "sq_dequant"]
 
 
 class W8A8Error(RuntimeError):
@@ -63,6 +63,8 @@ def _load() -> ctypes.CDLL:
         "w8a8_gemm_dequant_asym": ([P, P, P, P, P, P, I64, I64, I64, P, I, P, P], I),
         "sq_pack_int4": ([P, I64, I64, P, P], I),
         "sq_layernorm_quant": ([P, I, I64, I64, P, P, F, P, P, P, P], I),
+        "quant_act_given_scale": ([P, I, I64, I64, P, P, P, P], I),
+        "sq_dequant": ([P, P, P, I64, I64, P, I, P], I),
         "w4a8_gemm_dequant": ([P, P, P, P, I64, I64, I64, P, I, P, P], I),
     }
     for name, (args, res) in sig.items():
@@ -232,6 +234,26 @@ def sq_layernorm_quant(h: torch.Tensor, gamma: torch.Tensor | None, beta: torch.
     _check("sq_layernorm_quant", lib.sq_layernorm_quant(_ptr(h), _dtype(h), M, K, _ptr(gamma), _ptr(beta),
                                                          float(eps), _ptr(inv_s), _ptr(q_out), _ptr(scale_out),
                                                          _stream(stream)))
+
+
+def quant_act_given_scale(x: torch.Tensor, inv_s: torch.Tensor | None, sx: torch.Tensor, q_out: torch.Tensor,
+                          stream=None) -> None:
+    """int8 codes of x * inv_s at the given per-row scales sx."""
+    _need(inv_s, torch.float32, "inv_s")
+    _need(sx, torch.float32, "sx")
+    _need(q_out, torch.int8, "q_out")
+    M, K = x.shape
+    _check("quant_act_given_scale", lib.quant_act_given_scale(_ptr(x), _dtype(x), M, K, _ptr(inv_s), _ptr(sx),
+                                                               _ptr(q_out), _stream(stream)))
+
+
+def sq_dequant(acc: torch.Tensor, sx: torch.Tensor, sw: torch.Tensor, y: torch.Tensor, stream=None) -> None:
+    """y = ((float)acc * sx[row]) * sw[col] from int32 accumulators."""
+    _need(acc, torch.int32, "acc")
+    _need(sx, torch.float32, "sx")
+    _need(sw, torch.float32, "sw")
+    M, N = acc.shape
+    _check("sq_dequant", lib.sq_dequant(_ptr(acc), _ptr(sx), _ptr(sw), M, N, _ptr(y), _dtype(y), _stream(stream)))
 
 
 def sq_pack_int4(q: torch.Tensor, packed: torch.Tensor, stream=None) -> None:
