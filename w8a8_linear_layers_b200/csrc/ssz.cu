@@ -41,9 +41,9 @@
 // The search is a chain of rounds per channel, so the kernel is latency
 // bound; it keeps many channels in flight (small CTAs, shared-memory rows)
 // and keeps each round's serial tail short: warp trees skip warps whose
-// codes did not move, warp 0 alone takes the decision (the exact error in
-// fp64 and the next candidate) and shares it through shared memory, so the
-// other warps skip that fp64 work.
+// codes did not move, and with four or more warps a channel warp 0 alone
+// takes the decision (the exact error in fp64 and the next candidate) and
+// shares it through shared memory, so the other warps skip that fp64 work.
 #include "common.cuh"
 #include "dd.cuh"
 
@@ -359,7 +359,11 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
             if (lane == 0) part[par][warp] = {p.num, {0.0, 0.0}, p.den};
             __syncthreads();  // the candidate codes and all partials are in place
             ++it;
-            if (warp == 0) {  // warp 0 decides; the others read the decision
+            // The decision: every thread takes it (1-2 warps a channel), or
+            // warp 0 takes it and shares it (4 or more warps, where the
+            // saved fp64 work outweighs one more barrier; measured).
+            const bool shared_decision = nwarps >= 4;
+            if (!shared_decision || warp == 0) {
                 dd num_c = NUM;
                 int den_c = DEN;
                 for (int i = 0; i < nwarps; ++i) {
@@ -367,7 +371,8 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
                     den_c += part[par][i].den;
                 }
                 const double m_c = exact_error_k(W2, num_c, den_c, c);
-                const float c_next = ls_candidate(num_c, den_c, c);
+                const float c_next = ls_candidate(num_c, den_c, c);  // used only if c is kept
+                // on K-scaled errors: d/e < thr <=> dK < thr eK (eK > 0), |d| < thr <=> |dK| < thr K
                 const double delta = m_best - m_c;
                 bool dn = (m_best == 0.0) || (delta < kSszThreshold * m_best) || (fabs(delta) < thr_k) ||
                           it == max_iters;
@@ -377,19 +382,33 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
                     NUM = num_c;
                     DEN = den_c;
                 } else {
-                    dn = true;
+                    dn = true;  // implied by the tests above (m_best >= 0); stated for the restore below
                 }
-                if (lane == 0) decision[par] = {c_next, keep ? 1 : 0, dn ? 1 : 0};
+                if (shared_decision) {
+                    if (lane == 0) decision[par] = {c_next, keep ? 1 : 0, dn ? 1 : 0};
+                } else {
+                    done = dn;
+                    if (keep) {
+                        s_best = c;
+                        c = c_next;
+                    } else {
+                        rejected = true;
+                    }
+                }
             }
-            __syncthreads();
-            const Decision dcs = decision[par];
-            done = dcs.done != 0;
-            if (dcs.keep) {
-                s_best = c;
-                c = dcs.c_next;
-            } else {
-                rejected = true;
+            if (shared_decision) {
+                __syncthreads();
+                const Decision dcs = decision[par];
+                done = dcs.done != 0;
+                if (dcs.keep) {
+                    s_best = c;
+                    c = dcs.c_next;
+                } else {
+                    rejected = true;
+                }
             }
+            // part[par] and decision[par] are rewritten two rounds from now,
+            // after another barrier
         }
         if (rejected) restore_chunks(wrow, touched, s_best, qmax, wmax, q);
 
