@@ -1063,6 +1063,14 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     }
 }
 
+}  // namespace gemm
+}  // namespace w8a8
+
+#include "gemm_decode.cuh"
+
+namespace w8a8 {
+namespace gemm {
+
 // Packs int8 codes in [-8, 7] two per byte (element 2i in the low nibble);
 // one thread per 8 output bytes.
 __global__ void pack_int4_kernel(const int8_t *__restrict__ q, int64_t total_out8, uint8_t *__restrict__ out) {
@@ -1166,6 +1174,65 @@ static sq_status launch_w4(const int8_t *qx, const float *sx, const uint8_t *qw4
     return launch_status("w4a8_gemm_kernel");
 }
 
+// K split of the decode kernel: the largest power of two S <= 8 with
+// tiles x S CTAs <= two per SM and S <= k-blocks (every CTA gets one).
+static int decode_split(int N, int K, int sms) {
+    const int tiles = (N + kDecRows - 1) / kDecRows;
+    const int num_kb = (K + BK - 1) / BK;
+    int s = 1;
+    while (s < kDecMaxSplit && tiles * (2 * s) <= 2 * sms && 2 * s <= num_kb) s *= 2;
+    return s;
+}
+
+template <int NT, typename OutT, bool ASYM, bool INT4>
+static sq_status launch_decode(const int8_t *qx, const float *sx, const int32_t *rs, const void *qw,
+                               const float *sw, const float *ow, int M, int N, int K, void *y, int32_t *acc_out,
+                               int sms, cudaStream_t st) {
+    using C = CfgDec<NT, INT4>;
+    CUtensorMap mw, mx;
+    const bool okw = INT4 ? make_map_int4(&mw, qw, N, K, kDecRows) : make_map(&mw, qw, N, K, kDecRows);
+    if (!okw || !make_map(&mx, qx, M, K, NT))
+        return fail(SQ_ERR_CUDA, "w8a8 decode GEMM: cuTensorMapEncodeTiled failed");
+    auto kern = w8a8_gemm_decode_kernel<NT, OutT, ASYM, INT4>;
+    static int configured_dev[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !configured_dev[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        // the whole shared-memory carveout, so that two CTAs fit an SM
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return fail(SQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        configured_dev[dev] = 1;
+    }
+    const int split = decode_split(N, K, sms);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(((N + kDecRows - 1) / kDecRows) * split), 1, 1);
+    cfg.blockDim = dim3(dec_threads(INT4), 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mw, mx, sx, sw, rs, ow, (OutT *)y, acc_out, M, N, K);
+    if (e != cudaSuccess) return fail(SQ_ERR_CUDA, "w8a8_gemm_decode_kernel launch: %s", cudaGetErrorString(e));
+    return launch_status("w8a8_gemm_decode_kernel");
+}
+
+// Token-tile width of the decode kernel for M <= 64 tokens.
+template <typename OutT, bool ASYM, bool INT4>
+static sq_status dispatch_decode(const int8_t *qx, const float *sx, const int32_t *rs, const void *qw,
+                                 const float *sw, const float *ow, int M, int N, int K, void *y, int32_t *acc_out,
+                                 int sms, cudaStream_t st) {
+    if (M <= 16) return launch_decode<16, OutT, ASYM, INT4>(qx, sx, rs, qw, sw, ow, M, N, K, y, acc_out, sms, st);
+    if (M <= 32) return launch_decode<32, OutT, ASYM, INT4>(qx, sx, rs, qw, sw, ow, M, N, K, y, acc_out, sms, st);
+    return launch_decode<64, OutT, ASYM, INT4>(qx, sx, rs, qw, sw, ow, M, N, K, y, acc_out, sms, st);
+}
+
 template <int BN, typename OutT, bool ASYM>
 static sq_status launch(const int8_t *qx, const float *sx, const int32_t *rs, const int8_t *qw, const float *sw,
                         const float *ow, int M, int N, int K, void *y, int32_t *acc_out, int sms, cudaStream_t st) {
@@ -1242,7 +1309,17 @@ static sq_status gemm_entry(const char *fn, const int8_t *qx, const float *sx, c
     if (st != SQ_OK) return st;
     cudaStream_t cs = (cudaStream_t)stream;
     const int m = (int)M, n = (int)N, k = (int)K;
-    // M > 128: 256-row tiles on CTA pairs; otherwise one CTA per 128 x 256 tile
+    // M <= 64: the weight-streaming decode kernel; M > 128: 256-row tiles on
+    // CTA pairs; otherwise one CTA per 128 x 256 tile
+    if (M <= gemm::kDecMaxTokens) {
+        if (yt == SQ_BF16)
+            return asym ? gemm::dispatch_decode<__nv_bfloat16, true, false>(qx, sx, rs, qw, sw, ow, m, n, k, y,
+                                                                            acc_out, sms, cs)
+                        : gemm::dispatch_decode<__nv_bfloat16, false, false>(qx, sx, rs, qw, sw, ow, m, n, k, y,
+                                                                             acc_out, sms, cs);
+        return asym ? gemm::dispatch_decode<float, true, false>(qx, sx, rs, qw, sw, ow, m, n, k, y, acc_out, sms, cs)
+                    : gemm::dispatch_decode<float, false, false>(qx, sx, rs, qw, sw, ow, m, n, k, y, acc_out, sms, cs);
+    }
     if (M > gemm::BM) {
         if (yt == SQ_BF16)
             return asym ? gemm::launch_pair<__nv_bfloat16, true>(qx, sx, rs, qw, sw, ow, m, n, k, y, acc_out, sms, cs)
@@ -1293,6 +1370,14 @@ extern "C" sq_status w4a8_gemm_dequant(const int8_t *qx, const float *sx, const 
     sq_status st = check_device(&sms);
     if (st != SQ_OK) return st;
     cudaStream_t cs = (cudaStream_t)stream;
+    if (yt == SQ_BF16)
+    if (M <= gemm::kDecMaxTokens) {
+        if (yt == SQ_BF16)
+            return gemm::dispatch_decode<__nv_bfloat16, false, true>(qx, sx, nullptr, qw4, sw, nullptr, (int)M,
+                                                                     (int)N, (int)K, y, acc_out, sms, cs);
+        return gemm::dispatch_decode<float, false, true>(qx, sx, nullptr, qw4, sw, nullptr, (int)M, (int)N, (int)K, y,
+                                                         acc_out, sms, cs);
+    }
     if (yt == SQ_BF16)
         return gemm::launch_w4<__nv_bfloat16>(qx, sx, qw4, sw, (int)M, (int)N, (int)K, y, acc_out, sms, cs);
     return gemm::launch_w4<float>(qx, sx, qw4, sw, (int)M, (int)N, (int)K, y, acc_out, sms, cs);

@@ -1,0 +1,355 @@
+// gemm_decode.cuh -- the W8A8 / W4A8 GEMM for few tokens (M <= 64), included
+// by gemm.cu (it shares that file's PTX wrappers and fault word).
+//
+// Same operation as w8a8_gemm_kernel: y = dequant(qx qw^T) (CUDA INT8
+// quantization notes, aicoding.csdn.net, sections 3.2 and 4.2).  With few
+// tokens the product is bound by the weight bytes, and a 128 x 256 tile per
+// CTA leaves most of the tensor-core tile empty and only N/256 CTAs to
+// stream the weights.  Here the operands swap roles:
+//
+//   * the MMA's A operand (M = 128, TMEM lanes) is a 128-row weight tile,
+//     its B operand (N = NT = 16, 32 or 64) the token tile; D[n][t] lands
+//     in TMEM lane n, column t, so the epilogue thread of weight row n
+//     writes y[t][n] for every token (32 lanes = 32 consecutive columns of
+//     y: coalesced);
+//   * one CTA per 128 weight rows, about 108 KB of shared memory so that two
+//     CTAs share an SM, every CTA resident at once: the weight stream is
+//     spread over all SMs and HBM shares itself among the CTAs;
+//   * where N / 128 tiles are too few to fill the SMs, the K dimension is
+//     split over a thread-block cluster of S CTAs (S <= 8): each CTA
+//     accumulates its share of the k-blocks, writes the int32 partial to
+//     its shared memory, and after a cluster barrier CTA rank r sums the
+//     S partials of rows [r 128/S, (r+1) 128/S) through distributed shared
+//     memory (exact int32) and runs the dequant for them.  No global
+//     scratch memory;
+//   * int4 weights (two per byte) arrive packed and are unpacked to the
+//     int8 operand layout (three unpacked tiles in flight) by eight
+//     converter warps, the first four of which then run the epilogue.
+//
+// Warp roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps
+// 2..5 epilogue (int4: warps 2..9 convert first).  Every wait is bounded as in the
+// other GEMM kernels; no TMA multicast.
+
+namespace w8a8 {
+namespace gemm {
+
+#ifndef W8A8_DEC_OP_STAGES
+#define W8A8_DEC_OP_STAGES 3
+#endif
+#ifndef W8A8_DEC_CONV_WARPS
+#define W8A8_DEC_CONV_WARPS 8
+#endif
+constexpr int kDecRows = 128;  // weight rows per CTA (= MMA M = TMEM lanes)
+constexpr int kDecConvWarps = W8A8_DEC_CONV_WARPS;  // int4 unpacking warps (the first 4 also run the epilogue)
+// producer, MMA, then 4 epilogue warps (int4: the converter warps)
+__host__ __device__ constexpr int dec_threads(bool int4) { return 64 + 32 * (int4 ? kDecConvWarps : 4); }
+constexpr int kDecMaxSplit = 8;   // portable cluster size
+constexpr int kDecMaxTokens = 64;
+constexpr int kDecBudget = 108 * 1024;  // dynamic shared memory, two CTAs per SM
+
+template <int NT, bool INT4>
+struct CfgDec {
+    static constexpr int W_BYTES = kDecRows * BK;                         // int8 weight tile (MMA A)
+    static constexpr int RAW_BYTES = INT4 ? kDecRows * BK / 2 : W_BYTES;  // weight tile as loaded
+    static constexpr int X_BYTES = NT * BK;                               // token tile (MMA B)
+    static constexpr int IN_BYTES = RAW_BYTES + X_BYTES;
+    static constexpr int OP_STAGES = INT4 ? W8A8_DEC_OP_STAGES : 0;  // unpacked weight tiles
+    static constexpr int IN_OFFSET = OP_STAGES * W_BYTES;
+    static constexpr int STAGES_FIT = (kDecBudget - IN_OFFSET) / IN_BYTES;
+    static constexpr int STAGES = STAGES_FIT < 8 ? STAGES_FIT : 8;
+    static constexpr int SMEM = IN_OFFSET + STAGES * IN_BYTES + 1024;  // + alignment slack
+    static constexpr int TMEM_COLS = NT < 32 ? 32 : NT;
+    static constexpr int RED_BYTES = NT * kDecRows * 4;  // int32 partial, over the stages
+    static_assert(STAGES >= 3, "decode pipeline too shallow");
+    static_assert(IN_BYTES % 1024 == 0 && RAW_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
+    static_assert(RED_BYTES <= STAGES * IN_BYTES, "partial must fit over the stages");
+};
+
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t local, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
+    int v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+// 16 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// y[t][n] (and acc_out[t][n]) from the full accumulator of weight row n and
+// token t.
+template <typename OutT, bool ASYM>
+__device__ __forceinline__ void dec_store(int32_t acc, int t, int n, int N, const float *__restrict__ sx,
+                                          const int32_t *__restrict__ rs, float swv, float owv,
+                                          OutT *__restrict__ y, int32_t *__restrict__ acc_out) {
+    const float v = dequant1<ASYM>((uint32_t)acc, sx[t], ASYM ? rs[t] : 0, swv, owv);
+    const int64_t at = (int64_t)t * N + n;
+    if (sizeof(OutT) == 2)
+        reinterpret_cast<__nv_bfloat16 *>(y)[at] = __float2bfloat16_rn(v);
+    else
+        reinterpret_cast<float *>(y)[at] = v;
+    if (acc_out) acc_out[at] = acc;
+}
+
+// Synchronisation:
+//   in_full[s]  : producer's expect_tx; the weight and token TMAs complete it.
+//   in_empty[s] : MMA commit (the MMA is the last reader of a stage).
+//   op_full[p]  : int4: one arrival per converter thread after its fenced
+//                 writes (it waited for in_full first, so op_full implies it).
+//   op_empty[p] : int4: MMA commit.
+//   tfull       : MMA commit after the CTA's last k-block.
+template <int NT, typename OutT, bool ASYM, bool INT4>
+__global__ void __launch_bounds__(dec_threads(INT4), 2)
+w8a8_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+                        const float *__restrict__ sx, const float *__restrict__ sw,
+                        const int32_t *__restrict__ rs, const float *__restrict__ ow, OutT *__restrict__ y,
+                        int32_t *__restrict__ acc_out, int M, int N, int K) {
+    using C = CfgDec<NT, INT4>;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t in_full[C::STAGES];
+    __shared__ __align__(8) uint64_t in_empty[C::STAGES];
+    __shared__ __align__(8) uint64_t op_full[INT4 ? C::OP_STAGES : 1];
+    __shared__ __align__(8) uint64_t op_empty[INT4 ? C::OP_STAGES : 1];
+    __shared__ __align__(8) uint64_t tfull_bar;
+    __shared__ __align__(8) uint64_t drain_bar;
+    __shared__ uint32_t tmem_slot;
+    __shared__ volatile int abort_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;  // 1024-aligned for 128B swizzle
+    uint8_t *gbase = smem_raw + (smem_base - smem_u32(smem_raw));      // the same bytes, generic address
+
+    // K split over the cluster (1 CTA, rank 0, without a cluster launch)
+    const int split = (int)cluster_nctarank();
+    const int rank = (int)cluster_ctarank();
+    const int n0 = (int)(blockIdx.x / split) * kDecRows;
+    const int num_kb = (K + BK - 1) / BK;
+    const int kb0 = (int)((int64_t)num_kb * rank / split);
+    const int kb1 = (int)((int64_t)num_kb * (rank + 1) / split);  // the host keeps kb1 > kb0
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(smem_u32(&in_full[s]), 1);
+            mbar_init(smem_u32(&in_empty[s]), 1);
+        }
+        for (int p = 0; p < C::OP_STAGES; ++p) {
+            mbar_init(smem_u32(&op_full[p]), kDecConvWarps * 32);
+            mbar_init(smem_u32(&op_empty[p]), 1);
+        }
+        mbar_init(smem_u32(&tfull_bar), 1);
+        mbar_init(smem_u32(&drain_bar), 1);
+        abort_flag = 0;
+        fence_barrier_init();
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tmap_w) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tmap_x) : "memory");
+    }
+    if (warp == 1) tmem_alloc(smem_u32(&tmem_slot), C::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            bool ok = true;
+            for (int kb = kb0; kb < kb1; ++kb) {
+                if (!wait_bounded(smem_u32(&in_empty[stage]), phase ^ 1u, &abort_flag, kFaultProducer)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t w_dst = smem_base + C::IN_OFFSET + stage * C::IN_BYTES;
+                const uint32_t fb = smem_u32(&in_full[stage]);
+                mbar_arrive_expect_tx(fb, C::IN_BYTES);
+                tma_load_2d(w_dst, &tmap_w, fb, INT4 ? kb * (BK / 2) : kb * BK, n0);
+                tma_load_2d(w_dst + C::RAW_BYTES, &tmap_x, fb, kb * BK, 0);
+                ++issued;
+                if (++stage == C::STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) {
+                // drain: wait (bounded) for the copies of the last issued stages
+                int outstanding = issued < C::STAGES ? issued : C::STAGES;
+                int s = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < outstanding; ++i) {
+                    if (--s < 0) {
+                        s = C::STAGES - 1;
+                        ph ^= 1u;
+                    }
+                    const unsigned long long t0 = globaltimer();
+                    while (!mbar_try_wait(smem_u32(&in_full[s]), ph) && globaltimer() - t0 < kWaitNs) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_i8(kDecRows, NT);
+            int stage = 0, os = 0;
+            uint32_t phase = 0, oph = 0;
+            bool ok = true, issued_any = false;
+            for (int kb = kb0; kb < kb1; ++kb) {
+                const uint32_t bar = INT4 ? smem_u32(&op_full[os]) : smem_u32(&in_full[stage]);
+                if (!wait_bounded(bar, INT4 ? oph : phase, &abort_flag, kFaultMmaFull)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t in_addr = smem_base + C::IN_OFFSET + stage * C::IN_BYTES;
+                const uint32_t a_addr = INT4 ? smem_base + os * C::W_BYTES : in_addr;
+                const uint32_t b_addr = in_addr + C::RAW_BYTES;
+#pragma unroll
+                for (int k = 0; k < BK / UMMA_K; ++k)
+                    mma_i8(tmem_base, smem_desc_sw128(a_addr + k * UMMA_K), smem_desc_sw128(b_addr + k * UMMA_K),
+                           idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+                issued_any = true;
+                mma_commit(smem_u32(&in_empty[stage]));
+                if (INT4) mma_commit(smem_u32(&op_empty[os]));
+                if (++stage == C::STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+                if (++os == C::OP_STAGES) {
+                    os = 0;
+                    oph ^= 1u;
+                }
+            }
+            if (ok) {
+                mma_commit(smem_u32(&tfull_bar));
+            } else if (issued_any) {
+                // drain: every MMA issued so far completes before TMEM is freed
+                mma_commit(smem_u32(&drain_bar));
+                const unsigned long long t0 = globaltimer();
+                while (!mbar_try_wait(smem_u32(&drain_bar), 0) && globaltimer() - t0 < kWaitNs) {
+                }
+            }
+        }
+    } else {
+        const int ct = threadIdx.x - 64;
+        bool ok = true;
+        if (INT4) {
+            // ------------------------------------------ converters
+            // A packed tile is 128 rows x 64 bytes: 512 16-byte pieces over
+            // the converter threads; piece i = (row i/4, bytes 16 (i%4) ..),
+            // unpacked into 16-byte chunks 2 (i%4) and 2 (i%4) + 1 of the row
+            // (128B swizzle).
+            int stage = 0, os = 0;
+            uint32_t phase = 0, oph = 0;
+            for (int kb = kb0; kb < kb1; ++kb) {
+                if (!wait_bounded(smem_u32(&op_empty[os]), oph ^ 1u, &abort_flag, kFaultConvert) ||
+                    !wait_bounded(smem_u32(&in_full[stage]), phase, &abort_flag, kFaultConvert)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t *raw = gbase + C::IN_OFFSET + stage * C::IN_BYTES;
+                uint8_t *wdst = gbase + os * C::W_BYTES;
+#pragma unroll
+                for (int it = 0; it < 512 / (32 * kDecConvWarps); ++it) {
+                    const int i = it * (32 * kDecConvWarps) + ct;
+                    const int r = i >> 2, sub = i & 3;
+                    const uint4 p = *reinterpret_cast<const uint4 *>(raw + r * (BK / 2) + sub * 16);
+                    uint32_t o[8];
+                    unpack_int4x8(p.x, o[0], o[1]);
+                    unpack_int4x8(p.y, o[2], o[3]);
+                    unpack_int4x8(p.z, o[4], o[5]);
+                    unpack_int4x8(p.w, o[6], o[7]);
+                    uint8_t *rowp = wdst + (r >> 3) * 1024 + (r & 7) * 128;
+                    *reinterpret_cast<uint4 *>(rowp + (((2 * sub) ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<uint4 *>(rowp + (((2 * sub + 1) ^ (r & 7)) << 4)) =
+                        make_uint4(o[4], o[5], o[6], o[7]);
+                }
+                fence_proxy_async_smem();  // the MMA reads these bytes through the async proxy
+                mbar_arrive(smem_u32(&op_full[os]));
+                if (++stage == C::STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+                if (++os == C::OP_STAGES) {
+                    os = 0;
+                    oph ^= 1u;
+                }
+            }
+        }
+        // ---------------------------------------------- epilogue (warps 2..5)
+        const int quarter = warp & 3;  // TMEM lanes this warp may access
+        const int nl = quarter * 32 + lane;
+        const int n = n0 + nl;
+        if (ok && warp < 6) ok = wait_bounded(smem_u32(&tfull_bar), 0, &abort_flag, kFaultEpilogue);
+        // the TMEM loads below are warp-collective: all lanes or none
+        // (warps 6.. only convert)
+        if (warp < 6 && __all_sync(0xffffffffu, ok)) {
+            tc_fence_after();
+            const float swv = n < N ? sw[n] : 0.0f;
+            const float owv = (ASYM && n < N) ? ow[n] : 0.0f;
+            int32_t *red = reinterpret_cast<int32_t *>(gbase + C::IN_OFFSET);
+#pragma unroll
+            for (int c0 = 0; c0 < NT; c0 += 16) {
+                uint32_t acc[16];
+                tmem_ld16(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c0, acc);
+                if (split == 1) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (c0 + j < M && n < N)
+                            dec_store<OutT, ASYM>((int32_t)acc[j], c0 + j, n, N, sx, rs, swv, owv, y, acc_out);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) red[(c0 + j) * kDecRows + nl] = (int32_t)acc[j];
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (split > 1) {
+        // every CTA of the cluster holds its partial in shared memory: rank r
+        // sums rows [r R, (r + 1) R) of all S partials, R = 128 / S
+        cluster_sync_all();
+        const int rows = kDecRows / split;
+        const uint32_t red_base = smem_base + C::IN_OFFSET;
+        for (int e = threadIdx.x; e < NT * rows; e += (int)blockDim.x) {
+            const int t = e / rows, nl = rank * rows + e % rows;
+            const int n = n0 + nl;
+            if (t < M && n < N) {
+                const uint32_t local = red_base + (uint32_t)((t * kDecRows + nl) * 4);
+                int32_t sum = 0;
+                for (int p = 0; p < split; ++p) sum += ld_cluster_s32(map_to_rank(local, (uint32_t)p));
+                dec_store<OutT, ASYM>(sum, t, n, N, sx, rs, sw[n], ASYM ? ow[n] : 0.0f, y, acc_out);
+            }
+        }
+        cluster_sync_all();  // no CTA leaves while a peer still reads its partial
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+}  // namespace gemm
+}  // namespace w8a8
