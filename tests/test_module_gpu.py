@@ -98,3 +98,20 @@ def test_module_forward_ln_matches_calls(w):
     assert torch.equal(y.float(), yr.float())
     with pytest.raises(ValueError):
         w.W8A8Linear(wt, weights="asym8").forward_ln(x, g, b)
+
+
+@pytest.mark.parametrize("weights,act", [("sym8", "dynamic"), ("int4", "dynamic"), ("asym8", "static")])
+def test_graphed_forward_equals_eager(w, weights, act):
+    x, wt = _setup(seed=7)
+    lin = w.W8A8Linear(wt, alpha=0.5, weights=weights, act_scales=act)
+    lin.calibrate(x)
+    lin.quantize()
+    if act == "static":
+        lin.calibrate_static(x)
+    g = lin.graphed(16)
+    for seed in (1, 2):
+        xi, _ = synthetic.make_small(16, x.shape[1], 8, seed=seed)
+        g.x.copy_(xi.cuda())
+        yg = g.replay().clone()
+        ye = lin.forward(xi.cuda())
+        assert torch.equal(yg.float(), ye.float())

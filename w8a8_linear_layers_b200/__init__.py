@@ -416,6 +416,11 @@ class W8A8Linear:
         self._gemm(qx, sx, rs, y)
         return y
 
+    def graphed(self, M: int, x_dtype: torch.dtype | None = None) -> "GraphedLinear":
+        """forward() for M-token inputs captured in a CUDA graph (see
+        GraphedLinear)."""
+        return GraphedLinear(self, M, x_dtype or self.w.dtype)
+
     def forward_ln(self, h: torch.Tensor, gamma: torch.Tensor | None, beta: torch.Tensor | None,
                    eps: float = 1e-5, y: torch.Tensor | None = None) -> torch.Tensor:
         """forward(LayerNorm(h)) with the LayerNorm, the smoothing and the
@@ -430,3 +435,28 @@ class W8A8Linear:
             y = torch.empty(M, self.N, device=h.device, dtype=self.out_dtype)
         self._gemm(qx, sx, None, y)
         return y
+
+
+class GraphedLinear:
+    """A W8A8Linear's forward for M-token inputs captured once in a CUDA graph
+    (the activation quantization and the GEMM, two kernels): write the input
+    into .x, call replay(), read .y.  Built by W8A8Linear.graphed(M); the
+    layer must be quantized (and, for static scales, calibrated) first."""
+
+    def __init__(self, lin: "W8A8Linear", M: int, x_dtype: torch.dtype):
+        dev = lin.w.device
+        self.x = torch.zeros(M, lin.K, device=dev, dtype=x_dtype)
+        self.y = torch.empty(M, lin.N, device=dev, dtype=lin.out_dtype)
+        self._lin = lin
+        stream = torch.cuda.Stream(device=dev)
+        stream.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(stream):
+            lin.forward(self.x, self.y)  # one eager call: one-time kernel attributes are set outside the capture
+        torch.cuda.current_stream(dev).wait_stream(stream)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            lin.forward(self.x, self.y)
+
+    def replay(self) -> torch.Tensor:
+        self.graph.replay()
+        return self.y
