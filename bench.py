@@ -4,8 +4,9 @@ A step is one pass of the whole path over one batch: per-input-channel
 activation absmax (calibration) -> smoothing factor and weight column absmax
 -> SSZ int8 weight quantization of the smoothed weight -> per-token int8
 activation quantization -> INT8 GEMM with fused dequant.  Inputs are seeded
-synthetic LLM-shaped data resident in HBM; L2 is flushed (a 512 MB write)
-before every timed step, outside the timed events.
+synthetic LLM-shaped data resident in HBM; L2 is flushed (a 512 MB write,
+then a 384 MB read that writes the dirty lines back) before every timed step,
+outside the timed events.
 
 value  = 2*M*N*K int8 ops of the linear per step, over all ranks, divided by
          the step time (max over ranks), in TOPS.
@@ -224,7 +225,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     probs = make_problems(args, torch, rank, dev)
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(torch, dev)
     stream = torch.cuda.current_stream()
 
     def run(p, xin, wt, evs=None, base=0):
@@ -253,7 +254,7 @@ def run_ours(args, rank, world, local_rank):
             run(p, p.x, p.wt, evs, 6 * i)
 
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         step()
     torch.cuda.synchronize()
     if w.device_fault() != 0:
@@ -266,7 +267,7 @@ def run_ours(args, rank, world, local_rank):
     with ClockSampler(local_rank) as clk:
         wall0 = time.perf_counter()
         for i in range(args.steps):
-            flush.zero_()          # L2 flush, outside the timed events
+            flush()                # L2 flush, outside the timed events
             step(evs[i])
         torch.cuda.synchronize()
         wall1 = time.perf_counter()
@@ -292,6 +293,20 @@ def run_ours(args, rank, world, local_rank):
     return finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall1 - wall0, next_rows)
 
 
+class L2Flush:
+    """Evicts the inputs from L2 (126 MB) before a timed region: a 512 MB
+    write, then a 384 MB read, so that the lines the write left dirty are
+    written back here and not by the timed kernels."""
+
+    def __init__(self, torch, dev):
+        self.wbuf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+        self.rbuf = torch.ones(384 << 20, dtype=torch.uint8, device=dev)
+
+    def __call__(self):
+        self.wbuf.zero_()
+        self.rbuf.max()
+
+
 def time_next_rows(args, w, torch, probs, flush, stream, reps=50):
     """Kernels of the rows built beyond the five-step path, timed one launch
     at a time like the path's kernels (L2 flushed before each, outside the
@@ -303,7 +318,8 @@ def time_next_rows(args, w, torch, probs, flush, stream, reps=50):
     - ssz_quant_weight_asym, quant_act_per_token_rowsum and
       w8a8_gemm_dequant_asym: the asymmetric int8 weight path;
     - sq_pack_int4 and w4a8_gemm_dequant (packed int4 weights) against
-      w8a8_gemm_dequant on the 16 x 8192 -> 28672 decode shape.
+      w8a8_gemm_dequant on the 16 x 8192 -> 28672 decode shape;
+    - that decode linear's forward, eager and as a CUDA graph replay.
     Per-launch times include the launch gap that in-step events hide."""
     p = probs[0]
     peaks, _ = load_peaks()
@@ -314,7 +330,7 @@ def time_next_rows(args, w, torch, probs, flush, stream, reps=50):
     def timed(fn):
         ts = []
         for i in range(reps + 3):
-            flush.zero_()
+            flush()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             fn()
@@ -396,6 +412,25 @@ def time_next_rows(args, w, torch, probs, flush, stream, reps=50):
         out[name] = {"us": round(ms * 1e3, 2), "bound": "hbm", "achieved": round(gbs, 1),
                      "peak": round(peaks["hbm_gbs"], 1), "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
                      "algorithmic": {"bytes": nbytes, "ops": 2 * Md * Nd * Kd}, "shape": [Md, Nd, Kd]}
+    # the decode linear's forward (per-token codes, then the GEMM) issued
+    # from Python call by call, and the same two kernels replayed as one
+    # CUDA graph (W8A8Linear.graphed); weights set from the codes above
+    xd = torch.randn(Md, Kd, device=dev, dtype=torch.bfloat16, generator=g)
+    for kind in ("sym8", "int4"):
+        lin = w.W8A8Linear(torch.empty(Nd, Kd, device=dev, dtype=torch.bfloat16), weights=kind)
+        lin.inv_s.fill_(1.0)
+        lin.sw.copy_(swd)
+        if kind == "int4":
+            lin.qw4.copy_(packed)
+        else:
+            lin.qw.copy_(q4)
+        gl = lin.graphed(Md)
+        gl.x.copy_(xd)
+        ms_e = timed(lambda: lin.forward(xd, yd))
+        ms_g = timed(gl.replay)
+        out["decode_forward_" + kind] = {"eager_us": round(ms_e * 1e3, 2), "graph_us": round(ms_g * 1e3, 2),
+                                         "kernels": 2, "shape": [Md, Nd, Kd]}
+        del lin, gl
     ms = timed(lambda: w.sq_pack_int4(q4, packed))
     nbytes = Nd * Kd + Nd * Kd // 2
     gbs = nbytes / (ms * 1e-3) / 1e9
@@ -413,7 +448,7 @@ def run_e2e(args, w, wdist, torch, probs, run, flush, stream, ops_per_step, worl
               torch.empty_like(p.x), torch.empty_like(p.wt)) for p in probs]
     e2e_ms = []
     for i in range(args.warmup + args.e2e_steps):
-        flush.zero_()
+        flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for p, (xh, wh, yh, xd, wd) in zip(probs, hosts):
@@ -504,7 +539,7 @@ def finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall_s, next_
         "config": {"workload": args.workload, "linears": len(probs), "M_tokens_per_gpu": M, "K": K, "N": N,
                    "alpha": p0.alpha, "weight_bits": p0.bits, "ssz_max_iters": p0.max_iters,
                    "parallelism": "dp%d (replicas; MAX all-reduce of the calibration absmax)" % world,
-                   "l2": "flushed (512 MB write) before every timed step, outside the timed events"},
+                   "l2": "flushed (512 MB write, then 384 MB read) before every timed step, outside the timed events"},
         "roofline": roof,
         "kernels": kernels,
         "e2e": e2e,
