@@ -20,10 +20,12 @@
 //   * warp roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
 //     then epilogue warps (TMEM lanes 32*(warp%4) .. +31 each).
 //
-// Three kernels share these pieces: w8a8_gemm_kernel (one CTA per 128 x 256
-// tile, M <= 128), w8a8_gemm_pair_kernel (CTA pairs, cta_group::2, 256 x 256
-// tiles, 8 epilogue warps, M > 128) and w4a8_gemm_kernel (packed int4
-// weights unpacked on chip by converter warps).
+// Four kernels share these pieces: w8a8_gemm_kernel (one CTA per 128 x 256
+// tile, 64 < M <= 128), w8a8_gemm_pair_kernel (CTA pairs, cta_group::2,
+// 256 x 256 tiles, 8 epilogue warps, M > 128), w4a8_gemm_kernel (packed int4
+// weights unpacked on chip by converter warps, M > 64) and, for M <= 64,
+// w8a8_gemm_decode_kernel (gemm_decode.cuh: weights as the 128-row operand,
+// K split over a cluster where the weight tiles are few).
 //
 // Epilogue: tcgen05.ld of 32 accumulator columns per thread (thread = output
 // row), y = ((float)acc * sx[row]) * sw[col] (two fp32 multiplies, int->fp32
