@@ -3,7 +3,8 @@
 A step is one pass of the whole path over one batch: per-input-channel
 activation absmax (calibration) -> smoothing factor and weight column absmax
 -> SSZ int8 weight quantization of the smoothed weight -> per-token int8
-activation quantization -> INT8 GEMM with fused dequant.  Inputs are seeded
+activation quantization -> INT8 GEMM with fused dequant.  On one GPU the step
+is captured once as a CUDA graph and replayed.  Inputs are seeded
 synthetic LLM-shaped data resident in HBM; L2 is flushed (a 512 MB write,
 then a 384 MB read that writes the dirty lines back) before every timed step,
 outside the timed events.
@@ -47,6 +48,9 @@ def parse():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--eager", action="store_true",
+                   help="launch every call of a timed step from Python (default on one GPU: the step is "
+                        "captured once as a CUDA graph and replayed)")
     p.add_argument("--e2e-steps", type=int, default=20)
     p.add_argument("--no-next-rows", action="store_true",
                    help="skip the per-kernel timings of the rows beyond the five-step path")
@@ -231,7 +235,7 @@ def run_ours(args, rank, world, local_rank):
     def run(p, xin, wt, evs=None, base=0):
         def mark(i):
             if evs is not None:
-                evs[base + i].record(stream)
+                evs[base + i].record()  # the current stream: the launching one, or a graph's capture stream
         mark(0)
         w.sq_calib_absmax(xin, p.ax)
         mark(1)
@@ -260,7 +264,26 @@ def run_ours(args, rank, world, local_rank):
     if w.device_fault() != 0:
         raise RuntimeError("a kernel gave up on a bounded wait during warm-up")
 
+    # One GPU: the step is captured once as a CUDA graph (its per-kernel
+    # events included) and replayed every timed step, so that the host's
+    # launch of some 5 calls per linear never holds the GPU back.  Several
+    # ranks launch eagerly (no collective is captured).
+    graph = None
+    if world == 1 and not args.eager:
+        gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(6 * len(probs))]
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step(gev)
+        flush()
+        graph.replay()  # untimed
+        torch.cuda.synchronize()
+
+    def elapsed(e):
+        """Per linear j: [kernel i time for i in 0..4] from a step's events."""
+        return [[e[6 * j + i].elapsed_time(e[6 * j + i + 1]) for i in range(5)] for j in range(len(probs))]
+
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6 * len(probs))] for _ in range(args.steps)]
+    per_step = []
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -268,14 +291,20 @@ def run_ours(args, rank, world, local_rank):
         wall0 = time.perf_counter()
         for i in range(args.steps):
             flush()                # L2 flush, outside the timed events
-            step(evs[i])
+            if graph is not None:
+                graph.replay()
+                torch.cuda.synchronize()  # this step's events, before the next replay records them again
+                per_step.append(elapsed(gev))
+            else:
+                step(evs[i])
         torch.cuda.synchronize()
         wall1 = time.perf_counter()
     if world > 1:
         dist.barrier()
-    step_ms = [sum(e[6 * j].elapsed_time(e[6 * j + 5]) for j in range(len(probs))) for e in evs]
-    kern_ms = {n: statistics.mean(sum(e[6 * j + i].elapsed_time(e[6 * j + i + 1]) for j in range(len(probs)))
-                                  for e in evs) for i, n in enumerate(NAMES)}
+    if graph is None:
+        per_step = [elapsed(e) for e in evs]
+    step_ms = [sum(sum(lin) for lin in st) for st in per_step]
+    kern_ms = {n: statistics.mean(sum(lin[i] for lin in st) for st in per_step) for i, n in enumerate(NAMES)}
     total_ms = wdist.max_over_ranks(sum(step_ms), device=dev)
     if w.device_fault() != 0:
         raise RuntimeError("a kernel gave up on a bounded wait during timing")
@@ -290,7 +319,9 @@ def run_ours(args, rank, world, local_rank):
     e2e = None
     if args.e2e_steps > 0:
         e2e = run_e2e(args, w, wdist, torch, probs, run, flush, stream, ops_per_step, world)
-    return finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall1 - wall0, next_rows)
+    del graph
+    return finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall1 - wall0, next_rows,
+                  launch="eager" if world > 1 or args.eager else "cuda_graph")
 
 
 class L2Flush:
@@ -468,7 +499,7 @@ def run_e2e(args, w, wdist, torch, probs, run, flush, stream, ops_per_step, worl
             "ms_per_step": round(e2e_total / len(e2e_ms), 4)}
 
 
-def finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall_s, next_rows=None):
+def finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall_s, next_rows=None, launch="eager"):
     names = NAMES
     # ---- rooflines per kernel (algorithmic work summed over the workload's linears)
     peaks, src = load_peaks()
@@ -539,7 +570,10 @@ def finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall_s, next_
         "config": {"workload": args.workload, "linears": len(probs), "M_tokens_per_gpu": M, "K": K, "N": N,
                    "alpha": p0.alpha, "weight_bits": p0.bits, "ssz_max_iters": p0.max_iters,
                    "parallelism": "dp%d (replicas; MAX all-reduce of the calibration absmax)" % world,
-                   "l2": "flushed (512 MB write, then 384 MB read) before every timed step, outside the timed events"},
+                   "l2": "flushed (512 MB write, then 384 MB read) before every timed step, outside the timed events",
+                   "launch": {"cuda_graph": "each timed step one CUDA graph replay (captured once, per-kernel "
+                                            "events inside it)",
+                              "eager": "every call of a timed step launched from Python"}[launch]},
         "roofline": roof,
         "kernels": kernels,
         "e2e": e2e,

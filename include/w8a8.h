@@ -118,6 +118,15 @@ sq_status sq_smooth_fold(const float *x_absmax, const void *w, sq_dtype wt,
                          float *s_out, float *inv_s_out, float *w_folded_out,
                          void *stream);
 
+/* The smoothing factor alone, from both abs-max vectors [SQ]: s and inv_s
+ * exactly as sq_smooth_fold computes them, with w_absmax [K] fp32 given
+ * (sq_calib_absmax of w [N,K] is its w_absmax_out).  Splitting step 2 this
+ * way lets the column abs-max of W run on another stream, beside the
+ * activation calibration of step 1.  K a positive multiple of 16; alpha in
+ * [0,1]. */
+sq_status sq_smooth_factor(const float *x_absmax, const float *w_absmax, int64_t K, float alpha,
+                           float *s_out, float *inv_s_out, void *stream);
+
 /* ------------------------------------------------------------------ step 3
  * Per-output-channel symmetric weight quantization with the SSZ scale search
  * [SSZ].  For each output channel n, with w'[k] = w[n,k] * s[k] (s NULL: no

@@ -91,6 +91,15 @@ def test_smooth_fold_rejects_alpha(lib, alpha, status):
     assert "alpha" in _detail(lib)
 
 
+def test_smooth_factor_rejects(lib):
+    assert lib.sq_smooth_factor(NULL, P(4096), 32, 0.5, P(8192), P(12288), None) == 1
+    assert lib.sq_smooth_factor(P(), P(4096), 40, 0.5, P(8192), P(12288), None) == 2
+    assert lib.sq_smooth_factor(P(), P(4096), 0, 0.5, P(8192), P(12288), None) == 2
+    assert lib.sq_smooth_factor(P(), P(4096), 32, 1.5, P(8192), P(12288), None) == 5
+    assert "alpha" in _detail(lib)
+    assert lib.sq_smooth_factor(P(), P(4098), 32, 0.5, P(8192), P(12288), None) == 4
+
+
 @pytest.mark.parametrize("case,status", [
     ("bits6", 5), ("iters_neg", 5), ("iters_big", 5), ("k_big", 2), ("k_odd", 2), ("null_q", 1),
     ("misaligned_s", 4), ("dtype", 3),

@@ -109,6 +109,28 @@ def test_smooth_fold(w, orc, N, K, dtype, alpha):
     assert all(g.intact() for g in (aw_d, s_d, inv_d, fold))
 
 
+@pytest.mark.parametrize("N,K,dtype,alpha", [(13, 48, torch.float32, 0.5), (4096, 4096, torch.bfloat16, 0.5),
+                                             (301, 528, torch.bfloat16, 0.8)])
+def test_smooth_factor_split(w, orc, N, K, dtype, alpha):
+    """Step 2 split in two: the weight's column abs-max by sq_calib_absmax,
+    then sq_smooth_factor -- the same s and 1/s as sq_smooth_fold, and the
+    oracle's."""
+    x = make_x(256, K, dtype, seed=K + 1)
+    wt = (torch.randn(N, K, generator=torch.Generator().manual_seed(N + 1)) * 0.02).to(dtype)
+    ax = orc.calib_absmax(np32(x))
+    ax[1] = 0.0
+    axd = torch.from_numpy(ax).cuda()
+    aw, s1, inv1, aw2 = (torch.empty(K, device="cuda") for _ in range(4))
+    s2, inv2 = Guarded((K,), torch.float32), Guarded((K,), torch.float32)
+    w.sq_smooth_fold(axd, wt.cuda(), alpha, aw, s1, inv1)
+    w.sq_calib_absmax(wt.cuda(), aw2)
+    w.sq_smooth_factor(axd, aw2, alpha, s2.t, inv2.t)
+    assert torch.equal(aw2, aw) and torch.equal(s2.t, s1) and torch.equal(inv2.t, inv1)
+    s_ref, _ = orc.smooth_factor(ax, orc.weight_col_absmax(np32(wt)), alpha)
+    np.testing.assert_allclose(s2.t.cpu().numpy(), s_ref, rtol=1e-5, atol=0)
+    assert s2.intact() and inv2.intact()
+
+
 # --------------------------------------------------------------- step 4
 @pytest.mark.parametrize("M,K,dtype,smooth", [
     (1, 16, torch.float32, False), (5, 48, torch.bfloat16, True), (16, 256, torch.float32, True),

@@ -28,7 +28,7 @@ EXPORTS = ["sq_status_string", "sq_last_error_detail", "sq_abi_version", "sq_dev
            "sq_calib_absmax", "sq_smooth_fold", "ssz_quant_weight", "quant_act_per_token",
            "w8a8_gemm_dequant", "sq_static_range_update", "quant_act_static", "quant_act_per_token_rowsum",
            "ssz_quant_weight_asym", "w8a8_gemm_dequant_asym", "sq_pack_int4", "w4a8_gemm_dequant",
-           "sq_layernorm_quant", "quant_act_given_scale", "sq_dequant"]
+           "sq_layernorm_quant", "quant_act_given_scale", "sq_dequant", "sq_smooth_factor"]
 
 
 class W8A8Error(RuntimeError):
@@ -53,6 +53,7 @@ def _load() -> ctypes.CDLL:
         "sq_selftest_bounded_wait": ([ctypes.c_uint32, P], I),
         "sq_calib_absmax": ([P, I, I64, I64, P, I, P], I),
         "sq_smooth_fold": ([P, P, I, I64, I64, F, P, P, P, P, P], I),
+        "sq_smooth_factor": ([P, P, I64, F, P, P, P], I),
         "ssz_quant_weight": ([P, I, I64, I64, P, I, I, P, P, P, P, P], I),
         "quant_act_per_token": ([P, I, I64, I64, P, P, P, P], I),
         "w8a8_gemm_dequant": ([P, P, P, P, I64, I64, I64, P, I, P, P], I),
@@ -146,6 +147,19 @@ def sq_smooth_fold(x_absmax: torch.Tensor, w: torch.Tensor, alpha: float, w_absm
     _check("sq_smooth_fold", lib.sq_smooth_fold(_ptr(x_absmax), _ptr(w), _dtype(w), N, K, float(alpha),
                                                  _ptr(w_absmax_out), _ptr(s_out), _ptr(inv_s_out),
                                                  _ptr(w_folded_out), _stream(stream)))
+
+
+def sq_smooth_factor(x_absmax: torch.Tensor, w_absmax: torch.Tensor, alpha: float, s_out: torch.Tensor,
+                     inv_s_out: torch.Tensor, stream=None) -> None:
+    """s = ax^alpha / aw^(1-alpha) and 1/s from both abs-max vectors (w_absmax:
+    sq_calib_absmax of the weight), as sq_smooth_fold computes them."""
+    for t, n in ((x_absmax, "x_absmax"), (w_absmax, "w_absmax"), (s_out, "s_out"), (inv_s_out, "inv_s_out")):
+        _need(t, torch.float32, n)
+    K = x_absmax.numel()
+    if w_absmax.numel() != K or s_out.numel() != K or inv_s_out.numel() != K:
+        raise ValueError("x_absmax, w_absmax, s_out and inv_s_out must all hold K values")
+    _check("sq_smooth_factor", lib.sq_smooth_factor(_ptr(x_absmax), _ptr(w_absmax), K, float(alpha), _ptr(s_out),
+                                                     _ptr(inv_s_out), _stream(stream)))
 
 
 def ssz_quant_weight(w: torch.Tensor, s: torch.Tensor | None, bits: int, max_iters: int, q_out: torch.Tensor,

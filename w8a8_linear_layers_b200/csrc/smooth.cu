@@ -215,3 +215,20 @@ extern "C" sq_status sq_smooth_fold(const float *x_absmax, const void *w, sq_dty
         fold_kernel<float><<<blocks, 256, 0, cs>>>((const float *)w, N, K, s_out, w_folded_out);
     return launch_status("fold_kernel");
 }
+
+extern "C" sq_status sq_smooth_factor(const float *x_absmax, const float *w_absmax, int64_t K, float alpha,
+                                      float *s_out, float *inv_s_out, void *stream) {
+    if (!x_absmax || !w_absmax || !s_out || !inv_s_out) return fail(SQ_ERR_NULL, "sq_smooth_factor: NULL pointer");
+    if (K <= 0 || K % 16 != 0)
+        return fail(SQ_ERR_SHAPE, "sq_smooth_factor: K=%lld (a positive multiple of 16)", (long long)K);
+    if (!(alpha >= 0.0f && alpha <= 1.0f))
+        return fail(SQ_ERR_ARG, "sq_smooth_factor: alpha=%g outside [0,1]", (double)alpha);
+    if (!aligned(x_absmax, 4) || !aligned(w_absmax, 4) || !aligned(s_out, 4) || !aligned(inv_s_out, 4))
+        return fail(SQ_ERR_ALIGN, "sq_smooth_factor: misaligned pointer");
+    int sms;
+    sq_status st = check_device(&sms);
+    if (st != SQ_OK) return st;
+    smooth_factor_kernel<<<(unsigned)ceil_div(K, 256), 256, 0, (cudaStream_t)stream>>>(x_absmax, w_absmax, K, alpha,
+                                                                                      s_out, inv_s_out);
+    return launch_status("smooth_factor_kernel");
+}
