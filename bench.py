@@ -305,6 +305,8 @@ def run_ours(args, rank, world, local_rank):
         per_step = [elapsed(e) for e in evs]
     step_ms = [sum(sum(lin) for lin in st) for st in per_step]
     kern_ms = {n: statistics.mean(sum(lin[i] for lin in st) for st in per_step) for i, n in enumerate(NAMES)}
+    # per linear and kernel, mean over the timed steps (for the per-shape table)
+    lin_ms = [[statistics.mean(st[j][i] for st in per_step) for i in range(len(NAMES))] for j in range(len(probs))]
     total_ms = wdist.max_over_ranks(sum(step_ms), device=dev)
     if w.device_fault() != 0:
         raise RuntimeError("a kernel gave up on a bounded wait during timing")
@@ -321,7 +323,7 @@ def run_ours(args, rank, world, local_rank):
         e2e = run_e2e(args, w, wdist, torch, probs, run, flush, stream, ops_per_step, world)
     del graph
     return finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall1 - wall0, next_rows,
-                  launch="eager" if world > 1 or args.eager else "cuda_graph")
+                  launch="eager" if world > 1 or args.eager else "cuda_graph", lin_ms=lin_ms)
 
 
 class L2Flush:
@@ -499,7 +501,25 @@ def run_e2e(args, w, wdist, torch, probs, run, flush, stream, ops_per_step, worl
             "ms_per_step": round(e2e_total / len(e2e_ms), 4)}
 
 
-def finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall_s, next_rows=None, launch="eager"):
+def per_shape_table(probs, lin_ms, peaks):
+    """Workloads of several linears: per distinct (M, K, N) the number of
+    linears, the mean time of each kernel and the GEMM's TOPS."""
+    groups = {}
+    for p, ms in zip(probs, lin_ms):
+        groups.setdefault((p.M, p.K, p.N), []).append(ms)
+    out = {}
+    for (M, K, N), rows in groups.items():
+        mean = [statistics.mean(r[i] for r in rows) for i in range(len(NAMES))]
+        gemm_ms = mean[NAMES.index("w8a8_gemm_dequant")]
+        tops = 2.0 * M * N * K / (gemm_ms * 1e-3) / 1e12
+        out["%dx%d->%d" % (M, K, N)] = {
+            "linears": len(rows), "us": {n: round(m * 1e3, 2) for n, m in zip(NAMES, mean)},
+            "gemm_tops": round(tops, 1), "gemm_frac": round(tops / (peaks["bf16_tflops"] * INT8_OVER_BF16), 4)}
+    return out
+
+
+def finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall_s, next_rows=None, launch="eager",
+           lin_ms=None):
     names = NAMES
     # ---- rooflines per kernel (algorithmic work summed over the workload's linears)
     peaks, src = load_peaks()
@@ -581,6 +601,8 @@ def finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall_s, next_
         "clocks": clk.result,
         "wall_s_timed_region": round(wall_s, 3),
     }
+    if lin_ms is not None and len(probs) > 1:
+        result["per_shape"] = per_shape_table(probs, lin_ms, peaks)
     if next_rows:
         result["next_rows"] = next_rows
     return result

@@ -230,6 +230,7 @@ def _gemm_case(M, N, K, seed, extreme=False):
     (1, 16, 16, torch.bfloat16), (7, 24, 48, torch.bfloat16), (129, 264, 144, torch.bfloat16),
     (128, 256, 128, torch.bfloat16), (256, 512, 256, torch.float32), (16, 128, 256, torch.float32),
     (300, 520, 4096, torch.bfloat16), (1000, 2056, 1040, torch.bfloat16), (16, 28672, 512, torch.bfloat16),
+    (200, 24, 64, torch.bfloat16), (130, 12, 48, torch.float32), (520, 392, 272, torch.float32),
 ])
 def test_gemm_bit_exact(w, orc, M, N, K, ydt):
     qx, qw, sx, sw = _gemm_case(M, N, K, seed=M * 31 + N * 7 + K)

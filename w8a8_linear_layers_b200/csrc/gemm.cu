@@ -138,6 +138,12 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy accesses (TMA stores, tcgen05.mma operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void tmem_alloc(uint32_t slot_smem, uint32_t cols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_smem), "r"(cols)
                  : "memory");
@@ -607,13 +613,91 @@ struct Cfg2 {
     static constexpr int B_BYTES = (BN / 2) * BK;  // 16 KB: this CTA's half of B
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int TMEM_COLS = 2 * BN;    // two 128 x 256 accumulator buffers
-    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024;
+    static constexpr int OUT_BYTES = 32 * 128;  // per epilogue warp: 32 rows x 128 bytes of output
+    static constexpr int OUT_OFFSET = STAGES * STAGE_BYTES;
+    static constexpr int SMEM = OUT_OFFSET + kPairEpiWarps * OUT_BYTES + 1024;
 };
+
+// TMA store of a 2-D box from shared memory, tracked by this thread's bulk
+// groups; waits on the groups this thread committed.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"((uint64_t)map),
+                 "r"(src), "r"(x), "r"(y)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// One 32-row chunk of a warp's output, staged and stored by TMA: the 32
+// lanes' rows (lane = TMEM lane = output row) of CW = 128 / sizeof(OutT)
+// columns from TMEM at taddr, dequantized, packed into the 128B-swizzled
+// layout of the output tensor map's box (16-byte piece c of row r at piece
+// c ^ (r & 7)), fenced to the async proxy and stored at (col, row0) by
+// lane 0.  Columns past N read no scale and are clipped by the store, as are
+// rows past M; a box wholly past either edge is skipped.  `pending`: lane 0
+// has a store that may still read the buffer.
+template <typename OutT, bool ASYM>
+__device__ __forceinline__ void store_chunk_tma(const CUtensorMap *tmap_y, uint32_t taddr, uint32_t buf,
+                                                int lane, int col, int row0, int M, int N, float sxr, int Rr,
+                                                const float *__restrict__ sw, const float *__restrict__ ow,
+                                                bool &pending) {
+    constexpr int CW = 128 / (int)sizeof(OutT);
+    if (col >= N || row0 >= M) return;  // warp-uniform: the whole box lies past the output
+    uint32_t acc[CW];
+    tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&acc[0]));
+    if (CW == 64) tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&acc[CW == 64 ? 32 : 0]));
+    uint32_t packed[32];
+    const bool full = col + CW <= N;
+#pragma unroll
+    for (int j = 0; j < CW; j += 4) {
+        float4 f, o = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (full) {
+            f = __ldg(reinterpret_cast<const float4 *>(sw + col + j));
+            if (ASYM) o = __ldg(reinterpret_cast<const float4 *>(ow + col + j));
+        } else {
+            f.x = col + j < N ? sw[col + j] : 0.f;
+            f.y = col + j + 1 < N ? sw[col + j + 1] : 0.f;
+            f.z = col + j + 2 < N ? sw[col + j + 2] : 0.f;
+            f.w = col + j + 3 < N ? sw[col + j + 3] : 0.f;
+            if (ASYM) {
+                o.x = col + j < N ? ow[col + j] : 0.f;
+                o.y = col + j + 1 < N ? ow[col + j + 1] : 0.f;
+                o.z = col + j + 2 < N ? ow[col + j + 2] : 0.f;
+                o.w = col + j + 3 < N ? ow[col + j + 3] : 0.f;
+            }
+        }
+        const float v0 = dequant1<ASYM>(acc[j], sxr, Rr, f.x, o.x), v1 = dequant1<ASYM>(acc[j + 1], sxr, Rr, f.y, o.y);
+        const float v2 = dequant1<ASYM>(acc[j + 2], sxr, Rr, f.z, o.z), v3 = dequant1<ASYM>(acc[j + 3], sxr, Rr, f.w, o.w);
+        if (sizeof(OutT) == 2) {
+            __nv_bfloat162 lo = __floats2bfloat162_rn(v0, v1), hi = __floats2bfloat162_rn(v2, v3);
+            packed[j / 2] = *reinterpret_cast<uint32_t *>(&lo);
+            packed[j / 2 + 1] = *reinterpret_cast<uint32_t *>(&hi);
+        } else {
+            packed[j] = __float_as_uint(v0);
+            packed[j + 1] = __float_as_uint(v1);
+            packed[j + 2] = __float_as_uint(v2);
+            packed[j + 3] = __float_as_uint(v3);
+        }
+    }
+    if (lane == 0 && pending) bulk_wait_read_all();  // the previous store has read the buffer
+    __syncwarp();
+    const uint32_t rowp = buf + (uint32_t)lane * 128u;
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowp + (uint32_t)(((c ^ (lane & 7)) << 4))),
+                     "r"(packed[4 * c]), "r"(packed[4 * c + 1]), "r"(packed[4 * c + 2]), "r"(packed[4 * c + 3])
+                     : "memory");
+    fence_proxy_async_smem();  // the TMA store reads these bytes through the async proxy
+    __syncwarp();
+    if (lane == 0) tma_store_2d(tmap_y, buf, col, row0);
+    pending = true;
+}
 
 template <typename OutT, bool ASYM>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
 w8a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                      const float *__restrict__ sx, const float *__restrict__ sw, const int32_t *__restrict__ rs,
+                      const __grid_constant__ CUtensorMap tmap_y, const float *__restrict__ sx, const float *__restrict__ sw, const int32_t *__restrict__ rs,
                       const float *__restrict__ ow, OutT *__restrict__ y, int32_t *__restrict__ acc_out, int M,
                       int N, int K) {
     using C = Cfg2;
@@ -759,6 +843,8 @@ w8a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_c
         const int row_in_tile = (int)rank * BM + quarter * 32 + lane;
         constexpr int kCols = C::BN * 4 / kPairEpiWarps;   // columns of a tile per warp
         const int col0 = ((warp - 2) / 4) * kCols;
+        const uint32_t out_buf = smem_base + C::OUT_OFFSET + (uint32_t)(warp - 2) * C::OUT_BYTES;
+        bool store_pending = false;
         int buf = 0;
         uint32_t buf_phase = 0;
         for (int tile = pair; tile < num_tiles; tile += num_pairs) {
@@ -773,12 +859,23 @@ w8a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_c
             tc_fence_after();
             const uint32_t tbase =
                 tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * C::BN + col0);
-            epilogue_tile<OutT, ASYM>(tbase, row, M, n0 + col0, N, sxr, Rr, sw, ow, y, acc_out, kCols);
+            if (acc_out) {
+                // with the int32 accumulators requested: direct stores of both
+                epilogue_tile<OutT, ASYM>(tbase, row, M, n0 + col0, N, sxr, Rr, sw, ow, y, acc_out, kCols);
+            } else {
+                constexpr int CW = 128 / (int)sizeof(OutT);
+#pragma unroll 1
+                for (int c0 = 0; c0 < kCols; c0 += CW)
+                    store_chunk_tma<OutT, ASYM>(&tmap_y, tbase + (uint32_t)c0, out_buf, lane, n0 + col0 + c0,
+                                                m0 + (int)rank * BM + quarter * 32, M, N, sxr, Rr, sw, ow,
+                                                store_pending);
+            }
             tc_fence_before();
             mbar_arrive_leader(smem_u32(&tempty_bar[buf]));
             buf ^= 1;
             if (buf == 0) buf_phase ^= 1u;
         }
+        if (lane == 0 && store_pending) bulk_wait_all();  // this warp's stores are complete
     }
 
     tc_fence_before();
@@ -820,9 +917,6 @@ struct CfgW4 {
     static constexpr int SMEM = IN_OFFSET + IN_STAGES * IN_BYTES + 1024;
 };
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 // 8 int4 codes (one 32-bit word, element 2i in the low nibble of byte i) to
 // 8 int8 codes.  A nibble x sign-extends as ((x ^ 8) + 0x78) ^ 0x80: every
@@ -1139,6 +1233,23 @@ static bool make_map(CUtensorMap *map, const void *base, int64_t rows, int64_t K
     return r == CUDA_SUCCESS;
 }
 
+// Output y [rows, cols] (bf16 or fp32) for TMA stores: box [32 rows, 128
+// bytes], 128B swizzle.  cols * element size is a multiple of 16 (checked by
+// the entry points).
+static bool make_map_out(CUtensorMap *map, const void *base, int64_t rows, int64_t cols, bool bf16) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const int64_t esz = bf16 ? 2 : 4;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(cols * esz)};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / esz), 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                    const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // Packed int4 weights [rows, K/2 bytes]: box [box_rows, 64 bytes] (BK codes),
 // no swizzle (the converter warps read it with plain loads).
 static bool make_map_int4(CUtensorMap *map, const void *base, int64_t rows, int64_t K, int box_rows) {
@@ -1262,8 +1373,9 @@ static sq_status launch_pair(const int8_t *qx, const float *sx, const int32_t *r
                              const float *sw, const float *ow, int M, int N, int K, void *y, int32_t *acc_out,
                              int sms, cudaStream_t st) {
     using C = Cfg2;
-    CUtensorMap ma, mb;
-    if (!make_map(&ma, qx, M, K, BM) || !make_map(&mb, qw, N, K, C::BN / 2))
+    CUtensorMap ma, mb, my;
+    if (!make_map(&ma, qx, M, K, BM) || !make_map(&mb, qw, N, K, C::BN / 2) ||
+        !make_map_out(&my, y, M, N, sizeof(OutT) == 2))
         return fail(SQ_ERR_CUDA, "w8a8_gemm_dequant: cuTensorMapEncodeTiled failed");
     auto kern = w8a8_gemm_pair_kernel<OutT, ASYM>;
     static int configured_dev[64] = {0};
@@ -1276,7 +1388,7 @@ static sq_status launch_pair(const int8_t *qx, const float *sx, const int32_t *r
     }
     const int tiles = ((M + C::PM - 1) / C::PM) * ((N + C::BN - 1) / C::BN);
     const int pairs = std::min(tiles, sms / 2);
-    kern<<<2 * pairs, kThreadsPair, C::SMEM, st>>>(ma, mb, sx, sw, rs, ow, (OutT *)y, acc_out, M, N, K);
+    kern<<<2 * pairs, kThreadsPair, C::SMEM, st>>>(ma, mb, my, sx, sw, rs, ow, (OutT *)y, acc_out, M, N, K);
     return launch_status("w8a8_gemm_pair_kernel");
 }
 
