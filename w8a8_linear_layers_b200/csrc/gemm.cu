@@ -31,7 +31,9 @@
 // row), y = ((float)acc * sx[row]) * sw[col] (two fp32 multiplies, int->fp32
 // round-to-nearest-even), or with asymmetric weights
 // sx * (sw * (float)(acc + 128 R) + ow * (float)R), converted to bf16 (RNE) or
-// kept fp32, stored with 16-byte stores.  Optionally the raw int32
+// kept fp32, and stored: by the pair kernel through a 128B-swizzled
+// shared-memory buffer and TMA stores (32 rows x 128 bytes a warp), by the
+// others with 16-byte stores.  Optionally the raw int32
 // accumulators are stored too.
 //
 // No TMA multicast is used anywhere (each CTA loads its own tiles).
