@@ -23,36 +23,44 @@ namespace w8a8 {
 
 constexpr int kColThreads = 256;
 constexpr int kColWarps = kColThreads / 32;
+constexpr int kColDepth = 6;  // row loads in flight per thread
 
 template <typename T> struct ColVec;
 template <> struct ColVec<__nv_bfloat16> { static constexpr int N = 8; };
 template <> struct ColVec<float> { static constexpr int N = 4; };
 
-template <typename T>
-__device__ __forceinline__ void load_abs(const T *p, float (&v)[ColVec<T>::N]);
+// A 16-byte vector of VEC consecutive columns, raw, and its |.| folded into
+// the running maxima m.
+template <typename T> struct ColRaw;
+template <> struct ColRaw<__nv_bfloat16> { using type = uint4; };
+template <> struct ColRaw<float> { using type = float4; };
 
-template <>
-__device__ __forceinline__ void load_abs<__nv_bfloat16>(const __nv_bfloat16 *p, float (&v)[8]) {
-    uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
-    uint32_t w[4] = {u.x, u.y, u.z, u.w};
+template <typename T>
+__device__ __forceinline__ typename ColRaw<T>::type load_raw(const T *p) {
+    return __ldg(reinterpret_cast<const typename ColRaw<T>::type *>(p));
+}
+
+__device__ __forceinline__ void fold_abs(float (&m)[8], uint4 u) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        v[2 * i] = __uint_as_float((w[i] << 16) & 0x7fff0000u);
-        v[2 * i + 1] = __uint_as_float(w[i] & 0x7fff0000u);
+        m[2 * i] = fmaxf(m[2 * i], __uint_as_float((w[i] << 16) & 0x7fff0000u));
+        m[2 * i + 1] = fmaxf(m[2 * i + 1], __uint_as_float(w[i] & 0x7fff0000u));
     }
 }
 
-template <>
-__device__ __forceinline__ void load_abs<float>(const float *p, float (&v)[4]) {
-    float4 a = __ldg(reinterpret_cast<const float4 *>(p));
-    v[0] = fabsf(a.x); v[1] = fabsf(a.y); v[2] = fabsf(a.z); v[3] = fabsf(a.w);
+__device__ __forceinline__ void fold_abs(float (&m)[4], float4 a) {
+    m[0] = fmaxf(m[0], fabsf(a.x));
+    m[1] = fmaxf(m[1], fabsf(a.y));
+    m[2] = fmaxf(m[2], fabsf(a.z));
+    m[3] = fmaxf(m[3], fabsf(a.w));
 }
 
 // grid.x: column strips of 32 * VEC columns; grid.y: row slices.
 // out_bits: [K] fp32 maxima viewed as unsigned ints (non-negative floats
 // order like their bit patterns).
 template <typename T>
-__global__ void __launch_bounds__(kColThreads)
+__global__ void __launch_bounds__(kColThreads, 4)
 col_absmax_kernel(const T *__restrict__ a, int64_t R, int64_t K, int64_t rows_per_slice,
                   unsigned int *__restrict__ out_bits) {
     constexpr int VEC = ColVec<T>::N;
@@ -70,23 +78,18 @@ col_absmax_kernel(const T *__restrict__ a, int64_t R, int64_t K, int64_t rows_pe
 
     if (col < K) {
         const T *p = a + col;
-        int64_t r = r0 + warp;
-        // four independent 16-byte loads in flight per thread
-        for (; r + 3 * kColWarps < r1; r += 4 * kColWarps) {
-            float v0[VEC], v1[VEC], v2[VEC], v3[VEC];
-            load_abs<T>(p + r * K, v0);
-            load_abs<T>(p + (r + kColWarps) * K, v1);
-            load_abs<T>(p + (r + 2 * kColWarps) * K, v2);
-            load_abs<T>(p + (r + 3 * kColWarps) * K, v3);
+        // up to kColDepth independent 16-byte loads in flight per thread: a
+        // slice is a few dozen rows deep, so one or two round trips cover it
+        for (int64_t r = r0 + warp; r < r1; r += kColDepth * kColWarps) {
+            typename ColRaw<T>::type v[kColDepth];
 #pragma unroll
-            for (int i = 0; i < VEC; ++i)
-                m[i] = fmaxf(fmaxf(m[i], v0[i]), fmaxf(fmaxf(v1[i], v2[i]), v3[i]));
-        }
-        for (; r < r1; r += kColWarps) {
-            float v0[VEC];
-            load_abs<T>(p + r * K, v0);
+            for (int u = 0; u < kColDepth; ++u) {
+                const int64_t rr = r + u * kColWarps;
+                if (rr < r1) v[u] = load_raw<T>(p + rr * K);
+            }
 #pragma unroll
-            for (int i = 0; i < VEC; ++i) m[i] = fmaxf(m[i], v0[i]);
+            for (int u = 0; u < kColDepth; ++u)
+                if (r + u * kColWarps < r1) fold_abs(m, v[u]);
         }
     }
 #pragma unroll
