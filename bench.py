@@ -97,15 +97,16 @@ def algorithmic_work(cfg):
     return algorithmic_work_mnk(cfg.M, cfg.K, cfg.N, xb, yb, cfg.bits)
 
 
+# every source a step's kernels are compiled from (besides common.cuh)
 KERNEL_SOURCES = {
-    "calib_absmax": "smooth.cu", "smooth_fold": "smooth.cu", "ssz_quant_weight": "ssz.cu",
-    "quant_act_per_token": "quant_act.cu", "w8a8_gemm_dequant": "gemm.cu",
+    "calib_absmax": ("smooth.cu",), "smooth_fold": ("smooth.cu",), "ssz_quant_weight": ("ssz.cu", "dd.cuh"),
+    "quant_act_per_token": ("quant_act.cu",), "w8a8_gemm_dequant": ("gemm.cu", "gemm_decode.cuh"),
 }
 
 
-def source_sha(fname):
+def source_sha(files):
     h = hashlib.sha256()
-    for f in (fname, "common.cuh"):
+    for f in (*files, "common.cuh"):
         with open(os.path.join(ROOT, "w8a8_linear_layers_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

@@ -1,0 +1,55 @@
+"""Host-side pieces of bench.py (no GPU): the algorithmic work model, the
+per-shape table of multi-linear workloads, and the DRAM-traffic record that
+must match the current kernel sources."""
+import importlib.util
+import os
+from types import SimpleNamespace
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_algorithmic_work_of_the_prefill_linear(bench):
+    w = bench.algorithmic_work_mnk(2048, 4096, 4096, 2, 2, 8)
+    assert w["calib_absmax"]["bytes"] == 2 * 2048 * 4096 + 4 * 4096            # X once + absmax
+    assert w["w8a8_gemm_dequant"]["ops"] == 2 * 2048 * 4096 * 4096
+    assert w["w8a8_gemm_dequant"]["bytes"] == 2048 * 4096 + 4096 * 4096 + 4 * 2048 + 4 * 4096 + 2 * 2048 * 4096
+    w4 = bench.algorithmic_work_mnk(16, 8192, 28672, 2, 2, 4)
+    # int4: the codes are packed (read N K, write N K / 2) and read packed by the GEMM
+    assert w4["w8a8_gemm_dequant"]["bytes"] - 16 * 8192 - 4 * 16 - 4 * 28672 - 2 * 16 * 28672 == 2 * 28672 * 8192
+
+
+def test_per_shape_table_groups_linears_by_shape(bench):
+    probs = [SimpleNamespace(M=8192, K=1024, N=3072), SimpleNamespace(M=8192, K=1024, N=1024),
+             SimpleNamespace(M=8192, K=1024, N=3072)]
+    # ms per kernel (NAMES order) per linear
+    lin = [[0.01, 0.01, 0.05, 0.01, 0.030], [0.01, 0.01, 0.04, 0.01, 0.020], [0.03, 0.01, 0.07, 0.01, 0.030]]
+    t = bench.per_shape_table(probs, lin, {"bf16_tflops": 1000.0})
+    assert set(t) == {"8192x1024->3072", "8192x1024->1024"}
+    qkv = t["8192x1024->3072"]
+    assert qkv["linears"] == 2
+    assert qkv["us"]["calib_absmax"] == pytest.approx(20.0)
+    tops = 2 * 8192 * 1024 * 3072 / 30e-6 / 1e12
+    assert qkv["gemm_tops"] == pytest.approx(round(tops, 1))
+    assert qkv["gemm_frac"] == pytest.approx(round(tops / (1000.0 * bench.INT8_OVER_BF16), 4))
+
+
+def test_recorded_traffic_matches_the_current_sources(bench):
+    """profiles/dram_traffic.json is keyed by a hash of every source a step's
+    kernels are built from; a recorded entry is used only while it matches,
+    and each file named in the key exists."""
+    for step, files in bench.KERNEL_SOURCES.items():
+        for f in files:
+            assert os.path.exists(os.path.join(ROOT, "w8a8_linear_layers_b200", "csrc", f)), f
+        got = bench.dram_traffic(step, "prefill_2048x4096x4096")
+        assert got is None or got > 0
+    assert bench.dram_traffic("ssz_quant_weight", "no_such_workload") is None
