@@ -577,8 +577,9 @@ void oracle_dequant(const int32_t *acc, const float *sx, const float *sw,
 }
 
 /* ------------------------------------------------------- packed int4 */
-/* Two int4 codes per byte (SURVEY next row: packed int4 weights; the int4
- * codes themselves are the SSZ page's int4 per-channel symmetric case).
+/* Two int4 codes per byte (the pages print no packed layout, so this one is
+ * a reading; the int4 codes themselves are the int4 per-channel symmetric
+ * case of "SSZ：权重量化算法说明", 使用限制).
  * Reading: element 2i in the low nibble, 2i+1 in the high nibble, each in
  * 4-bit two's complement; codes must lie in [-8, 7].  K is even. */
 void oracle_pack_int4(const int8_t *q, int64_t N, int64_t K, uint8_t *packed)
