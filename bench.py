@@ -57,6 +57,10 @@ def parse():
     p.add_argument("--record-traffic", metavar="NCU_CSV",
                    help="read an ncu --csv capture (gpu__time_duration.sum, dram__bytes_read.sum, "
                         "dram__bytes_write.sum) of this workload and write profiles/dram_traffic.json")
+    p.add_argument("--decode-launches", action="store_true",
+                   help="only launch the 16 x 8192 -> 28672 decode GEMMs on random codes, three with int8 "
+                        "weights then three with packed int4 weights, and exit (the workload of the decode "
+                        "kernel's ncu capture)")
     return p.parse_args()
 
 
@@ -757,8 +761,37 @@ def record_traffic(csv_path, workload):
     print(json.dumps(out, indent=1))
 
 
+def decode_launches():
+    """Three w8a8_gemm_dequant then three w4a8_gemm_dequant launches on the
+    16 x 8192 -> 28672 decode shape (random codes in the int4 range, seed 0),
+    for an ncu capture of the few-token GEMM kernel."""
+    import torch
+
+    import w8a8_linear_layers_b200 as w
+    dev = "cuda"
+    g = torch.Generator(device=dev).manual_seed(0)
+    M, N, K = 16, 28672, 8192
+    qx = torch.randint(-127, 128, (M, K), device=dev, dtype=torch.int8, generator=g)
+    qw = torch.randint(-7, 8, (N, K), device=dev, dtype=torch.int8, generator=g)
+    sx = torch.rand(M, device=dev, generator=g) * 1e-2
+    sw = torch.rand(N, device=dev, generator=g) * 1e-2
+    packed = torch.empty(N, K // 2, device=dev, dtype=torch.uint8)
+    w.sq_pack_int4(qw, packed)
+    y = torch.empty(M, N, device=dev, dtype=torch.bfloat16)
+    for _ in range(3):
+        w.w8a8_gemm_dequant(qx, sx, qw, sw, y)
+    for _ in range(3):
+        w.w4a8_gemm_dequant(qx, sx, packed, sw, y)
+    torch.cuda.synchronize()
+    if w.device_fault() != 0:
+        raise RuntimeError("a kernel gave up on a bounded wait")
+
+
 def main():
     args = parse()
+    if args.decode_launches:
+        decode_launches()
+        return
     if args.record_traffic:
         record_traffic(args.record_traffic, args.workload)
         return
