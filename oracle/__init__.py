@@ -83,13 +83,15 @@ def _L():
             "oracle_channel_mse_asym": [P, I64, ctypes.c_float, ctypes.c_float],
             "oracle_act_rowsum": [P, I64, I64, P],
             "oracle_pack_int4": [P, I64, I64, P],
-            "oracle_layernorm_quant": [P, I64, I64, P, P, ctypes.c_float, P, P, P, P],
+            "oracle_layernorm_quant": [P, I64, I64, P, P, ctypes.c_float, P, P, P, P, P],
             "oracle_quant_act_given_scale": [P, I64, I64, P, P, P],
             "oracle_unpack_int4": [P, I64, I64, P],
             "oracle_dequant_asym": [P, P, P, P, P, I64, I64, P, P],
             "oracle_static_ema": [ctypes.c_float, ctypes.c_float, ctypes.c_float, I],
             "oracle_quant_act_static": [P, I64, I64, P, ctypes.c_float, P],
             "oracle_to_bf16": [P, I64, P],
+            "oracle_weight_codes_asym": [P, I64, I64, P, P, P],
+            "oracle_pairwise_sum": [P, I64],
         }
         for name, args in sig.items():
             fn = getattr(_lib, name)
@@ -101,6 +103,7 @@ def _L():
         _lib.oracle_ssz_quant_weight_asym.restype = ctypes.c_int
         _lib.oracle_channel_mse_asym.restype = ctypes.c_double
         _lib.oracle_static_ema.restype = ctypes.c_float
+        _lib.oracle_pairwise_sum.restype = ctypes.c_double
     return _lib
 
 
@@ -229,6 +232,16 @@ def ssz_quant_weight_asym(w, max_iters: int = SSZ_ITERS, s=None, trace: bool = F
     return out
 
 
+def weight_codes_asym(w, scale, offset) -> np.ndarray:
+    """Stored asymmetric codes q = clamp(rint(fl(w - offset[n]) / scale[n]),
+    0, 255) - 128 of a folded weight at given per-row (scale, offset)."""
+    w, scale, offset = _f32(w), _f32(scale), _f32(offset)
+    N, K = w.shape
+    q = np.empty((N, K), np.int8)
+    _L().oracle_weight_codes_asym(_ptr(w), N, K, _ptr(scale), _ptr(offset), _ptr(q))
+    return q
+
+
 def channel_mse_asym(w_row, S, m) -> float:
     w_row = _f32(w_row)
     return float(_L().oracle_channel_mse_asym(_ptr(w_row), w_row.shape[0], float(S), float(m)))
@@ -245,9 +258,17 @@ def quant_act_given_scale(x, inv_s, sx):
     return q
 
 
-def layernorm_quant(h, gamma=None, beta=None, eps: float = 1e-5, inv_s=None):
-    """LayerNorm (fp64 statistics, fp32 output) of h [M,K] times inv_s, then
-    per-token int8 codes.  Returns (q, sx, y) with y the LayerNorm output."""
+def pairwise_sum(v) -> float:
+    """The pairwise (recursive halving, zero-padded to a power of two) fp64
+    sum the LayerNorm statistics use."""
+    v = np.ascontiguousarray(np.asarray(v, dtype=np.float64))
+    return float(_L().oracle_pairwise_sum(_ptr(v), v.shape[0]))
+
+
+def layernorm_quant(h, gamma=None, beta=None, eps: float = 1e-5, inv_s=None, stats: bool = False):
+    """LayerNorm (fp64 pairwise statistics, fp32 output) of h [M,K] times
+    inv_s, then per-token int8 codes.  Returns (q, sx, y) with y the
+    LayerNorm output, and with stats=True also [M,2] fp64 (mean, var)."""
     h = _f32(h)
     M, K = h.shape
     g = None if gamma is None else _f32(gamma)
@@ -256,8 +277,10 @@ def layernorm_quant(h, gamma=None, beta=None, eps: float = 1e-5, inv_s=None):
     q = np.empty((M, K), np.int8)
     sx = np.empty(M, np.float32)
     y = np.empty((M, K), np.float32)
-    _L().oracle_layernorm_quant(_ptr(h), M, K, _ptr(g), _ptr(b), float(eps), _ptr(inv), _ptr(q), _ptr(sx), _ptr(y))
-    return q, sx, y
+    st = np.empty((M, 2), np.float64) if stats else None
+    _L().oracle_layernorm_quant(_ptr(h), M, K, _ptr(g), _ptr(b), float(eps), _ptr(inv), _ptr(q), _ptr(sx), _ptr(y),
+                                _ptr(st))
+    return (q, sx, y, st) if stats else (q, sx, y)
 
 
 def pack_int4(q) -> np.ndarray:

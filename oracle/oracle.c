@@ -387,6 +387,16 @@ int oracle_ssz_quant_weight_asym(const float *w, int64_t N, int64_t K, int max_i
     return 0;
 }
 
+/* Codes of a [N,K] weight at given per-row (S, m) (stage-wise parity: the
+ * stored codes q = u - 128 a scale and offset imply, [SSZ] 迭代优化阶段). */
+void oracle_weight_codes_asym(const float *w, int64_t N, int64_t K, const float *S,
+                              const float *m, int8_t *q)
+{
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            q[n * K + k] = (int8_t)((int)asym_code(w[n * K + k], S[n], m[n]) - 128);
+}
+
 /* The error of one channel at a given (S, m) (exposed for the pins). */
 double oracle_channel_mse_asym(const float *w, int64_t K, float S, float m)
 {
@@ -421,32 +431,64 @@ void oracle_quant_act_per_token(const float *x, int64_t M, int64_t K,
 }
 
 /* ------------------------------------------- LayerNorm fused with step 4 */
+/* Pairwise (recursive halving) fp64 sum of v[0..K-1] padded with zeros to a
+ * power of two P >= K: S(lo, len) = S(lo, len/2) + S(lo + len/2, len/2),
+ * S(i, 1) = v[i] (0 past K).  The order is fixed by the definition, not by
+ * an implementation, so any evaluation of this tree gives the same bits
+ * (zero subtrees add exactly 0; padding to a larger power of two changes at
+ * most the sign of a zero sum). */
+static double pairwise(const double *v, int64_t K, int64_t lo, int64_t len)
+{
+    if (lo >= K)
+        return 0.0;
+    if (len == 1)
+        return v[lo];
+    int64_t h = len / 2;
+    return pairwise(v, K, lo, h) + pairwise(v, K, lo + h, h);
+}
+
+double oracle_pairwise_sum(const double *v, int64_t K)
+{
+    int64_t P = 1;
+    while (P < K)
+        P *= 2;
+    return K > 0 ? pairwise(v, K, 0, P) : 0.0;
+}
+
 /* Activation quantization fused upstream: the smoothing 1/s folded into the
  * LayerNorm that produces X (SmoothQuant page, section 1: the scaling is an
  * equivalent transform; CUDA INT8 notes 4.2: fuse quantization with the
  * neighbouring op so the intermediate never goes to memory).  Per row t of
  * h [M,K]:
- *     mu  = sum_j h_j / K,  var = sum_j (h_j - mu)^2 / K      (fp64, index order)
+ *     mu  = P(h) / K,  var = P(d^2) / K,  d_j = h_j - mu         (fp64)
  *     m = fp32(mu), r = fp32(1 / sqrt(var + eps))
+ * with P the pairwise sum above (the pages fix no summation order; a fixed
+ * tree makes the statistics, and hence the codes, reproducible bit for bit);
  *     y_j = ((h_j - m) * r) * gamma_j + beta_j                  (fp32, each op rounded)
  *     x'_j = y_j * inv_s_j (fp32), then the per-token codes and scale of step 4.
  * gamma, beta, inv_s nullable (1, 0, 1).  Also writes y (the LayerNorm
- * output, nullable) so the pins can check it. */
+ * output, nullable) and stats (nullable, [M,2]: mu and var in fp64) so the
+ * pins can check them. */
 void oracle_layernorm_quant(const float *h, int64_t M, int64_t K, const float *gamma,
                             const float *beta, float eps, const float *inv_s, int8_t *q,
-                            float *sx, float *y_out)
+                            float *sx, float *y_out, double *stats)
 {
 #pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < M; ++t) {
         const float *row = h + t * K;
-        double sum = 0.0;
+        double *tmp = (double *)malloc((size_t)K * sizeof(double));
         for (int64_t j = 0; j < K; ++j)
-            sum += (double)row[j];
-        double mu = sum / (double)K;
-        double ss = 0.0;
+            tmp[j] = (double)row[j];
+        double mu = oracle_pairwise_sum(tmp, K) / (double)K;
         for (int64_t j = 0; j < K; ++j) {
             double d = (double)row[j] - mu;
-            ss += d * d;
+            tmp[j] = d * d;
+        }
+        double ss = oracle_pairwise_sum(tmp, K);
+        free(tmp);
+        if (stats) {
+            stats[2 * t] = mu;
+            stats[2 * t + 1] = ss / (double)K;
         }
         double rstd = 1.0 / sqrt(ss / (double)K + (double)eps);
         float m32 = (float)mu, r32 = (float)rstd;

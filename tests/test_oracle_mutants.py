@@ -77,6 +77,13 @@ MUTANTS = [
      "double rstd = 1.0 / sqrt(ss / (double)(K - 1) + (double)eps);"),
     ("ln_drops_beta", "float b = beta ? beta[j] : 0.0f;", "float b = 0.0f;"),
     ("ln_smooths_before_norm", "float v = inv_s ? yj * inv_s[j] : yj;", "float v = yj;"),
+    ("ln_sequential_mean", "double mu = oracle_pairwise_sum(tmp, K) / (double)K;",
+     "double mu = 0.0;\n        for (int64_t j = 0; j < K; ++j)\n            mu += tmp[j];\n        mu /= (double)K;"),
+    ("ln_sequential_variance", "double ss = oracle_pairwise_sum(tmp, K);",
+     "double ss = 0.0;\n        for (int64_t j = 0; j < K; ++j)\n            ss += tmp[j];"),
+    ("pairwise_unpadded_split", "while (P < K)\n        P *= 2;", "P = K;"),
+    ("asym_given_codes_not_offset", "q[n * K + k] = (int8_t)((int)asym_code(w[n * K + k], S[n], m[n]) - 128);",
+     "q[n * K + k] = (int8_t)((int)asym_code(w[n * K + k], S[n], m[n]) - 127);"),
     ("int4_nibbles_swapped", "packed[n * (K / 2) + i] = (uint8_t)(lo | (hi << 4));",
      "packed[n * (K / 2) + i] = (uint8_t)(hi | (lo << 4));"),
     ("int4_unpack_no_sign", "q[n * K + 2 * i] = (int8_t)(lo >= 8 ? lo - 16 : lo);", "q[n * K + 2 * i] = (int8_t)lo;"),

@@ -14,6 +14,7 @@ CUDA INT8 notes (aicoding.csdn.net) section 2.1 for Q = round(R/S) + Z;
 "PaddleNLP GPT 量化感知训练（QAT）实战指南" section 六 for the moving-average
 activation range.
 """
+import math
 import os
 
 import numpy as np
@@ -400,6 +401,26 @@ def test_ssz_asym_scale_equivariance(orc):
     np.testing.assert_array_equal(2 * a["offset"], b["offset"])
 
 
+def test_asym_codes_at_given_scale(orc):
+    # hand-derived: S = 0.5, m = -1 (both exact); u = rint((w - m) / S)
+    # clamped to [0, 255] with ties to even, stored as q = u - 128
+    w = np.array([[0.25, 0.75, -1.0, -3.0, 126.75, 200.0, -0.75, 0.0]], np.float32)
+    #       (w-m)/S:   2.5   3.5    0    -4   255.5   402    0.5   2
+    want = np.array([[2, 4, 0, 0, 255, 255, 0, 2]], np.int32) - 128
+    q = orc.weight_codes_asym(w, np.float32([0.5]), np.float32([-1.0]))
+    np.testing.assert_array_equal(q, want)
+    # the codes the searched (S, m) imply are the codes the search returns
+    r = np.random.default_rng(46)
+    w = (r.standard_normal((10, 144)) * 0.5 + 0.3).astype(np.float32)
+    out = orc.ssz_quant_weight_asym(w)
+    np.testing.assert_array_equal(orc.weight_codes_asym(w, out["scale"], out["offset"]), out["q"])
+    # in range, each code reconstructs its weight within half a step
+    u = orc.weight_codes_asym(w, out["scale"], out["offset"]).astype(np.float64) + 128
+    rec = out["scale"][:, None].astype(np.float64) * u + out["offset"][:, None]
+    inside = (u > 0) & (u < 255)
+    assert np.all(np.abs(rec - w)[inside] <= 0.5 * out["scale"][:, None].repeat(144, 1)[inside] * (1 + 1e-6))
+
+
 def test_act_rowsum_and_asym_dequant(orc):
     r = np.random.default_rng(45)
     qx = r.integers(-127, 128, (9, 64)).astype(np.int8)
@@ -454,6 +475,64 @@ def test_k_sharded_linear_equals_unsharded(orc):
 # ------------------------------------------------- LayerNorm fused with step 4
 # SmoothQuant page section 1 (the scaling moves into the op that produces X);
 # CUDA INT8 notes 4.2 (fuse quantization with the neighbouring kernel).
+def _pairwise_golden():
+    def val(t):
+        return 2.0 ** int(t[2:]) if t.startswith("2^") else (-(2.0 ** int(t[3:])) if t.startswith("-2^")
+                                                               else float(t))
+    cases = []
+    for line in open(os.path.join(GOLDEN, "pairwise_sum.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        f = line.split()
+        k = int(f[1])
+        cases.append((f[0], val(f[2]), np.array([val(t) for t in f[3:3 + k]])))
+    return cases
+
+
+def test_pairwise_sum_golden(orc):
+    # see tests/golden/pairwise_sum.txt for the derivations
+    cases = _pairwise_golden()
+    assert [c[0] for c in cases] == ["A", "B", "C", "D"]
+    for name, want, x in cases:
+        assert orc.pairwise_sum(x) == want, name
+
+
+def test_pairwise_sum_error_bound(orc):
+    # within the pairwise-summation bound |S - s| <= g(ceil(log2 n)) sum|x|,
+    # g(k) = k u / (1 - k u), u = 2^-53 (Higham), against the exact fsum;
+    # exact on small integers
+    r = np.random.default_rng(80)
+    u = 2.0 ** -53
+    for n in (1, 2, 3, 7, 8, 100, 1000, 4096, 5000):
+        x = r.standard_normal(n) * np.exp(r.standard_normal(n) * 6)
+        k = max(1, int(np.ceil(np.log2(n))))
+        bound = k * u / (1 - k * u) * np.abs(x).sum()
+        assert abs(orc.pairwise_sum(x) - math.fsum(x)) <= bound
+        xi = r.integers(-1000, 1000, n).astype(np.float64)
+        assert orc.pairwise_sum(xi) == xi.sum()
+
+
+def test_layernorm_statistics_are_pairwise(orc):
+    # rows of the golden cases A and B: mean and variance from the
+    # hand-derived pairwise sums, the rest by the stated fp32 formulas
+    cases = {c[0]: c[2] for c in _pairwise_golden()}
+    for name, mean, ss in (("A", 0.25, 2.0 ** 107), ("B", 0.5, 2.0 ** 107)):
+        # A: d = [2^53, 0.75, 0.75, -2^53] after rounding, squares sum to 2^107
+        # B: d = [2^53, 0.5, 0.5, -2^53, 0.5, 0.5], sum 2^107 + 0.5 -> 2^107
+        h = cases[name].astype(np.float32)[None, :]
+        K = h.shape[1]
+        _, _, y = orc.layernorm_quant(h, None, None, 0.0)
+        r32 = np.float32(1.0 / np.sqrt(ss / K))
+        want = (h[0] - np.float32(mean)) * r32
+        np.testing.assert_array_equal(y[0], want)
+    # row D's squares are golden case D: mean 0, var = (2 + 2^-51) / 16 exactly
+    b = np.float32(2.0 ** -27)
+    h = np.array([[1] + [b] * 7 + [-1] + [-b] * 7], np.float32)
+    _, _, _, st = orc.layernorm_quant(h, None, None, 1e-5, stats=True)
+    assert st[0, 0] == 0.0 and st[0, 1] == (2.0 + 2.0 ** -51) / 16
+    assert math.fsum(cases["D"]) / 16 != st[0, 1]  # the exact sum would differ: the order is pinned
+
+
 def test_layernorm_matches_torch_fp64(orc):
     r = np.random.default_rng(60)
     for scale, eps in ((3.0, 1e-5), (0.01, 1e-5), (1.0, 0.0)):
