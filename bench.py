@@ -7,12 +7,19 @@ activation quantization -> INT8 GEMM with fused dequant.  On one GPU the step
 is captured once as a CUDA graph and replayed.  Inputs are seeded
 synthetic LLM-shaped data resident in HBM; L2 is flushed (a 512 MB write,
 then a 384 MB read that writes the dirty lines back) before every timed step,
-outside the timed events.
+outside the timed events.  Default workload: the MLP up-projection
+8192 x 4096 -> 11008 (the largest single-GPU linear; compute-bound GEMM).
 
-value  = 2*M*N*K int8 ops of the linear per step, over all ranks, divided by
-         the step time (max over ranks), in TOPS.
-e2e    = the same, through the C ABI with the inputs copied from pinned host
-         memory every step and the output copied back (copies timed).
+value  = the W8A8 linear's INT8 TOPS: 2*M*N*K int8 ops per step, over all
+         ranks, divided by the device time of the per-inference part of each
+         step (per-token activation quantization + GEMM with dequant; max over
+         ranks).  The once-per-weight part (calibration, smoothing, SSZ) runs
+         inside every timed step too and is reported beside it in GB/s and as
+         a fraction of its roofline (`weight_path`); `ms_per_step` is the whole
+         step, `path` gives its TOPS.
+e2e    = the same metric through the C ABI with the activations copied from
+         pinned host memory every step and the output copied back (copies
+         timed), the quantized weights resident on the device.
 
 Multi-GPU (torchrun): data parallel, each rank a replica of the layer with its
 own batch of tokens (weak scaling).  The one exchange is the calibration
@@ -35,7 +42,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-DEFAULT_WORKLOAD = "prefill_2048x4096x4096"
+DEFAULT_WORKLOAD = "mlp_up_8192x4096x11008"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 
@@ -85,13 +92,12 @@ def algorithmic_work_mnk(M, K, N, xb, yb, bits=8):
         "calib_absmax": {"bytes": xb * M * K + 4 * K},
         "smooth_fold": {"bytes": xb * N * K + 3 * 4 * K},
         "ssz_quant_weight": {"bytes": xb * N * K + N * K + 4 * K + 4 * N + 8 * N + 4 * N},
+        # int4 weights: the codes packed two per byte (N K read, N K / 2 written)
+        "sq_pack_int4": {"bytes": N * K + N * K // 2 if bits == 4 else 0},
         "quant_act_per_token": {"bytes": xb * M * K + M * K + 4 * K + 4 * M},
-        # int4: the step packs the codes (N K read, N K / 2 written) and the
-        # W4A8 GEMM reads them packed
-        "w8a8_gemm_dequant": ({"ops": 2 * M * N * K, "bytes": M * K + N * K + 4 * M + 4 * N + yb * M * N}
-                              if bits == 8 else
-                              {"ops": 2 * M * N * K,
-                               "bytes": N * K + N * K // 2 + M * K + N * K // 2 + 4 * M + 4 * N + yb * M * N}),
+        # int4: the W4A8 GEMM reads the weight codes packed
+        "w8a8_gemm_dequant": {"ops": 2 * M * N * K,
+                              "bytes": M * K + (N * K if bits == 8 else N * K // 2) + 4 * M + 4 * N + yb * M * N},
     }
 
 
@@ -104,7 +110,8 @@ def algorithmic_work(cfg):
 # every source a step's kernels are compiled from (besides common.cuh)
 KERNEL_SOURCES = {
     "calib_absmax": ("smooth.cu",), "smooth_fold": ("smooth.cu",), "ssz_quant_weight": ("ssz.cu", "dd.cuh"),
-    "quant_act_per_token": ("quant_act.cu",), "w8a8_gemm_dequant": ("gemm.cu", "gemm_decode.cuh"),
+    "sq_pack_int4": ("gemm.cu",), "quant_act_per_token": ("quant_act.cu",),
+    "w8a8_gemm_dequant": ("gemm.cu", "gemm_decode.cuh"),
 }
 
 
@@ -182,7 +189,11 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ our arm
-NAMES = ["calib_absmax", "smooth_fold", "ssz_quant_weight", "quant_act_per_token", "w8a8_gemm_dequant"]
+NAMES = ["calib_absmax", "smooth_fold", "ssz_quant_weight", "sq_pack_int4", "quant_act_per_token",
+         "w8a8_gemm_dequant"]
+WEIGHT_PATH = ("calib_absmax", "smooth_fold", "ssz_quant_weight", "sq_pack_int4")  # once per weight
+LINEAR = ("quant_act_per_token", "w8a8_gemm_dequant")  # every inference
+NM = len(NAMES) + 1  # events per linear
 GPT_WORKLOAD = "gpt345m_8x1024"
 
 
@@ -237,30 +248,40 @@ def run_ours(args, rank, world, local_rank):
     flush = L2Flush(torch, dev)
     stream = torch.cuda.current_stream()
 
-    def run(p, xin, wt, evs=None, base=0):
-        def mark(i):
-            if evs is not None:
-                evs[base + i].record()  # the current stream: the launching one, or a graph's capture stream
-        mark(0)
-        w.sq_calib_absmax(xin, p.ax)
-        mark(1)
-        wdist.allreduce_calibration(p.ax)
-        w.sq_smooth_fold(p.ax, wt, p.alpha, p.aw, p.s, p.inv)
-        mark(2)
-        w.ssz_quant_weight(wt, p.s, p.bits, p.max_iters, p.qw, p.sw, iters_out=p.iters)
-        mark(3)
+    def forward(p, xin, evs=None, base=0):
+        """The per-inference part: per-token codes, then the GEMM."""
         w.quant_act_per_token(xin, p.inv, p.qx, p.sx)
-        mark(4)
+        if evs is not None:
+            evs[base + 5].record()
         if p.bits == 8:
             w.w8a8_gemm_dequant(p.qx, p.sx, p.qw, p.sw, p.y)
-        else:  # int4 weights: packed two per byte, W4A8 GEMM
-            w.sq_pack_int4(p.qw, p.qw4)
+        else:
             w.w4a8_gemm_dequant(p.qx, p.sx, p.qw4, p.sw, p.y)
-        mark(5)
+
+    def run(p, evs=None, base=0):
+        """The whole path on one linear; with evs, an event before each
+        kernel (NAMES order) and one after the last, on the current stream
+        (the launching one, or a graph's capture stream)."""
+        def mark(i):
+            if evs is not None:
+                evs[base + i].record()
+        mark(0)
+        w.sq_calib_absmax(p.x, p.ax)
+        mark(1)
+        wdist.allreduce_calibration(p.ax)
+        w.sq_smooth_fold(p.ax, p.wt, p.alpha, p.aw, p.s, p.inv)
+        mark(2)
+        w.ssz_quant_weight(p.wt, p.s, p.bits, p.max_iters, p.qw, p.sw, iters_out=p.iters)
+        mark(3)
+        if p.bits == 4:  # int4 weights: packed two per byte for the W4A8 GEMM
+            w.sq_pack_int4(p.qw, p.qw4)
+        mark(4)
+        forward(p, p.x, evs, base)
+        mark(6)
 
     def step(evs=None):
         for i, p in enumerate(probs):
-            run(p, p.x, p.wt, evs, 6 * i)
+            run(p, evs, NM * i)
 
     for _ in range(args.warmup):
         flush()
@@ -275,7 +296,7 @@ def run_ours(args, rank, world, local_rank):
     # ranks launch eagerly (no collective is captured).
     graph = None
     if world == 1 and not args.eager:
-        gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(6 * len(probs))]
+        gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(NM * len(probs))]
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
             step(gev)
@@ -284,10 +305,10 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
 
     def elapsed(e):
-        """Per linear j: [kernel i time for i in 0..4] from a step's events."""
-        return [[e[6 * j + i].elapsed_time(e[6 * j + i + 1]) for i in range(5)] for j in range(len(probs))]
+        """Per linear j: [kernel i time for i in NAMES] from a step's events."""
+        return [[e[NM * j + i].elapsed_time(e[NM * j + i + 1]) for i in range(len(NAMES))] for j in range(len(probs))]
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6 * len(probs))] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(NM * len(probs))] for _ in range(args.steps)]
     per_step = []
     if world > 1:
         dist.barrier()
@@ -309,15 +330,19 @@ def run_ours(args, rank, world, local_rank):
     if graph is None:
         per_step = [elapsed(e) for e in evs]
     step_ms = [sum(sum(lin) for lin in st) for st in per_step]
+    li = [NAMES.index(n) for n in LINEAR]
+    linear_step_ms = [sum(lin[i] for lin in st for i in li) for st in per_step]
     kern_ms = {n: statistics.mean(sum(lin[i] for lin in st) for st in per_step) for i, n in enumerate(NAMES)}
     # per linear and kernel, mean over the timed steps (for the per-shape table)
     lin_ms = [[statistics.mean(st[j][i] for st in per_step) for i in range(len(NAMES))] for j in range(len(probs))]
     total_ms = wdist.max_over_ranks(sum(step_ms), device=dev)
+    linear_ms = wdist.max_over_ranks(sum(linear_step_ms), device=dev)
     if w.device_fault() != 0:
         raise RuntimeError("a kernel gave up on a bounded wait during timing")
 
     ops_per_step = sum(2.0 * p.M * p.N * p.K for p in probs)
-    value = ops_per_step * world * args.steps / (total_ms * 1e-3) / 1e12
+    value = ops_per_step * world * args.steps / (linear_ms * 1e-3) / 1e12
+    path_value = ops_per_step * world * args.steps / (total_ms * 1e-3) / 1e12
 
     next_rows = (time_next_rows(args, w, torch, probs, flush, stream)
                  if world == 1 and not args.no_next_rows else None)
@@ -325,10 +350,10 @@ def run_ours(args, rank, world, local_rank):
     # ---- end to end through the C ABI with host buffers
     e2e = None
     if args.e2e_steps > 0:
-        e2e = run_e2e(args, w, wdist, torch, probs, run, flush, stream, ops_per_step, world)
+        e2e = run_e2e(args, w, wdist, torch, probs, forward, flush, stream, ops_per_step, world)
     del graph
-    return finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall1 - wall0, next_rows,
-                  launch="eager" if world > 1 or args.eager else "cuda_graph", lin_ms=lin_ms)
+    return finish(args, world, probs, kern_ms, total_ms, linear_ms, value, path_value, e2e, clk, wall1 - wall0,
+                  next_rows, launch="eager" if world > 1 or args.eager else "cuda_graph", lin_ms=lin_ms)
 
 
 class L2Flush:
@@ -479,20 +504,21 @@ def time_next_rows(args, w, torch, probs, flush, stream, reps=50):
     return out
 
 
-def run_e2e(args, w, wdist, torch, probs, run, flush, stream, ops_per_step, world):
-    """Inputs copied from pinned host memory and outputs copied back every
-    step, inside the timed region."""
-    hosts = [(p.x.cpu().pin_memory(), p.wt.cpu().pin_memory(), torch.empty_like(p.y, device="cpu").pin_memory(),
-              torch.empty_like(p.x), torch.empty_like(p.wt)) for p in probs]
+def run_e2e(args, w, wdist, torch, probs, forward, flush, stream, ops_per_step, world):
+    """The per-inference linear end to end: every step copies the
+    activations from pinned host memory, quantizes them, runs the GEMM and
+    copies the output back, all inside the timed events; the quantized
+    weights (the layer's parameters) stay resident on the device."""
+    hosts = [(p.x.cpu().pin_memory(), torch.empty_like(p.y, device="cpu").pin_memory(), torch.empty_like(p.x))
+             for p in probs]
     e2e_ms = []
     for i in range(args.warmup + args.e2e_steps):
         flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for p, (xh, wh, yh, xd, wd) in zip(probs, hosts):
+        for p, (xh, yh, xd) in zip(probs, hosts):
             xd.copy_(xh, non_blocking=True)
-            wd.copy_(wh, non_blocking=True)
-            run(p, xd, wd)
+            forward(p, xd)
             yh.copy_(p.y, non_blocking=True)
         e1.record(stream)
         e1.synchronize()
@@ -500,37 +526,46 @@ def run_e2e(args, w, wdist, torch, probs, run, flush, stream, ops_per_step, worl
             e2e_ms.append(e0.elapsed_time(e1))
     e2e_total = wdist.max_over_ranks(sum(e2e_ms), device=probs[0].x.device)
     e2e_value = ops_per_step * world * len(e2e_ms) / (e2e_total * 1e-3) / 1e12
-    h2d = sum(p.x.numel() * p.x.element_size() + p.wt.numel() * p.wt.element_size() for p in probs)
+    h2d = sum(p.x.numel() * p.x.element_size() for p in probs)
     d2h = sum(p.y.numel() * p.y.element_size() for p in probs)
     return {"value": round(e2e_value, 3), "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "ms_per_step": round(e2e_total / len(e2e_ms), 4)}
+            "ms_per_step": round(e2e_total / len(e2e_ms), 4),
+            "what": "activations copied host->device from pinned memory, per-token quantization, GEMM + dequant, "
+                    "output copied device->host, every step; quantized weights resident"}
 
 
 def per_shape_table(probs, lin_ms, peaks):
     """Workloads of several linears: per distinct (M, K, N) the number of
-    linears, the mean time of each kernel and the GEMM's TOPS."""
+    linears, the mean time of each kernel, the GEMM's TOPS and the linear's
+    (activation quantization + GEMM)."""
     groups = {}
     for p, ms in zip(probs, lin_ms):
         groups.setdefault((p.M, p.K, p.N), []).append(ms)
     out = {}
+    peak = peaks["bf16_tflops"] * INT8_OVER_BF16
     for (M, K, N), rows in groups.items():
         mean = [statistics.mean(r[i] for r in rows) for i in range(len(NAMES))]
         gemm_ms = mean[NAMES.index("w8a8_gemm_dequant")]
+        lin = gemm_ms + mean[NAMES.index("quant_act_per_token")]
         tops = 2.0 * M * N * K / (gemm_ms * 1e-3) / 1e12
         out["%dx%d->%d" % (M, K, N)] = {
             "linears": len(rows), "us": {n: round(m * 1e3, 2) for n, m in zip(NAMES, mean)},
-            "gemm_tops": round(tops, 1), "gemm_frac": round(tops / (peaks["bf16_tflops"] * INT8_OVER_BF16), 4)}
+            "gemm_tops": round(tops, 1), "gemm_frac": round(tops / peak, 4),
+            "linear_tops": round(2.0 * M * N * K / (lin * 1e-3) / 1e12, 1)}
     return out
 
 
-def finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall_s, next_rows=None, launch="eager",
-           lin_ms=None):
-    names = NAMES
+def finish(args, world, probs, kern_ms, total_ms, linear_ms, value, path_value, e2e, clk, wall_s, next_rows=None,
+           launch="eager", lin_ms=None):
+    names = [n for n in NAMES if n != "sq_pack_int4" or any(p.bits == 4 for p in probs)]
     # ---- rooflines per kernel (algorithmic work summed over the workload's linears)
     peaks, src = load_peaks()
+    int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
     work = {n: {} for n in names}
     for p in probs:
         for n, v in algorithmic_work_mnk(p.M, p.K, p.N, p.x.element_size(), p.y.element_size(), p.bits).items():
+            if n not in work:
+                continue
             for key, val in v.items():
                 work[n][key] = work[n].get(key, 0) + val
     # SSZ is bound by its search rounds, not by HBM: ALU work = c N K (1 + iters)
@@ -554,12 +589,11 @@ def finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall_s, next_
                               "frac": round(hbm / peaks["hbm_gbs"], 4)})
             work[n] = dict(work[n], ops=ssz_ops)
         elif "ops" in work[n] and (work[n]["ops"] / max(work[n]["bytes"], 1)
-                                   >= peaks["bf16_tflops"] * INT8_OVER_BF16 * 1e12 / (peaks["hbm_gbs"] * 1e9)):
+                                   >= int8_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)):
             # at or above the ridge point: bound by the tensor cores
             ach = work[n]["ops"] / t_s / 1e12
-            peak = peaks["bf16_tflops"] * INT8_OVER_BF16
-            entry.update(bound="tensor", achieved=round(ach, 1), peak=round(peak, 1), unit="TFLOP/s",
-                         frac=round(ach / peak, 4))
+            entry.update(bound="tensor", achieved=round(ach, 1), peak=round(int8_peak, 1), unit="TFLOP/s",
+                         frac=round(ach / int8_peak, 4))
         else:
             ach = work[n]["bytes"] / t_s / 1e9
             peak = peaks["hbm_gbs"]
@@ -576,9 +610,10 @@ def finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall_s, next_
                            }[roof["bound"]]
 
     p0 = probs[0]
-    launches_per_step = {"calib_absmax": 1, "smooth_fold": 2, "ssz_quant_weight": 1, "quant_act_per_token": 1,
-                         "w8a8_gemm_dequant": 1 if p0.bits == 8 else 2}
+    launches_per_step = {"calib_absmax": 1, "smooth_fold": 2, "ssz_quant_weight": 1, "sq_pack_int4": int(p0.bits == 4),
+                         "quant_act_per_token": 1, "w8a8_gemm_dequant": 1}
     M, K, N = p0.M, p0.K, p0.N
+    lin_step = linear_ms / args.steps
     result = {
         "metric": "W8A8 linear INT8 TOPS (% of peak); quant/SSZ GB/s (% of HBM) on 1 B200",
         "value": round(value, 2),
@@ -599,6 +634,15 @@ def finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall_s, next_
                    "launch": {"cuda_graph": "each timed step one CUDA graph replay (captured once, per-kernel "
                                             "events inside it)",
                               "eager": "every call of a timed step launched from Python"}[launch]},
+        "value_definition": ("2*M*N*K int8 ops over the device time of the per-inference linear (per-token "
+                             "activation quantization + GEMM with fused dequant) inside each timed step; every "
+                             "timed step also runs the once-per-weight path (calibration, smoothing, SSZ), whose "
+                             "time is in ms_per_step and whose throughput is in weight_path"),
+        "linear": {"ms_per_step": round(lin_step, 4), "tops": round(value, 2), "peak": round(int8_peak, 1),
+                   "frac": round(value / int8_peak, 4), "kernels": list(LINEAR)},
+        "path": {"ms_per_step": round(total_ms / args.steps, 4), "tops": round(path_value, 2),
+                 "what": "the whole path per step: calibration, smoothing, SSZ, activation quantization, GEMM"},
+        "weight_path": {n: kernels[n] for n in names if n in WEIGHT_PATH},
         "roofline": roof,
         "kernels": kernels,
         "e2e": e2e,
@@ -614,43 +658,47 @@ def finish(args, world, probs, kern_ms, total_ms, value, e2e, clk, wall_s, next_
 
 
 # ------------------------------------------------------------------ oracle arm
-def oracle_sample(cfg, frac=1.0):
-    """Time the CPU oracle on one step of the workload.  frac < 1 runs the
-    SSZ search, the activation quantization and the GEMM+dequant on that
-    fraction of their rows (rows are independent in all three) and scales
-    their times back up; the calibration and weight-absmax passes always run
-    in full.  Returns (seconds per full step, per-stage seconds, description)."""
+def oracle_linear_times(x, wt, alpha, bits, max_iters, frac=1.0):
+    """Time the CPU oracle on one linear (x [M,K], wt [N,K] fp32 numpy).
+    frac < 1 runs the SSZ search, the activation quantization and the
+    GEMM+dequant on that fraction of their rows (rows are independent in all
+    three) and scales their times back up; the calibration and weight-absmax
+    passes always run in full.  Returns (per-stage seconds scaled to the full
+    linear, description, per-stage seconds actually spent)."""
     import oracle
-    import synthetic
-    x, wt = _oracle_inputs(cfg)
-    M, K, N = cfg.M, cfg.K, cfg.N
-    t = {}
+    M, K = x.shape
+    N = wt.shape[0]
+    t, spent = {}, {}
     t0 = time.perf_counter()
     ax = oracle.calib_absmax(x)
     t["calib_absmax"] = time.perf_counter() - t0
     t0 = time.perf_counter()
     aw = oracle.weight_col_absmax(wt)
-    s, inv_s = oracle.smooth_factor(ax, aw, cfg.alpha)
+    s, inv_s = oracle.smooth_factor(ax, aw, alpha)
     t["smooth_fold"] = time.perf_counter() - t0
     n_s = max(1, min(N, int(round(N * frac))))
     m_s = max(1, min(M, int(round(M * frac))))
     t0 = time.perf_counter()
-    wq = oracle.ssz_quant_weight(wt[:n_s], bits=cfg.bits, max_iters=cfg.max_iters, s=s)
-    t["ssz_quant_weight"] = (time.perf_counter() - t0) * N / n_s
+    wq = oracle.ssz_quant_weight(wt[:n_s], bits=bits, max_iters=max_iters, s=s)
+    spent["ssz_quant_weight"] = time.perf_counter() - t0
+    t["ssz_quant_weight"] = spent["ssz_quant_weight"] * N / n_s
     t0 = time.perf_counter()
     qx, sx = oracle.quant_act_per_token(x[:m_s], inv_s)
-    t["quant_act_per_token"] = (time.perf_counter() - t0) * M / m_s
+    spent["quant_act_per_token"] = time.perf_counter() - t0
+    t["quant_act_per_token"] = spent["quant_act_per_token"] * M / m_s
     t0 = time.perf_counter()
     acc = oracle.gemm_i8(qx, wq["q"])
     oracle.dequant(acc, sx, wq["scale"])
-    t["w8a8_gemm_dequant"] = (time.perf_counter() - t0) * (M * N) / (m_s * n_s)
+    spent["w8a8_gemm_dequant"] = time.perf_counter() - t0
+    t["w8a8_gemm_dequant"] = spent["w8a8_gemm_dequant"] * (M * N) / (m_s * n_s)
+    spent["calib_absmax"], spent["smooth_fold"] = t["calib_absmax"], t["smooth_fold"]
     if frac >= 1.0:
-        sample = "the whole workload, one step (%d tokens x %d -> %d)" % (M, K, N)
+        sample = "whole linear (%d tokens x %d -> %d)" % (M, K, N)
     else:
-        sample = ("calibration and weight absmax in full; SSZ on %d of %d channels, activation quantization on "
-                  "%d of %d tokens, GEMM+dequant on their %dx%d block; each scaled to the full step"
-                  % (n_s, N, m_s, M, m_s, n_s))
-    return sum(t.values()), t, sample
+        sample = ("%d tokens x %d -> %d: calibration and weight absmax in full; SSZ on %d of %d channels, "
+                  "activation quantization on %d of %d tokens, GEMM+dequant on their %dx%d block; each scaled "
+                  "to the full linear" % (M, K, N, n_s, N, m_s, M, m_s, n_s))
+    return t, sample, spent
 
 
 _INPUTS = {}
@@ -664,6 +712,67 @@ def _oracle_inputs(cfg):
     return _INPUTS[cfg.name]
 
 
+def _gpt_sample_inputs():
+    """Layer 0 of the GPT-345M-shaped harness on the CPU over one of the 8
+    sequences (1024 tokens): the four linears' inputs and weights."""
+    if GPT_WORKLOAD not in _INPUTS:
+        import torch
+        from synthetic import gpt
+        weights = gpt.make_weights(0, "cpu")
+        cap = {}
+        gpt.forward(weights, gpt.make_tokens(0)[:1], capture=cap, layers=1)
+        _INPUTS[GPT_WORKLOAD] = [(cap[(0, n)].float().numpy(), weights[(0, n)].float().numpy()) for n in gpt.LINEARS]
+        del weights, torch
+    return _INPUTS[GPT_WORKLOAD]
+
+
+def oracle_workload(workload, frac=1.0):
+    """The oracle on one step of a workload: (int8 ops per step, per-stage
+    seconds scaled to the full step, sample description, per-stage seconds
+    actually spent).  The GPT-345M
+    workload is sampled as layer 0 over one sequence, its token-proportional
+    stages (calibration, activation quantization, GEMM) scaled by 8 to the
+    8 x 1024 batch and every stage by the 24 layers."""
+    import synthetic
+    if workload == GPT_WORKLOAD:
+        from synthetic import gpt
+        tot, descs, spent = {}, [], {}
+        for x, wt in _gpt_sample_inputs():
+            t, d, sp = oracle_linear_times(x, wt, 0.5, 8, 20, frac)
+            for k, v in sp.items():
+                spent[k] = spent.get(k, 0.0) + v
+            for k, v in t.items():
+                per_token = k in ("calib_absmax", "quant_act_per_token", "w8a8_gemm_dequant")
+                tot[k] = tot.get(k, 0.0) + v * gpt.LAYERS * (gpt.BATCH if per_token else 1)
+            descs.append(d)
+        sample = ("layer 0 of the GPT-345M-shaped harness over 1 of 8 sequences (" + "; ".join(descs) +
+                  "); token-proportional stages x8, all stages x24 layers")
+        return gpt.flops_per_pass(), tot, sample, spent
+    cfg = synthetic.CONFIGS[workload]
+    x, wt = _oracle_inputs(cfg)
+    t, sample, spent = oracle_linear_times(x, wt, cfg.alpha, cfg.bits, cfg.max_iters, frac)
+    return 2.0 * cfg.M * cfg.N * cfg.K, t, sample, spent
+
+
+def oracle_metric(ops, t):
+    """(linear TOPS, whole-path TOPS) of the oracle's per-stage seconds."""
+    lin = t["quant_act_per_token"] + t["w8a8_gemm_dequant"]
+    return ops / lin / 1e12, ops / sum(t.values()) / 1e12
+
+
+def oracle_frac(workload, seconds):
+    """The sample fraction that makes one oracle step take about `seconds`:
+    a 1/64 probe, then fixed + (SSZ + act) f + GEMM f^2 = seconds (the GEMM
+    runs on an f M x f N block, the row-sampled stages on f of their rows)."""
+    f0 = 1.0 / 64
+    _, _, _, t = oracle_workload(workload, frac=f0)  # seconds spent on the probe
+    c = t["calib_absmax"] + t["smooth_fold"] - seconds  # always run in full
+    b = (t["ssz_quant_weight"] + t["quant_act_per_token"]) / f0
+    a = t["w8a8_gemm_dequant"] / (f0 * f0)
+    f = (-b + (b * b - 4 * a * c) ** 0.5) / (2 * a) if a > 0 else -c / max(b, 1e-9)
+    return min(1.0, max(1.0 / 1024, f))
+
+
 def cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -671,35 +780,42 @@ def cores():
         return os.cpu_count()
 
 
+def cpu_baseline(workload):
+    """The oracle as it stands on the host cores, one step of the workload
+    sampled to about 15 s, in the bench's metric."""
+    frac = oracle_frac(workload, 15.0)
+    ops, t, sample, _ = oracle_workload(workload, frac)
+    lin, path = oracle_metric(ops, t)
+    return {"value": round(lin, 6), "unit": "TOPS", "cores": cores(), "kind": "oracle", "sample": sample,
+            "path_tops": round(path, 6), "seconds_per_step": round(sum(t.values()), 3),
+            "stage_seconds": {k: round(v, 3) for k, v in t.items()}}
+
+
 def run_reference(args, rank):
-    """The oracle as it stands, timed on the host cores.  Each step is a
-    sample of the workload sized so that warm-up + steps take about two
-    minutes; its time is scaled to one full step."""
-    import synthetic
+    """The oracle as it stands, timed on the host cores in the bench's
+    metric.  Each step is a sample of the workload sized so that warm-up +
+    steps take about two minutes; its times are scaled to one full step."""
     if rank != 0:
         return None
-    if args.workload not in synthetic.CONFIGS:
-        return {"impl": "reference", "unavailable": "the oracle arm times the single-linear workloads only"}
-    cfg = synthetic.CONFIGS[args.workload]
-    probe, _, _ = oracle_sample(cfg, frac=1.0 / 16)
-    budget = 120.0 / max(1, args.warmup + args.steps)
-    frac = min(1.0, max(1.0 / 256, budget / max(probe, 1e-9)))
+    frac = oracle_frac(args.workload, 120.0 / max(1, args.warmup + args.steps))
     steps = []
     for _ in range(args.warmup + args.steps):
-        total, parts, sample = oracle_sample(cfg, frac)
-        steps.append(total)
+        ops, t, sample, _ = oracle_workload(args.workload, frac)
+        steps.append(t)
     timed = steps[args.warmup:]
-    ops = 2.0 * cfg.M * cfg.N * cfg.K
-    value = ops * len(timed) / sum(timed) / 1e12
+    tot = {k: sum(t[k] for t in timed) for k in timed[0]}
+    lin, path = oracle_metric(ops * len(timed), tot)
     return {
         "impl": "reference",
         "metric": "W8A8 linear INT8 TOPS (% of peak); quant/SSZ GB/s (% of HBM) on 1 B200",
-        "value": value, "unit": "TOPS", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * sum(timed) / len(timed), "higher_is_better": True, "scaling": "weak",
+        "value": lin, "unit": "TOPS", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * sum(tot.values()) / len(timed), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8 codes, int32 acc, fp32 decisions, fp64 sums (CPU)",
-        "data": "synthetic", "config": {"workload": args.workload, "M_tokens_per_gpu": cfg.M, "K": cfg.K, "N": cfg.N},
-        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cores(), "kind": "oracle", "sample": sample},
-        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "data": "synthetic", "config": {"workload": args.workload},
+        "value_definition": "2*M*N*K over the oracle's activation quantization + GEMM+dequant time",
+        "path": {"tops": path},
+        "cpu_baseline": {"value": lin, "unit": "TOPS", "cores": cores(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": lin, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
 
@@ -815,14 +931,8 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
     try:
         res = run_ours(args, rank, world, local_rank)
-        if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload != GPT_WORKLOAD:
-            import synthetic
-            total, parts, sample = oracle_sample(synthetic.CONFIGS[args.workload], frac=1.0)
-            cfg = synthetic.CONFIGS[args.workload]
-            res["cpu_baseline"] = {"value": round(2.0 * cfg.M * cfg.N * cfg.K / total / 1e12, 6), "unit": "TOPS",
-                                   "cores": cores(), "kind": "oracle", "sample": sample,
-                                   "seconds_per_step": round(total, 3),
-                                   "stage_seconds": {k: round(v, 3) for k, v in parts.items()}}
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(args.workload)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

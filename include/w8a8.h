@@ -112,7 +112,9 @@ sq_status sq_calib_absmax(const void *x, sq_dtype xt, int64_t M, int64_t K,
  * x_absmax: [K] fp32 from sq_calib_absmax.  w: [N,K] of dtype wt.
  * alpha in [0,1].  w_absmax_out, s_out, inv_s_out: [K] fp32 outputs
  * (required).  w_folded_out: [N,K] fp32 or NULL (the fold is otherwise
- * applied on the fly by ssz_quant_weight and quant_act_per_token). */
+ * applied on the fly by ssz_quant_weight and quant_act_per_token).
+ * With w_folded_out given, s_out must be 16-byte aligned (the fold reads s
+ * with 16-byte loads); SQ_ERR_ALIGN otherwise. */
 sq_status sq_smooth_fold(const float *x_absmax, const void *w, sq_dtype wt,
                          int64_t N, int64_t K, float alpha, float *w_absmax_out,
                          float *s_out, float *inv_s_out, float *w_folded_out,
@@ -223,15 +225,17 @@ sq_status w4a8_gemm_dequant(const int8_t *qx, const float *sx, const uint8_t *qw
  * equivalent rescaling) and the quantization fused with it so that X never
  * goes to memory (CUDA INT8 notes 4.2, kernel fusion).  Per row t of
  * h [M,K] (dtype ht):
- *     mu = sum_j h_j / K, var = sum_j (h_j - mu)^2 / K          (fp64)
+ *     mu = P(h) / K, var = P(d^2) / K, d_j = h_j - mu            (fp64)
  *     m = fp32(mu), r = fp32(1 / sqrt(var + eps))
  *     y_j = ((h_j - m) * r) * gamma_j + beta_j                   (fp32, each op rounded)
  *     x'_j = y_j * inv_s_j (fp32); codes and scale as quant_act_per_token.
+ * P is the pairwise sum: the row padded with zeros to a power of two and
+ * summed by recursive halving, S(lo, len) = S(lo, len/2) + S(lo + len/2,
+ * len/2).  The pages fix no summation order; this tree fixes one, so the
+ * statistics and the codes are reproducible bit for bit by any evaluation
+ * of the same tree.
  * gamma, beta, inv_s: [K] fp32 or NULL (1, 0, 1), 16-byte aligned.  eps >= 0.
- * K: a multiple of 16 up to 16384 (one row is held in registers).
- * The fp64 sums are taken in tree order; they equal a sequential sum
- * whenever they are exact (bf16 inputs of moderate range), otherwise they
- * may differ in the last bit. */
+ * K: a multiple of 16 up to 16384 (one row is held in registers). */
 sq_status sq_layernorm_quant(const void *h, sq_dtype ht, int64_t M, int64_t K, const float *gamma,
                              const float *beta, float eps, const float *inv_s, int8_t *q_out,
                              float *scale_out, void *stream);

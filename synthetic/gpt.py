@@ -41,9 +41,10 @@ def make_tokens(seed: int = 0, batch: int = BATCH, seq: int = SEQ):
 
 
 @torch.no_grad()
-def forward(weights, tokens, linear=None, capture=None):
+def forward(weights, tokens, linear=None, capture=None, layers=LAYERS):
     """bf16 forward.  `linear(layer, name, x2d, W)` computes each linear
-    (default x W^T); `capture` (dict) receives every linear's input [B*T, K]."""
+    (default x W^T); `capture` (dict) receives every linear's input [B*T, K];
+    `layers` < 24 stops after that many layers (input synthesis for a sample)."""
     dev = weights["wte"].device
     B, T = tokens.shape
     x = weights["wte"][tokens.to(dev)] + weights["wpe"][:T][None]
@@ -55,7 +56,7 @@ def forward(weights, tokens, linear=None, capture=None):
             capture[(layer, name)] = a2
         return lin(layer, name, a2, weights[(layer, name)]).reshape(*a.shape[:-1], -1)
 
-    for layer in range(LAYERS):
+    for layer in range(layers):
         h = F.layer_norm(x, (HIDDEN,))
         qkv = run(layer, "qkv", h)
         q, k, v = qkv.split(HIDDEN, dim=-1)

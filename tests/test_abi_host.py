@@ -91,6 +91,14 @@ def test_smooth_fold_rejects_alpha(lib, alpha, status):
     assert "alpha" in _detail(lib)
 
 
+def test_smooth_fold_fold_needs_16_byte_s(lib):
+    # s_out at a 4-byte offset is a valid vector, but the materialised fold
+    # reads it 16 bytes at a time
+    rc = lib.sq_smooth_fold(P(), P(4096), 1, 8, 32, 0.5, P(8192), P(12292), P(16384), P(32768), None)
+    assert rc == 4, _detail(lib)
+    assert "s_out" in _detail(lib)
+
+
 def test_smooth_factor_rejects(lib):
     assert lib.sq_smooth_factor(NULL, P(4096), 32, 0.5, P(8192), P(12288), None) == 1
     assert lib.sq_smooth_factor(P(), P(4096), 40, 0.5, P(8192), P(12288), None) == 2

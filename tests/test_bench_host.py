@@ -23,16 +23,21 @@ def test_algorithmic_work_of_the_prefill_linear(bench):
     assert w["calib_absmax"]["bytes"] == 2 * 2048 * 4096 + 4 * 4096            # X once + absmax
     assert w["w8a8_gemm_dequant"]["ops"] == 2 * 2048 * 4096 * 4096
     assert w["w8a8_gemm_dequant"]["bytes"] == 2048 * 4096 + 4096 * 4096 + 4 * 2048 + 4 * 4096 + 2 * 2048 * 4096
+    assert w["sq_pack_int4"]["bytes"] == 0
     w4 = bench.algorithmic_work_mnk(16, 8192, 28672, 2, 2, 4)
     # int4: the codes are packed (read N K, write N K / 2) and read packed by the GEMM
-    assert w4["w8a8_gemm_dequant"]["bytes"] - 16 * 8192 - 4 * 16 - 4 * 28672 - 2 * 16 * 28672 == 2 * 28672 * 8192
+    assert w4["sq_pack_int4"]["bytes"] == 28672 * 8192 * 3 // 2
+    assert w4["w8a8_gemm_dequant"]["bytes"] - 16 * 8192 - 4 * 16 - 4 * 28672 - 2 * 16 * 28672 == 28672 * 8192 // 2
 
 
 def test_per_shape_table_groups_linears_by_shape(bench):
     probs = [SimpleNamespace(M=8192, K=1024, N=3072), SimpleNamespace(M=8192, K=1024, N=1024),
              SimpleNamespace(M=8192, K=1024, N=3072)]
-    # ms per kernel (NAMES order) per linear
-    lin = [[0.01, 0.01, 0.05, 0.01, 0.030], [0.01, 0.01, 0.04, 0.01, 0.020], [0.03, 0.01, 0.07, 0.01, 0.030]]
+    # ms per kernel (NAMES order: calib, smooth, ssz, pack, act quant, gemm) per linear
+    assert bench.NAMES == ["calib_absmax", "smooth_fold", "ssz_quant_weight", "sq_pack_int4", "quant_act_per_token",
+                           "w8a8_gemm_dequant"]
+    lin = [[0.01, 0.01, 0.05, 0.0, 0.01, 0.030], [0.01, 0.01, 0.04, 0.0, 0.01, 0.020],
+           [0.03, 0.01, 0.07, 0.0, 0.01, 0.030]]
     t = bench.per_shape_table(probs, lin, {"bf16_tflops": 1000.0})
     assert set(t) == {"8192x1024->3072", "8192x1024->1024"}
     qkv = t["8192x1024->3072"]
@@ -41,6 +46,24 @@ def test_per_shape_table_groups_linears_by_shape(bench):
     tops = 2 * 8192 * 1024 * 3072 / 30e-6 / 1e12
     assert qkv["gemm_tops"] == pytest.approx(round(tops, 1))
     assert qkv["gemm_frac"] == pytest.approx(round(tops / (1000.0 * bench.INT8_OVER_BF16), 4))
+    assert qkv["linear_tops"] == pytest.approx(round(2 * 8192 * 1024 * 3072 / 40e-6 / 1e12, 1))
+
+
+def test_default_workload_is_the_mlp_up_projection(bench):
+    assert bench.DEFAULT_WORKLOAD == "mlp_up_8192x4096x11008"
+
+
+def test_oracle_arm_reports_the_linear_metric(bench):
+    """The oracle arm times the whole path on a small linear and reports
+    2 M N K over its activation quantization + GEMM time, like our arm."""
+    ops, t, sample, spent = bench.oracle_workload("single_linear_16x256x128", frac=1.0)
+    assert ops == 2 * 16 * 256 * 128
+    assert set(t) == {"calib_absmax", "smooth_fold", "ssz_quant_weight", "quant_act_per_token", "w8a8_gemm_dequant"}
+    lin, path = bench.oracle_metric(ops, t)
+    assert lin == pytest.approx(ops / (t["quant_act_per_token"] + t["w8a8_gemm_dequant"]) / 1e12)
+    assert path < lin
+    ops2, t2, sample2, _ = bench.oracle_workload("single_linear_16x256x128", frac=0.5)
+    assert "8 of 16 tokens" in sample2 and "64 of 128 channels" in sample2
 
 
 def test_recorded_traffic_matches_the_current_sources(bench):

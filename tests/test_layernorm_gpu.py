@@ -3,9 +3,9 @@ quantization (activation quantization fused upstream) against the oracle.
 
 SmoothQuant page section 1 (the smoothing moves into the op that produces
 X) and the CUDA INT8 notes 4.2 (fused kernel, no intermediate in memory).
-Both sides compute the statistics in fp64; the GPU sums in tree order, so a
-last-bit difference is possible where a sum is inexact.  Scales must agree
-within 1e-6 relative and the codes in all but a 1e-4 fraction (by at most 1).
+Both sides compute the statistics as fp64 pairwise sums (the row padded
+with zeros to a power of two, summed by recursive halving), so the
+statistics, the scales and the int8 codes must match bit for bit.
 """
 import numpy as np
 import pytest
@@ -20,6 +20,7 @@ pytestmark = pytest.mark.gpu
     (1, 16, torch.float32, False, False), (7, 48, torch.bfloat16, True, False), (300, 528, torch.bfloat16, True, True),
     (129, 1040, torch.float32, True, True), (2048, 4096, torch.bfloat16, True, True),
     (33, 8192, torch.bfloat16, False, True), (5, 16384, torch.float32, True, True),
+    (64, 3072, torch.bfloat16, True, True), (17, 272, torch.float32, False, True),
 ])
 def test_layernorm_quant_parity(w, orc, M, K, dtype, affine, smooth):
     h = make_x(M, K, dtype, seed=M + K, scale=20.0)
@@ -32,9 +33,31 @@ def test_layernorm_quant_parity(w, orc, M, K, dtype, affine, smooth):
     sx = Guarded((M,), torch.float32)
     w.sq_layernorm_quant(h.cuda(), d(g), d(b), 1e-5, d(inv), q.t, sx.t)
     qo, sxo, _ = orc.layernorm_quant(np32(h), g, b, 1e-5, inv)
-    np.testing.assert_allclose(sx.t.cpu().numpy(), sxo, rtol=1e-6, atol=0)
-    qg = q.t.cpu().numpy()
-    assert np.mean(qg != qo) < 1e-4 and np.abs(qg.astype(int) - qo).max() <= 1
+    np.testing.assert_array_equal(sx.t.cpu().numpy(), sxo)
+    np.testing.assert_array_equal(q.t.cpu().numpy(), qo)
+    assert q.intact() and sx.intact()
+
+
+@pytest.mark.parametrize("K", [16, 48, 1024, 4096])
+def test_layernorm_quant_order_sensitive_rows(w, orc, K):
+    """Rows whose fp64 sums depend on the summation order (entries of
+    magnitude 2^53 beside small ones): the codes and scales still match the
+    oracle's pairwise tree bit for bit."""
+    r = np.random.default_rng(K + 5)
+    h = (r.standard_normal((6, K)) * 4.0).astype(np.float32)
+    big = np.float32(2.0 ** 53)
+    for t in range(6):
+        cols = r.choice(K, 4, replace=False)
+        h[t, cols[:2]] = big
+        h[t, cols[2:]] = -big
+        h[t, r.choice(K, 3, replace=False)] += np.float32(0.5)
+    inv = (r.random(K) + 0.5).astype(np.float32)
+    q = Guarded((6, K), torch.int8)
+    sx = Guarded((6,), torch.float32)
+    w.sq_layernorm_quant(torch.from_numpy(h).cuda(), None, None, 1e-5, torch.from_numpy(inv).cuda(), q.t, sx.t)
+    qo, sxo, _ = orc.layernorm_quant(h, None, None, 1e-5, inv)
+    np.testing.assert_array_equal(sx.t.cpu().numpy(), sxo)
+    np.testing.assert_array_equal(q.t.cpu().numpy(), qo)
     assert q.intact() and sx.intact()
 
 

@@ -235,20 +235,47 @@ static void launch_quant_act(const void *x, int64_t M, int64_t K, const float *i
 }
 
 // ------------------------------------------------ LayerNorm fused with step 4
-// One CTA per row (as quant_act_kernel), the raw row in registers for the
-// whole computation: fp64 mean, then fp64 sum of squared deviations (two
-// passes over registers), rstd = 1 / sqrt(var + eps) (IEEE fp64); m and r
-// rounded to fp32, then per element y = ((h - m) r) gamma + beta and
+// One CTA per row, the raw row in registers for the whole computation.  The
+// row statistics are fp64 pairwise sums: the tree that halves the row padded
+// with zeros to a power of two (S(lo, len) = S(lo, len/2) + S(lo + len/2,
+// len/2)), so they do not depend on how the work is split.  Thread t owns the
+// E contiguous columns [t E, t E + E): it sums its 8-column chunks as
+// subtrees of 8 and combines them pairwise; the xor butterfly of a warp
+// combines neighbouring threads' subtrees (a + b == b + a exactly, so every
+// lane ends with the same sum), and one more butterfly over the warps' sums
+// finishes the tree (T and E are powers of two).  Then mean = S / K,
+// var = S(d^2) / K with d = h - mean, rstd = 1 / sqrt(var + eps) (IEEE fp64);
+// m and r rounded to fp32, then per element y = ((h - m) r) gamma + beta and
 // x' = y inv_s in fp32 with no fused multiply-add (the build contracts
-// nothing), the row abs-max and the packed per-token codes.  X' never goes
-// to memory.
-__device__ __forceinline__ double block_sum_d(double v, double (&red)[32], int lane, int warp, int nwarps) {
+// nothing), the row abs-max and the packed per-token codes.  X' never goes to
+// memory.
+
+// Pairwise sum of 8 values (a subtree of 8 leaves).
+__device__ __forceinline__ double tree8(const double (&a)[8]) {
+    return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+}
+
+// Pairwise sum of C chunk subtrees (C a power of two).
+template <int C>
+__device__ __forceinline__ double tree_chunks(double (&c)[C]) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    for (int len = C; len > 1; len >>= 1) {
+#pragma unroll
+        for (int i = 0; i < len / 2; ++i) c[i] = c[2 * i] + c[2 * i + 1];
+    }
+    return c[0];
+}
+
+// The thread subtrees of the whole CTA combined in tree order: warp
+// butterfly, then a butterfly over the nwarps (a power of two) warp sums.
+__device__ __forceinline__ double block_tree_sum(double v, double (&red)[32], int lane, int warp, int nwarps) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     if (lane == 0) red[warp] = v;
     __syncthreads();
-    double t = red[0];
-    for (int w = 1; w < nwarps; ++w) t += red[w];
+    double t = lane < nwarps ? red[lane] : 0.0;
+    for (int o = 1; o < nwarps; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    t = __shfl_sync(0xffffffffu, t, 0);
     __syncthreads();  // red is reused by the next reduction
     return t;
 }
@@ -263,44 +290,48 @@ ln_quant_kernel(const T *__restrict__ h, int64_t M, int64_t K, const float *__re
     __shared__ float redf[32];
     const int T_ = blockDim.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = T_ >> 5;
-    bool live[C];
+    const int64_t base = (int64_t)threadIdx.x * E;  // this thread's first column
+    bool live[C];  // K is a multiple of 8: a chunk is wholly inside the row or wholly past it
 #pragma unroll
-    for (int c = 0; c < C; ++c) live[c] = ((int64_t)c * T_ + threadIdx.x) * 8 < K;
+    for (int c = 0; c < C; ++c) live[c] = base + 8 * c < K;
     const double kd = (double)K;
 
     for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
         Raw8<T> raw[C];
 #pragma unroll
         for (int c = 0; c < C; ++c) {
-            if (live[c]) raw[c].load(h + row * K + ((int64_t)c * T_ + threadIdx.x) * 8);
+            if (live[c]) raw[c].load(h + row * K + base + 8 * c);
             else raw[c].zero();
         }
-        double sum = 0.0;
+        double part[C];
 #pragma unroll
         for (int c = 0; c < C; ++c) {
             float v[8];
-            raw[c].widen(v);
+            raw[c].widen(v);  // zeros past the row
+            double a[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) sum += (double)v[i];
+            for (int i = 0; i < 8; ++i) a[i] = (double)v[i];
+            part[c] = tree8(a);
         }
-        const double mu = block_sum_d(sum, redd, lane, warp, nwarps) / kd;
-        double ss = 0.0;
+        const double mu = block_tree_sum(tree_chunks<C>(part), redd, lane, warp, nwarps) / kd;
 #pragma unroll
         for (int c = 0; c < C; ++c) {
-            if (!live[c]) continue;
             float v[8];
             raw[c].widen(v);
+            double a[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const double d = (double)v[i] - mu;
-                ss += d * d;
+                a[i] = live[c] ? d * d : 0.0;  // the padding adds zeros, not (0 - mu)^2
             }
+            part[c] = tree8(a);
         }
-        const double rstd = 1.0 / sqrt(block_sum_d(ss, redd, lane, warp, nwarps) / kd + (double)eps);
+        const double var = block_tree_sum(tree_chunks<C>(part), redd, lane, warp, nwarps) / kd;
+        const double rstd = 1.0 / sqrt(var + (double)eps);
         const float m32 = (float)mu, r32 = (float)rstd;
         // x' of chunk c: ((h - m) r) gamma + beta, times inv_s, each op in fp32
         auto xs = [&](int c, float (&x)[8]) {
-            const int64_t j = ((int64_t)c * T_ + threadIdx.x) * 8;
+            const int64_t j = base + 8 * c;
             float v[8], g[8], b[8], f[8];
             raw[c].widen(v);
             if (gamma) load8_f32(gamma + j, g);
@@ -350,15 +381,20 @@ ln_quant_kernel(const T *__restrict__ h, int64_t M, int64_t K, const float *__re
             } else {
                 code = fast_codes_tied(x, s, r, narrow, tie_bound);
             }
-            *reinterpret_cast<uint2 *>(q + row * K + ((int64_t)c * T_ + threadIdx.x) * 8) = code;
+            *reinterpret_cast<uint2 *>(q + row * K + base + 8 * c) = code;
         }
     }
 }
 
+// T threads of E contiguous columns each, T * E the power of two at or above
+// K (at least one warp of E = 8): E = 8, 16, 32 up to K = 1024, then 32
+// columns a thread and up to 512 threads (K <= 16384).
 template <typename T, int E>
 static void launch_ln_quant(const void *h, int64_t M, int64_t K, const float *gamma, const float *beta, float eps,
                             const float *inv_s, int8_t *q, float *scale, int sms, cudaStream_t st) {
-    const int threads = (int)ceil_div(ceil_div(K, E), 32) * 32;
+    int64_t P = 32 * E;
+    while (P < K) P *= 2;
+    const int threads = (int)(P / E);
     const int per_sm = std::max(1, std::min(32, 2048 / threads));
     const int64_t grid = std::min<int64_t>(M, (int64_t)sms * per_sm);
     ln_quant_kernel<T, E><<<(unsigned)grid, threads, 0, st>>>((const T *)h, M, K, gamma, beta, eps, inv_s, q, scale);
@@ -494,18 +530,15 @@ extern "C" sq_status sq_layernorm_quant(const void *h, sq_dtype ht, int64_t M, i
     if (st != SQ_OK) return st;
     cudaStream_t cs = (cudaStream_t)stream;
     const bool bf = ht == SQ_BF16;
-    // E elements per thread: one warp per row up to K = 32 E, at most 32
-    // (measured faster than 64, which spills); K <= 16384 keeps a row within
-    // 512 threads
+    // E contiguous columns per thread: one warp per row up to K = 32 E, then
+    // E = 32 (measured faster than 64, which spills); K <= 16384 keeps a row
+    // within 512 threads
     if (K <= 256) {
         if (bf) launch_ln_quant<__nv_bfloat16, 8>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);
         else launch_ln_quant<float, 8>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);
     } else if (K <= 512) {
         if (bf) launch_ln_quant<__nv_bfloat16, 16>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);
         else launch_ln_quant<float, 16>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);
-    } else if (K <= 1024) {
-        if (bf) launch_ln_quant<__nv_bfloat16, 32>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);
-        else launch_ln_quant<float, 32>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);
     } else {
         if (bf) launch_ln_quant<__nv_bfloat16, 32>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);
         else launch_ln_quant<float, 32>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);

@@ -200,6 +200,9 @@ extern "C" sq_status sq_smooth_fold(const float *x_absmax, const void *w, sq_dty
     if ((w && !aligned(w, 16)) || (w_folded_out && !aligned(w_folded_out, 16)) ||
         !aligned(x_absmax, 4) || !aligned(w_absmax_out, 4) || !aligned(s_out, 4) || !aligned(inv_s_out, 4))
         return fail(SQ_ERR_ALIGN, "sq_smooth_fold: misaligned pointer");
+    // the fold reads s eight columns at a time with 16-byte loads
+    if (w_folded_out && !aligned(s_out, 16))
+        return fail(SQ_ERR_ALIGN, "sq_smooth_fold: s_out must be 16-byte aligned when w_folded_out is given");
     int sms;
     sq_status st = check_device(&sms);
     if (st != SQ_OK) return st;
