@@ -22,9 +22,12 @@ e2e    = the same metric through the C ABI with the activations copied from
          timed), the quantized weights resident on the device.
 
 Multi-GPU (torchrun): data parallel, each rank a replica of the layer with its
-own batch of tokens (weak scaling).  The one exchange is the calibration
-statistic: the [K] activation absmax is all-reduced with MAX over NCCL so all
-replicas derive the same smoothing factor and the same quantized weight.
+own batch of tokens (weak scaling).  The calibration statistic, the [K]
+activation absmax, is all-reduced with MAX over NCCL so all replicas derive
+the same smoothing factor; the SSZ search is split by output channel (each
+rank searches N/G channels) and its codes, scales and rounds are
+all-gathered, so every replica holds the same quantized weight without
+repeating the search.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 """
@@ -271,7 +274,10 @@ def run_ours(args, rank, world, local_rank):
         wdist.allreduce_calibration(p.ax)
         w.sq_smooth_fold(p.ax, p.wt, p.alpha, p.aw, p.s, p.inv)
         mark(2)
-        w.ssz_quant_weight(p.wt, p.s, p.bits, p.max_iters, p.qw, p.sw, iters_out=p.iters)
+        if world > 1:  # each rank searches its block of output channels, then all-gather
+            wdist.ssz_quant_weight_sharded(p.wt, p.s, p.bits, p.max_iters, p.qw, p.sw, p.iters)
+        else:
+            w.ssz_quant_weight(p.wt, p.s, p.bits, p.max_iters, p.qw, p.sw, iters_out=p.iters)
         mark(3)
         if p.bits == 4:  # int4 weights: packed two per byte for the W4A8 GEMM
             w.sq_pack_int4(p.qw, p.qw4)
@@ -629,7 +635,8 @@ def finish(args, world, probs, kern_ms, total_ms, linear_ms, value, path_value, 
         "data": "synthetic (seeded LLM-shaped activations with outlier channels, N(0,std) weights)",
         "config": {"workload": args.workload, "linears": len(probs), "M_tokens_per_gpu": M, "K": K, "N": N,
                    "alpha": p0.alpha, "weight_bits": p0.bits, "ssz_max_iters": p0.max_iters,
-                   "parallelism": "dp%d (replicas; MAX all-reduce of the calibration absmax)" % world,
+                   "parallelism": ("dp%d (replicas; MAX all-reduce of the calibration absmax; SSZ split by output "
+                                   "channel and all-gathered)" % world),
                    "l2": "flushed (512 MB write, then 384 MB read) before every timed step, outside the timed events",
                    "launch": {"cuda_graph": "each timed step one CUDA graph replay (captured once, per-kernel "
                                             "events inside it)",

@@ -86,6 +86,20 @@ int sq_abi_version(void);
  * 4 GEMM epilogue, 6 sq_selftest_bounded_wait, 7 W4A8 GEMM unpacking. */
 sq_status sq_device_fault(void *stream, uint32_t *fault_out /* host */);
 
+/* Debug counters (the pages' debugging advice, CUDA INT8 notes section 5:
+ * copy the parameters back and compare stage by stage, in place of a
+ * sanitizer).  A debug build of this library (compiled with -DW8A8_DEBUG,
+ * shipped as libw8a8_debug.so) counts, in device counters, the non-finite
+ * values among the input matrices the kernels read (x of sq_calib_absmax and
+ * quant_act_per_token / _static / _rowsum, w of sq_smooth_fold, the smoothed
+ * w of ssz_quant_weight / _asym, h of sq_layernorm_quant; each element once
+ * per call) and the index checks that failed (the access is then skipped).
+ * Nothing traps.  This call synchronizes `stream`, writes both totals to
+ * the host and clears them; *enabled_out is 1 in a debug build.  In a
+ * release build it writes zeros and *enabled_out = 0. */
+sq_status sq_debug_status(void *stream, uint64_t *nonfinite_out /* host */, uint64_t *index_out /* host */,
+                          int *enabled_out /* host */);
+
 /* Test hook for the bounded waits: launches one CTA that waits, with the same
  * bounded wait the GEMM uses and a limit of limit_ms (1..10000), on an
  * mbarrier nothing ever arrives at.  The wait runs out, records fault code 6

@@ -267,3 +267,22 @@ def test_python_binding_refuses_cpu_tensors():
     ax = torch.zeros(32)
     with pytest.raises(ValueError):
         w.sq_calib_absmax(x, ax)
+
+
+def test_debug_status_release_build(lib):
+    nf, ix, en = ctypes.c_uint64(7), ctypes.c_uint64(7), ctypes.c_int(7)
+    assert lib.sq_debug_status(None, ctypes.byref(nf), ctypes.byref(ix), ctypes.byref(en)) == 0
+    assert (nf.value, ix.value, en.value) == (0, 0, 0)
+    assert lib.sq_debug_status(None, None, ctypes.byref(ix), ctypes.byref(en)) == 1
+
+
+def test_debug_library_exports_every_declared_symbol():
+    """The debug build (-DW8A8_DEBUG) is the same library with counters: it
+    exports every declared entry point."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("w8a8_build", os.path.join(ROOT, "w8a8_linear_layers_b200",
+                                                                             "build.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    dbg = ctypes.CDLL(b.build(debug=True))
+    assert [f for f in declared_functions() if not hasattr(dbg, f)] == []

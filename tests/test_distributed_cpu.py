@@ -125,6 +125,25 @@ class _OracleOps:
     def dequant(self, acc, sx, sw, y):
         y.copy_(torch.from_numpy(self.o.dequant(acc.numpy(), sx.numpy(), sw.numpy(), out="f32")))
 
+    def ssz(self, w_rows, s, bits, max_iters, q_out, scale_out, iters_out):
+        r = self.o.ssz_quant_weight(w_rows.float().numpy(), bits=bits, max_iters=max_iters,
+                                    s=None if s is None else s.numpy())
+        q_out.copy_(torch.from_numpy(r["q"]))
+        scale_out.copy_(torch.from_numpy(r["scale"]))
+        iters_out.copy_(torch.from_numpy(r["iters"]))
+
+    def quant_act(self, x, inv_s, qx, sx):
+        q, s = self.o.quant_act_per_token(x.float().numpy(), None if inv_s is None else inv_s.numpy())
+        qx.copy_(torch.from_numpy(q))
+        sx.copy_(torch.from_numpy(s))
+
+    def gemm(self, qx, sx, qw, sw, y):
+        acc = self.o.gemm_i8(qx.numpy(), qw.numpy())
+        if y.dtype == torch.bfloat16:
+            y.view(torch.int16).copy_(torch.from_numpy(self.o.dequant(acc, sx.numpy(), sw.numpy()).view(np.int16)))
+        else:
+            y.copy_(torch.from_numpy(self.o.dequant(acc, sx.numpy(), sw.numpy(), out="f32")))
+
 
 def _row_parallel_worker(rank, world, port, outdir):
     _init(rank, world, port)
@@ -164,3 +183,70 @@ def test_row_parallel_linear_equals_unsharded():
     want = oracle.dequant(oracle.gemm_i8(q, qw), sx, sw, out="f32")
     for y in ys:
         np.testing.assert_array_equal(y, want)
+
+
+# ------------------------------------------------- N-sharded SSZ and linear
+def _sharded_inputs():
+    import synthetic
+    x, wt = synthetic.make_small(20, 96, 37, seed=5, w_outliers=4)  # N = 37: blocks of 19 and 18
+    K = 96
+    inv = (np.random.default_rng(6).random(K) + 0.5).astype(np.float32)
+    s = (np.float32(1.0) / inv).astype(np.float32)
+    return x, wt, s, inv
+
+
+def _sharded_worker(rank, world, port, outdir):
+    _init(rank, world, port)
+    try:
+        import oracle
+        from w8a8_linear_layers_b200 import distributed as wdist
+        x, wt, s, inv = _sharded_inputs()
+        N, K = wt.shape
+        ops = _OracleOps(oracle)
+        # SSZ split by output channel, all-gathered
+        q = torch.empty(N, K, dtype=torch.int8)
+        sc = torch.empty(N)
+        its = torch.empty(N, dtype=torch.int32)
+        wdist.ssz_quant_weight_sharded(wt.float(), torch.from_numpy(s), 8, 20, q, sc, its, ops=ops)
+        # column-parallel linear on this rank's block of the gathered weight
+        a, b = wdist.shard_rows(N, world, rank)
+        y_shard = torch.empty(x.shape[0], b - a, dtype=torch.bfloat16)
+        y_full = torch.empty(x.shape[0], N, dtype=torch.bfloat16)
+        wdist.column_parallel_linear(x.float(), torch.from_numpy(inv), q[a:b].contiguous(), sc[a:b].contiguous(),
+                                     y_shard, y_full, ops=ops)
+        np.savez(os.path.join(outdir, "rank%d.npz" % rank), q=q.numpy(), sc=sc.numpy(), its=its.numpy(),
+                 y=y_full.view(torch.int16).numpy(), ys=y_shard.view(torch.int16).numpy(), a=a, b=b)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_shard_rows_cover_every_row_once():
+    from w8a8_linear_layers_b200.distributed import shard_rows
+    for n in (1, 7, 37, 4096, 11008):
+        for g in (1, 2, 3, 8):
+            blocks = [shard_rows(n, g, r) for r in range(g)]
+            assert blocks[0][0] == 0 and blocks[-1][1] == n
+            assert all(blocks[i][1] == blocks[i + 1][0] for i in range(g - 1))
+            sizes = [b - a for a, b in blocks]
+            assert max(sizes) - min(sizes) <= 1
+
+
+def test_sharded_ssz_and_column_parallel_equal_unsharded():
+    """SSZ split by output channel over 2 ranks and all-gathered equals the
+    unsharded search (codes, scales, rounds bit for bit); the column-parallel
+    linear's gathered output equals the unsharded linear's, and each rank's
+    block equals its columns."""
+    import oracle
+    with tempfile.TemporaryDirectory() as d:
+        mp.spawn(_sharded_worker, args=(2, _free_port(), d), nprocs=2, join=True)
+        rs = [np.load(os.path.join(d, "rank%d.npz" % r)) for r in range(2)]
+    x, wt, s, inv = _sharded_inputs()
+    ref = oracle.ssz_quant_weight(wt.float().numpy(), bits=8, max_iters=20, s=s)
+    qx, sx = oracle.quant_act_per_token(x.float().numpy(), inv)
+    y_ref = oracle.dequant(oracle.gemm_i8(qx, ref["q"]), sx, ref["scale"]).view(np.int16)
+    for r in rs:
+        np.testing.assert_array_equal(r["q"], ref["q"])
+        np.testing.assert_array_equal(r["sc"], ref["scale"])
+        np.testing.assert_array_equal(r["its"], ref["iters"])
+        np.testing.assert_array_equal(r["y"], y_ref)
+        np.testing.assert_array_equal(r["ys"], y_ref[:, int(r["a"]):int(r["b"])])

@@ -62,3 +62,48 @@ def test_row_parallel_emulated_equals_unsharded(w):
     y = torch.empty(M, N, device="cuda")
     ops.dequant(acc.to(torch.int32), sx_g, sw, y)
     assert torch.equal(y, y_full)
+
+
+@pytest.mark.parametrize("G", [2, 3])
+def test_ssz_by_output_channel_blocks_equals_unsharded(w, G):
+    """SSZ on each rank's block of output channels (ranks emulated in turn)
+    concatenates to the unsharded search: codes, scales and rounds bit for
+    bit (the channels are independent)."""
+    import synthetic
+    from w8a8_linear_layers_b200.distributed import shard_rows
+    x, wt = synthetic.make_small(64, 1040, 203, seed=11, w_outliers=20)
+    wt = wt.cuda()
+    N, K = wt.shape
+    s = torch.rand(K, device="cuda") + 0.5
+    q, sc, its = (torch.empty(N, K, dtype=torch.int8, device="cuda"), torch.empty(N, device="cuda"),
+                  torch.empty(N, dtype=torch.int32, device="cuda"))
+    w.ssz_quant_weight(wt, s, 8, 20, q, sc, iters_out=its)
+    for r in range(G):
+        a, b = shard_rows(N, G, r)
+        qr, sr, ir = (torch.empty(b - a, K, dtype=torch.int8, device="cuda"), torch.empty(b - a, device="cuda"),
+                      torch.empty(b - a, dtype=torch.int32, device="cuda"))
+        w.ssz_quant_weight(wt[a:b].contiguous(), s, 8, 20, qr, sr, iters_out=ir)
+        assert torch.equal(qr, q[a:b]) and torch.equal(sr, sc[a:b]) and torch.equal(ir, its[a:b])
+
+
+def test_column_parallel_blocks_equal_unsharded_columns(w):
+    """The column-parallel linear's per-rank products (ranks emulated in
+    turn, each on its block of output channels) are the unsharded output's
+    columns, bit for bit."""
+    from w8a8_linear_layers_b200.distributed import KernelOps, column_parallel_linear, shard_rows
+    M, K, N, G = 300, 1024, 1032, 3
+    x = make_x(M, K, torch.bfloat16, seed=12).cuda()
+    inv = torch.rand(K, device="cuda") + 0.5
+    qw = torch.randint(-127, 128, (N, K), dtype=torch.int8, device="cuda")
+    sw = torch.rand(N, device="cuda") * 1e-3
+    qx, sx = torch.empty(M, K, dtype=torch.int8, device="cuda"), torch.empty(M, device="cuda")
+    w.quant_act_per_token(x, inv, qx, sx)
+    y_full = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    w.w8a8_gemm_dequant(qx, sx, qw, sw, y_full)
+    ops = KernelOps(w)
+    for r in range(G):
+        a, b = shard_rows(N, G, r)
+        assert (b - a) % 8 == 0  # bf16 output rows of 16 bytes
+        y_r = torch.empty(M, b - a, dtype=torch.bfloat16, device="cuda")
+        column_parallel_linear(x, inv, qw[a:b].contiguous(), sw[a:b].contiguous(), y_r, ops=ops)
+        assert torch.equal(y_r, y_full[:, a:b])

@@ -16,7 +16,9 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libw8a8.so")
+# W8A8_LIBRARY=debug loads the debug build (libw8a8_debug.so: the kernels
+# count non-finite inputs and failed index checks, see sq_debug_status)
+LIB_PATH = os.path.join(_HERE, "libw8a8_debug.so" if os.environ.get("W8A8_LIBRARY") == "debug" else "libw8a8.so")
 
 SQ_F32, SQ_BF16 = 0, 1
 STATUS = ["SQ_OK", "SQ_ERR_NULL", "SQ_ERR_SHAPE", "SQ_ERR_DTYPE", "SQ_ERR_ALIGN", "SQ_ERR_ARG",
@@ -28,7 +30,7 @@ EXPORTS = ["sq_status_string", "sq_last_error_detail", "sq_abi_version", "sq_dev
            "sq_calib_absmax", "sq_smooth_fold", "ssz_quant_weight", "quant_act_per_token",
            "w8a8_gemm_dequant", "sq_static_range_update", "quant_act_static", "quant_act_per_token_rowsum",
            "ssz_quant_weight_asym", "w8a8_gemm_dequant_asym", "sq_pack_int4", "w4a8_gemm_dequant",
-           "sq_layernorm_quant", "quant_act_given_scale", "sq_dequant", "sq_smooth_factor"]
+           "sq_layernorm_quant", "quant_act_given_scale", "sq_dequant", "sq_smooth_factor", "sq_debug_status"]
 
 
 class W8A8Error(RuntimeError):
@@ -42,7 +44,7 @@ class W8A8Error(RuntimeError):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            "libw8a8.so is not built (%s); run `python -m w8a8_linear_layers_b200.build`" % LIB_PATH)
+            "%s is not built; run `python w8a8_linear_layers_b200/build.py`" % LIB_PATH)
     lib = ctypes.CDLL(LIB_PATH)
     P, I64, I, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
     sig = {
@@ -67,6 +69,7 @@ def _load() -> ctypes.CDLL:
         "quant_act_given_scale": ([P, I, I64, I64, P, P, P, P], I),
         "sq_dequant": ([P, P, P, I64, I64, P, I, P], I),
         "w4a8_gemm_dequant": ([P, P, P, P, I64, I64, I64, P, I, P, P], I),
+        "sq_debug_status": ([P, P, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -114,6 +117,15 @@ def _stream(stream) -> ctypes.c_void_p:
 
 def abi_version() -> int:
     return lib.sq_abi_version()
+
+
+def debug_status(stream=None) -> tuple[int, int, bool]:
+    """(non-finite inputs, failed index checks, debug build?) counted since the
+    last call, read and cleared (sq_debug_status; zeros in a release build)."""
+    nf, ix, en = ctypes.c_uint64(0), ctypes.c_uint64(0), ctypes.c_int(0)
+    _check("sq_debug_status", lib.sq_debug_status(_stream(stream), ctypes.byref(nf), ctypes.byref(ix),
+                                                  ctypes.byref(en)))
+    return int(nf.value), int(ix.value), bool(en.value)
 
 
 def device_fault(stream=None) -> int:

@@ -1,6 +1,9 @@
 """Build libw8a8.so (the C-ABI CUDA library) in-tree with nvcc for sm_100a.
 
-    python w8a8_linear_layers_b200/build.py [--verbose]
+    python w8a8_linear_layers_b200/build.py [--verbose] [--debug]
+
+(--debug builds libw8a8_debug.so: the same kernels compiled with -DW8A8_DEBUG,
+which count non-finite inputs and failed index checks for sq_debug_status.)
 
 (Run it by path, or load it with importlib by path: importing the package
 itself loads libw8a8.so, which is what this script produces.)
@@ -19,6 +22,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libw8a8.so")
+LIB_DEBUG = os.path.join(PKG, "libw8a8_debug.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 NVCC_FLAGS = [
@@ -32,10 +36,10 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + [os.path.join(ROOT, "include", "w8a8.h")]
     return any(os.path.getmtime(d) > t for d in deps)
 
@@ -49,17 +53,19 @@ def load_build_module():
     return mod
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every kernel source into libw8a8.so; returns its path."""
-    if not force and not _stale():
-        return LIB
-    tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [NVCC, *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), *sources(), "-o", tmp,
-           "-lcudart"]
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Compile every kernel source into libw8a8.so (debug: libw8a8_debug.so
+    with -DW8A8_DEBUG); returns its path."""
+    lib = LIB_DEBUG if debug else LIB
+    if not force and not _stale(lib):
+        return lib
+    tmp = lib + ".tmp%d" % os.getpid()
+    cmd = [NVCC, *NVCC_FLAGS, *(["-DW8A8_DEBUG"] if debug else []), *(["-Xptxas", "-v"] if verbose else []),
+           *sources(), "-o", tmp, "-lcudart"]
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force=True, verbose="--verbose" in sys.argv))
+    print(build(force=True, verbose="--verbose" in sys.argv, debug="--debug" in sys.argv))

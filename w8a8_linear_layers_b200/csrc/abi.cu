@@ -65,3 +65,32 @@ extern "C" const char *sq_status_string(sq_status s) {
 extern "C" const char *sq_last_error_detail(void) { return w8a8::g_detail; }
 
 extern "C" int sq_abi_version(void) { return 1; }
+
+extern "C" sq_status sq_debug_status(void *stream, uint64_t *nonfinite_out, uint64_t *index_out, int *enabled_out) {
+    if (!nonfinite_out || !index_out || !enabled_out) return w8a8::fail(SQ_ERR_NULL, "sq_debug_status: NULL pointer");
+#ifdef W8A8_DEBUG
+    int sms;
+    sq_status st = w8a8::check_device(&sms);
+    if (st != SQ_OK) return st;
+    cudaStream_t cs = (cudaStream_t)stream;
+    unsigned long long total[2] = {0ull, 0ull};
+    cudaError_t (*readers[])(cudaStream_t, unsigned long long (&)[2]) = {
+        w8a8::dbg_take_smooth, w8a8::dbg_take_quant_act, w8a8::dbg_take_ssz, w8a8::dbg_take_ssz_asym};
+    for (auto rd : readers) {
+        unsigned long long c[2];
+        const cudaError_t e = rd(cs, c);
+        if (e != cudaSuccess) return w8a8::fail(SQ_ERR_CUDA, "sq_debug_status: %s", cudaGetErrorString(e));
+        total[0] += c[0];
+        total[1] += c[1];
+    }
+    *nonfinite_out = total[0];
+    *index_out = total[1];
+    *enabled_out = 1;
+#else
+    (void)stream;
+    *nonfinite_out = 0;
+    *index_out = 0;
+    *enabled_out = 0;
+#endif
+    return SQ_OK;
+}

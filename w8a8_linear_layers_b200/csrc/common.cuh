@@ -203,4 +203,82 @@ __device__ __forceinline__ uint2 fast_codes8(const float4 a, const float4 b, flo
     return make_uint2(p0, p1);
 }
 
+// ------------------------------------------------------------ debug counters
+// Debug builds (-DW8A8_DEBUG, libw8a8_debug.so): the kernels count the
+// non-finite values they read from their inputs, and the index checks that
+// fail (the access is then skipped), into two device counters per source
+// file; sq_debug_status adds them up and clears them.  Nothing traps.  In
+// release builds the checks compile to nothing.
+#ifdef W8A8_DEBUG
+static __device__ unsigned long long g_dbg_counts[2];  // [non-finite inputs, failed index checks]
+
+__device__ __forceinline__ void dbg_count_nonfinite(int n) {
+    if (n) atomicAdd(&g_dbg_counts[0], (unsigned long long)n);
+}
+__device__ __forceinline__ bool dbg_index_ok(bool ok) {
+    if (!ok) atomicAdd(&g_dbg_counts[1], 1ull);
+    return ok;
+}
+// reads and clears this source file's counters (host)
+static inline cudaError_t dbg_take(cudaStream_t st, unsigned long long (&out)[2]) {
+    unsigned long long zero[2] = {0ull, 0ull};
+    cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_dbg_counts, sizeof out, 0, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaMemcpyToSymbolAsync(g_dbg_counts, zero, sizeof zero, 0, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    return e;
+}
+// per-file readers (each file's counters are its own)
+cudaError_t dbg_take_smooth(cudaStream_t st, unsigned long long (&out)[2]);
+cudaError_t dbg_take_quant_act(cudaStream_t st, unsigned long long (&out)[2]);
+cudaError_t dbg_take_ssz(cudaStream_t st, unsigned long long (&out)[2]);
+cudaError_t dbg_take_ssz_asym(cudaStream_t st, unsigned long long (&out)[2]);
+// the same check again, not counted (the paired use of a skipped access)
+__device__ __forceinline__ bool dbg_index_again(bool ok) { return ok; }
+#define W8A8_DEBUG_READER(name) \
+    cudaError_t dbg_take_##name(cudaStream_t st, unsigned long long (&out)[2]) { return dbg_take(st, out); }
+#else
+__device__ __forceinline__ void dbg_count_nonfinite(int) {}
+__device__ __forceinline__ bool dbg_index_ok(bool) { return true; }
+__device__ __forceinline__ bool dbg_index_again(bool) { return true; }
+#define W8A8_DEBUG_READER(name)
+#endif
+
+// Non-finite values among 8 (4) fp32 values (debug builds only).
+__device__ __forceinline__ void dbg_check8(const float (&v)[8]) {
+#ifdef W8A8_DEBUG
+    int n = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) n += !isfinite(v[i]);
+    dbg_count_nonfinite(n);
+#else
+    (void)v;
+#endif
+}
+__device__ __forceinline__ void dbg_check4(float4 a) {
+#ifdef W8A8_DEBUG
+    dbg_count_nonfinite(!isfinite(a.x) + !isfinite(a.y) + !isfinite(a.z) + !isfinite(a.w));
+#else
+    (void)a;
+#endif
+}
+// Non-finite values among 8 raw bf16 values (exponent bits all ones).
+__device__ __forceinline__ void dbg_check_bf16x8(uint4 u) {
+#ifdef W8A8_DEBUG
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    int n = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) n += ((w[i] & 0x7f80u) == 0x7f80u) + ((w[i] & 0x7f800000u) == 0x7f800000u);
+    dbg_count_nonfinite(n);
+#else
+    (void)u;
+#endif
+}
+__device__ __forceinline__ void dbg_check1(float a) {
+#ifdef W8A8_DEBUG
+    dbg_count_nonfinite(!isfinite(a));
+#else
+    (void)a;
+#endif
+}
+
 }  // namespace w8a8

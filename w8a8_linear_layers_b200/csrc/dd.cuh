@@ -39,6 +39,14 @@ __device__ __forceinline__ dd warp_sum_dd(dd a) {
     return a;
 }
 
+// Plain fp64 butterfly sum: every lane ends with the same value (a + b ==
+// b + a exactly).
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
 __device__ __forceinline__ int warp_sum_i(int v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

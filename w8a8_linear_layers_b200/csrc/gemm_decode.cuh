@@ -39,8 +39,16 @@ namespace gemm {
 #ifndef W8A8_DEC_CONV_WARPS
 #define W8A8_DEC_CONV_WARPS 8
 #endif
+#ifndef W8A8_DEC_CONV_GROUPS
+#define W8A8_DEC_CONV_GROUPS 2
+#endif
 constexpr int kDecRows = 128;  // weight rows per CTA (= MMA M = TMEM lanes)
 constexpr int kDecConvWarps = W8A8_DEC_CONV_WARPS;  // int4 unpacking warps (the first 4 also run the epilogue)
+// the converter warps form groups that take alternate k-blocks, so that
+// several stages are unpacked at once (the unpacking of one stage is
+// latency-bound: shared load, ALU, shared store, proxy fence, arrive)
+constexpr int kDecConvGroups = W8A8_DEC_CONV_GROUPS;
+constexpr int kDecConvGroupThreads = kDecConvWarps * 32 / kDecConvGroups;
 // producer, MMA, then 4 epilogue warps (int4: the converter warps)
 __host__ __device__ constexpr int dec_threads(bool int4) { return 64 + 32 * (int4 ? kDecConvWarps : 4); }
 constexpr int kDecMaxSplit = 8;   // portable cluster size
@@ -61,6 +69,14 @@ struct CfgDec {
     static constexpr int TMEM_COLS = NT < 32 ? 32 : NT;
     static constexpr int RED_BYTES = NT * kDecRows * 4;  // int32 partial, over the stages
     static_assert(STAGES >= 3, "decode pipeline too shallow");
+    // a converter group's previous k-block (kb - G) made it wait for the MMA
+    // to consume kb - G - OP_STAGES, so every barrier it waits on next is at
+    // most one phase behind (an mbarrier parity wait cannot tell two phases
+    // apart): G <= OP_STAGES
+    static_assert(!INT4 || (kDecConvGroups >= 1 && kDecConvGroups <= OP_STAGES && STAGES >= OP_STAGES),
+                  "converter groups must not run more than one phase ahead");
+    static_assert(kDecConvWarps * 32 % kDecConvGroups == 0 && 512 % kDecConvGroupThreads == 0,
+                  "a packed tile splits evenly over a group");
     static_assert(IN_BYTES % 1024 == 0 && RAW_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
     static_assert(RED_BYTES <= STAGES * IN_BYTES, "partial must fit over the stages");
 };
@@ -152,7 +168,7 @@ w8a8_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
             mbar_init(smem_u32(&in_empty[s]), 1);
         }
         for (int p = 0; p < C::OP_STAGES; ++p) {
-            mbar_init(smem_u32(&op_full[p]), kDecConvWarps * 32);
+            mbar_init(smem_u32(&op_full[p]), kDecConvGroupThreads);  // one group unpacks a stage
             mbar_init(smem_u32(&op_empty[p]), 1);
         }
         mbar_init(smem_u32(&tfull_bar), 1);
@@ -256,12 +272,17 @@ w8a8_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
         if (INT4) {
             // ------------------------------------------ converters
             // A packed tile is 128 rows x 64 bytes: 512 16-byte pieces over
-            // the converter threads; piece i = (row i/4, bytes 16 (i%4) ..),
-            // unpacked into 16-byte chunks 2 (i%4) and 2 (i%4) + 1 of the row
-            // (128B swizzle).
-            int stage = 0, os = 0;
-            uint32_t phase = 0, oph = 0;
-            for (int kb = kb0; kb < kb1; ++kb) {
+            // the threads of one converter group; piece i = (row i/4, bytes
+            // 16 (i%4) ..), unpacked into 16-byte chunks 2 (i%4) and
+            // 2 (i%4) + 1 of the row (128B swizzle).  Group g takes the
+            // k-blocks kb0 + g, kb0 + g + G, ...; the ring positions and
+            // phases follow from the k-block's index.
+            constexpr int kOps = INT4 ? C::OP_STAGES : 1;  // (this branch only runs for int4)
+            const int grp = ct / kDecConvGroupThreads, gt = ct % kDecConvGroupThreads;
+            for (int kb = kb0 + grp; kb < kb1; kb += kDecConvGroups) {
+                const int u = kb - kb0;
+                const int stage = u % C::STAGES, os = u % kOps;
+                const uint32_t phase = (uint32_t)(u / C::STAGES) & 1u, oph = (uint32_t)(u / kOps) & 1u;
                 if (!wait_bounded(smem_u32(&op_empty[os]), oph ^ 1u, &abort_flag, kFaultConvert) ||
                     !wait_bounded(smem_u32(&in_full[stage]), phase, &abort_flag, kFaultConvert)) {
                     ok = false;
@@ -270,8 +291,8 @@ w8a8_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
                 const uint8_t *raw = gbase + C::IN_OFFSET + stage * C::IN_BYTES;
                 uint8_t *wdst = gbase + os * C::W_BYTES;
 #pragma unroll
-                for (int it = 0; it < 512 / (32 * kDecConvWarps); ++it) {
-                    const int i = it * (32 * kDecConvWarps) + ct;
+                for (int it = 0; it < 512 / kDecConvGroupThreads; ++it) {
+                    const int i = it * kDecConvGroupThreads + gt;
                     const int r = i >> 2, sub = i & 3;
                     const uint4 p = *reinterpret_cast<const uint4 *>(raw + r * (BK / 2) + sub * 16);
                     uint32_t o[8];
@@ -286,14 +307,6 @@ w8a8_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
                 }
                 fence_proxy_async_smem();  // the MMA reads these bytes through the async proxy
                 mbar_arrive(smem_u32(&op_full[os]));
-                if (++stage == C::STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-                if (++os == C::OP_STAGES) {
-                    os = 0;
-                    oph ^= 1u;
-                }
             }
         }
         // ---------------------------------------------- epilogue (warps 2..5)

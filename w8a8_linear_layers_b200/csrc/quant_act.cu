@@ -84,7 +84,10 @@ __device__ __forceinline__ uint2 fast_codes_tied(const float (&v)[8], float s, f
 // ROWS token rows per CTA iteration, all loaded before the first reduction.
 // Measured on B200: one row per small CTA (32 elements per thread) with many
 // CTAs per SM beats several rows per larger CTA and beats staging rows in
-// shared memory with bulk copies.
+// shared memory with bulk copies.  The CTAs are persistent (as many as fit
+// on the SMs at once) and software-pipelined: the loads of a CTA's next row
+// are issued before the current row's reduction, so that two rows per CTA
+// are in flight while one is quantized.
 //
 // STATIC: one scale for the whole tensor, S = range[0] / 127 (a range
 // calibrated beforehand, see sq_static_range_update); no per-row reduction,
@@ -131,19 +134,26 @@ quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__r
         }
     };
 
-    int parity = 0;
-    for (int64_t row0 = (int64_t)blockIdx.x * ROWS; row0 < M; row0 += (int64_t)gridDim.x * ROWS, parity ^= 1) {
-        Raw8<T> raw[ROWS][C];
+    auto load_rows = [&](Raw8<T> (&dst)[ROWS][C], int64_t r0) {
 #pragma unroll
         for (int rr = 0; rr < ROWS; ++rr) {
 #pragma unroll
             for (int c = 0; c < C; ++c) {
-                if (live[c] && row0 + rr < M)
-                    raw[rr][c].load(x + (row0 + rr) * K + ((int64_t)c * T_ + threadIdx.x) * 8);
+                if (live[c] && r0 + rr < M &&
+                    dbg_index_ok(((int64_t)c * T_ + threadIdx.x) * 8 + 8 <= K))
+                    dst[rr][c].load(x + (r0 + rr) * K + ((int64_t)c * T_ + threadIdx.x) * 8);
                 else
-                    raw[rr][c].zero();
+                    dst[rr][c].zero();
             }
         }
+    };
+    const int64_t rstride = (int64_t)gridDim.x * ROWS;
+    int parity = 0;
+    Raw8<T> raw[ROWS][C];
+    if ((int64_t)blockIdx.x * ROWS < M) load_rows(raw, (int64_t)blockIdx.x * ROWS);
+    for (int64_t row0 = (int64_t)blockIdx.x * ROWS; row0 < M; row0 += rstride, parity ^= 1) {
+        Raw8<T> nxt[ROWS][C];  // the next rows of this CTA, loading while these are quantized
+        load_rows(nxt, row0 + rstride);
         float amax[ROWS];  // dynamic: the row's abs-max; static: this thread's
 #pragma unroll
         for (int rr = 0; rr < ROWS; ++rr) {
@@ -151,6 +161,10 @@ quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__r
 #pragma unroll
             for (int c = 0; c < C; ++c) {
                 float v[8];
+#ifdef W8A8_DEBUG
+                raw[rr][c].widen(v);
+                dbg_check8(v);  // the input itself (zeros past the row)
+#endif
                 scaled(raw[rr][c], c, v);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) amax[rr] = fmaxf(amax[rr], fabsf(v[i]));
@@ -220,6 +234,10 @@ quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__r
                 }
             }
         }
+#pragma unroll
+        for (int rr = 0; rr < ROWS; ++rr)
+#pragma unroll
+            for (int c = 0; c < C; ++c) raw[rr][c] = nxt[rr][c];
     }
 }
 
@@ -227,23 +245,28 @@ template <typename T, int E, int ROWS, bool STATIC>
 static void launch_quant_act(const void *x, int64_t M, int64_t K, const float *inv_s, const float *range,
                              int8_t *q, float *scale, int32_t *rowsum, int sms, cudaStream_t st) {
     int threads = (int)ceil_div(ceil_div(K, E), 32) * 32;
-    // enough CTAs to fill the machine; each strides over groups of ROWS rows
-    int per_sm = std::max(1, std::min(32, 2048 / threads));
+    // persistent: as many CTAs as fit on the SMs at once, each striding over
+    // groups of ROWS rows
+    int per_sm = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_act_kernel<T, E, ROWS, STATIC>, threads, 0);
+    per_sm = std::max(1, std::min(per_sm, 2048 / threads));
     int64_t grid = std::min<int64_t>(ceil_div(M, ROWS), (int64_t)sms * per_sm);
     quant_act_kernel<T, E, ROWS, STATIC>
         <<<(unsigned)grid, threads, 0, st>>>((const T *)x, M, K, inv_s, range, q, scale, rowsum);
 }
 
 // ------------------------------------------------ LayerNorm fused with step 4
-// One CTA per row, the raw row in registers for the whole computation.  The
-// row statistics are fp64 pairwise sums: the tree that halves the row padded
-// with zeros to a power of two (S(lo, len) = S(lo, len/2) + S(lo + len/2,
-// len/2)), so they do not depend on how the work is split.  Thread t owns the
-// E contiguous columns [t E, t E + E): it sums its 8-column chunks as
-// subtrees of 8 and combines them pairwise; the xor butterfly of a warp
-// combines neighbouring threads' subtrees (a + b == b + a exactly, so every
-// lane ends with the same sum), and one more butterfly over the warps' sums
-// finishes the tree (T and E are powers of two).  Then mean = S / K,
+// Persistent CTAs of T threads, one row at a time; thread t owns the E (8 or
+// 16) contiguous columns [t E, t E + E), so its gamma, beta and inv_s stay in
+// registers for every row, and the next row's loads are issued before the
+// current row's reductions.  The row statistics are fp64 pairwise sums: the
+// tree that halves the row padded with zeros to a power of two
+// (S(lo, len) = S(lo, len/2) + S(lo + len/2, len/2)), so they do not depend on
+// how the work is split.  A thread sums its 8-column chunks as subtrees of 8
+// and combines them pairwise; the xor butterfly of a warp combines
+// neighbouring threads' subtrees (a + b == b + a exactly, so every lane ends
+// with the same sum), and one more butterfly over the warps' sums finishes
+// the tree (T and E are powers of two).  Then mean = S / K,
 // var = S(d^2) / K with d = h - mean, rstd = 1 / sqrt(var + eps) (IEEE fp64);
 // m and r rounded to fp32, then per element y = ((h - m) r) gamma + beta and
 // x' = y inv_s in fp32 with no fused multiply-add (the build contracts
@@ -255,65 +278,78 @@ __device__ __forceinline__ double tree8(const double (&a)[8]) {
     return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
 }
 
-// Pairwise sum of C chunk subtrees (C a power of two).
-template <int C>
-__device__ __forceinline__ double tree_chunks(double (&c)[C]) {
-#pragma unroll
-    for (int len = C; len > 1; len >>= 1) {
-#pragma unroll
-        for (int i = 0; i < len / 2; ++i) c[i] = c[2 * i] + c[2 * i + 1];
-    }
-    return c[0];
-}
-
 // The thread subtrees of the whole CTA combined in tree order: warp
 // butterfly, then a butterfly over the nwarps (a power of two) warp sums.
-__device__ __forceinline__ double block_tree_sum(double v, double (&red)[32], int lane, int warp, int nwarps) {
+// red: this reduction's slot array; a slot is reused two rows later, after
+// other barriers, so one barrier per reduction suffices.
+__device__ __forceinline__ double block_tree_sum(double v, double *red, int lane, int warp, int nwarps) {
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     if (lane == 0) red[warp] = v;
     __syncthreads();
     double t = lane < nwarps ? red[lane] : 0.0;
     for (int o = 1; o < nwarps; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-    t = __shfl_sync(0xffffffffu, t, 0);
-    __syncthreads();  // red is reused by the next reduction
-    return t;
+    return __shfl_sync(0xffffffffu, t, 0);
 }
 
 template <typename T, int E>
-__global__ void __launch_bounds__(512)
+__global__ void __launch_bounds__(1024)
 ln_quant_kernel(const T *__restrict__ h, int64_t M, int64_t K, const float *__restrict__ gamma,
                 const float *__restrict__ beta, float eps, const float *__restrict__ inv_s, int8_t *__restrict__ q,
                 float *__restrict__ scale) {
     constexpr int C = E / 8;
-    __shared__ double redd[32];
-    __shared__ float redf[32];
+    __shared__ double redd[2][2][32];  // [row parity][mean, variance][warp]
+    __shared__ float redf[2][32];      // [row parity][warp]: abs-max
     const int T_ = blockDim.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = T_ >> 5;
     const int64_t base = (int64_t)threadIdx.x * E;  // this thread's first column
     bool live[C];  // K is a multiple of 8: a chunk is wholly inside the row or wholly past it
+    float g[C][8], bt[C][8], f[C][8];
 #pragma unroll
-    for (int c = 0; c < C; ++c) live[c] = base + 8 * c < K;
+    for (int c = 0; c < C; ++c) {
+        live[c] = base + 8 * c < K;
+        const int64_t j = base + 8 * c;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            g[c][i] = 1.0f;
+            bt[c][i] = 0.0f;
+            f[c][i] = 1.0f;
+        }
+        if (live[c]) {
+            if (gamma) load8_f32(gamma + j, g[c]);
+            if (beta) load8_f32(beta + j, bt[c]);
+            if (inv_s) load8_f32(inv_s + j, f[c]);
+        }
+    }
     const double kd = (double)K;
-
-    for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
-        Raw8<T> raw[C];
+    auto load_row = [&](Raw8<T> (&dst)[C], int64_t r) {
 #pragma unroll
         for (int c = 0; c < C; ++c) {
-            if (live[c]) raw[c].load(h + row * K + base + 8 * c);
-            else raw[c].zero();
+            if (live[c] && r < M && dbg_index_ok(base + 8 * c + 8 <= K)) dst[c].load(h + r * K + base + 8 * c);
+            else dst[c].zero();
         }
+    };
+
+    Raw8<T> raw[C];
+    load_row(raw, blockIdx.x);
+    int par = 0;
+    for (int64_t row = blockIdx.x; row < M; row += gridDim.x, par ^= 1) {
+        Raw8<T> nxt[C];
+        load_row(nxt, row + gridDim.x);
         double part[C];
 #pragma unroll
         for (int c = 0; c < C; ++c) {
             float v[8];
             raw[c].widen(v);  // zeros past the row
+            dbg_check8(v);
             double a[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) a[i] = (double)v[i];
             part[c] = tree8(a);
         }
-        const double mu = block_tree_sum(tree_chunks<C>(part), redd, lane, warp, nwarps) / kd;
+        double tsum = part[0];
+        if (C == 2) tsum = part[0] + part[C - 1];
+        const double mu = block_tree_sum(tsum, redd[par][0], lane, warp, nwarps) / kd;
 #pragma unroll
         for (int c = 0; c < C; ++c) {
             float v[8];
@@ -326,40 +362,31 @@ ln_quant_kernel(const T *__restrict__ h, int64_t M, int64_t K, const float *__re
             }
             part[c] = tree8(a);
         }
-        const double var = block_tree_sum(tree_chunks<C>(part), redd, lane, warp, nwarps) / kd;
+        tsum = part[0];
+        if (C == 2) tsum = part[0] + part[C - 1];
+        const double var = block_tree_sum(tsum, redd[par][1], lane, warp, nwarps) / kd;
         const double rstd = 1.0 / sqrt(var + (double)eps);
         const float m32 = (float)mu, r32 = (float)rstd;
-        // x' of chunk c: ((h - m) r) gamma + beta, times inv_s, each op in fp32
-        auto xs = [&](int c, float (&x)[8]) {
-            const int64_t j = base + 8 * c;
-            float v[8], g[8], b[8], f[8];
-            raw[c].widen(v);
-            if (gamma) load8_f32(gamma + j, g);
-            if (beta) load8_f32(beta + j, b);
-            if (inv_s) load8_f32(inv_s + j, f);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float n = (v[i] - m32) * r32;
-                const float gn = gamma ? n * g[i] : n;
-                const float y = beta ? gn + b[i] : gn;
-                x[i] = inv_s ? y * f[i] : y;
-            }
-        };
+        // x' = ((h - m) r) gamma + beta, times inv_s, each op in fp32
+        float x[C][8];
         float amax = 0.0f;
 #pragma unroll
         for (int c = 0; c < C; ++c) {
-            if (!live[c]) continue;
-            float x[8];
-            xs(c, x);
+            float v[8];
+            raw[c].widen(v);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
+            for (int i = 0; i < 8; ++i) {
+                const float n = __fmul_rn(__fsub_rn(v[i], m32), r32);
+                const float y = __fadd_rn(__fmul_rn(n, g[c][i]), bt[c][i]);
+                x[c][i] = __fmul_rn(y, f[c][i]);
+                if (live[c]) amax = fmaxf(amax, fabsf(x[c][i]));
+            }
         }
         amax = warp_max(amax);
-        if (lane == 0) redf[warp] = amax;
+        if (lane == 0) redf[par][warp] = amax;
         __syncthreads();
-        float am = redf[0];
-        for (int w = 1; w < nwarps; ++w) am = fmaxf(am, redf[w]);
-        __syncthreads();  // redf is rewritten for the next row
+        float am = redf[par][0];
+        for (int w = 1; w < nwarps; ++w) am = fmaxf(am, redf[par][w]);
         const float s = __fdiv_rn(am, 127.0f);
         if (threadIdx.x == 0) scale[row] = s;
         const float r = __fdiv_rn(1.0f, s);
@@ -369,33 +396,35 @@ ln_quant_kernel(const T *__restrict__ h, int64_t M, int64_t K, const float *__re
 #pragma unroll
         for (int c = 0; c < C; ++c) {
             if (!live[c]) continue;
-            float x[8];
-            xs(c, x);
             uint2 code = make_uint2(0u, 0u);
             if (s == 0.0f) {
             } else if (exact_only) {
                 int e[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) e[i] = (int)sym_code(x[i], s, r, 127.0f, true);
+                for (int i = 0; i < 8; ++i) e[i] = (int)sym_code(x[c][i], s, r, 127.0f, true);
                 code = pack8_codes(e);
             } else {
-                code = fast_codes_tied(x, s, r, narrow, tie_bound);
+                code = fast_codes_tied(x[c], s, r, narrow, tie_bound);
             }
             *reinterpret_cast<uint2 *>(q + row * K + base + 8 * c) = code;
         }
+#pragma unroll
+        for (int c = 0; c < C; ++c) raw[c] = nxt[c];
     }
 }
 
 // T threads of E contiguous columns each, T * E the power of two at or above
-// K (at least one warp of E = 8): E = 8, 16, 32 up to K = 1024, then 32
-// columns a thread and up to 512 threads (K <= 16384).
+// K (at least one warp): E = 8 up to K = 8192 (T <= 1024), 16 above
+// (K <= 16384).  Persistent: as many CTAs as fit on the SMs at once.
 template <typename T, int E>
 static void launch_ln_quant(const void *h, int64_t M, int64_t K, const float *gamma, const float *beta, float eps,
                             const float *inv_s, int8_t *q, float *scale, int sms, cudaStream_t st) {
     int64_t P = 32 * E;
     while (P < K) P *= 2;
     const int threads = (int)(P / E);
-    const int per_sm = std::max(1, std::min(32, 2048 / threads));
+    int per_sm = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ln_quant_kernel<T, E>, threads, 0);
+    per_sm = std::max(1, std::min(per_sm, 2048 / threads));
     const int64_t grid = std::min<int64_t>(M, (int64_t)sms * per_sm);
     ln_quant_kernel<T, E><<<(unsigned)grid, threads, 0, st>>>((const T *)h, M, K, gamma, beta, eps, inv_s, q, scale);
 }
@@ -445,6 +474,8 @@ static_range_kernel(const float *__restrict__ ax, const float *__restrict__ inv_
         range[0] = first ? a : __fadd_rn(__fmul_rn(rate, range[0]), __fmul_rn(__fsub_rn(1.0f, rate), a));
     }
 }
+
+W8A8_DEBUG_READER(quant_act)
 
 }  // namespace w8a8
 
@@ -530,18 +561,12 @@ extern "C" sq_status sq_layernorm_quant(const void *h, sq_dtype ht, int64_t M, i
     if (st != SQ_OK) return st;
     cudaStream_t cs = (cudaStream_t)stream;
     const bool bf = ht == SQ_BF16;
-    // E contiguous columns per thread: one warp per row up to K = 32 E, then
-    // E = 32 (measured faster than 64, which spills); K <= 16384 keeps a row
-    // within 512 threads
-    if (K <= 256) {
+    if (K <= 8192) {
         if (bf) launch_ln_quant<__nv_bfloat16, 8>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);
         else launch_ln_quant<float, 8>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);
-    } else if (K <= 512) {
+    } else {
         if (bf) launch_ln_quant<__nv_bfloat16, 16>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);
         else launch_ln_quant<float, 16>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);
-    } else {
-        if (bf) launch_ln_quant<__nv_bfloat16, 32>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);
-        else launch_ln_quant<float, 32>(h, M, K, gamma, beta, eps, inv_s, q_out, scale_out, sms, cs);
     }
     return launch_status("ln_quant_kernel");
 }

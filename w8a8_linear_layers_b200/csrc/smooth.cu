@@ -41,6 +41,7 @@ __device__ __forceinline__ typename ColRaw<T>::type load_raw(const T *p) {
 }
 
 __device__ __forceinline__ void fold_abs(float (&m)[8], uint4 u) {
+    dbg_check_bf16x8(u);
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -50,6 +51,7 @@ __device__ __forceinline__ void fold_abs(float (&m)[8], uint4 u) {
 }
 
 __device__ __forceinline__ void fold_abs(float (&m)[4], float4 a) {
+    dbg_check4(a);
     m[0] = fmaxf(m[0], fabsf(a.x));
     m[1] = fmaxf(m[1], fabsf(a.y));
     m[2] = fmaxf(m[2], fabsf(a.z));
@@ -85,11 +87,12 @@ col_absmax_kernel(const T *__restrict__ a, int64_t R, int64_t K, int64_t rows_pe
 #pragma unroll
             for (int u = 0; u < kColDepth; ++u) {
                 const int64_t rr = r + u * kColWarps;
-                if (rr < r1) v[u] = load_raw<T>(p + rr * K);
+                if (rr < r1 && dbg_index_ok(rr < R && col + VEC <= K)) v[u] = load_raw<T>(p + rr * K);
             }
 #pragma unroll
             for (int u = 0; u < kColDepth; ++u)
-                if (r + u * kColWarps < r1) fold_abs(m, v[u]);
+                if (r + u * kColWarps < r1 && dbg_index_again(r + u * kColWarps < R && col + VEC <= K))
+                    fold_abs(m, v[u]);
         }
     }
 #pragma unroll
@@ -166,6 +169,8 @@ __global__ void fold_kernel(const T *__restrict__ w, int64_t N, int64_t K,
         o[1] = make_float4(v[4] * f[4], v[5] * f[5], v[6] * f[6], v[7] * f[7]);
     }
 }
+
+W8A8_DEBUG_READER(smooth)
 
 }  // namespace w8a8
 

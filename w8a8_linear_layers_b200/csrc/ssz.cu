@@ -20,21 +20,29 @@
 // stops for good once it meets them; the minimum scale floors the MinMax
 // scale and every candidate; int4 codes are [-7, 7].
 //
-// Design.  One CTA of R warps per output channel; the folded fp32 row stays
-// resident in shared memory for the whole search (W is read from HBM once,
-// the codes written once), next to one buffer of kept codes: a candidate
-// that is not kept ends the search, so a round writes its codes over the
-// kept ones and the chunks it touched are restored in that one case.
+// Design.  One CTA of R warps per output channel; the row stays resident in
+// shared memory for the whole search (W is read from HBM once, the codes
+// written once), next to one buffer of kept codes: a candidate that is not
+// kept ends the search, so a round writes its codes over the kept ones and
+// the chunks it touched are restored in that one case.  A bf16 row is kept
+// as loaded (2 bytes an element) and folded again, fl(w s_j) with the same
+// single fp32 rounding, wherever it is read (s through L1); an fp32 row is
+// kept folded.  At K = 4096 a channel then takes 12 KB instead of 20, and up
+// to 16 channels (32 warps) fit on an SM.
 //
 // The error is evaluated exactly instead of by a per-element fp64 sum:
 //     K e(c) = W2 - 2 c NUM + c^2 DEN,  W2 = sum w^2, NUM = sum w q, DEN = sum q^2,
 // with W2 and NUM held in double-double (error-free transformations: Knuth's
 // TwoSum and the FMA TwoProduct), DEN exact, and the cancelling sum taken
-// with TwoSum, so e(c) is the exact error rounded once -- never further from
-// the true value than a direct fp64 sum.  NUM and DEN change only where a
-// code changes, so a round is one pass that computes the codes at the
-// candidate scale on the FP32 pipe (magic-constant rounding), compares them
-// 8 at a time with the kept codes and updates NUM/DEN for the few that moved.
+// with TwoSum.  NUM and DEN change only where a code changes, so a round is
+// one pass that computes the codes at the candidate scale on the FP32 pipe
+// (magic-constant rounding), compares them 8 at a time with the kept codes
+// and updates NUM/DEN for the few that moved: DEN exactly, NUM by the exact
+// products w (q' - q) summed in fp64 (a handful of terms per thread and
+// round, each sum off by at most 2^-52 of the terms' magnitudes) and added
+// to the double-double NUM with TwoSum.  The evaluated error is then within
+// a few 2^-52 of |w| c per moved code of the exact one, far below the 1e-10
+// thresholds the decisions test.
 // Codes are exact: an element whose scaled value lies within |y| 2^-21 of a
 // half-integer takes the IEEE quotient (see sym_code_i for the bound).
 //
@@ -83,19 +91,70 @@ __device__ __forceinline__ int code_byte(uint2 p, int b) {
 }
 
 struct PassOut {
-    dd num;          // init: NUM; update: change of NUM
+    dd num;          // init: NUM
     dd w2;           // init only
+    double dnum;     // update: change of NUM (exact products, fp64 sum)
     int den;         // init: DEN; update: change of DEN
     bool moved;      // update: some code of this thread changed
     uint32_t touched;  // update: chunks whose codes were rewritten (moved or near a tie)
 };
 
+// The channel's row in shared memory, read as folded fp32 values.  fp32
+// input: the folded row itself.  bf16 input: the raw bf16 row, widened
+// (exact) and, with FOLD, multiplied by s_j (one IEEE fp32 multiply, the
+// value the fp32 path stores).
+template <typename T, bool FOLD> struct Row;
+
+template <bool FOLD> struct Row<float, FOLD> {
+    const float *w;
+    __device__ __forceinline__ void load8(int j, float4 &a, float4 &b) const {
+        a = *reinterpret_cast<const float4 *>(w + j);
+        b = *reinterpret_cast<const float4 *>(w + j + 4);
+    }
+    __device__ __forceinline__ float load1(int j) const { return w[j]; }
+};
+
+template <bool FOLD> struct Row<__nv_bfloat16, FOLD> {
+    const uint16_t *w;     // raw bf16 bits
+    const float *s;        // smoothing factor (global, read through L1); unused without FOLD
+    __device__ __forceinline__ void load8(int j, float4 &a, float4 &b) const {
+        const uint4 u = *reinterpret_cast<const uint4 *>(w + j);
+        a = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                        __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+        b = make_float4(__uint_as_float(u.z << 16), __uint_as_float(u.z & 0xffff0000u),
+                        __uint_as_float(u.w << 16), __uint_as_float(u.w & 0xffff0000u));
+        if (FOLD) {
+            const float4 f0 = __ldg(reinterpret_cast<const float4 *>(s + j));
+            const float4 f1 = __ldg(reinterpret_cast<const float4 *>(s + j) + 1);
+            a = make_float4(__fmul_rn(a.x, f0.x), __fmul_rn(a.y, f0.y), __fmul_rn(a.z, f0.z), __fmul_rn(a.w, f0.w));
+            b = make_float4(__fmul_rn(b.x, f1.x), __fmul_rn(b.y, f1.y), __fmul_rn(b.z, f1.z), __fmul_rn(b.w, f1.w));
+        }
+    }
+    __device__ __forceinline__ float load1(int j) const {
+        const float v = __uint_as_float((uint32_t)w[j] << 16);
+        return FOLD ? __fmul_rn(v, __ldg(s + j)) : v;
+    }
+    // the folded values of 8 raw elements u at column j (staging)
+    __device__ __forceinline__ void load8_global(uint4 u, int j, float4 &a, float4 &b) const {
+        a = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                        __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+        b = make_float4(__uint_as_float(u.z << 16), __uint_as_float(u.z & 0xffff0000u),
+                        __uint_as_float(u.w << 16), __uint_as_float(u.w & 0xffff0000u));
+        if (FOLD) {
+            const float4 f0 = __ldg(reinterpret_cast<const float4 *>(s + j));
+            const float4 f1 = __ldg(reinterpret_cast<const float4 *>(s + j) + 1);
+            a = make_float4(__fmul_rn(a.x, f0.x), __fmul_rn(a.y, f0.y), __fmul_rn(a.z, f0.z), __fmul_rn(a.w, f0.w));
+            b = make_float4(__fmul_rn(b.x, f1.x), __fmul_rn(b.y, f1.y), __fmul_rn(b.z, f1.z), __fmul_rn(b.w, f1.w));
+        }
+    }
+};
+
 // Fast codes of the chunk at j for scale 1/r (see fast_codes8); dmax as there.
-template <bool NARROW>
-__device__ __forceinline__ uint2 chunk_codes(const float *__restrict__ wrow, int j, float r, float lo, float hi,
+template <bool NARROW, typename R>
+__device__ __forceinline__ uint2 chunk_codes(const R &row, int j, float r, float lo, float hi,
                                              uint32_t lo2, uint32_t hi2, float &dmax) {
-    const float4 a = *reinterpret_cast<const float4 *>(wrow + j);
-    const float4 b = *reinterpret_cast<const float4 *>(wrow + j + 4);
+    float4 a, b;
+    row.load8(j, a, b);
     return fast_codes8<NARROW>(a, b, r, lo, hi, lo2, hi2, dmax);
 }
 
@@ -104,8 +163,8 @@ __device__ __forceinline__ uint2 chunk_codes(const float *__restrict__ wrow, int
 // the candidate with the kept codes in q and marks the chunks that moved;
 // they are rewritten afterwards, once (a warp would otherwise run the update
 // path whenever any lane had a moved chunk).  Both mark near-tie chunks.
-template <bool INIT, bool NARROW>
-__device__ __forceinline__ void pass_chunks(const float *__restrict__ wrow, int K, float r, float lo, float hi,
+template <bool INIT, bool NARROW, typename R>
+__device__ __forceinline__ void pass_chunks(const R &row, int K, float r, float lo, float hi,
                                             uint32_t lo2, uint32_t hi2, float tie_bound, int8_t *__restrict__ q,
                                             PassOut &out, uint32_t &moved, uint32_t &tie) {
     const int stride = blockDim.x * 8;
@@ -113,12 +172,12 @@ __device__ __forceinline__ void pass_chunks(const float *__restrict__ wrow, int 
 #pragma unroll 2
     for (int j = threadIdx.x * 8; j < K; j += stride, ++m) {
         float dmax = 0.0f;
-        const uint2 nw = chunk_codes<NARROW>(wrow, j, r, lo, hi, lo2, hi2, dmax);
+        float4 a, b;
+        row.load8(j, a, b);
+        const uint2 nw = fast_codes8<NARROW>(a, b, r, lo, hi, lo2, hi2, dmax);
         if (dmax >= tie_bound) tie |= 1u << m;
         if (INIT) {
             *reinterpret_cast<uint2 *>(q + j) = nw;
-            const float4 a = *reinterpret_cast<const float4 *>(wrow + j);
-            const float4 b = *reinterpret_cast<const float4 *>(wrow + j + 4);
             const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -137,8 +196,15 @@ __device__ __forceinline__ void pass_chunks(const float *__restrict__ wrow, int 
 
 // Moved chunks: the change of NUM and DEN, and the new codes written over
 // the kept ones.
-template <bool NARROW>
-__device__ __forceinline__ void rewrite_moved(const float *__restrict__ wrow, uint32_t moved, float r, float lo,
+// The change of DEN for a chunk whose codes go from od to nw (exact: dp4a
+// of the signed bytes).
+__device__ __forceinline__ int den_change(uint2 nw, uint2 od) {
+    return __dp4a((int)nw.x, (int)nw.x, __dp4a((int)nw.y, (int)nw.y, 0)) -
+           __dp4a((int)od.x, (int)od.x, __dp4a((int)od.y, (int)od.y, 0));
+}
+
+template <bool NARROW, typename R>
+__device__ __forceinline__ void rewrite_moved(const R &row, uint32_t moved, float r, float lo,
                                               float hi, uint32_t lo2, uint32_t hi2, int8_t *__restrict__ q,
                                               PassOut &out) {
     const int stride = blockDim.x * 8;
@@ -147,15 +213,16 @@ __device__ __forceinline__ void rewrite_moved(const float *__restrict__ wrow, ui
         moved &= moved - 1u;
         const int j = threadIdx.x * 8 + mm * stride;
         float dmax = 0.0f;
-        const uint2 nw = chunk_codes<NARROW>(wrow, j, r, lo, hi, lo2, hi2, dmax);
+        const uint2 nw = chunk_codes<NARROW>(row, j, r, lo, hi, lo2, hi2, dmax);
         const uint2 od = *reinterpret_cast<const uint2 *>(q + j);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int qn = code_byte(nw, i), qo = code_byte(od, i);
-            if (qn != qo) {
-                out.den += qn * qn - qo * qo;
-                dd_acc(out.num, (double)wrow[j + i] * code_to_f64(qn - qo));  // exact product
-            }
+        out.den += den_change(nw, od);
+        // only the bytes that differ: 0x80 marks each
+        const unsigned long long diff =
+            ((unsigned long long)__vcmpne4(nw.y, od.y) << 32 | __vcmpne4(nw.x, od.x)) & 0x8080808080808080ull;
+        for (unsigned long long d = diff; d;) {
+            const int i = (__ffsll((long long)d) - 1) >> 3;
+            d &= d - 1ull;
+            out.dnum += (double)row.load1(j + i) * code_to_f64(code_byte(nw, i) - code_byte(od, i));  // exact product
         }
         *reinterpret_cast<uint2 *>(q + j) = nw;
     }
@@ -165,8 +232,10 @@ __device__ __forceinline__ void rewrite_moved(const float *__restrict__ wrow, ui
 // whose fast codes are already in q.  With SUMS, the change of NUM and DEN
 // is accumulated.  Visiting only the flagged chunks keeps the warp's detour
 // short when one lane has a near tie.
-template <bool SUMS>
-__device__ __forceinline__ void fix_ties(const float *__restrict__ wrow, uint32_t tie, float c, float r, float qmax,
+// SUMS: 1 adds the change to the init sums (double-double NUM), 2 to the
+// update's fp64 change of NUM, 0 to nothing.
+template <int SUMS, typename R>
+__device__ __forceinline__ void fix_ties(const R &row, uint32_t tie, float c, float r, float qmax,
                                          int8_t *__restrict__ q, PassOut &out) {
     const int stride = blockDim.x * 8;
     while (tie) {
@@ -175,7 +244,7 @@ __device__ __forceinline__ void fix_ties(const float *__restrict__ wrow, uint32_
         const int j = threadIdx.x * 8 + mm * stride;
 #pragma unroll 1
         for (int i = 0; i < 8; ++i) {
-            const float v = wrow[j + i];
+            const float v = row.load1(j + i);
             const float t = fmaf(v, r, kRoundMagic);
             const float rq = t - kRoundMagic;
             const float d = fmaf(v, r, -rq);
@@ -186,7 +255,8 @@ __device__ __forceinline__ void fix_ties(const float *__restrict__ wrow, uint32_
                     q[j + i] = (int8_t)qe;
                     if (SUMS) {
                         out.den += qe * qe - qf * qf;
-                        dd_acc(out.num, (double)v * code_to_f64(qe - qf));
+                        if (SUMS == 1) dd_acc(out.num, (double)v * code_to_f64(qe - qf));
+                        else out.dnum += (double)v * code_to_f64(qe - qf);
                         out.moved = true;
                     }
                 }
@@ -223,29 +293,30 @@ __device__ __forceinline__ ScaleConsts scale_consts(float c, float qmax, float w
 // where they differ and the change of NUM and DEN is returned; `touched`
 // names the chunks rewritten, so that the kept codes can be restored if c
 // is rejected.  wmax is the thread's max |w|.  Called by whole warps.
-template <bool INIT>
-__device__ __forceinline__ PassOut row_pass(const float *__restrict__ wrow, int K, float c, float qmax, float wmax,
+template <bool INIT, typename R>
+__device__ __forceinline__ PassOut row_pass(const R &row, int K, float c, float qmax, float wmax,
                                             int8_t *__restrict__ q) {
     const ScaleConsts k = scale_consts(c, qmax, wmax);
-    PassOut out = {{0.0, 0.0}, {0.0, 0.0}, 0, false, 0u};
+    PassOut out = {{0.0, 0.0}, {0.0, 0.0}, 0.0, 0, false, 0u};
     uint32_t moved = 0u;  // bit m: chunk m of this thread moved (at most 32 chunks per thread)
     uint32_t tie = 0u;    // bit m: chunk m holds an element near a rounding tie
     if (k.narrow)
-        pass_chunks<INIT, true>(wrow, K, k.r, k.lo, k.hi, k.lo2, k.hi2, k.tie_bound, q, out, moved, tie);
+        pass_chunks<INIT, true>(row, K, k.r, k.lo, k.hi, k.lo2, k.hi2, k.tie_bound, q, out, moved, tie);
     else
-        pass_chunks<INIT, false>(wrow, K, k.r, k.lo, k.hi, k.lo2, k.hi2, k.tie_bound, q, out, moved, tie);
+        pass_chunks<INIT, false>(row, K, k.r, k.lo, k.hi, k.lo2, k.hi2, k.tie_bound, q, out, moved, tie);
     if (!INIT) {
         out.moved = moved != 0u;
         out.touched = moved | tie;
-        if (k.narrow) rewrite_moved<true>(wrow, moved, k.r, k.lo, k.hi, k.lo2, k.hi2, q, out);
-        else rewrite_moved<false>(wrow, moved, k.r, k.lo, k.hi, k.lo2, k.hi2, q, out);
+        if (k.narrow) rewrite_moved<true>(row, moved, k.r, k.lo, k.hi, k.lo2, k.hi2, q, out);
+        else rewrite_moved<false>(row, moved, k.r, k.lo, k.hi, k.lo2, k.hi2, q, out);
     }
-    fix_ties<true>(wrow, tie, c, k.r, qmax, q, out);
+    fix_ties<INIT ? 1 : 2>(row, tie, c, k.r, qmax, q, out);
     return out;
 }
 
 // Writes the exact codes at scale c over the chunks named in `touched`.
-__device__ __forceinline__ void restore_chunks(const float *__restrict__ wrow, uint32_t touched, float c,
+template <typename R>
+__device__ __forceinline__ void restore_chunks(const R &row, uint32_t touched, float c,
                                                float qmax, float wmax, int8_t *__restrict__ q) {
     const ScaleConsts k = scale_consts(c, qmax, wmax);
     const int stride = blockDim.x * 8;
@@ -255,19 +326,20 @@ __device__ __forceinline__ void restore_chunks(const float *__restrict__ wrow, u
         t &= t - 1u;
         const int j = threadIdx.x * 8 + mm * stride;
         float dmax = 0.0f;
-        const uint2 nw = k.narrow ? chunk_codes<true>(wrow, j, k.r, k.lo, k.hi, k.lo2, k.hi2, dmax)
-                                  : chunk_codes<false>(wrow, j, k.r, k.lo, k.hi, k.lo2, k.hi2, dmax);
+        const uint2 nw = k.narrow ? chunk_codes<true>(row, j, k.r, k.lo, k.hi, k.lo2, k.hi2, dmax)
+                                  : chunk_codes<false>(row, j, k.r, k.lo, k.hi, k.lo2, k.hi2, dmax);
         if (dmax >= k.tie_bound) tie |= 1u << mm;
         *reinterpret_cast<uint2 *>(q + j) = nw;
     }
     PassOut unused;
-    fix_ties<false>(wrow, tie, c, k.r, qmax, q, unused);
+    fix_ties<0>(row, tie, c, k.r, qmax, q, unused);
 }
 
 struct WarpPart {
-    dd num, w2;
+    dd num, w2;  // init: the warp's NUM and W2; update: num.hi is the warp's change of NUM
     int den;
 };
+
 
 template <typename T, bool FOLD>
 __global__ void __launch_bounds__(512, 2)
@@ -275,8 +347,15 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
            int8_t *__restrict__ q_out, float *__restrict__ scale_out, double *__restrict__ mse_out,
            int32_t *__restrict__ iters_out) {
     extern __shared__ __align__(16) uint8_t smem[];
-    float *wrow = reinterpret_cast<float *>(smem);            // K floats: the folded row
-    int8_t *q = reinterpret_cast<int8_t *>(wrow + K);         // K codes: the kept codes
+    T *wrow = reinterpret_cast<T *>(smem);                     // K elements: the row (see Row)
+    int8_t *q = reinterpret_cast<int8_t *>(smem) + (size_t)K * sizeof(T);  // K codes: the kept codes
+    Row<T, FOLD> row;
+    if constexpr (sizeof(T) == 2) {
+        row.w = reinterpret_cast<const uint16_t *>(wrow);
+        row.s = s;
+    } else {
+        row.w = reinterpret_cast<const float *>(wrow);
+    }
     __shared__ WarpPart part[2][16];
     struct Decision {
         float c_next;
@@ -290,23 +369,33 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
     const double thr_k = kSszThreshold * kd;  // absolute threshold on K-scaled errors
 
     for (int64_t n = blockIdx.x; n < N; n += gridDim.x) {
-        // ---- stage the folded row in shared memory
+        // ---- stage the row in shared memory (bf16 as loaded, fp32 folded)
         float amax = 0.0f;
 #pragma unroll 4
         for (int j = threadIdx.x * 8; j < K; j += T_ * 8) {
             float v[8];
-            Vec8<T>::load(wg + n * K + j, v);
-            if (FOLD) {
-                float f[8];
-                load8_f32(s + j, f);
+            if constexpr (sizeof(T) == 2) {
+                const uint4 u = __ldg(reinterpret_cast<const uint4 *>(wg + n * K + j));
+                *reinterpret_cast<uint4 *>(wrow + j) = u;
+                float4 a, b;
+                row.load8_global(u, j, a, b);
+                v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+                v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+            } else {
+                Vec8<T>::load(wg + n * K + j, v);
+                if (FOLD) {
+                    float f[8];
+                    load8_f32(s + j, f);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = v[i] * f[i];
+                    for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], f[i]);
+                }
+                float4 *dst = reinterpret_cast<float4 *>(wrow + j);
+                dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+                dst[1] = make_float4(v[4], v[5], v[6], v[7]);
             }
+            dbg_check8(v);  // the (smoothed) weights the search reads
 #pragma unroll
             for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-            float4 *dst = reinterpret_cast<float4 *>(wrow + j);
-            dst[0] = make_float4(v[0], v[1], v[2], v[3]);
-            dst[1] = make_float4(v[4], v[5], v[6], v[7]);
         }
         const float wmax = amax;  // this thread's max |w| (tie bound)
         amax = warp_max(amax);
@@ -319,7 +408,7 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
         float s_best = fmaxf(__fdiv_rn(amax, qmax), kSszMinScale);
         int par = 0;
         {
-            PassOut p = row_pass<true>(wrow, K, s_best, qmax, wmax, q);
+            PassOut p = row_pass<true>(row, K, s_best, qmax, wmax, q);
             p.num = warp_sum_dd(p.num);
             p.w2 = warp_sum_dd(p.w2);
             p.den = warp_sum_i(p.den);
@@ -347,16 +436,16 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
         // touched chunks restored in that one case.
         while (!done) {
             par ^= 1;
-            PassOut p = row_pass<false>(wrow, K, c, qmax, wmax, q);
+            PassOut p = row_pass<false>(row, K, c, qmax, wmax, q);
             touched = p.touched;
             if (__any_sync(0xffffffffu, p.moved)) {
-                p.num = warp_sum_dd(p.num);
+                p.dnum = warp_sum_d(p.dnum);
                 p.den = warp_sum_i(p.den);
             } else {
-                p.num = {0.0, 0.0};
+                p.dnum = 0.0;
                 p.den = 0;
             }
-            if (lane == 0) part[par][warp] = {p.num, {0.0, 0.0}, p.den};
+            if (lane == 0) part[par][warp] = {{p.dnum, 0.0}, {0.0, 0.0}, p.den};
             __syncthreads();  // the candidate codes and all partials are in place
             ++it;
             // The decision: every thread takes it (1-2 warps a channel), or
@@ -367,7 +456,7 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
                 dd num_c = NUM;
                 int den_c = DEN;
                 for (int i = 0; i < nwarps; ++i) {
-                    num_c = dd_add_cascade(num_c, part[par][i].num);
+                    dd_acc(num_c, part[par][i].num.hi);
                     den_c += part[par][i].den;
                 }
                 const double m_c = exact_error_k(W2, num_c, den_c, c);
@@ -410,7 +499,7 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
             // part[par] and decision[par] are rewritten two rounds from now,
             // after another barrier
         }
-        if (rejected) restore_chunks(wrow, touched, s_best, qmax, wmax, q);
+        if (rejected) restore_chunks(row, touched, s_best, qmax, wmax, q);
 
         // ---- kept codes out (each thread wrote and now reads its own chunks)
         for (int j = threadIdx.x * 8; j < K; j += T_ * 8)
@@ -442,7 +531,7 @@ static sq_status launch_ssz(const void *w, int64_t N, int64_t K, const float *s,
                             int8_t *q, float *scale, double *mse, int32_t *iters, int sms, cudaStream_t st) {
     const int threads = 32 * ssz_warps(K);
     const float qmax = (float)((1 << (bits - 1)) - 1);
-    const size_t smem = 5 * (size_t)K;  // fp32 row + codes
+    const size_t smem = (size_t)K * (sizeof(T) + 1);  // the row (bf16 raw or fp32 folded) + codes
     auto kern = s ? ssz_kernel<T, true> : ssz_kernel<T, false>;
     if (smem > 32 * 1024) {  // dynamic + static shared memory may pass the 48 KB default
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -454,6 +543,8 @@ static sq_status launch_ssz(const void *w, int64_t N, int64_t K, const float *s,
     kern<<<(unsigned)grid, threads, smem, st>>>((const T *)w, N, (int)K, s, qmax, max_iters, q, scale, mse, iters);
     return launch_status("ssz_kernel");
 }
+
+W8A8_DEBUG_READER(ssz)
 
 }  // namespace w8a8
 

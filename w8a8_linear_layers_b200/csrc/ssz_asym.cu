@@ -292,6 +292,7 @@ ssz_asym_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restr
 #pragma unroll
                 for (int i = 0; i < 8; ++i) v[i] = v[i] * f[i];
             }
+            dbg_check8(v);  // the (smoothed) weights the search reads
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 lo = fminf(lo, v[i]);
@@ -430,6 +431,8 @@ static sq_status launch(const void *w, int64_t N, int64_t K, const float *s, int
 }
 
 }  // namespace asym
+W8A8_DEBUG_READER(ssz_asym)
+
 }  // namespace w8a8
 
 using namespace w8a8;
