@@ -136,6 +136,9 @@ def test_smooth_factor_split(w, orc, N, K, dtype, alpha):
     (1, 16, torch.float32, False), (5, 48, torch.bfloat16, True), (16, 256, torch.float32, True),
     (2048, 4096, torch.bfloat16, True), (33, 8192, torch.bfloat16, True), (3, 12304, torch.bfloat16, True),
     (2, 32768, torch.float32, True), (257, 1040, torch.bfloat16, False),
+    # rows staged by bulk copies (M, K >= 1024): ragged token counts, fp32 rows of 16 KB
+    (1500, 1040, torch.float32, True), (4099, 2064, torch.bfloat16, True), (1100, 4096, torch.float32, False),
+    (1024, 8192, torch.bfloat16, True),
 ])
 def test_quant_act_bit_exact(w, orc, M, K, dtype, smooth):
     x = make_x(M, K, dtype, seed=3 * M + K)
