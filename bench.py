@@ -281,7 +281,7 @@ def run_ours(args, rank, world, local_rank):
         mark(3)
         if p.bits == 4:  # int4 weights: packed two per byte for the W4A8 GEMM
             w.sq_pack_int4(p.qw, p.qw4)
-        mark(4)
+            mark(4)  # int8 records no packing event: an empty pair would time only the gap
         forward(p, p.x, evs, base)
         mark(6)
 
@@ -310,9 +310,25 @@ def run_ours(args, rank, world, local_rank):
         graph.replay()  # untimed
         torch.cuda.synchronize()
 
+    pack = NAMES.index("sq_pack_int4")
+
     def elapsed(e):
-        """Per linear j: [kernel i time for i in NAMES] from a step's events."""
-        return [[e[NM * j + i].elapsed_time(e[NM * j + i + 1]) for i in range(len(NAMES))] for j in range(len(probs))]
+        """Per linear j: [kernel i time for i in NAMES] from a step's events
+        (int8 weights: no packing event, the activation quantization timed
+        from the SSZ's end event)."""
+        out = []
+        for j, p in enumerate(probs):
+            b = NM * j
+            t = []
+            for i in range(len(NAMES)):
+                if p.bits != 4 and i == pack:
+                    t.append(0.0)
+                elif p.bits != 4 and i == pack + 1:
+                    t.append(e[b + i - 1].elapsed_time(e[b + i + 1]))
+                else:
+                    t.append(e[b + i].elapsed_time(e[b + i + 1]))
+            out.append(t)
+        return out
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(NM * len(probs))] for _ in range(args.steps)]
     per_step = []
