@@ -178,7 +178,9 @@ __device__ __forceinline__ uint32_t clamp_s16x2(uint32_t w, uint32_t lo2, uint32
 // NARROW (every |v r| < 2^14): bits(t) - bits(M) is the code, so the low
 // halves of bits(t) are the codes as int16 and are clamped two at a time;
 // otherwise t is clamped as a float (|v r| may leave the integer range of M).
-template <bool NARROW>
+// !CLAMP: the caller guarantees every |v r| < qmax + 0.5, so rint(v r) is
+// already in range and the low byte of bits(t) is the code as it stands.
+template <bool NARROW, bool CLAMP = true>
 __device__ __forceinline__ uint2 fast_codes8(const float4 a, const float4 b, float r, float lo, float hi,
                                              uint32_t lo2, uint32_t hi2, float &dmax) {
     const float2 v[4] = {make_float2(a.x, a.y), make_float2(a.z, a.w), make_float2(b.x, b.y), make_float2(b.z, b.w)};
@@ -189,10 +191,10 @@ __device__ __forceinline__ uint2 fast_codes8(const float4 a, const float4 b, flo
         const float2 tt = f2_fma(v[i], r2, m2);
         const float2 d = f2_fma(v[i], r2, f2_sub(m2, tt));
         dmax = fmax3(dmax, fabsf(d.x), fabsf(d.y));
-        t[2 * i] = __float_as_uint(NARROW ? tt.x : fminf(fmaxf(tt.x, lo), hi));  // code = low byte
-        t[2 * i + 1] = __float_as_uint(NARROW ? tt.y : fminf(fmaxf(tt.y, lo), hi));
+        t[2 * i] = __float_as_uint(NARROW || !CLAMP ? tt.x : fminf(fmaxf(tt.x, lo), hi));  // code = low byte
+        t[2 * i + 1] = __float_as_uint(NARROW || !CLAMP ? tt.y : fminf(fmaxf(tt.y, lo), hi));
     }
-    if (NARROW) {
+    if (NARROW && CLAMP) {
         uint32_t h[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) h[i] = clamp_s16x2(__byte_perm(t[2 * i], t[2 * i + 1], 0x5410), lo2, hi2);

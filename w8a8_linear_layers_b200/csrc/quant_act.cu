@@ -58,12 +58,19 @@ constexpr uint32_t kLo2 = 0xFF81FF81u, kHi2 = 0x007F007Fu;
 
 // Codes of 8 scaled elements at scale s (r = 1/s): packed fast path, then
 // the exact quotient for any element near a rounding tie (rare).
+// IN_RANGE: s and r come from this row's own abs-max am (s = am / 127,
+// r = 1 / s, r finite), so no code needs the clamp: every |v| r <= am r <
+// 127 (1 + 2^-22) once r is finite (s >= 2^-128: the relative error of s
+// is at most 2^-22 even where s is subnormal, and a smaller s makes r
+// overflow), so rint(v r) is within [-127, 127].
+template <bool IN_RANGE>
 __device__ __forceinline__ uint2 fast_codes_tied(const float (&v)[8], float s, float r, bool narrow,
                                                  float tie_bound) {
     const float4 a = make_float4(v[0], v[1], v[2], v[3]), b = make_float4(v[4], v[5], v[6], v[7]);
     float dmax = 0.0f;
-    uint2 code = narrow ? fast_codes8<true>(a, b, r, kLo, kHi, kLo2, kHi2, dmax)
-                        : fast_codes8<false>(a, b, r, kLo, kHi, kLo2, kHi2, dmax);
+    uint2 code = IN_RANGE ? fast_codes8<true, false>(a, b, r, kLo, kHi, kLo2, kHi2, dmax)
+                 : narrow ? fast_codes8<true>(a, b, r, kLo, kHi, kLo2, kHi2, dmax)
+                          : fast_codes8<false>(a, b, r, kLo, kHi, kLo2, kHi2, dmax);
     if (dmax >= tie_bound) {
 #pragma unroll  // unrolled: v stays in registers
         for (int i = 0; i < 8; ++i) {
@@ -213,7 +220,7 @@ quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__r
                     for (int i = 0; i < 8; ++i) e[i] = (int)sym_code(v[i], s, r, 127.0f, true);
                     code = pack8_codes(e);
                 } else {
-                    code = fast_codes_tied(v, s, r, narrow, tie_bound);
+                    code = fast_codes_tied<!STATIC>(v, s, r, narrow, tie_bound);
                 }
                 *reinterpret_cast<uint2 *>(qr + ((int64_t)c * T_ + threadIdx.x) * 8) = code;
                 if (rowsum) rsum = __dp4a((int)code.y, 0x01010101, __dp4a((int)code.x, 0x01010101, rsum));
@@ -404,7 +411,7 @@ ln_quant_kernel(const T *__restrict__ h, int64_t M, int64_t K, const float *__re
                 for (int i = 0; i < 8; ++i) e[i] = (int)sym_code(x[c][i], s, r, 127.0f, true);
                 code = pack8_codes(e);
             } else {
-                code = fast_codes_tied(x[c], s, r, narrow, tie_bound);
+                code = fast_codes_tied<true>(x[c], s, r, narrow, tie_bound);
             }
             *reinterpret_cast<uint2 *>(q + row * K + base + 8 * c) = code;
         }
