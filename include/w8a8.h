@@ -228,7 +228,9 @@ sq_status sq_pack_int4(const int8_t *q, int64_t N, int64_t K, uint8_t *packed, v
 /* w4a8_gemm_dequant: w8a8_gemm_dequant with the weight codes packed by
  * sq_pack_int4 (qw4: [N, K/2] bytes, 16-byte aligned).  The codes are
  * unpacked on chip; acc and y are exactly those of w8a8_gemm_dequant on
- * the unpacked codes.  K a multiple of 32. */
+ * the unpacked codes.  K a multiple of 32, at most 131040 (the tensor
+ * cores take the codes as 16 q, so the int32 accumulator holds 16 acc and
+ * stays below 2^31 for any int8 qx and codes in [-8, 7]). */
 sq_status w4a8_gemm_dequant(const int8_t *qx, const float *sx, const uint8_t *qw4, const float *sw,
                             int64_t M, int64_t N, int64_t K, void *y, sq_dtype yt, int32_t *acc_out,
                             void *stream);

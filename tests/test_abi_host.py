@@ -163,11 +163,12 @@ def test_gemm_asym_rejects(lib, case, status):
     assert rc == status, _detail(lib)
 
 
-@pytest.mark.parametrize("case,status", [("null", 1), ("k16", 2), ("align", 4), ("dtype", 3)])
+@pytest.mark.parametrize("case,status", [("null", 1), ("k16", 2), ("k_limit", 2), ("align", 4), ("dtype", 3)])
 def test_w4a8_rejects(lib, case, status):
     a = dict(qx=P(), sx=P(4096), qw=P(8192), sw=P(12288), M=4, N=16, K=64, y=P(16384), yt=1)
     if case == "null": a["qw"] = NULL
     if case == "k16": a["K"] = 48
+    if case == "k_limit": a["K"] = 131072  # 16 * 128 * 8 * K would pass 2^31
     if case == "align": a["qw"] = P(8200)
     if case == "dtype": a["yt"] = 2
     rc = lib.w4a8_gemm_dequant(a["qx"], a["sx"], a["qw"], a["sw"], a["M"], a["N"], a["K"], a["y"], a["yt"], NULL,

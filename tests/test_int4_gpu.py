@@ -52,6 +52,32 @@ def test_w4a8_gemm_bit_exact(w, orc, M, N, K, ydt):
     assert y.intact()
 
 
+@pytest.mark.parametrize("M", [16, 300])  # the decode kernel and the W4A8 kernel
+def test_w4a8_extreme_accumulators(w, orc, M):
+    """Largest |acc| the signed operands allow: a row of qx at -128 against
+    codes at -8 (and at 7), over K = 16384; acc exact, signs kept."""
+    N, K = 256, 16384
+    r = np.random.default_rng(M)
+    qx = r.integers(-127, 128, (M, K)).astype(np.int8)
+    qx[0, :] = -128
+    qx[1, :] = 127
+    q4 = r.integers(-8, 8, (N, K)).astype(np.int8)
+    q4[0, :] = -8
+    q4[1, :] = 7
+    sx = np.full(M, 1e-6, np.float32)
+    sw = np.full(N, 1e-3, np.float32)
+    d = lambda a: torch.from_numpy(a).cuda()  # noqa: E731
+    p = torch.empty(N, K // 2, dtype=torch.uint8, device="cuda")
+    w.sq_pack_int4(d(q4), p)
+    y = torch.empty(M, N, dtype=torch.float32, device="cuda")
+    acc = torch.empty(M, N, dtype=torch.int32, device="cuda")
+    w.w4a8_gemm_dequant(d(qx), d(sx), p, d(sw), y, acc)
+    acc_o = orc.gemm_i8(qx, q4)
+    assert acc_o[0, 0] == 128 * 8 * K and acc_o[1, 1] == 127 * 7 * K and acc_o[0, 1] == -128 * 7 * K
+    np.testing.assert_array_equal(acc.cpu().numpy(), acc_o)
+    np.testing.assert_array_equal(y.cpu().numpy(), orc.dequant(acc_o, sx, sw, out="f32"))
+
+
 def test_w4a8_equals_w8a8_on_the_same_codes(w):
     r = np.random.default_rng(7)
     M, N, K = 200, 1024, 4096

@@ -562,7 +562,9 @@ __device__ __forceinline__ void mbar_arrive_leader(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar & kPeerMask) : "memory");
 }
 
-template <typename OutT, bool ASYM>
+// SHIFT: the accumulator holds 2^SHIFT times the product (int4 operands, see
+// unpack_int4x8) and is shifted back first.
+template <typename OutT, bool ASYM, int SHIFT = 0>
 __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int row, int M, int n0, int N, const float sxr,
                                               int Rr, const float *__restrict__ sw, const float *__restrict__ ow,
                                               OutT *__restrict__ y, int32_t *__restrict__ acc_out, int BNc) {
@@ -572,6 +574,10 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int row, int M, in
     for (int c0 = 0; c0 < BNc; c0 += 32) {
         uint32_t acc[32];
         tmem_ld32(tbase + (uint32_t)c0, acc);  // warp-collective
+        if (SHIFT) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[j] = (uint32_t)((int32_t)acc[j] >> SHIFT);  // exact: a multiple of 2^SHIFT
+        }
         const int col = n0 + c0;
         if (row < M && col < N) {
             const int valid = N - col;
@@ -921,12 +927,16 @@ struct CfgW4 {
 
 
 // 8 int4 codes (one 32-bit word, element 2i in the low nibble of byte i) to
-// 8 int8 codes.  A nibble x sign-extends as ((x ^ 8) + 0x78) ^ 0x80: every
-// byte stays below 0x88 before the last step, so one 32-bit add serves four
-// bytes without carries.  Low and high nibble values are then interleaved.
+// 8 int8 operands 16 q: a nibble moved to the high half of its byte, low
+// half zero, is 16 times its signed value as an int8, so no sign extension
+// is needed (|16 q| <= 128 stays in the int8 range).  The accumulator is then
+// 16 times the product of the codes, exactly (every term is a multiple of
+// 16, and |16 acc| < 2^31 for the sizes the GEMMs accept); the epilogues
+// shift it right by 4 (exact) before the dequant.
+constexpr int kInt4AccShift = 4;
 __device__ __forceinline__ void unpack_int4x8(uint32_t w, uint32_t &o0, uint32_t &o1) {
-    const uint32_t lo = (((w & 0x0F0F0F0Fu) ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
-    const uint32_t hi = ((((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
+    const uint32_t hi = w & 0xF0F0F0F0u;          // 16 q[2i+1]
+    const uint32_t lo = (w << 4) & 0xF0F0F0F0u;   // 16 q[2i]
     o0 = __byte_perm(lo, hi, 0x5140);
     o1 = __byte_perm(lo, hi, 0x7362);
 }
@@ -1145,7 +1155,7 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
             const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BNw);
-            epilogue_tile<OutT, false>(tbase, row, M, n0, N, sxr, 0, sw, nullptr, y, acc_out, BNw);
+            epilogue_tile<OutT, false, kInt4AccShift>(tbase, row, M, n0, N, sxr, 0, sw, nullptr, y, acc_out, BNw);
             tc_fence_before();
             mbar_arrive(smem_u32(&tempty_bar[buf]));
             buf ^= 1;
@@ -1470,8 +1480,9 @@ extern "C" sq_status w4a8_gemm_dequant(const int8_t *qx, const float *sx, const 
     const char *fn = "w4a8_gemm_dequant";
     if (M > 0 && N > 0 && (!qx || !sx || !qw4 || !sw || !y)) return fail(SQ_ERR_NULL, "%s: NULL pointer", fn);
     if (yt != SQ_F32 && yt != SQ_BF16) return fail(SQ_ERR_DTYPE, "%s: output dtype %d", fn, (int)yt);
-    if (M < 0 || N < 0 || K <= 0 || K % 32 != 0 || K > 133144 || M > INT32_MAX || N > INT32_MAX)
-        return fail(SQ_ERR_SHAPE, "%s: M=%lld N=%lld K=%lld (K a multiple of 32 in [32, 133144])", fn, (long long)M,
+    // the accumulator holds 16 acc (unpack_int4x8): 16 * 128 * 8 * K < 2^31
+    if (M < 0 || N < 0 || K <= 0 || K % 32 != 0 || K > 131040 || M > INT32_MAX || N > INT32_MAX)
+        return fail(SQ_ERR_SHAPE, "%s: M=%lld N=%lld K=%lld (K a multiple of 32 in [32, 131040])", fn, (long long)M,
                     (long long)N, (long long)K);
     if (M == 0 || N == 0) return SQ_OK;
     const int out_vec = (yt == SQ_BF16) ? 8 : 4;

@@ -325,6 +325,10 @@ w8a8_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
             for (int c0 = 0; c0 < NT; c0 += 16) {
                 uint32_t acc[16];
                 tmem_ld16(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c0, acc);
+                if (INT4) {  // 16 times the product (see unpack_int4x8); exact
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) acc[j] = (uint32_t)((int32_t)acc[j] >> kInt4AccShift);
+                }
                 if (split == 1) {
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
