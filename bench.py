@@ -196,7 +196,7 @@ NAMES = ["calib_absmax", "smooth_fold", "ssz_quant_weight", "sq_pack_int4", "qua
          "w8a8_gemm_dequant"]
 WEIGHT_PATH = ("calib_absmax", "smooth_fold", "ssz_quant_weight", "sq_pack_int4")  # once per weight
 LINEAR = ("quant_act_per_token", "w8a8_gemm_dequant")  # every inference
-NM = len(NAMES) + 1  # events per linear
+NW = len(WEIGHT_PATH) + 1  # weight-path events per linear
 GPT_WORKLOAD = "gpt345m_8x1024"
 
 
@@ -252,19 +252,24 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream()
 
     def forward(p, xin, evs=None, base=0):
-        """The per-inference part: per-token codes, then the GEMM."""
+        """The per-inference part: per-token codes, then the GEMM (with evs:
+        an event before, between and after, for the per-kernel split)."""
+        if evs is not None:
+            evs[base].record()
         w.quant_act_per_token(xin, p.inv, p.qx, p.sx)
         if evs is not None:
-            evs[base + 5].record()
+            evs[base + 1].record()
         if p.bits == 8:
             w.w8a8_gemm_dequant(p.qx, p.sx, p.qw, p.sw, p.y)
         else:
             w.w4a8_gemm_dequant(p.qx, p.sx, p.qw4, p.sw, p.y)
+        if evs is not None:
+            evs[base + 2].record()
 
-    def run(p, evs=None, base=0):
-        """The whole path on one linear; with evs, an event before each
-        kernel (NAMES order) and one after the last, on the current stream
-        (the launching one, or a graph's capture stream)."""
+    def weight_path(p, evs=None, base=0):
+        """The once-per-weight part of one linear; with evs, an event before
+        each kernel (WEIGHT_PATH order) and one after the last, on the
+        current stream (the launching one, or a graph's capture stream)."""
         def mark(i):
             if evs is not None:
                 evs[base + i].record()
@@ -282,12 +287,24 @@ def run_ours(args, rank, world, local_rank):
         if p.bits == 4:  # int4 weights: packed two per byte for the W4A8 GEMM
             w.sq_pack_int4(p.qw, p.qw4)
             mark(4)  # int8 records no packing event: an empty pair would time only the gap
-        forward(p, p.x, evs, base)
-        mark(6)
+
+    nw_ev = NW * len(probs)  # events of the weight path; then two around the linears
 
     def step(evs=None):
+        """One pass of the whole path over every linear: the once-per-weight
+        part of each (its kernels bracketed by events), then the per-inference
+        part of each, back to back with events only around the block (an
+        event node between two kernels adds its own latency and keeps the
+        next kernel from starting early, so the linears' time is taken
+        without them; the per-kernel split comes from instrumented replays)."""
         for i, p in enumerate(probs):
-            run(p, evs, NM * i)
+            weight_path(p, evs, NW * i)
+        if evs is not None:
+            evs[nw_ev].record()
+        for p in probs:
+            forward(p, p.x)
+        if evs is not None:
+            evs[nw_ev + 1].record()
 
     for _ in range(args.warmup):
         flush()
@@ -302,7 +319,7 @@ def run_ours(args, rank, world, local_rank):
     # ranks launch eagerly (no collective is captured).
     graph = None
     if world == 1 and not args.eager:
-        gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(NM * len(probs))]
+        gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(nw_ev + 2)]
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
             step(gev)
@@ -310,27 +327,18 @@ def run_ours(args, rank, world, local_rank):
         graph.replay()  # untimed
         torch.cuda.synchronize()
 
-    pack = NAMES.index("sq_pack_int4")
-
     def elapsed(e):
-        """Per linear j: [kernel i time for i in NAMES] from a step's events
-        (int8 weights: no packing event, the activation quantization timed
-        from the SSZ's end event)."""
+        """Per linear j: {weight-path kernel: ms} from a step's events (int8
+        weights: no packing event), and the per-inference block's ms."""
         out = []
         for j, p in enumerate(probs):
-            b = NM * j
-            t = []
-            for i in range(len(NAMES)):
-                if p.bits != 4 and i == pack:
-                    t.append(0.0)
-                elif p.bits != 4 and i == pack + 1:
-                    t.append(e[b + i - 1].elapsed_time(e[b + i + 1]))
-                else:
-                    t.append(e[b + i].elapsed_time(e[b + i + 1]))
+            b = NW * j
+            t = {n: e[b + i].elapsed_time(e[b + i + 1]) for i, n in enumerate(WEIGHT_PATH[:3])}
+            t["sq_pack_int4"] = e[b + 3].elapsed_time(e[b + 4]) if p.bits == 4 else 0.0
             out.append(t)
-        return out
+        return out, e[nw_ev].elapsed_time(e[nw_ev + 1])
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(NM * len(probs))] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nw_ev + 2)] for _ in range(args.steps)]
     per_step = []
     if world > 1:
         dist.barrier()
@@ -351,16 +359,68 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     if graph is None:
         per_step = [elapsed(e) for e in evs]
-    step_ms = [sum(sum(lin) for lin in st) for st in per_step]
-    li = [NAMES.index(n) for n in LINEAR]
-    linear_step_ms = [sum(lin[i] for lin in st for i in li) for st in per_step]
-    kern_ms = {n: statistics.mean(sum(lin[i] for lin in st) for st in per_step) for i, n in enumerate(NAMES)}
-    # per linear and kernel, mean over the timed steps (for the per-shape table)
-    lin_ms = [[statistics.mean(st[j][i] for st in per_step) for i in range(len(NAMES))] for j in range(len(probs))]
+    step_ms = [sum(sum(t.values()) for t in st) + blk for st, blk in per_step]
+    linear_step_ms = [blk for _, blk in per_step]
     total_ms = wdist.max_over_ranks(sum(step_ms), device=dev)
     linear_ms = wdist.max_over_ranks(sum(linear_step_ms), device=dev)
     if w.device_fault() != 0:
         raise RuntimeError("a kernel gave up on a bounded wait during timing")
+
+    # ---- outside the timed region: the per-inference block again, (a) with
+    # an event before, between and after the two kernels of every linear (the
+    # per-kernel split; each time then carries an event node's latency), and
+    # (b) with events only around each group of linears of one shape (the
+    # per-shape linear time, as in the timed block)
+    groups = {}
+    for j, p in enumerate(probs):
+        groups.setdefault((p.M, p.K, p.N), []).append(j)
+    iev = [torch.cuda.Event(enable_timing=True, external=graph is not None) for _ in range(3 * len(probs))]
+    gev2 = [torch.cuda.Event(enable_timing=True, external=graph is not None) for _ in range(2 * len(groups))]
+
+    def inst_split():
+        for j, p in enumerate(probs):
+            forward(p, p.x, iev, 3 * j)
+
+    def inst_groups():
+        for g, idx in enumerate(groups.values()):
+            gev2[2 * g].record()
+            for j in idx:
+                forward(probs[j], probs[j].x)
+            gev2[2 * g + 1].record()
+
+    reps = max(3, min(args.steps, 10))
+    split = [[0.0, 0.0] for _ in probs]
+    grp_ms = [0.0] * len(groups)
+    for fn, sink in ((inst_split, "split"), (inst_groups, "groups")):
+        g2 = None
+        if graph is not None:
+            g2 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g2):
+                fn()
+        for r in range(reps + 1):
+            flush()
+            if g2 is not None:
+                g2.replay()
+            else:
+                fn()
+            torch.cuda.synchronize()
+            if r == 0:
+                continue  # warm-up replay
+            if sink == "split":
+                for j in range(len(probs)):
+                    split[j][0] += iev[3 * j].elapsed_time(iev[3 * j + 1]) / reps
+                    split[j][1] += iev[3 * j + 1].elapsed_time(iev[3 * j + 2]) / reps
+            else:
+                for g in range(len(groups)):
+                    grp_ms[g] += gev2[2 * g].elapsed_time(gev2[2 * g + 1]) / reps
+        del g2
+    # per kernel (summed over the linears, mean over steps) and per linear and kernel
+    kern_ms = {n: statistics.mean(sum(t[n] for t in st) for st, _ in per_step) for n in WEIGHT_PATH}
+    kern_ms["quant_act_per_token"] = sum(a for a, _ in split)
+    kern_ms["w8a8_gemm_dequant"] = sum(b for _, b in split)
+    lin_ms = [[statistics.mean(st[j][n] for st, _ in per_step) for n in WEIGHT_PATH] + split[j]
+              for j in range(len(probs))]
+    shape_ms = {"%dx%d->%d" % k: grp_ms[g] / len(idx) for g, (k, idx) in enumerate(groups.items())}
 
     ops_per_step = sum(2.0 * p.M * p.N * p.K for p in probs)
     value = ops_per_step * world * args.steps / (linear_ms * 1e-3) / 1e12
@@ -375,7 +435,8 @@ def run_ours(args, rank, world, local_rank):
         e2e = run_e2e(args, w, wdist, torch, probs, forward, flush, stream, ops_per_step, world)
     del graph
     return finish(args, world, probs, kern_ms, total_ms, linear_ms, value, path_value, e2e, clk, wall1 - wall0,
-                  next_rows, launch="eager" if world > 1 or args.eager else "cuda_graph", lin_ms=lin_ms)
+                  next_rows, launch="eager" if world > 1 or args.eager else "cuda_graph", lin_ms=lin_ms,
+                  shape_ms=shape_ms)
 
 
 class L2Flush:
@@ -556,10 +617,13 @@ def run_e2e(args, w, wdist, torch, probs, forward, flush, stream, ops_per_step, 
                     "output copied device->host, every step; quantized weights resident"}
 
 
-def per_shape_table(probs, lin_ms, peaks):
+def per_shape_table(probs, lin_ms, peaks, shape_ms=None):
     """Workloads of several linears: per distinct (M, K, N) the number of
-    linears, the mean time of each kernel, the GEMM's TOPS and the linear's
-    (activation quantization + GEMM)."""
+    linears, the mean time of each kernel (the activation quantization and
+    the GEMM each from events around it, which add an event node's
+    latency), the GEMM's TOPS and the linear's (activation quantization +
+    GEMM, from events around the shape's group of linears run back to back,
+    as in the timed block)."""
     groups = {}
     for p, ms in zip(probs, lin_ms):
         groups.setdefault((p.M, p.K, p.N), []).append(ms)
@@ -569,6 +633,8 @@ def per_shape_table(probs, lin_ms, peaks):
         mean = [statistics.mean(r[i] for r in rows) for i in range(len(NAMES))]
         gemm_ms = mean[NAMES.index("w8a8_gemm_dequant")]
         lin = gemm_ms + mean[NAMES.index("quant_act_per_token")]
+        if shape_ms:
+            lin = shape_ms["%dx%d->%d" % (M, K, N)]
         tops = 2.0 * M * N * K / (gemm_ms * 1e-3) / 1e12
         out["%dx%d->%d" % (M, K, N)] = {
             "linears": len(rows), "us": {n: round(m * 1e3, 2) for n, m in zip(NAMES, mean)},
@@ -578,7 +644,7 @@ def per_shape_table(probs, lin_ms, peaks):
 
 
 def finish(args, world, probs, kern_ms, total_ms, linear_ms, value, path_value, e2e, clk, wall_s, next_rows=None,
-           launch="eager", lin_ms=None):
+           launch="eager", lin_ms=None, shape_ms=None):
     names = [n for n in NAMES if n != "sq_pack_int4" or any(p.bits == 4 for p in probs)]
     # ---- rooflines per kernel (algorithmic work summed over the workload's linears)
     peaks, src = load_peaks()
@@ -654,13 +720,17 @@ def finish(args, world, probs, kern_ms, total_ms, linear_ms, value, path_value, 
                    "parallelism": ("dp%d (replicas; MAX all-reduce of the calibration absmax; SSZ split by output "
                                    "channel and all-gathered)" % world),
                    "l2": "flushed (512 MB write, then 384 MB read) before every timed step, outside the timed events",
-                   "launch": {"cuda_graph": "each timed step one CUDA graph replay (captured once, per-kernel "
-                                            "events inside it)",
+                   "launch": {"cuda_graph": "each timed step one CUDA graph replay (captured once, events "
+                                            "inside it)",
                               "eager": "every call of a timed step launched from Python"}[launch]},
-        "value_definition": ("2*M*N*K int8 ops over the device time of the per-inference linear (per-token "
-                             "activation quantization + GEMM with fused dequant) inside each timed step; every "
-                             "timed step also runs the once-per-weight path (calibration, smoothing, SSZ), whose "
-                             "time is in ms_per_step and whose throughput is in weight_path"),
+        "value_definition": ("2*M*N*K int8 ops over the device time of the per-inference linears (per-token "
+                             "activation quantization + GEMM with fused dequant), run back to back inside each "
+                             "timed step with events only around them; every timed step first runs the "
+                             "once-per-weight path of every linear (calibration, smoothing, SSZ, each kernel "
+                             "between events), whose time is in ms_per_step and whose throughput is in "
+                             "weight_path.  The activation-quantization and GEMM entries of kernels come from "
+                             "replays of the linears outside the timed region with an event around each kernel "
+                             "(each carries an event node's latency)"),
         "linear": {"ms_per_step": round(lin_step, 4), "tops": round(value, 2), "peak": round(int8_peak, 1),
                    "frac": round(value / int8_peak, 4), "kernels": list(LINEAR)},
         "path": {"ms_per_step": round(total_ms / args.steps, 4), "tops": round(path_value, 2),
@@ -674,7 +744,7 @@ def finish(args, world, probs, kern_ms, total_ms, linear_ms, value, path_value, 
         "wall_s_timed_region": round(wall_s, 3),
     }
     if lin_ms is not None and len(probs) > 1:
-        result["per_shape"] = per_shape_table(probs, lin_ms, peaks)
+        result["per_shape"] = per_shape_table(probs, lin_ms, peaks, shape_ms)
     if next_rows:
         result["next_rows"] = next_rows
     return result
