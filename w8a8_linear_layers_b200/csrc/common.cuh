@@ -44,6 +44,35 @@ inline sq_status launch_status(const char *what) {
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// ------------------------------------------------ programmatic dependent launch
+// The per-inference kernels (activation quantization, GEMM) are launched with
+// programmatic stream serialization: such a kernel may be scheduled before
+// its predecessor in the stream has finished, as soon as every CTA of the
+// predecessor has called pdl_trigger (or exited), so that its launch and
+// prologue overlap the predecessor's tail.  Before its first access to global
+// memory that the predecessor may write or read, every thread calls pdl_wait,
+// which returns once the predecessor grid has completed and its writes are
+// visible.  Without the attribute (or after a kernel that never triggers)
+// both are no-ops and the launch is ordinary.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...);
+}
+
 // ----------------------------------------------------------------- device side
 // Load 8 consecutive elements (16 bytes of bf16, or 32 bytes of fp32) as fp32.
 // bf16 widens exactly (its bits are the high half of an fp32).

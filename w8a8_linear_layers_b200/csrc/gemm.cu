@@ -322,6 +322,8 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = tmem_slot;
+    pdl_wait();     // the codes and scales come from the previous kernel (prologue above overlapped it)
+    pdl_trigger();  // the next kernel may launch; it waits for this grid before touching memory
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -749,6 +751,8 @@ w8a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_c
     cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated
     tc_fence_after();
     const uint32_t tmem_base = tmem_slot;
+    pdl_wait();     // the codes and scales come from the previous kernel (prologue above overlapped it)
+    pdl_trigger();  // the next kernel may launch; it waits for this grid before touching memory
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (both CTAs)
@@ -998,6 +1002,8 @@ w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = tmem_slot;
+    pdl_wait();     // the codes and scales come from the previous kernel (prologue above overlapped it)
+    pdl_trigger();  // the next kernel may launch; it waits for this grid before touching memory
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (A + packed B)
@@ -1295,7 +1301,7 @@ static sq_status launch_w4(const int8_t *qx, const float *sx, const uint8_t *qw4
     }
     const int tiles = ((M + BM - 1) / BM) * ((N + C::BN - 1) / C::BN);
     const int grid = std::min(tiles, sms);
-    kern<<<grid, kThreadsW4, C::SMEM, st>>>(ma, mb, sx, sw, (OutT *)y, acc_out, M, N, K);
+    launch_pdl(kern, dim3(grid), dim3(kThreadsW4), C::SMEM, st, ma, mb, sx, sw, (OutT *)y, acc_out, M, N, K);
     return launch_status("w4a8_gemm_kernel");
 }
 
@@ -1336,13 +1342,15 @@ static sq_status launch_decode(const int8_t *qx, const float *sx, const int32_t 
     cfg.blockDim = dim3(dec_threads(INT4), 1, 1);
     cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)split;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see pdl_wait
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mw, mx, sx, sw, rs, ow, (OutT *)y, acc_out, M, N, K);
     if (e != cudaSuccess) return fail(SQ_ERR_CUDA, "w8a8_gemm_decode_kernel launch: %s", cudaGetErrorString(e));
     return launch_status("w8a8_gemm_decode_kernel");
@@ -1376,7 +1384,7 @@ static sq_status launch(const int8_t *qx, const float *sx, const int32_t *rs, co
     }
     const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int grid = std::min(tiles, sms);
-    kern<<<grid, kThreads, C::SMEM, st>>>(ma, mb, sx, sw, rs, ow, (OutT *)y, acc_out, M, N, K);
+    launch_pdl(kern, dim3(grid), dim3(kThreads), C::SMEM, st, ma, mb, sx, sw, rs, ow, (OutT *)y, acc_out, M, N, K);
     return launch_status("w8a8_gemm_kernel");
 }
 
@@ -1400,7 +1408,8 @@ static sq_status launch_pair(const int8_t *qx, const float *sx, const int32_t *r
     }
     const int tiles = ((M + C::PM - 1) / C::PM) * ((N + C::BN - 1) / C::BN);
     const int pairs = std::min(tiles, sms / 2);
-    kern<<<2 * pairs, kThreadsPair, C::SMEM, st>>>(ma, mb, my, sx, sw, rs, ow, (OutT *)y, acc_out, M, N, K);
+    launch_pdl(kern, dim3(2 * pairs), dim3(kThreadsPair), C::SMEM, st, ma, mb, my, sx, sw, rs, ow, (OutT *)y, acc_out,
+               M, N, K);
     return launch_status("w8a8_gemm_pair_kernel");
 }
 

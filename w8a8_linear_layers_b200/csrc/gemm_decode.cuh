@@ -183,6 +183,8 @@ w8a8_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = tmem_slot;
+    pdl_wait();     // the codes and scales come from the previous kernel (prologue above overlapped it)
+    pdl_trigger();  // the next kernel may launch; it waits for this grid before touching memory
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer

@@ -115,6 +115,8 @@ quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__r
     __shared__ int rsum_red[2][ROWS][32];
     const int T_ = blockDim.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = T_ >> 5;
+    pdl_wait();     // x, inv_s and the outputs may belong to the previous kernel
+    pdl_trigger();  // the GEMM that follows may launch (it waits for this grid)
 
     float f[kCacheInvS ? C : 1][8];  // inv_s for this thread's columns (constant across rows)
     bool live[C];
@@ -258,8 +260,8 @@ static void launch_quant_act(const void *x, int64_t M, int64_t K, const float *i
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_act_kernel<T, E, ROWS, STATIC>, threads, 0);
     per_sm = std::max(1, std::min(per_sm, 2048 / threads));
     int64_t grid = std::min<int64_t>(ceil_div(M, ROWS), (int64_t)sms * per_sm);
-    quant_act_kernel<T, E, ROWS, STATIC>
-        <<<(unsigned)grid, threads, 0, st>>>((const T *)x, M, K, inv_s, range, q, scale, rowsum);
+    launch_pdl(quant_act_kernel<T, E, ROWS, STATIC>, dim3((unsigned)grid), dim3(threads), 0, st, (const T *)x, M, K,
+               inv_s, range, q, scale, rowsum);
 }
 
 // ------------------------------------------------ LayerNorm fused with step 4
@@ -310,6 +312,8 @@ ln_quant_kernel(const T *__restrict__ h, int64_t M, int64_t K, const float *__re
     const int T_ = blockDim.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = T_ >> 5;
     const int64_t base = (int64_t)threadIdx.x * E;  // this thread's first column
+    pdl_wait();     // h, gamma, beta, inv_s and the outputs may belong to the previous kernel
+    pdl_trigger();  // the GEMM that follows may launch (it waits for this grid)
     bool live[C];  // K is a multiple of 8: a chunk is wholly inside the row or wholly past it
     float g[C][8], bt[C][8], f[C][8];
 #pragma unroll
@@ -433,7 +437,8 @@ static void launch_ln_quant(const void *h, int64_t M, int64_t K, const float *ga
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ln_quant_kernel<T, E>, threads, 0);
     per_sm = std::max(1, std::min(per_sm, 2048 / threads));
     const int64_t grid = std::min<int64_t>(M, (int64_t)sms * per_sm);
-    ln_quant_kernel<T, E><<<(unsigned)grid, threads, 0, st>>>((const T *)h, M, K, gamma, beta, eps, inv_s, q, scale);
+    launch_pdl(ln_quant_kernel<T, E>, dim3((unsigned)grid), dim3(threads), 0, st, (const T *)h, M, K, gamma, beta, eps,
+               inv_s, q, scale);
 }
 
 // E elements per thread: one warp per row up to K = 1024, then 32 elements
