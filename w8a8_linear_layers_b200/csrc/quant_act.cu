@@ -164,26 +164,26 @@ quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__r
         Raw8<T> nxt[ROWS][C];  // the next rows of this CTA, loading while these are quantized
         load_rows(nxt, row0 + rstride);
         float amax[ROWS];  // dynamic: the row's abs-max; static: this thread's
+        float v[ROWS][C][8];  // x * inv_s of these rows, kept for the codes
 #pragma unroll
         for (int rr = 0; rr < ROWS; ++rr) {
             amax[rr] = 0.0f;
 #pragma unroll
             for (int c = 0; c < C; ++c) {
-                float v[8];
 #ifdef W8A8_DEBUG
-                raw[rr][c].widen(v);
-                dbg_check8(v);  // the input itself (zeros past the row)
+                raw[rr][c].widen(v[rr][c]);
+                dbg_check8(v[rr][c]);  // the input itself (zeros past the row)
 #endif
-                scaled(raw[rr][c], c, v);
+                scaled(raw[rr][c], c, v[rr][c]);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) amax[rr] = fmaxf(amax[rr], fabsf(v[i]));
+                for (int i = 0; i < 8; i += 2) amax[rr] = fmax3(amax[rr], fabsf(v[rr][c][i]), fabsf(v[rr][c][i + 1]));
             }
             if (!STATIC) {
                 amax[rr] = warp_max(amax[rr]);
-                if (lane == 0) red[parity][rr][warp] = amax[rr];
+                if (nwarps > 1 && lane == 0) red[parity][rr][warp] = amax[rr];
             }
         }
-        if (!STATIC) __syncthreads();  // red[parity] complete; red[parity^1] free for the next rows
+        if (!STATIC && nwarps > 1) __syncthreads();  // red[parity] complete; red[parity^1] free for the next rows
 #pragma unroll
         for (int rr = 0; rr < ROWS; ++rr) {
             const int64_t row = row0 + rr;
@@ -193,8 +193,10 @@ quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__r
                 s = __fdiv_rn(__ldg(range), 127.0f);
                 if (scale && threadIdx.x == 0) scale[row] = s;
             } else {
-                am = red[parity][rr][0];
-                for (int w = 1; w < nwarps; ++w) am = fmaxf(am, red[parity][rr][w]);
+                if (nwarps > 1) {  // (one warp: its butterfly already holds the row's abs-max)
+                    am = red[parity][rr][0];
+                    for (int w = 1; w < nwarps; ++w) am = fmaxf(am, red[parity][rr][w]);
+                }
                 s = __fdiv_rn(am, 127.0f);
                 if (threadIdx.x == 0) scale[row] = s;
             }
@@ -211,18 +213,17 @@ quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__r
 #pragma unroll
             for (int c = 0; c < C; ++c) {
                 if (!live[c]) continue;
-                float v[8];
-                scaled(raw[rr][c], c, v);
+                const float(&vc)[8] = v[rr][c];
                 uint2 code = make_uint2(0u, 0u);
                 if (s == 0.0f) {
                     // all-zero row: every code is 0
                 } else if (exact_only) {
                     int e[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) e[i] = (int)sym_code(v[i], s, r, 127.0f, true);
+                    for (int i = 0; i < 8; ++i) e[i] = (int)sym_code(vc[i], s, r, 127.0f, true);
                     code = pack8_codes(e);
                 } else {
-                    code = fast_codes_tied<!STATIC>(v, s, r, narrow, tie_bound);
+                    code = fast_codes_tied<!STATIC>(vc, s, r, narrow, tie_bound);
                 }
                 *reinterpret_cast<uint2 *>(qr + ((int64_t)c * T_ + threadIdx.x) * 8) = code;
                 if (rowsum) rsum = __dp4a((int)code.y, 0x01010101, __dp4a((int)code.x, 0x01010101, rsum));
