@@ -161,8 +161,6 @@ quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__r
     Raw8<T> raw[ROWS][C];
     if ((int64_t)blockIdx.x * ROWS < M) load_rows(raw, (int64_t)blockIdx.x * ROWS);
     for (int64_t row0 = (int64_t)blockIdx.x * ROWS; row0 < M; row0 += rstride, parity ^= 1) {
-        Raw8<T> nxt[ROWS][C];  // the next rows of this CTA, loading while these are quantized
-        load_rows(nxt, row0 + rstride);
         float amax[ROWS];  // dynamic: the row's abs-max; static: this thread's
         float v[ROWS][C][8];  // x * inv_s of these rows, kept for the codes
 #pragma unroll
@@ -183,6 +181,9 @@ quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__r
                 if (nwarps > 1 && lane == 0) red[parity][rr][warp] = amax[rr];
             }
         }
+        // these rows now live in v: the registers take the CTA's next rows,
+        // which load while these are reduced and quantized
+        load_rows(raw, row0 + rstride);
         if (!STATIC && nwarps > 1) __syncthreads();  // red[parity] complete; red[parity^1] free for the next rows
 #pragma unroll
         for (int rr = 0; rr < ROWS; ++rr) {
@@ -244,10 +245,6 @@ quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__r
                 }
             }
         }
-#pragma unroll
-        for (int rr = 0; rr < ROWS; ++rr)
-#pragma unroll
-            for (int c = 0; c < C; ++c) raw[rr][c] = nxt[rr][c];
     }
 }
 
