@@ -22,13 +22,13 @@
 //
 // Design.  One CTA of R warps per output channel; the row stays resident in
 // shared memory for the whole search (W is read from HBM once, the codes
-// written once), next to one buffer of kept codes: a candidate that is not
-// kept ends the search, so a round writes its codes over the kept ones and
-// the chunks it touched are restored in that one case.  A bf16 row is kept
-// as loaded (2 bytes an element) and folded again, fl(w s_j) with the same
-// single fp32 rounding, wherever it is read (s through L1); an fp32 row is
-// kept folded.  At K = 4096 a channel then takes 12 KB instead of 20, and up
-// to 16 channels (32 warps) fit on an SM.
+// written once), next to two code buffers: a round writes the candidate's
+// codes into one while the kept codes stay in the other, and a kept
+// candidate swaps them (the moved chunks' change of NUM and DEN reads both,
+// with no code computed twice).  A bf16 row is kept as loaded (2 bytes an
+// element) and folded again, fl(w s_j) with the same single fp32 rounding,
+// wherever it is read (s through L1); an fp32 row is kept folded.  At
+// K = 4096 a channel takes 16 KB.
 //
 // The error is evaluated exactly instead of by a per-element fp64 sum:
 //     K e(c) = W2 - 2 c NUM + c^2 DEN,  W2 = sum w^2, NUM = sum w q, DEN = sum q^2,
@@ -96,7 +96,6 @@ struct PassOut {
     double dnum;     // update: change of NUM (exact products, fp64 sum)
     int den;         // init: DEN; update: change of DEN
     bool moved;      // update: some code of this thread changed
-    uint32_t touched;  // update: chunks whose codes were rewritten (moved or near a tie)
 };
 
 // The channel's row in shared memory, read as folded fp32 values.  fp32
@@ -149,24 +148,17 @@ template <bool FOLD> struct Row<__nv_bfloat16, FOLD> {
     }
 };
 
-// Fast codes of the chunk at j for scale 1/r (see fast_codes8); dmax as there.
-template <bool NARROW, typename R>
-__device__ __forceinline__ uint2 chunk_codes(const R &row, int j, float r, float lo, float hi,
-                                             uint32_t lo2, uint32_t hi2, float &dmax) {
-    float4 a, b;
-    row.load8(j, a, b);
-    return fast_codes8<NARROW>(a, b, r, lo, hi, lo2, hi2, dmax);
-}
-
 // Main loop of a pass over this thread's chunks.  init: writes the codes
-// into q and accumulates W2, NUM, DEN.  update: only compares the codes at
-// the candidate with the kept codes in q and marks the chunks that moved;
-// they are rewritten afterwards, once (a warp would otherwise run the update
-// path whenever any lane had a moved chunk).  Both mark near-tie chunks.
+// into q and accumulates W2, NUM, DEN.  update: writes the codes at the
+// candidate into qc, compares them with the kept codes in q and marks the
+// chunks that moved; their change of NUM and DEN is taken afterwards, once
+// (a warp would otherwise run that path whenever any lane had a moved
+// chunk).  Both mark near-tie chunks.
 template <bool INIT, bool NARROW, typename R>
 __device__ __forceinline__ void pass_chunks(const R &row, int K, float r, float lo, float hi,
                                             uint32_t lo2, uint32_t hi2, float tie_bound, int8_t *__restrict__ q,
-                                            PassOut &out, uint32_t &moved, uint32_t &tie) {
+                                            int8_t *__restrict__ qc, PassOut &out, uint32_t &moved,
+                                            uint32_t &tie) {
     const int stride = blockDim.x * 8;
     int m = 0;
 #pragma unroll 2
@@ -188,14 +180,15 @@ __device__ __forceinline__ void pass_chunks(const R &row, int K, float r, float 
                 out.den += qq * qq;
             }
         } else {
+            *reinterpret_cast<uint2 *>(qc + j) = nw;
             const uint2 od = *reinterpret_cast<const uint2 *>(q + j);
             if ((nw.x ^ od.x) | (nw.y ^ od.y)) moved |= 1u << m;
         }
     }
 }
 
-// Moved chunks: the change of NUM and DEN, and the new codes written over
-// the kept ones.
+// Moved chunks: the change of NUM and DEN from the kept codes (q) to the
+// candidate's (qc).
 // The change of DEN for a chunk whose codes go from od to nw (exact: dp4a
 // of the signed bytes).
 __device__ __forceinline__ int den_change(uint2 nw, uint2 od) {
@@ -203,17 +196,15 @@ __device__ __forceinline__ int den_change(uint2 nw, uint2 od) {
            __dp4a((int)od.x, (int)od.x, __dp4a((int)od.y, (int)od.y, 0));
 }
 
-template <bool NARROW, typename R>
-__device__ __forceinline__ void rewrite_moved(const R &row, uint32_t moved, float r, float lo,
-                                              float hi, uint32_t lo2, uint32_t hi2, int8_t *__restrict__ q,
-                                              PassOut &out) {
+template <typename R>
+__device__ __forceinline__ void sum_moved(const R &row, uint32_t moved, const int8_t *__restrict__ q,
+                                          const int8_t *__restrict__ qc, PassOut &out) {
     const int stride = blockDim.x * 8;
     while (moved) {
         const int mm = __ffs(moved) - 1;
         moved &= moved - 1u;
         const int j = threadIdx.x * 8 + mm * stride;
-        float dmax = 0.0f;
-        const uint2 nw = chunk_codes<NARROW>(row, j, r, lo, hi, lo2, hi2, dmax);
+        const uint2 nw = *reinterpret_cast<const uint2 *>(qc + j);
         const uint2 od = *reinterpret_cast<const uint2 *>(q + j);
         out.den += den_change(nw, od);
         // only the bytes that differ: 0x80 marks each
@@ -224,7 +215,6 @@ __device__ __forceinline__ void rewrite_moved(const R &row, uint32_t moved, floa
             d &= d - 1ull;
             out.dnum += (double)row.load1(j + i) * code_to_f64(code_byte(nw, i) - code_byte(od, i));  // exact product
         }
-        *reinterpret_cast<uint2 *>(q + j) = nw;
     }
 }
 
@@ -287,52 +277,29 @@ __device__ __forceinline__ ScaleConsts scale_consts(float c, float qmax, float w
     return k;
 }
 
-// One pass at scale c over this thread's chunks of the row in shared memory,
-// against the codes in q (one buffer).  init: q receives the codes at c and
-// W2, NUM, DEN are accumulated.  update: the codes at c are written over q
-// where they differ and the change of NUM and DEN is returned; `touched`
-// names the chunks rewritten, so that the kept codes can be restored if c
-// is rejected.  wmax is the thread's max |w|.  Called by whole warps.
+// One pass at scale c over this thread's chunks of the row in shared memory.
+// init: q receives the codes at c and W2, NUM, DEN are accumulated.  update:
+// qc receives the codes at c (q keeps the kept codes) and the change of NUM
+// and DEN from q to qc is returned; if c is kept the caller swaps the two
+// buffers, if not q still holds the kept codes.  wmax is the thread's max
+// |w|.  Called by whole warps.
 template <bool INIT, typename R>
 __device__ __forceinline__ PassOut row_pass(const R &row, int K, float c, float qmax, float wmax,
-                                            int8_t *__restrict__ q) {
+                                            int8_t *__restrict__ q, int8_t *__restrict__ qc) {
     const ScaleConsts k = scale_consts(c, qmax, wmax);
-    PassOut out = {{0.0, 0.0}, {0.0, 0.0}, 0.0, 0, false, 0u};
+    PassOut out = {{0.0, 0.0}, {0.0, 0.0}, 0.0, 0, false};
     uint32_t moved = 0u;  // bit m: chunk m of this thread moved (at most 32 chunks per thread)
     uint32_t tie = 0u;    // bit m: chunk m holds an element near a rounding tie
     if (k.narrow)
-        pass_chunks<INIT, true>(row, K, k.r, k.lo, k.hi, k.lo2, k.hi2, k.tie_bound, q, out, moved, tie);
+        pass_chunks<INIT, true>(row, K, k.r, k.lo, k.hi, k.lo2, k.hi2, k.tie_bound, q, qc, out, moved, tie);
     else
-        pass_chunks<INIT, false>(row, K, k.r, k.lo, k.hi, k.lo2, k.hi2, k.tie_bound, q, out, moved, tie);
+        pass_chunks<INIT, false>(row, K, k.r, k.lo, k.hi, k.lo2, k.hi2, k.tie_bound, q, qc, out, moved, tie);
     if (!INIT) {
         out.moved = moved != 0u;
-        out.touched = moved | tie;
-        if (k.narrow) rewrite_moved<true>(row, moved, k.r, k.lo, k.hi, k.lo2, k.hi2, q, out);
-        else rewrite_moved<false>(row, moved, k.r, k.lo, k.hi, k.lo2, k.hi2, q, out);
+        sum_moved(row, moved, q, qc, out);
     }
-    fix_ties<INIT ? 1 : 2>(row, tie, c, k.r, qmax, q, out);
+    fix_ties<INIT ? 1 : 2>(row, tie, c, k.r, qmax, INIT ? q : qc, out);
     return out;
-}
-
-// Writes the exact codes at scale c over the chunks named in `touched`.
-template <typename R>
-__device__ __forceinline__ void restore_chunks(const R &row, uint32_t touched, float c,
-                                               float qmax, float wmax, int8_t *__restrict__ q) {
-    const ScaleConsts k = scale_consts(c, qmax, wmax);
-    const int stride = blockDim.x * 8;
-    uint32_t tie = 0u;
-    for (uint32_t t = touched; t;) {
-        const int mm = __ffs(t) - 1;
-        t &= t - 1u;
-        const int j = threadIdx.x * 8 + mm * stride;
-        float dmax = 0.0f;
-        const uint2 nw = k.narrow ? chunk_codes<true>(row, j, k.r, k.lo, k.hi, k.lo2, k.hi2, dmax)
-                                  : chunk_codes<false>(row, j, k.r, k.lo, k.hi, k.lo2, k.hi2, dmax);
-        if (dmax >= k.tie_bound) tie |= 1u << mm;
-        *reinterpret_cast<uint2 *>(q + j) = nw;
-    }
-    PassOut unused;
-    fix_ties<0>(row, tie, c, k.r, qmax, q, unused);
 }
 
 struct WarpPart {
@@ -341,6 +308,13 @@ struct WarpPart {
 };
 
 
+// Dynamic shared memory: the row (K elements, bf16 raw or fp32 folded), two
+// code buffers (K bytes each), then the per-warp partials of two rounds
+// (8-byte aligned).
+__host__ __device__ __forceinline__ size_t ssz_parts_offset(int K, size_t elem) {
+    return ((size_t)K * elem + 2 * (size_t)K + 7) & ~(size_t)7;
+}
+
 template <typename T, bool FOLD>
 __global__ void __launch_bounds__(512, 2)
 ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__ s, float qmax, int max_iters,
@@ -348,7 +322,12 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
            int32_t *__restrict__ iters_out) {
     extern __shared__ __align__(16) uint8_t smem[];
     T *wrow = reinterpret_cast<T *>(smem);                     // K elements: the row (see Row)
-    int8_t *q = reinterpret_cast<int8_t *>(smem) + (size_t)K * sizeof(T);  // K codes: the kept codes
+    // two code buffers of K bytes: the kept codes (q) and a round's candidate
+    // codes (qc), swapped when the candidate is kept; then the per-warp
+    // partials of two rounds
+    int8_t *q = reinterpret_cast<int8_t *>(smem) + (size_t)K * sizeof(T);
+    int8_t *qc = q + K;
+    WarpPart *parts = reinterpret_cast<WarpPart *>(smem + ssz_parts_offset(K, sizeof(T)));
     Row<T, FOLD> row;
     if constexpr (sizeof(T) == 2) {
         row.w = reinterpret_cast<const uint16_t *>(wrow);
@@ -356,12 +335,11 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
     } else {
         row.w = reinterpret_cast<const float *>(wrow);
     }
-    __shared__ WarpPart part[2][16];
     struct Decision {
         float c_next;
         int keep, done;
     };
-    __shared__ Decision decision[2];  // warp 0's decision of a round, by parity                          // per-warp partials, by round parity
+    __shared__ Decision decision[2];  // warp 0's decision of a round, by parity
     __shared__ float redmax[16];
     const int T_ = blockDim.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = T_ >> 5;
@@ -408,36 +386,33 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
         float s_best = fmaxf(__fdiv_rn(amax, qmax), kSszMinScale);
         int par = 0;
         {
-            PassOut p = row_pass<true>(row, K, s_best, qmax, wmax, q);
+            PassOut p = row_pass<true>(row, K, s_best, qmax, wmax, q, qc);
             p.num = warp_sum_dd(p.num);
             p.w2 = warp_sum_dd(p.w2);
             p.den = warp_sum_i(p.den);
-            if (lane == 0) part[par][warp] = {p.num, p.w2, p.den};
+            if (lane == 0) parts[par * nwarps + warp] = {p.num, p.w2, p.den};
         }
         __syncthreads();
         // every thread holds the (identical) channel state
-        dd W2 = part[par][0].w2, NUM = part[par][0].num;
-        int DEN = part[par][0].den;
+        dd W2 = parts[par * nwarps].w2, NUM = parts[par * nwarps].num;
+        int DEN = parts[par * nwarps].den;
         for (int i = 1; i < nwarps; ++i) {
-            W2 = dd_add_cascade(W2, part[par][i].w2);
-            NUM = dd_add_cascade(NUM, part[par][i].num);
-            DEN += part[par][i].den;
+            W2 = dd_add_cascade(W2, parts[par * nwarps + i].w2);
+            NUM = dd_add_cascade(NUM, parts[par * nwarps + i].num);
+            DEN += parts[par * nwarps + i].den;
         }
         double m_best = exact_error_k(W2, NUM, DEN, s_best);  // K x error
         float c = ls_candidate(NUM, DEN, s_best);
         int it = 0;
         bool done = max_iters == 0;
-        uint32_t touched = 0u;  // this thread's chunks rewritten by the last round
-        bool rejected = false;  // the last round's candidate was not kept
 
-        // ---- least-squares rounds.  A round whose candidate is not kept
-        // ends the search (its improvement is <= 0, below both thresholds),
-        // so the candidate's codes can be written over the kept ones and the
-        // touched chunks restored in that one case.
+        // ---- least-squares rounds.  A round writes its candidate codes into
+        // qc; a kept candidate swaps the buffers, a rejected one (which ends
+        // the search: its improvement is <= 0, below both thresholds) leaves
+        // the kept codes in q.
         while (!done) {
             par ^= 1;
-            PassOut p = row_pass<false>(row, K, c, qmax, wmax, q);
-            touched = p.touched;
+            PassOut p = row_pass<false>(row, K, c, qmax, wmax, q, qc);
             if (__any_sync(0xffffffffu, p.moved)) {
                 p.dnum = warp_sum_d(p.dnum);
                 p.den = warp_sum_i(p.den);
@@ -445,7 +420,7 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
                 p.dnum = 0.0;
                 p.den = 0;
             }
-            if (lane == 0) part[par][warp] = {{p.dnum, 0.0}, {0.0, 0.0}, p.den};
+            if (lane == 0) parts[par * nwarps + warp] = {{p.dnum, 0.0}, {0.0, 0.0}, p.den};
             __syncthreads();  // the candidate codes and all partials are in place
             ++it;
             // The decision: every thread takes it (1-2 warps a channel), or
@@ -456,8 +431,8 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
                 dd num_c = NUM;
                 int den_c = DEN;
                 for (int i = 0; i < nwarps; ++i) {
-                    dd_acc(num_c, part[par][i].num.hi);
-                    den_c += part[par][i].den;
+                    dd_acc(num_c, parts[par * nwarps + i].num.hi);
+                    den_c += parts[par * nwarps + i].den;
                 }
                 const double m_c = exact_error_k(W2, num_c, den_c, c);
                 const float c_next = ls_candidate(num_c, den_c, c);  // used only if c is kept
@@ -471,7 +446,7 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
                     NUM = num_c;
                     DEN = den_c;
                 } else {
-                    dn = true;  // implied by the tests above (m_best >= 0); stated for the restore below
+                    dn = true;  // implied by the tests above (m_best >= 0); q keeps the kept codes
                 }
                 if (shared_decision) {
                     if (lane == 0) decision[par] = {c_next, keep ? 1 : 0, dn ? 1 : 0};
@@ -480,8 +455,9 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
                     if (keep) {
                         s_best = c;
                         c = c_next;
-                    } else {
-                        rejected = true;
+                        int8_t *t = q;  // the candidate's codes become the kept ones
+                        q = qc;
+                        qc = t;
                     }
                 }
             }
@@ -492,14 +468,14 @@ ssz_kernel(const T *__restrict__ wg, int64_t N, int K, const float *__restrict__
                 if (dcs.keep) {
                     s_best = c;
                     c = dcs.c_next;
-                } else {
-                    rejected = true;
+                    int8_t *t = q;  // the candidate's codes become the kept ones
+                    q = qc;
+                    qc = t;
                 }
             }
             // part[par] and decision[par] are rewritten two rounds from now,
             // after another barrier
         }
-        if (rejected) restore_chunks(row, touched, s_best, qmax, wmax, q);
 
         // ---- kept codes out (each thread wrote and now reads its own chunks)
         for (int j = threadIdx.x * 8; j < K; j += T_ * 8)
@@ -531,7 +507,7 @@ static sq_status launch_ssz(const void *w, int64_t N, int64_t K, const float *s,
                             int8_t *q, float *scale, double *mse, int32_t *iters, int sms, cudaStream_t st) {
     const int threads = 32 * ssz_warps(K);
     const float qmax = (float)((1 << (bits - 1)) - 1);
-    const size_t smem = (size_t)K * (sizeof(T) + 1);  // the row (bf16 raw or fp32 folded) + codes
+    const size_t smem = ssz_parts_offset((int)K, sizeof(T)) + sizeof(WarpPart) * 2 * (threads / 32);
     auto kern = s ? ssz_kernel<T, true> : ssz_kernel<T, false>;
     if (smem > 32 * 1024) {  // dynamic + static shared memory may pass the 48 KB default
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
