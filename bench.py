@@ -313,8 +313,8 @@ def run_ours(args, rank, world, local_rank):
     if w.device_fault() != 0:
         raise RuntimeError("a kernel gave up on a bounded wait during warm-up")
 
-    # One GPU: the step is captured once as a CUDA graph (its per-kernel
-    # events included) and replayed every timed step, so that the host's
+    # One GPU: the step is captured once as a CUDA graph (its events
+    # included) and replayed every timed step, so that the host's
     # launch of some 5 calls per linear never holds the GPU back.  Several
     # ranks launch eagerly (no collective is captured).
     graph = None
