@@ -331,6 +331,11 @@ ln_quant_kernel(const T *__restrict__ h, int64_t M, int64_t K, const float *__re
         }
     }
     const double kd = (double)K;
+    // S / K: a power-of-two K scales exactly (the same correctly rounded value
+    // as the division), any other K divides
+    const bool k_pow2 = (K & (K - 1)) == 0;
+    const double inv_kd = 1.0 / kd;
+    auto over_k = [&](double sum) { return k_pow2 ? sum * inv_kd : sum / kd; };
     auto load_row = [&](Raw8<T> (&dst)[C], int64_t r) {
 #pragma unroll
         for (int c = 0; c < C; ++c) {
@@ -358,7 +363,7 @@ ln_quant_kernel(const T *__restrict__ h, int64_t M, int64_t K, const float *__re
         }
         double tsum = part[0];
         if (C == 2) tsum = part[0] + part[C - 1];
-        const double mu = block_tree_sum(tsum, redd[par][0], lane, warp, nwarps) / kd;
+        const double mu = over_k(block_tree_sum(tsum, redd[par][0], lane, warp, nwarps));
 #pragma unroll
         for (int c = 0; c < C; ++c) {
             float v[8];
@@ -373,7 +378,7 @@ ln_quant_kernel(const T *__restrict__ h, int64_t M, int64_t K, const float *__re
         }
         tsum = part[0];
         if (C == 2) tsum = part[0] + part[C - 1];
-        const double var = block_tree_sum(tsum, redd[par][1], lane, warp, nwarps) / kd;
+        const double var = over_k(block_tree_sum(tsum, redd[par][1], lane, warp, nwarps));
         const double rstd = 1.0 / sqrt(var + (double)eps);
         const float m32 = (float)mu, r32 = (float)rstd;
         // x' = ((h - m) r) gamma + beta, times inv_s, each op in fp32
@@ -394,8 +399,7 @@ ln_quant_kernel(const T *__restrict__ h, int64_t M, int64_t K, const float *__re
         amax = warp_max(amax);
         if (lane == 0) redf[par][warp] = amax;
         __syncthreads();
-        float am = redf[par][0];
-        for (int w = 1; w < nwarps; ++w) am = fmaxf(am, redf[par][w]);
+        const float am = warp_max(lane < nwarps ? redf[par][lane] : 0.0f);
         const float s = __fdiv_rn(am, 127.0f);
         if (threadIdx.x == 0) scale[row] = s;
         const float r = __fdiv_rn(1.0f, s);
