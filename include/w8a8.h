@@ -13,7 +13,12 @@
  *    unless stated otherwise.  The library keeps no pointer after a call
  *    returns and allocates no device memory.
  *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
- *    the legacy default stream).  Nothing synchronizes the host.
+ *    the legacy default stream).  Nothing synchronizes the host.  The
+ *    per-token quantization kernels and the GEMMs are launched with
+ *    programmatic stream serialization: they may be scheduled while the
+ *    previous kernel on the stream is finishing, but wait for it to
+ *    complete before reading or writing any memory, so stream order holds
+ *    as for an ordinary launch.
  *  - K must be a positive multiple of 16; M and N may be 0 (nothing is done)
  *    or any positive size.  Matrix base pointers must be 16-byte aligned and
  *    vector pointers 4-byte aligned (8-byte for fp64 outputs).
