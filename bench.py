@@ -597,75 +597,37 @@ def run_e2e(args, w, wdist, torch, probs, forward, flush, stream, ops_per_step, 
     activations from pinned host memory, quantizes them, runs the GEMM and
     copies the output back, all inside the timed events; the quantized
     weights (the layers' parameters) stay resident on the device.  The
-    tokens are cut into chunks (M / E2E_CHUNKS rows, within [256,
-    E2E_CHUNK_ROWS]; per-token codes and the GEMM are row-independent) that
-    flow through three streams: the
-    host->device copy of one chunk, the codes + GEMM of the previous one and
-    the device->host copy of the one before run at once, on the two copy
-    engines and the SMs, through E2E_SLOTS device buffers in rotation."""
+    library's HostStreamer cuts the tokens into chunks (M / E2E_CHUNKS rows,
+    within [256, E2E_CHUNK_ROWS]) whose copy in, codes + GEMM and copy out
+    overlap on three streams through E2E_SLOTS device buffers."""
     hosts = [(p.x.cpu().pin_memory(), torch.empty_like(p.y, device="cpu").pin_memory()) for p in probs]
     dev = probs[0].x.device
-    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     M_max = max(p.M for p in probs)
     R = max(256, min(E2E_CHUNK_ROWS, -(-M_max // E2E_CHUNKS)))
-    K_max = max(p.K for p in probs)
-    N_max = max(p.N for p in probs)
-    xdt, ydt = probs[0].x.dtype, probs[0].y.dtype
-    slots = [dict(x=torch.empty(R * K_max, device=dev, dtype=xdt), qx=torch.empty(R * K_max, device=dev, dtype=torch.int8),
-                  sx=torch.empty(R, device=dev, dtype=torch.float32), y=torch.empty(R * N_max, device=dev, dtype=ydt))
-             for _ in range(E2E_SLOTS)]
-    units = [(j, r0, min(R, p.M - r0)) for j, p in enumerate(probs) for r0 in range(0, p.M, R)]
+    streamer = w.HostStreamer(dev, R, max(p.K for p in probs), max(p.N for p in probs), probs[0].x.dtype,
+                              probs[0].y.dtype, slots=E2E_SLOTS)
 
-    def chunk_forward(p, sl, r):
-        x = sl["x"][: r * p.K].view(r, p.K)
-        qx = sl["qx"][: r * p.K].view(r, p.K)
-        sx = sl["sx"][:r]
-        y = sl["y"][: r * p.N].view(r, p.N)
-        w.quant_act_per_token(x, p.inv, qx, sx)
-        if p.bits == 8:
-            w.w8a8_gemm_dequant(qx, sx, p.qw, p.sw, y)
-        else:
-            w.w4a8_gemm_dequant(qx, sx, p.qw4, p.sw, y)
-        return y
+    def chunk_fn(p):
+        def fn(x, qx, sx, y):
+            w.quant_act_per_token(x, p.inv, qx, sx)
+            if p.bits == 8:
+                w.w8a8_gemm_dequant(qx, sx, p.qw, p.sw, y)
+            else:
+                w.w4a8_gemm_dequant(qx, sx, p.qw4, p.sw, y)
+        return fn
 
+    jobs = [(xh, yh, chunk_fn(p)) for p, (xh, yh) in zip(probs, hosts)]
     e2e_ms = []
     for i in range(args.warmup + args.e2e_steps):
         flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        s_in.wait_event(e0)
-        s_out.wait_event(e0)
-        x_free = [None] * E2E_SLOTS  # event: the slot's x (and codes) no longer read
-        y_free = [None] * E2E_SLOTS  # event: the slot's y copied out
-        for k, (j, r0, r) in enumerate(units):
-            p, (xh, yh) = probs[j], hosts[j]
-            si = k % E2E_SLOTS
-            sl = slots[si]
-            with torch.cuda.stream(s_in):
-                if x_free[si] is not None:
-                    s_in.wait_event(x_free[si])
-                sl["x"][: r * p.K].view(r, p.K).copy_(xh[r0:r0 + r], non_blocking=True)
-                ev_in = torch.cuda.Event()
-                ev_in.record(s_in)
-            stream.wait_event(ev_in)
-            if y_free[si] is not None:
-                stream.wait_event(y_free[si])
-            y = chunk_forward(p, sl, r)
-            ev_c = torch.cuda.Event()
-            ev_c.record(stream)
-            x_free[si] = ev_c
-            with torch.cuda.stream(s_out):
-                s_out.wait_event(ev_c)
-                yh[r0:r0 + r].copy_(y, non_blocking=True)
-                ev_o = torch.cuda.Event()
-                ev_o.record(s_out)
-            y_free[si] = ev_o
-        stream.wait_stream(s_out)
+        streamer.run(jobs, stream)
         e1.record(stream)
         e1.synchronize()
         if i >= args.warmup:
             e2e_ms.append(e0.elapsed_time(e1))
-    # the pipeline must reproduce the resident path's output
+    # the chunked pipeline must reproduce the resident path's output
     for p, (xh, yh) in zip(probs, hosts):
         forward(p, p.x)
         if not torch.equal(yh, p.y.cpu()):
@@ -678,7 +640,7 @@ def run_e2e(args, w, wdist, torch, probs, forward, flush, stream, ops_per_step, 
             "ms_per_step": round(e2e_total / len(e2e_ms), 4), "chunk_rows": R,
             "what": "activations copied host->device from pinned memory, per-token quantization, GEMM + dequant, "
                     "output copied device->host, every step, in chunks of %d tokens whose copies in, compute and "
-                    "copies out overlap on three streams; quantized weights resident" % R}
+                    "copies out overlap on three streams (HostStreamer); quantized weights resident" % R}
 
 
 def per_shape_table(probs, lin_ms, peaks, shape_ms=None):

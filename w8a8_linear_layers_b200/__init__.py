@@ -426,21 +426,43 @@ class W8A8Linear:
         else:
             w8a8_gemm_dequant(qx, sx, self.qw, self.sw, y)
 
-    def forward(self, x: torch.Tensor, y: torch.Tensor | None = None) -> torch.Tensor:
-        M = x.shape[0]
-        qx = torch.empty(M, self.K, device=x.device, dtype=torch.int8)
-        sx = torch.empty(M, device=x.device, dtype=torch.float32)
-        rs = torch.empty(M, device=x.device, dtype=torch.int32) if self.weights == "asym8" else None
+    def _forward_into(self, x, qx, sx, rs, y) -> None:
+        """The per-inference kernels into caller buffers: codes qx [M, K],
+        scales sx [M], row sums rs [M] (asym8 only, else None), output y."""
         if self.act_scales == "static":
             if self._static_batches == 0:
                 raise RuntimeError("static activation scales need calibrate_static() first")
             quant_act_static(x, self.inv_s, self.range, qx, sx, rs)
         else:
             quant_act_per_token_rowsum(x, self.inv_s, qx, sx, rs)
+        self._gemm(qx, sx, rs, y)
+
+    def forward(self, x: torch.Tensor, y: torch.Tensor | None = None) -> torch.Tensor:
+        M = x.shape[0]
+        qx = torch.empty(M, self.K, device=x.device, dtype=torch.int8)
+        sx = torch.empty(M, device=x.device, dtype=torch.float32)
+        rs = torch.empty(M, device=x.device, dtype=torch.int32) if self.weights == "asym8" else None
         if y is None:
             y = torch.empty(M, self.N, device=x.device, dtype=self.out_dtype)
-        self._gemm(qx, sx, rs, y)
+        self._forward_into(x, qx, sx, rs, y)
         return y
+
+    def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, chunk_rows: int = 2048,
+                     streamer: "HostStreamer | None" = None) -> None:
+        """forward() on activations in pinned host memory: y_host [M, N]
+        (pinned, out_dtype) receives the output, the copies in and out
+        overlapped with the kernels chunk by chunk (HostStreamer; pass one
+        to reuse its device buffers).  Returns once enqueued: synchronize the
+        current stream before reading y_host."""
+        st = streamer or HostStreamer(self.w.device, chunk_rows, self.K, self.N, x_host.dtype, self.out_dtype)
+        # the kernels of all chunks run in order on one stream, so one
+        # row-sum buffer serves them all
+        rs = torch.empty(st.rows, device=self.w.device, dtype=torch.int32) if self.weights == "asym8" else None
+
+        def fn(x, qx, sx, y):
+            self._forward_into(x, qx, sx, None if rs is None else rs[: x.shape[0]], y)
+
+        st.run([(x_host, y_host, fn)])
 
     def graphed(self, M: int, x_dtype: torch.dtype | None = None) -> "GraphedLinear":
         """forward() for M-token inputs captured in a CUDA graph (see
@@ -486,3 +508,6 @@ class GraphedLinear:
     def replay(self) -> torch.Tensor:
         self.graph.replay()
         return self.y
+
+
+from .host import HostStreamer  # noqa: E402  (pinned-host linears with overlapped copies)
