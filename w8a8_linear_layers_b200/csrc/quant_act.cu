@@ -56,13 +56,25 @@ template <> struct Raw8<float> {
 constexpr float kLo = kRoundMagic - 127.0f, kHi = kRoundMagic + 127.0f;
 constexpr uint32_t kLo2 = 0xFF81FF81u, kHi2 = 0x007F007Fu;
 
-// Codes of 8 scaled elements at scale s (r = 1/s): packed fast path, then
-// the exact quotient for any element near a rounding tie (rare).
+// r = 1/s to within one ulp (rcp.approx; a subnormal s is flushed to 0 and
+// gives r = inf, which sends the row to the exact path).  The fast codes'
+// tie test flags every element within |y| 2^-21 + 2^-22 of a half-integer
+// and so allows v r to be off the exact quotient by up to 2^-21 |y|: an
+// exactly rounded r needs 2^-23 |y| (its own rounding and the quotient's),
+// one ulp more 1.5 2^-23 |y|, still inside.  The codes stay exact.
+__device__ __forceinline__ float approx_rcp(float s) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s));
+    return r;
+}
+
+// Codes of 8 scaled elements at scale s (r ~ 1/s, see approx_rcp): packed
+// fast path, then the exact quotient for any element near a rounding tie
+// (rare).
 // IN_RANGE: s and r come from this row's own abs-max am (s = am / 127,
-// r = 1 / s, r finite), so no code needs the clamp: every |v| r <= am r <
-// 127 (1 + 2^-22) once r is finite (s >= 2^-128: the relative error of s
-// is at most 2^-22 even where s is subnormal, and a smaller s makes r
-// overflow), so rint(v r) is within [-127, 127].
+// r ~ 1 / s finite, so s is normal), so no code needs the clamp: every
+// |v| r <= am r < 127 (1 + 2^-24)(1 + 2^-23)^2 < 127.5, so rint(v r) is
+// within [-127, 127].
 template <bool IN_RANGE>
 __device__ __forceinline__ uint2 fast_codes_tied(const float (&v)[8], float s, float r, bool narrow,
                                                  float tie_bound) {
@@ -201,7 +213,7 @@ quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__r
                 s = __fdiv_rn(am, 127.0f);
                 if (threadIdx.x == 0) scale[row] = s;
             }
-            const float r = __fdiv_rn(1.0f, s);
+            const float r = approx_rcp(s);
             const bool exact_only = !(fabsf(r) <= 3.402823466e38f);  // 1/s overflowed (or s == 0)
             // |v r| <= am r (about 127 in the dynamic case): below 2^14 the
             // int16 clamp of fast_codes8 applies; a fast code can differ from
@@ -211,23 +223,28 @@ quant_act_kernel(const T *__restrict__ x, int64_t M, int64_t K, const float *__r
             const float tie_bound = 0.5f - fmaf(am * r, 4.76837158203125e-07f, 2.384185791015625e-07f);
             int8_t *qr = q + row * K;
             int rsum = 0;
+            if (s != 0.0f && !exact_only) {  // the usual row: fast codes
 #pragma unroll
-            for (int c = 0; c < C; ++c) {
-                if (!live[c]) continue;
-                const float(&vc)[8] = v[rr][c];
-                uint2 code = make_uint2(0u, 0u);
-                if (s == 0.0f) {
-                    // all-zero row: every code is 0
-                } else if (exact_only) {
-                    int e[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) e[i] = (int)sym_code(vc[i], s, r, 127.0f, true);
-                    code = pack8_codes(e);
-                } else {
-                    code = fast_codes_tied<!STATIC>(vc, s, r, narrow, tie_bound);
+                for (int c = 0; c < C; ++c) {
+                    if (!live[c]) continue;
+                    const uint2 code = fast_codes_tied<!STATIC>(v[rr][c], s, r, narrow, tie_bound);
+                    *reinterpret_cast<uint2 *>(qr + ((int64_t)c * T_ + threadIdx.x) * 8) = code;
+                    if (rowsum) rsum = __dp4a((int)code.y, 0x01010101, __dp4a((int)code.x, 0x01010101, rsum));
                 }
-                *reinterpret_cast<uint2 *>(qr + ((int64_t)c * T_ + threadIdx.x) * 8) = code;
-                if (rowsum) rsum = __dp4a((int)code.y, 0x01010101, __dp4a((int)code.x, 0x01010101, rsum));
+            } else {  // an all-zero row (every code 0), or 1/s not finite: exact quotients
+#pragma unroll
+                for (int c = 0; c < C; ++c) {
+                    if (!live[c]) continue;
+                    uint2 code = make_uint2(0u, 0u);
+                    if (s != 0.0f) {
+                        int e[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) e[i] = (int)sym_code(v[rr][c][i], s, r, 127.0f, true);
+                        code = pack8_codes(e);
+                    }
+                    *reinterpret_cast<uint2 *>(qr + ((int64_t)c * T_ + threadIdx.x) * 8) = code;
+                    if (rowsum) rsum = __dp4a((int)code.y, 0x01010101, __dp4a((int)code.x, 0x01010101, rsum));
+                }
             }
             if (rowsum) {  // uniform: every thread of the CTA takes this branch
 #pragma unroll
@@ -402,7 +419,7 @@ ln_quant_kernel(const T *__restrict__ h, int64_t M, int64_t K, const float *__re
         const float am = warp_max(lane < nwarps ? redf[par][lane] : 0.0f);
         const float s = __fdiv_rn(am, 127.0f);
         if (threadIdx.x == 0) scale[row] = s;
-        const float r = __fdiv_rn(1.0f, s);
+        const float r = approx_rcp(s);
         const bool exact_only = !(fabsf(r) <= 3.402823466e38f);
         const bool narrow = am * r < 16384.0f;
         const float tie_bound = 0.5f - fmaf(am * r, 4.76837158203125e-07f, 2.384185791015625e-07f);
