@@ -592,6 +592,11 @@ E2E_CHUNKS = 4         # at least this many chunks a linear where its rows allow
 E2E_SLOTS = 3          # device buffers in rotation: one filling, one computing, one draining
 
 
+def e2e_chunk_rows(M):
+    """Rows of an end-to-end transfer chunk for linears of up to M tokens."""
+    return max(256, min(E2E_CHUNK_ROWS, -(-M // E2E_CHUNKS)))
+
+
 def run_e2e(args, w, wdist, torch, probs, forward, flush, stream, ops_per_step, world):
     """The per-inference linears end to end: every step copies the
     activations from pinned host memory, quantizes them, runs the GEMM and
@@ -602,8 +607,7 @@ def run_e2e(args, w, wdist, torch, probs, forward, flush, stream, ops_per_step, 
     overlap on three streams through E2E_SLOTS device buffers."""
     hosts = [(p.x.cpu().pin_memory(), torch.empty_like(p.y, device="cpu").pin_memory()) for p in probs]
     dev = probs[0].x.device
-    M_max = max(p.M for p in probs)
-    R = max(256, min(E2E_CHUNK_ROWS, -(-M_max // E2E_CHUNKS)))
+    R = e2e_chunk_rows(max(p.M for p in probs))
     streamer = w.HostStreamer(dev, R, max(p.K for p in probs), max(p.N for p in probs), probs[0].x.dtype,
                               probs[0].y.dtype, slots=E2E_SLOTS)
 

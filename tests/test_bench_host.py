@@ -49,6 +49,26 @@ def test_per_shape_table_groups_linears_by_shape(bench):
     assert qkv["linear_tops"] == pytest.approx(round(2 * 8192 * 1024 * 3072 / 40e-6 / 1e12, 1))
 
 
+def test_per_shape_linear_time_comes_from_the_group_timing(bench):
+    """With the shape groups timed back to back (shape_ms: ms a linear), the
+    linear's TOPS uses that time, not the per-kernel sum (which carries the
+    event nodes' latency)."""
+    probs = [SimpleNamespace(M=8192, K=1024, N=1024)] * 2
+    lin = [[0.0, 0.0, 0.0, 0.0, 0.012, 0.018]] * 2
+    t = bench.per_shape_table(probs, lin, {"bf16_tflops": 1000.0}, {"8192x1024->1024": 0.020})
+    row = t["8192x1024->1024"]
+    assert row["linear_tops"] == pytest.approx(round(2 * 8192 * 1024 * 1024 / 20e-6 / 1e12, 1))
+    assert row["gemm_tops"] == pytest.approx(round(2 * 8192 * 1024 * 1024 / 18e-6 / 1e12, 1))
+
+
+def test_e2e_chunks(bench):
+    """The end-to-end chunks: about four a linear, 256 to 2048 rows each."""
+    assert bench.e2e_chunk_rows(8192) == 2048 and bench.e2e_chunk_rows(2048) == 512
+    assert bench.e2e_chunk_rows(16) == 256 and bench.e2e_chunk_rows(1000) == 256
+    assert bench.e2e_chunk_rows(1 << 20) == 2048
+    assert bench.E2E_SLOTS >= 2
+
+
 def test_default_workload_is_the_mlp_up_projection(bench):
     assert bench.DEFAULT_WORKLOAD == "mlp_up_8192x4096x11008"
 
