@@ -52,11 +52,12 @@ def test_w4a8_gemm_bit_exact(w, orc, M, N, K, ydt):
     assert y.intact()
 
 
-@pytest.mark.parametrize("M", [16, 300])  # the decode kernel and the W4A8 kernel
-def test_w4a8_extreme_accumulators(w, orc, M):
+# the decode kernel and the W4A8 kernel; K = 131040 is the largest the call
+# accepts (16 * 128 * 8 * K just below 2^31) and ends in a partial k-block
+@pytest.mark.parametrize("M,N,K", [(16, 256, 16384), (300, 256, 16384), (16, 16, 131040), (130, 16, 131040)])
+def test_w4a8_extreme_accumulators(w, orc, M, N, K):
     """Largest |acc| the signed operands allow: a row of qx at -128 against
-    codes at -8 (and at 7), over K = 16384; acc exact, signs kept."""
-    N, K = 256, 16384
+    codes at -8 (and at 7); acc exact, signs kept."""
     r = np.random.default_rng(M)
     qx = r.integers(-127, 128, (M, K)).astype(np.int8)
     qx[0, :] = -128

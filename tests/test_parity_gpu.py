@@ -254,8 +254,11 @@ def test_gemm_bit_exact(w, orc, M, N, K, ydt):
     assert torch.equal(y2, y.t)
 
 
-def test_gemm_extreme_codes_do_not_overflow(w, orc):
-    M, N, K = 130, 264, 8192
+# the pair kernel at K = 8192; then K = 133136, the largest multiple of 16
+# the call accepts (127 * 127 * K just below 2^31, a partial last k-block),
+# on the one-CTA kernel (M <= 128) and the pair kernel
+@pytest.mark.parametrize("M,N,K", [(130, 264, 8192), (100, 16, 133136), (130, 16, 133136)])
+def test_gemm_extreme_codes_do_not_overflow(w, orc, M, N, K):
     qx, qw, sx, sw = _gemm_case(M, N, K, seed=5, extreme=True)
     acc = torch.empty(M, N, dtype=torch.int32, device="cuda")
     y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")

@@ -1506,7 +1506,6 @@ extern "C" sq_status w4a8_gemm_dequant(const int8_t *qx, const float *sx, const 
     sq_status st = check_device(&sms);
     if (st != SQ_OK) return st;
     cudaStream_t cs = (cudaStream_t)stream;
-    if (yt == SQ_BF16)
     if (M <= gemm::kDecMaxTokens) {
         if (yt == SQ_BF16)
             return gemm::dispatch_decode<__nv_bfloat16, false, true>(qx, sx, nullptr, qw4, sw, nullptr, (int)M,
