@@ -71,6 +71,11 @@ def parse():
                    help="only launch the 16 x 8192 -> 28672 decode GEMMs on random codes, three with int8 "
                         "weights then three with packed int4 weights, and exit (the workload of the decode "
                         "kernel's ncu capture)")
+    p.add_argument("--gemm-sweep", choices=["time", "launch"],
+                   help="time: w8a8_gemm_dequant over a sweep of K and M at N = 1024 and the two prefill "
+                        "shapes, 20 back-to-back launches per CUDA-graph replay, beside torch._int_mm "
+                        "(cuBLASLt, int32 out) as the library ceiling, one JSON line a shape; launch: only "
+                        "launch w8a8_gemm_dequant twice a shape (the launch list's workload); then exit")
     return p.parse_args()
 
 
@@ -1026,8 +1031,69 @@ def decode_launches():
         raise RuntimeError("a kernel gave up on a bounded wait")
 
 
+GEMM_SWEEP = ([(8192, k, 1024) for k in (128, 256, 512, 1024, 2048, 4096, 8192)]
+              + [(m, 1024, 1024) for m in (512, 2048, 4096, 6144, 10240, 16384, 32768)]
+              + [(2048, 4096, 4096), (8192, 4096, 1024)])
+
+
+def gemm_sweep(mode, rep=20, replays=8):
+    """The int8 GEMM + dequant alone on random codes (seed 0) of each
+    GEMM_SWEEP shape (M, K, N).  Back-to-back launches in one CUDA graph
+    show the per-launch cost a chain of linears pays (launch, prologue,
+    pipeline fill, final epilogue) beside the main loop's; torch._int_mm
+    beside it is the library's int8 GEMM (no dequant, int32 out), a
+    ceiling for comparison only."""
+    import torch
+
+    import w8a8_linear_layers_b200 as w
+    dev = "cuda"
+    for M, K, N in GEMM_SWEEP:
+        g = torch.Generator(device=dev).manual_seed(0)
+        qx = torch.randint(-127, 128, (M, K), device=dev, dtype=torch.int8, generator=g)
+        qw = torch.randint(-127, 128, (N, K), device=dev, dtype=torch.int8, generator=g)
+        sx = torch.rand(M, device=dev, generator=g) * 1e-2
+        sw = torch.rand(N, device=dev, generator=g) * 1e-2
+        y = torch.empty(M, N, device=dev, dtype=torch.bfloat16)
+        if mode == "launch":
+            for _ in range(2):
+                w.w8a8_gemm_dequant(qx, sx, qw, sw, y)
+            torch.cuda.synchronize()
+            continue
+        line = dict(M=M, K=K, N=N)
+        for name, fn in (("w8a8_gemm_dequant", lambda: w.w8a8_gemm_dequant(qx, sx, qw, sw, y)),
+                         ("library_int_mm", lambda: torch._int_mm(qx, qw.t()))):
+            s = torch.cuda.Stream()
+            s.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(s):
+                for _ in range(3):
+                    fn()
+            torch.cuda.current_stream().wait_stream(s)
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for _ in range(rep):
+                    fn()
+            ts = []
+            for _ in range(replays):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                torch.cuda.synchronize()
+                e0.record()
+                graph.replay()
+                e1.record()
+                torch.cuda.synchronize()
+                ts.append(e0.elapsed_time(e1) * 1e3 / rep)
+            del graph
+            us = sorted(ts)[len(ts) // 2]
+            line[name] = dict(us=round(us, 2), tops=round(2.0 * M * N * K / us / 1e6, 1))
+        print(json.dumps(line), flush=True)
+    if w.device_fault() != 0:
+        raise RuntimeError("a kernel gave up on a bounded wait")
+
+
 def main():
     args = parse()
+    if args.gemm_sweep:
+        gemm_sweep(args.gemm_sweep)
+        return
     if args.decode_launches:
         decode_launches()
         return
