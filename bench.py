@@ -71,6 +71,10 @@ def parse():
                    help="only launch the 16 x 8192 -> 28672 decode GEMMs on random codes, three with int8 "
                         "weights then three with packed int4 weights, and exit (the workload of the decode "
                         "kernel's ncu capture)")
+    p.add_argument("--next-row-launches", action="store_true",
+                   help="only launch, on the MLP up-projection inputs (8192 x 4096 -> 11008, seed 0), the "
+                        "asymmetric SSZ twice, then the int4 SSZ, packing and three W4A8 GEMMs, and exit (the "
+                        "workload of those kernels' ncu captures)")
     p.add_argument("--gemm-sweep", choices=["time", "launch"],
                    help="time: w8a8_gemm_dequant over a sweep of K and M at N = 1024 and the two prefill "
                         "shapes, 20 back-to-back launches per CUDA-graph replay, beside torch._int_mm "
@@ -1089,8 +1093,46 @@ def gemm_sweep(mode, rep=20, replays=8):
         raise RuntimeError("a kernel gave up on a bounded wait")
 
 
+def next_row_launches():
+    """The asymmetric SSZ (twice), then the int4 SSZ, its packing and three
+    W4A8 GEMMs on the 8192 x 4096 -> 11008 MLP up-projection inputs (seed 0,
+    alpha 0.8, 20 rounds), for ncu captures of those kernels."""
+    import torch
+
+    import synthetic
+    import w8a8_linear_layers_b200 as w
+    cfg = synthetic.CONFIGS[DEFAULT_WORKLOAD]
+    x_cpu, w_cpu = synthetic.make_linear(cfg, seed=0)
+    x, wt = x_cpu.cuda(), w_cpu.cuda()
+    M, K = x.shape
+    N = wt.shape[0]
+    f32 = dict(device="cuda", dtype=torch.float32)
+    ax, aw, s, inv_s = (torch.empty(K, **f32) for _ in range(4))
+    w.sq_calib_absmax(x, ax)
+    w.sq_smooth_fold(ax, wt, cfg.alpha, aw, s, inv_s)
+    q = torch.empty(N, K, device="cuda", dtype=torch.int8)
+    sw, ow = torch.empty(N, **f32), torch.empty(N, **f32)
+    for _ in range(2):
+        w.ssz_quant_weight_asym(wt, s, 20, q, sw, ow)
+    w.ssz_quant_weight(wt, s, 4, 20, q, sw)
+    packed = torch.empty(N, K // 2, device="cuda", dtype=torch.uint8)
+    w.sq_pack_int4(q, packed)
+    qx = torch.empty(M, K, device="cuda", dtype=torch.int8)
+    sx = torch.empty(M, **f32)
+    w.quant_act_per_token(x, inv_s, qx, sx)
+    y = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
+    for _ in range(3):
+        w.w4a8_gemm_dequant(qx, sx, packed, sw, y)
+    torch.cuda.synchronize()
+    if w.device_fault() != 0:
+        raise RuntimeError("a kernel gave up on a bounded wait")
+
+
 def main():
     args = parse()
+    if args.next_row_launches:
+        next_row_launches()
+        return
     if args.gemm_sweep:
         gemm_sweep(args.gemm_sweep)
         return
