@@ -167,6 +167,18 @@ __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t
         : "memory");
 }
 
+// The same MMA with the A operand (M = 128 rows, K-major, four int8 per
+// 32-bit column) read from tensor memory at column a_tmem.
+__device__ __forceinline__ void mma_i8_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive on `bar` once every tcgen05 op this thread issued so far completes.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -187,6 +199,21 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr)
         : "memory");
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// 32 consecutive 32-bit TMEM columns of this thread's lane from registers
+// (warp-collective), then wait until the stores are done.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+          "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+          "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // Shared-memory matrix descriptor for a K-major operand tile written by TMA
@@ -1270,7 +1297,10 @@ static bool make_map_out(CUtensorMap *map, const void *base, int64_t rows, int64
 
 // Packed int4 weights [rows, K/2 bytes]: box [box_rows, 64 bytes] (BK codes),
 // no swizzle (the converter warps read it with plain loads).
-static bool make_map_int4(CUtensorMap *map, const void *base, int64_t rows, int64_t K, int box_rows) {
+// swizzle64: the 64-byte rows of a box land in shared memory with 16-byte
+// piece j of row r at piece j ^ ((r >> 1) & 3) (TMA 64B swizzle)
+static bool make_map_int4(CUtensorMap *map, const void *base, int64_t rows, int64_t K, int box_rows,
+                          bool swizzle64 = false) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
@@ -1278,8 +1308,8 @@ static bool make_map_int4(CUtensorMap *map, const void *base, int64_t rows, int6
     cuuint32_t box[2] = {(cuuint32_t)(BK / 2), (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -1321,7 +1351,7 @@ static sq_status launch_decode(const int8_t *qx, const float *sx, const int32_t 
                                int sms, cudaStream_t st) {
     using C = CfgDec<NT, INT4>;
     CUtensorMap mw, mx;
-    const bool okw = INT4 ? make_map_int4(&mw, qw, N, K, kDecRows) : make_map(&mw, qw, N, K, kDecRows);
+    const bool okw = INT4 ? make_map_int4(&mw, qw, N, K, kDecRows, true) : make_map(&mw, qw, N, K, kDecRows);
     if (!okw || !make_map(&mx, qx, M, K, NT))
         return fail(SQ_ERR_CUDA, "w8a8 decode GEMM: cuTensorMapEncodeTiled failed");
     auto kern = w8a8_gemm_decode_kernel<NT, OutT, ASYM, INT4>;

@@ -22,12 +22,14 @@
 //     S partials of rows [r 128/S, (r+1) 128/S) through distributed shared
 //     memory (exact int32) and runs the dequant for them.  No global
 //     scratch memory;
-//   * int4 weights (two per byte) arrive packed and are unpacked to the
-//     int8 operand layout (three unpacked tiles in flight) by eight
-//     converter warps, the first four of which then run the epilogue.
+//   * int4 weights (two per byte) arrive packed (64-byte rows, TMA 64B
+//     swizzle) and are unpacked by eight converter warps straight into
+//     tensor memory, which the MMA reads as its A operand (three unpacked
+//     tiles in flight); the first four converter warps then run the
+//     epilogue.
 //
 // Warp roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps
-// 2..5 epilogue (int4: warps 2..9 convert first).  Every wait is bounded as in the
+// 2..5 epilogue (int4: warps 2..9 convert first, in two groups of four).  Every wait is bounded as in the
 // other GEMM kernels; no TMA multicast.
 
 namespace w8a8 {
@@ -44,9 +46,10 @@ namespace gemm {
 #endif
 constexpr int kDecRows = 128;  // weight rows per CTA (= MMA M = TMEM lanes)
 constexpr int kDecConvWarps = W8A8_DEC_CONV_WARPS;  // int4 unpacking warps (the first 4 also run the epilogue)
-// the converter warps form groups that take alternate k-blocks, so that
-// several stages are unpacked at once (the unpacking of one stage is
-// latency-bound: shared load, ALU, shared store, proxy fence, arrive)
+// the converter warps form groups of four (one warp per TMEM lane quarter,
+// one weight row per thread) that take alternate k-blocks, so that several
+// stages are unpacked at once (the unpacking of one stage is latency-bound:
+// shared loads, ALU, TMEM store, fence, arrive)
 constexpr int kDecConvGroups = W8A8_DEC_CONV_GROUPS;
 constexpr int kDecConvGroupThreads = kDecConvWarps * 32 / kDecConvGroups;
 // producer, MMA, then 4 epilogue warps (int4: the converter warps)
@@ -61,12 +64,18 @@ struct CfgDec {
     static constexpr int RAW_BYTES = INT4 ? kDecRows * BK / 2 : W_BYTES;  // weight tile as loaded
     static constexpr int X_BYTES = NT * BK;                               // token tile (MMA B)
     static constexpr int IN_BYTES = RAW_BYTES + X_BYTES;
-    static constexpr int OP_STAGES = INT4 ? W8A8_DEC_OP_STAGES : 0;  // unpacked weight tiles
-    static constexpr int IN_OFFSET = OP_STAGES * W_BYTES;
+    static constexpr int OP_STAGES = INT4 ? W8A8_DEC_OP_STAGES : 0;  // unpacked weight tiles (in TMEM)
+    static constexpr int IN_OFFSET = 0;
     static constexpr int STAGES_FIT = (kDecBudget - IN_OFFSET) / IN_BYTES;
     static constexpr int STAGES = STAGES_FIT < 8 ? STAGES_FIT : 8;
     static constexpr int SMEM = IN_OFFSET + STAGES * IN_BYTES + 1024;  // + alignment slack
-    static constexpr int TMEM_COLS = NT < 32 ? 32 : NT;
+    // TMEM: the accumulator (NT columns), then OP_STAGES unpacked weight
+    // tiles of BK / 4 columns (128 rows x 128 int8, four per 32-bit column)
+    static constexpr int ACC_COLS = NT < 32 ? 32 : NT;
+    static constexpr int A_COLS = BK / 4;
+    static constexpr int USED_COLS = ACC_COLS + OP_STAGES * A_COLS;
+    static constexpr int TMEM_COLS = USED_COLS <= 32 ? 32 : USED_COLS <= 64 ? 64 : USED_COLS <= 128 ? 128 : 256;
+    static_assert(USED_COLS <= 256, "two CTAs per SM share 512 TMEM columns");
     static constexpr int RED_BYTES = NT * kDecRows * 4;  // int32 partial, over the stages
     static_assert(STAGES >= 3, "decode pipeline too shallow");
     // a converter group's previous k-block (kb - G) made it wait for the MMA
@@ -75,8 +84,7 @@ struct CfgDec {
     // apart): G <= OP_STAGES
     static_assert(!INT4 || (kDecConvGroups >= 1 && kDecConvGroups <= OP_STAGES && STAGES >= OP_STAGES),
                   "converter groups must not run more than one phase ahead");
-    static_assert(kDecConvWarps * 32 % kDecConvGroups == 0 && 512 % kDecConvGroupThreads == 0,
-                  "a packed tile splits evenly over a group");
+    static_assert(!INT4 || kDecConvGroupThreads == kDecRows, "a converter group is one thread per weight row");
     static_assert(IN_BYTES % 1024 == 0 && RAW_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
     static_assert(RED_BYTES <= STAGES * IN_BYTES, "partial must fit over the stages");
 };
@@ -129,9 +137,11 @@ __device__ __forceinline__ void dec_store(int32_t acc, int t, int n, int N, cons
 // Synchronisation:
 //   in_full[s]  : producer's expect_tx; the weight and token TMAs complete it.
 //   in_empty[s] : MMA commit (the MMA is the last reader of a stage).
-//   op_full[p]  : int4: one arrival per converter thread after its fenced
-//                 writes (it waited for in_full first, so op_full implies it).
-//   op_empty[p] : int4: MMA commit.
+//   op_full[p]  : int4: one arrival per converter thread after its TMEM
+//                 stores completed and were fenced (it waited for in_full
+//                 first, so op_full implies it).
+//   op_empty[p] : int4: MMA commit (the MMA is the last reader of the
+//                 unpacked tile in TMEM).
 //   tfull       : MMA commit after the CTA's last k-block.
 template <int NT, typename OutT, bool ASYM, bool INT4>
 __global__ void __launch_bounds__(dec_threads(INT4), 2)
@@ -240,12 +250,17 @@ w8a8_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
                 }
                 tc_fence_after();
                 const uint32_t in_addr = smem_base + C::IN_OFFSET + stage * C::IN_BYTES;
-                const uint32_t a_addr = INT4 ? smem_base + os * C::W_BYTES : in_addr;
                 const uint32_t b_addr = in_addr + C::RAW_BYTES;
 #pragma unroll
-                for (int k = 0; k < BK / UMMA_K; ++k)
-                    mma_i8(tmem_base, smem_desc_sw128(a_addr + k * UMMA_K), smem_desc_sw128(b_addr + k * UMMA_K),
-                           idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+                for (int k = 0; k < BK / UMMA_K; ++k) {
+                    const uint32_t acc = (kb > kb0 || k > 0) ? 1u : 0u;
+                    if (INT4)  // A: the unpacked tile in TMEM, UMMA_K / 4 columns per step
+                        mma_i8_tmem_a(tmem_base, tmem_base + (uint32_t)(C::ACC_COLS + os * C::A_COLS + k * (UMMA_K / 4)),
+                                      smem_desc_sw128(b_addr + k * UMMA_K), idesc, acc);
+                    else
+                        mma_i8(tmem_base, smem_desc_sw128(in_addr + k * UMMA_K), smem_desc_sw128(b_addr + k * UMMA_K),
+                               idesc, acc);
+                }
                 issued_any = true;
                 mma_commit(smem_u32(&in_empty[stage]));
                 if (INT4) mma_commit(smem_u32(&op_empty[os]));
@@ -273,41 +288,43 @@ w8a8_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
         bool ok = true;
         if (INT4) {
             // ------------------------------------------ converters
-            // A packed tile is 128 rows x 64 bytes: 512 16-byte pieces over
-            // the threads of one converter group; piece i = (row i/4, bytes
-            // 16 (i%4) ..), unpacked into 16-byte chunks 2 (i%4) and
-            // 2 (i%4) + 1 of the row (128B swizzle).  Group g takes the
-            // k-blocks kb0 + g, kb0 + g + G, ...; the ring positions and
-            // phases follow from the k-block's index.
+            // A packed tile is 128 rows x 64 bytes (TMA 64B swizzle: piece
+            // j of row r at piece j ^ ((r >> 1) & 3), so the 8 rows a
+            // quarter-warp reads at once fall in distinct banks).  Each
+            // thread unpacks one weight row r = 32 (warp % 4) + lane (a
+            // warp may only access TMEM lanes 32 (warp % 4) ..) into 32
+            // words and stores them to lane r, columns [ACC_COLS + 32 p,
+            // +32) for unpacked tile p.  Group g takes the k-blocks kb0 + g,
+            // kb0 + g + G, ...; the ring positions and phases follow from
+            // the k-block's index.
             constexpr int kOps = INT4 ? C::OP_STAGES : 1;  // (this branch only runs for int4)
-            const int grp = ct / kDecConvGroupThreads, gt = ct % kDecConvGroupThreads;
+            const int grp = ct / kDecConvGroupThreads;
+            const int row = (warp & 3) * 32 + lane;  // this thread's TMEM lane = weight row of the tile
+            const uint32_t lane_base = tmem_base + ((uint32_t)((warp & 3) * 32) << 16);
+            const int rot = (row >> 1) & 3;
             for (int kb = kb0 + grp; kb < kb1; kb += kDecConvGroups) {
                 const int u = kb - kb0;
                 const int stage = u % C::STAGES, os = u % kOps;
                 const uint32_t phase = (uint32_t)(u / C::STAGES) & 1u, oph = (uint32_t)(u / kOps) & 1u;
-                if (!wait_bounded(smem_u32(&op_empty[os]), oph ^ 1u, &abort_flag, kFaultConvert) ||
-                    !wait_bounded(smem_u32(&in_full[stage]), phase, &abort_flag, kFaultConvert)) {
+                const bool got = wait_bounded(smem_u32(&op_empty[os]), oph ^ 1u, &abort_flag, kFaultConvert) &&
+                                 wait_bounded(smem_u32(&in_full[stage]), phase, &abort_flag, kFaultConvert);
+                if (!__all_sync(0xffffffffu, got)) {  // the TMEM store below is warp-collective
                     ok = false;
                     break;
                 }
-                const uint8_t *raw = gbase + C::IN_OFFSET + stage * C::IN_BYTES;
-                uint8_t *wdst = gbase + os * C::W_BYTES;
+                tc_fence_after();  // the MMA that last read this tile is done
+                const uint8_t *rowp = gbase + C::IN_OFFSET + stage * C::IN_BYTES + row * (BK / 2);
+                uint32_t o[32];
 #pragma unroll
-                for (int it = 0; it < 512 / kDecConvGroupThreads; ++it) {
-                    const int i = it * kDecConvGroupThreads + gt;
-                    const int r = i >> 2, sub = i & 3;
-                    const uint4 p = *reinterpret_cast<const uint4 *>(raw + r * (BK / 2) + sub * 16);
-                    uint32_t o[8];
-                    unpack_int4x8(p.x, o[0], o[1]);
-                    unpack_int4x8(p.y, o[2], o[3]);
-                    unpack_int4x8(p.z, o[4], o[5]);
-                    unpack_int4x8(p.w, o[6], o[7]);
-                    uint8_t *rowp = wdst + (r >> 3) * 1024 + (r & 7) * 128;
-                    *reinterpret_cast<uint4 *>(rowp + (((2 * sub) ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-                    *reinterpret_cast<uint4 *>(rowp + (((2 * sub + 1) ^ (r & 7)) << 4)) =
-                        make_uint4(o[4], o[5], o[6], o[7]);
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 p = *reinterpret_cast<const uint4 *>(rowp + ((j ^ rot) << 4));
+                    unpack_int4x8(p.x, o[8 * j + 0], o[8 * j + 1]);
+                    unpack_int4x8(p.y, o[8 * j + 2], o[8 * j + 3]);
+                    unpack_int4x8(p.z, o[8 * j + 4], o[8 * j + 5]);
+                    unpack_int4x8(p.w, o[8 * j + 6], o[8 * j + 7]);
                 }
-                fence_proxy_async_smem();  // the MMA reads these bytes through the async proxy
+                tmem_st32(lane_base + (uint32_t)(C::ACC_COLS + os * C::A_COLS), o);
+                tc_fence_before();  // the stores are ordered before the arrive the MMA waits on
                 mbar_arrive(smem_u32(&op_full[os]));
             }
         }
