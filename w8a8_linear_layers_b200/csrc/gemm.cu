@@ -1297,18 +1297,19 @@ static bool make_map_out(CUtensorMap *map, const void *base, int64_t rows, int64
 
 // Packed int4 weights [rows, K/2 bytes]: box [box_rows, 64 bytes] (BK codes),
 // no swizzle (the converter warps read it with plain loads).
-// swizzle64: the 64-byte rows of a box land in shared memory with 16-byte
-// piece j of row r at piece j ^ ((r >> 1) & 3) (TMA 64B swizzle)
+// box_bytes packed bytes of each of box_rows rows; swizzle128: the 128-byte
+// rows of a box land in shared memory with 16-byte piece j of row r at
+// piece j ^ (r & 7) (TMA 128B swizzle)
 static bool make_map_int4(CUtensorMap *map, const void *base, int64_t rows, int64_t K, int box_rows,
-                          bool swizzle64 = false) {
+                          int box_bytes = BK / 2, bool swizzle128 = false) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-    cuuint32_t box[2] = {(cuuint32_t)(BK / 2), (cuuint32_t)box_rows};
+    cuuint32_t box[2] = {(cuuint32_t)box_bytes, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -1336,10 +1337,11 @@ static sq_status launch_w4(const int8_t *qx, const float *sx, const uint8_t *qw4
 }
 
 // K split of the decode kernel: the largest power of two S <= 8 with
-// tiles x S CTAs <= two per SM and S <= k-blocks (every CTA gets one).
-static int decode_split(int N, int K, int sms) {
+// tiles x S CTAs <= two per SM and S <= k-blocks of kblock K each (every
+// CTA gets one).
+static int decode_split(int N, int K, int sms, int kblock) {
     const int tiles = (N + kDecRows - 1) / kDecRows;
-    const int num_kb = (K + BK - 1) / BK;
+    const int num_kb = (K + kblock - 1) / kblock;
     int s = 1;
     while (s < kDecMaxSplit && tiles * (2 * s) <= 2 * sms && 2 * s <= num_kb) s *= 2;
     return s;
@@ -1351,7 +1353,7 @@ static sq_status launch_decode(const int8_t *qx, const float *sx, const int32_t 
                                int sms, cudaStream_t st) {
     using C = CfgDec<NT, INT4>;
     CUtensorMap mw, mx;
-    const bool okw = INT4 ? make_map_int4(&mw, qw, N, K, kDecRows, true) : make_map(&mw, qw, N, K, kDecRows);
+    const bool okw = INT4 ? make_map_int4(&mw, qw, N, K, kDecRows, C::KB / 2, true) : make_map(&mw, qw, N, K, kDecRows);
     if (!okw || !make_map(&mx, qx, M, K, NT))
         return fail(SQ_ERR_CUDA, "w8a8 decode GEMM: cuTensorMapEncodeTiled failed");
     auto kern = w8a8_gemm_decode_kernel<NT, OutT, ASYM, INT4>;
@@ -1366,7 +1368,7 @@ static sq_status launch_decode(const int8_t *qx, const float *sx, const int32_t 
         if (e != cudaSuccess) return fail(SQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
         configured_dev[dev] = 1;
     }
-    const int split = decode_split(N, K, sms);
+    const int split = decode_split(N, K, sms, C::KB);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(((N + kDecRows - 1) / kDecRows) * split), 1, 1);
     cfg.blockDim = dim3(dec_threads(INT4), 1, 1);

@@ -22,11 +22,11 @@
 //     S partials of rows [r 128/S, (r+1) 128/S) through distributed shared
 //     memory (exact int32) and runs the dequant for them.  No global
 //     scratch memory;
-//   * int4 weights (two per byte) arrive packed (64-byte rows, TMA 64B
-//     swizzle) and are unpacked by eight converter warps straight into
-//     tensor memory, which the MMA reads as its A operand (three unpacked
-//     tiles in flight); the first four converter warps then run the
-//     epilogue.
+//   * int4 weights (two per byte) arrive packed, 256 K a k-block (128-byte
+//     rows, TMA 128B swizzle), and are unpacked by eight converter warps
+//     straight into tensor memory, which the MMA reads as its A operand
+//     (three unpacked tiles in flight); the first four converter warps
+//     then run the epilogue.
 //
 // Warp roles: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps
 // 2..5 epilogue (int4: warps 2..9 convert first, in two groups of four).  Every wait is bounded as in the
@@ -58,11 +58,18 @@ constexpr int kDecMaxSplit = 8;   // portable cluster size
 constexpr int kDecMaxTokens = 64;
 constexpr int kDecBudget = 108 * 1024;  // dynamic shared memory, two CTAs per SM
 
+// K per k-block: int4 weights take 256 (128 packed bytes a row, as many
+// bytes a stage as int8's 128), which halves the k-blocks and so the
+// per-k-block handshakes of the unpacking pipeline
+__host__ __device__ constexpr int dec_kblock(bool int4) { return int4 ? 2 * BK : BK; }
+
 template <int NT, bool INT4>
 struct CfgDec {
+    static constexpr int KB = dec_kblock(INT4);
     static constexpr int W_BYTES = kDecRows * BK;                         // int8 weight tile (MMA A)
-    static constexpr int RAW_BYTES = INT4 ? kDecRows * BK / 2 : W_BYTES;  // weight tile as loaded
-    static constexpr int X_BYTES = NT * BK;                               // token tile (MMA B)
+    static constexpr int RAW_BYTES = INT4 ? kDecRows * KB / 2 : W_BYTES;  // weight tile as loaded
+    static constexpr int X_ATOM = NT * BK;                                // token rows x 128 bytes (one swizzle atom)
+    static constexpr int X_BYTES = NT * KB;                               // token tile (MMA B), KB / 128 atoms
     static constexpr int IN_BYTES = RAW_BYTES + X_BYTES;
     static constexpr int OP_STAGES = INT4 ? W8A8_DEC_OP_STAGES : 0;  // unpacked weight tiles (in TMEM)
     static constexpr int IN_OFFSET = 0;
@@ -70,9 +77,9 @@ struct CfgDec {
     static constexpr int STAGES = STAGES_FIT < 8 ? STAGES_FIT : 8;
     static constexpr int SMEM = IN_OFFSET + STAGES * IN_BYTES + 1024;  // + alignment slack
     // TMEM: the accumulator (NT columns), then OP_STAGES unpacked weight
-    // tiles of BK / 4 columns (128 rows x 128 int8, four per 32-bit column)
+    // tiles of KB / 4 columns (128 rows x KB int8, four per 32-bit column)
     static constexpr int ACC_COLS = NT < 32 ? 32 : NT;
-    static constexpr int A_COLS = BK / 4;
+    static constexpr int A_COLS = KB / 4;
     static constexpr int USED_COLS = ACC_COLS + OP_STAGES * A_COLS;
     static constexpr int TMEM_COLS = USED_COLS <= 32 ? 32 : USED_COLS <= 64 ? 64 : USED_COLS <= 128 ? 128 : 256;
     static_assert(USED_COLS <= 256, "two CTAs per SM share 512 TMEM columns");
@@ -168,7 +175,7 @@ w8a8_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
     const int split = (int)cluster_nctarank();
     const int rank = (int)cluster_ctarank();
     const int n0 = (int)(blockIdx.x / split) * kDecRows;
-    const int num_kb = (K + BK - 1) / BK;
+    const int num_kb = (K + C::KB - 1) / C::KB;
     const int kb0 = (int)((int64_t)num_kb * rank / split);
     const int kb1 = (int)((int64_t)num_kb * (rank + 1) / split);  // the host keeps kb1 > kb0
 
@@ -210,9 +217,12 @@ w8a8_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
                 }
                 const uint32_t w_dst = smem_base + C::IN_OFFSET + stage * C::IN_BYTES;
                 const uint32_t fb = smem_u32(&in_full[stage]);
-                mbar_arrive_expect_tx(fb, C::IN_BYTES);
-                tma_load_2d(w_dst, &tmap_w, fb, INT4 ? kb * (BK / 2) : kb * BK, n0);
-                tma_load_2d(w_dst + C::RAW_BYTES, &tmap_x, fb, kb * BK, 0);
+                // token atoms that start inside K (the weights' tail is zero-filled)
+                const int atoms = min(C::KB / BK, (K - kb * C::KB + BK - 1) / BK);
+                mbar_arrive_expect_tx(fb, C::RAW_BYTES + atoms * C::X_ATOM);
+                tma_load_2d(w_dst, &tmap_w, fb, INT4 ? kb * (C::KB / 2) : kb * BK, n0);
+                for (int a = 0; a < atoms; ++a)
+                    tma_load_2d(w_dst + C::RAW_BYTES + a * C::X_ATOM, &tmap_x, fb, kb * C::KB + a * BK, 0);
                 ++issued;
                 if (++stage == C::STAGES) {
                     stage = 0;
@@ -251,15 +261,19 @@ w8a8_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
                 tc_fence_after();
                 const uint32_t in_addr = smem_base + C::IN_OFFSET + stage * C::IN_BYTES;
                 const uint32_t b_addr = in_addr + C::RAW_BYTES;
+                // MMA steps that start inside K (K is a multiple of 16, and of 32 for int4)
+                const int steps = min(C::KB / UMMA_K, (K - kb * C::KB + UMMA_K - 1) / UMMA_K);
 #pragma unroll
-                for (int k = 0; k < BK / UMMA_K; ++k) {
+                for (int k = 0; k < C::KB / UMMA_K; ++k) {
+                    if (k >= steps) break;
                     const uint32_t acc = (kb > kb0 || k > 0) ? 1u : 0u;
+                    // B: token atom k / 4, 32 bytes per step within its 128-byte rows
+                    const uint32_t bk = b_addr + (uint32_t)((k / (BK / UMMA_K)) * C::X_ATOM + (k % (BK / UMMA_K)) * UMMA_K);
                     if (INT4)  // A: the unpacked tile in TMEM, UMMA_K / 4 columns per step
                         mma_i8_tmem_a(tmem_base, tmem_base + (uint32_t)(C::ACC_COLS + os * C::A_COLS + k * (UMMA_K / 4)),
-                                      smem_desc_sw128(b_addr + k * UMMA_K), idesc, acc);
+                                      smem_desc_sw128(bk), idesc, acc);
                     else
-                        mma_i8(tmem_base, smem_desc_sw128(in_addr + k * UMMA_K), smem_desc_sw128(b_addr + k * UMMA_K),
-                               idesc, acc);
+                        mma_i8(tmem_base, smem_desc_sw128(in_addr + k * UMMA_K), smem_desc_sw128(bk), idesc, acc);
                 }
                 issued_any = true;
                 mma_commit(smem_u32(&in_empty[stage]));
@@ -288,20 +302,20 @@ w8a8_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
         bool ok = true;
         if (INT4) {
             // ------------------------------------------ converters
-            // A packed tile is 128 rows x 64 bytes (TMA 64B swizzle: piece
-            // j of row r at piece j ^ ((r >> 1) & 3), so the 8 rows a
+            // A packed tile is 128 rows x 128 bytes (TMA 128B swizzle:
+            // piece j of row r at piece j ^ (r & 7), so the 8 rows a
             // quarter-warp reads at once fall in distinct banks).  Each
             // thread unpacks one weight row r = 32 (warp % 4) + lane (a
-            // warp may only access TMEM lanes 32 (warp % 4) ..) into 32
-            // words and stores them to lane r, columns [ACC_COLS + 32 p,
-            // +32) for unpacked tile p.  Group g takes the k-blocks kb0 + g,
-            // kb0 + g + G, ...; the ring positions and phases follow from
-            // the k-block's index.
+            // warp may only access TMEM lanes 32 (warp % 4) ..), 256 codes,
+            // into 64 words, stored in two halves to lane r, columns
+            // [ACC_COLS + 64 p, +64) for unpacked tile p.  Group g takes the
+            // k-blocks kb0 + g, kb0 + g + G, ...; the ring positions and
+            // phases follow from the k-block's index.
             constexpr int kOps = INT4 ? C::OP_STAGES : 1;  // (this branch only runs for int4)
             const int grp = ct / kDecConvGroupThreads;
             const int row = (warp & 3) * 32 + lane;  // this thread's TMEM lane = weight row of the tile
             const uint32_t lane_base = tmem_base + ((uint32_t)((warp & 3) * 32) << 16);
-            const int rot = (row >> 1) & 3;
+            const int rot = row & 7;
             for (int kb = kb0 + grp; kb < kb1; kb += kDecConvGroups) {
                 const int u = kb - kb0;
                 const int stage = u % C::STAGES, os = u % kOps;
@@ -313,17 +327,20 @@ w8a8_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid
                     break;
                 }
                 tc_fence_after();  // the MMA that last read this tile is done
-                const uint8_t *rowp = gbase + C::IN_OFFSET + stage * C::IN_BYTES + row * (BK / 2);
-                uint32_t o[32];
+                const uint8_t *rowp = gbase + C::IN_OFFSET + stage * C::IN_BYTES + row * (C::KB / 2);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint4 p = *reinterpret_cast<const uint4 *>(rowp + ((j ^ rot) << 4));
-                    unpack_int4x8(p.x, o[8 * j + 0], o[8 * j + 1]);
-                    unpack_int4x8(p.y, o[8 * j + 2], o[8 * j + 3]);
-                    unpack_int4x8(p.z, o[8 * j + 4], o[8 * j + 5]);
-                    unpack_int4x8(p.w, o[8 * j + 6], o[8 * j + 7]);
+                for (int h = 0; h < C::KB / 128; ++h) {
+                    uint32_t o[32];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint4 p = *reinterpret_cast<const uint4 *>(rowp + (((4 * h + j) ^ rot) << 4));
+                        unpack_int4x8(p.x, o[8 * j + 0], o[8 * j + 1]);
+                        unpack_int4x8(p.y, o[8 * j + 2], o[8 * j + 3]);
+                        unpack_int4x8(p.z, o[8 * j + 4], o[8 * j + 5]);
+                        unpack_int4x8(p.w, o[8 * j + 6], o[8 * j + 7]);
+                    }
+                    tmem_st32(lane_base + (uint32_t)(C::ACC_COLS + os * C::A_COLS + 32 * h), o);
                 }
-                tmem_st32(lane_base + (uint32_t)(C::ACC_COLS + os * C::A_COLS), o);
                 tc_fence_before();  // the stores are ordered before the arrive the MMA waits on
                 mbar_arrive(smem_u32(&op_full[os]));
             }
