@@ -959,7 +959,8 @@ NCU_KERNELS = [("col_absmax_kernel", None), ("smooth_factor_kernel", "smooth_fol
 
 def record_traffic(csv_path, workload):
     """DRAM bytes per launch of each kernel from an ncu capture of this
-    bench's workload; written with the hash of each kernel's source so the
+    bench's workload (all its kernels, or some of them: the others keep their
+    earlier records); written with the hash of each kernel's source so the
     numbers are dropped once the kernel changes."""
     import csv
     import collections
@@ -1003,7 +1004,7 @@ def record_traffic(csv_path, workload):
                          "src_sha": source_sha(KERNEL_SOURCES[step])}
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     allw = json.load(open(path)) if os.path.exists(path) else {}
-    allw[workload] = out
+    allw.setdefault(workload, {}).update(out)  # a capture of some kernels keeps the others' records
     with open(path, "w") as f:
         json.dump(allw, f, indent=1, sort_keys=True)
     print(json.dumps(out, indent=1))
