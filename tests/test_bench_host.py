@@ -96,3 +96,28 @@ def test_recorded_traffic_matches_the_current_sources(bench):
         got = bench.dram_traffic(step, "prefill_2048x4096x4096")
         assert got is None or got > 0
     assert bench.dram_traffic("ssz_quant_weight", "no_such_workload") is None
+
+
+def test_partial_traffic_capture_keeps_other_records(bench, tmp_path, monkeypatch):
+    """A capture of one kernel updates that step's record and leaves the
+    workload's other records as they were."""
+    import csv
+    import json
+    (tmp_path / "profiles").mkdir()
+    path = tmp_path / "profiles" / "dram_traffic.json"
+    old = {"w": {"ssz_quant_weight": {"bytes_per_launch": 7, "launches": 1, "src_sha": "a"},
+                 "w8a8_gemm_dequant": {"bytes_per_launch": 5, "launches": 1, "src_sha": "old"}}}
+    path.write_text(json.dumps(old))
+    rows = [["ID", "Kernel Name", "Metric Name", "Metric Unit", "Metric Value"]]
+    name = "void w8a8_gemm_pair_kernel<__nv_bfloat16, 0>(...)"
+    rows += [["0", name, "dram__bytes_read.sum", "Mbyte", "98.5"], ["0", name, "dram__bytes_write.sum", "byte", "1,500"],
+             ["0", name, "gpu__time_duration.sum", "usecond", "240"]]
+    cap = tmp_path / "cap.csv"
+    with open(cap, "w", newline="") as f:
+        csv.writer(f, quoting=csv.QUOTE_ALL).writerows(rows)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "source_sha", lambda files: "new")
+    bench.record_traffic(str(cap), "w")
+    got = json.loads(path.read_text())["w"]
+    assert got["ssz_quant_weight"] == old["w"]["ssz_quant_weight"]
+    assert got["w8a8_gemm_dequant"] == {"bytes_per_launch": 98501500, "launches": 1, "src_sha": "new"}
