@@ -88,6 +88,7 @@ def test_quant_rowsum_bit_exact(w, orc, M, K, dtype):
 @pytest.mark.parametrize("M,N,K,ydt", [
     (1, 8, 16, torch.bfloat16), (77, 264, 272, torch.float32), (128, 512, 1024, torch.bfloat16),
     (300, 520, 4096, torch.bfloat16), (1000, 1032, 2064, torch.float32),
+    (128, 520, 4096, torch.bfloat16), (90, 264, 2080, torch.float32),  # 128-token decode tiles
 ])
 def test_gemm_asym_bit_exact(w, orc, M, N, K, ydt):
     r = np.random.default_rng(M * N + K)

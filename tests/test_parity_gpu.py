@@ -234,6 +234,9 @@ def _gemm_case(M, N, K, seed, extreme=False):
     (128, 256, 128, torch.bfloat16), (256, 512, 256, torch.float32), (16, 128, 256, torch.float32),
     (300, 520, 4096, torch.bfloat16), (1000, 2056, 1040, torch.bfloat16), (16, 28672, 512, torch.bfloat16),
     (200, 24, 64, torch.bfloat16), (130, 12, 48, torch.float32), (520, 392, 272, torch.float32),
+    # 64 < M <= 128 with few column tiles and a long K: the decode kernel's
+    # 128-token tiles (split K); then the one-CTA kernel with a short K
+    (120, 1040, 4096, torch.bfloat16), (65, 264, 2048, torch.float32), (100, 264, 1024, torch.bfloat16),
 ])
 def test_gemm_bit_exact(w, orc, M, N, K, ydt):
     qx, qw, sx, sw = _gemm_case(M, N, K, seed=M * 31 + N * 7 + K)

@@ -1388,13 +1388,17 @@ static sq_status launch_decode(const int8_t *qx, const float *sx, const int32_t 
     return launch_status("w8a8_gemm_decode_kernel");
 }
 
-// Token-tile width of the decode kernel for M <= 64 tokens.
+// Token-tile width of the decode kernel: 16, 32 or 64 tokens, and 128 for
+// int8 weights with 64 < M <= 128 (see gemm_entry).
 template <typename OutT, bool ASYM, bool INT4>
 static sq_status dispatch_decode(const int8_t *qx, const float *sx, const int32_t *rs, const void *qw,
                                  const float *sw, const float *ow, int M, int N, int K, void *y, int32_t *acc_out,
                                  int sms, cudaStream_t st) {
     if (M <= 16) return launch_decode<16, OutT, ASYM, INT4>(qx, sx, rs, qw, sw, ow, M, N, K, y, acc_out, sms, st);
     if (M <= 32) return launch_decode<32, OutT, ASYM, INT4>(qx, sx, rs, qw, sw, ow, M, N, K, y, acc_out, sms, st);
+    if constexpr (!INT4) {
+        if (M > 64) return launch_decode<128, OutT, ASYM, false>(qx, sx, rs, qw, sw, ow, M, N, K, y, acc_out, sms, st);
+    }
     return launch_decode<64, OutT, ASYM, INT4>(qx, sx, rs, qw, sw, ow, M, N, K, y, acc_out, sms, st);
 }
 
@@ -1477,8 +1481,14 @@ static sq_status gemm_entry(const char *fn, const int8_t *qx, const float *sx, c
     cudaStream_t cs = (cudaStream_t)stream;
     const int m = (int)M, n = (int)N, k = (int)K;
     // M <= 64: the weight-streaming decode kernel; M > 128: 256-row tiles on
-    // CTA pairs; otherwise one CTA per 128 x 256 tile
-    if (M <= gemm::kDecMaxTokens) {
+    // CTA pairs; otherwise one CTA per 128 x 256 tile, except where those
+    // tiles would leave most SMs idle over a long K: the decode kernel with
+    // 128-token tiles then splits K over a cluster (measured on B200 at 100
+    // to 128 tokens: 128 x 4096 -> 4096 20.5 against 26.6 us, 100 x 133136
+    // -> 16 74 against 372 us; with 43 column tiles, 128 x 4096 -> 11008, or
+    // a short K the one-CTA kernel stays ahead: 28.7 against 34.8 us)
+    const bool few_tiles = M <= 2 * gemm::kDecMaxTokens && (N + 255) / 256 <= sms / 8 && K >= 2048;
+    if (M <= gemm::kDecMaxTokens || few_tiles) {
         if (yt == SQ_BF16)
             return asym ? gemm::dispatch_decode<__nv_bfloat16, true, false>(qx, sx, rs, qw, sw, ow, m, n, k, y,
                                                                             acc_out, sms, cs)

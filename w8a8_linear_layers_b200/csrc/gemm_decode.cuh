@@ -1,5 +1,7 @@
-// gemm_decode.cuh -- the W8A8 / W4A8 GEMM for few tokens (M <= 64), included
-// by gemm.cu (it shares that file's PTX wrappers and fault word).
+// gemm_decode.cuh -- the W8A8 / W4A8 GEMM for few tokens (M <= 64; int8
+// weights also up to 128 tokens where the one-CTA kernel's tiles would leave
+// most SMs idle), included by gemm.cu (it shares that file's PTX wrappers
+// and fault word).
 //
 // Same operation as w8a8_gemm_kernel: y = dequant(qx qw^T) (CUDA INT8
 // quantization notes, aicoding.csdn.net, sections 3.2 and 4.2).  With few
@@ -8,7 +10,7 @@
 // stream the weights.  Here the operands swap roles:
 //
 //   * the MMA's A operand (M = 128, TMEM lanes) is a 128-row weight tile,
-//     its B operand (N = NT = 16, 32 or 64) the token tile; D[n][t] lands
+//     its B operand (N = NT = 16, 32, 64 or 128) the token tile; D[n][t] lands
 //     in TMEM lane n, column t, so the epilogue thread of weight row n
 //     writes y[t][n] for every token (32 lanes = 32 consecutive columns of
 //     y: coalesced);
